@@ -1,0 +1,386 @@
+"""Pins of the float64 oracle against facts fixed outside the oracle itself.
+
+* a hand-worked example with exact fractions (tests/golden/worked_example_block2.txt);
+* a library routine: torch's CPU scaled_dot_product_attention in float64;
+* closed forms (zero queries, one dominant key, saturated gates);
+* invariants stated by the pages (k covering every block -> dense attention,
+  window >= N -> dense attention, selected indices never past the causal
+  position, forced tokens always attended);
+* brute force: a scalar pure-Python transcription on N <= 256.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests import brute_force as BF
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "worked_example_block2.txt")
+
+
+def _gold():
+    vals = {}
+    with open(GOLD) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, rest = line.split(":", 1)
+            vals[key.strip()] = np.array([float(Fraction(x)) for x in rest.split()])
+    return vals
+
+
+def _sdpa(q, k, v):
+    """torch float64 causal SDPA with GQA by repeating K/V heads. q [Hq,N,D], k/v [Hkv,N,D]."""
+    G = q.shape[0] // k.shape[0]
+    kk = torch.from_numpy(np.repeat(k, G, axis=0)).double()
+    vv = torch.from_numpy(np.repeat(v, G, axis=0)).double()
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).double(), kk, vv, is_causal=True).numpy()
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# ----------------------------------------------------------------------------- worked example
+class TestWorkedExample:
+    g = _gold()
+    q = np.ones((1, 1, 4, 1))
+    k = np.array([0.0, math.log(2.0), 0.0, math.log(3.0)]).reshape(1, 1, 4, 1)
+    v = np.array([1.0, 2.0, 3.0, 4.0]).reshape(1, 1, 4, 1)
+
+    def test_dense(self):
+        o, lse = O.full_attention(self.q, self.k, self.v)
+        np.testing.assert_allclose(o[0, 0, :, 0], self.g["o"], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(np.exp(lse[0, 0]), self.g["lse_exp"], rtol=1e-13)
+
+    def test_block_max(self):
+        rows = np.arange(4)
+        p, _, _ = O.causal_softmax(self.q[0, 0], rows, self.k[0, 0])
+        s = O.block_max_probs(p, rows, block=2)
+        for t in range(4):
+            np.testing.assert_allclose(s[t], self.g[f"smax_t{t}"], atol=1e-13)
+
+    @pytest.mark.parametrize("red", ["sum", "max"])
+    def test_scores_and_topk(self, red):
+        sc = O.block_scores(self.q, self.k, red, block=2)
+        for I in range(2):
+            np.testing.assert_allclose(sc[0, 0, I], self.g[f"score_{red}_tile{I}"], atol=1e-13)
+        idx = O.topk_blocks(sc, 1)
+        assert idx[0, 0, 0, 0] == self.g["topk1_tile0"][0]
+        assert idx[0, 0, 1, 0] == self.g["topk1_tile1"][0]
+
+    def test_sparse_layer(self):
+        sel = np.zeros((1, 1, 2, 1), dtype=np.int64)
+        rows = np.arange(4)
+        o_sp = np.concatenate([O.sparse_branch_rows(self.q[0, 0][r], r, self.k[0, 0], self.v[0, 0], [0], 2)
+                               for r in (rows[:2], rows[2:])])[:, 0]
+        np.testing.assert_allclose(o_sp, self.g["sparse_branch"], atol=1e-13)
+        o_sw = O.swa_branch_rows(self.q[0, 0], rows, self.k[0, 0], self.v[0, 0], 1)[:, 0]
+        np.testing.assert_allclose(o_sw, self.g["swa_branch"], atol=1e-13)
+        gate = np.zeros((1, 1, 4, 2))
+        o = O.sparse_attention(self.q, self.k, self.v, sel, self.k, self.v, 1, gate, block=2)
+        np.testing.assert_allclose(o[0, 0, :, 0], self.g["gated"], atol=1e-13)
+
+    def test_token_variant(self):
+        for I in range(2):
+            ts = O.token_scores_tile(self.q[0], self.k[0, 0], I, block=2)
+            np.testing.assert_allclose(ts, self.g[f"token_score_tile{I}"], atol=1e-13)
+            sel = O.topk_tokens_tile(ts, I, 4, 1, 1, block=2)
+            assert sel[0] == self.g[f"token_top1_tile{I}"][0]
+            rows = O.tile_rows(I, 4, 2)
+            o = O.token_sparse_rows(self.q[0, 0][rows], rows, self.k[0, 0], self.v[0, 0], sel, 1)[:, 0]
+            np.testing.assert_allclose(o, self.g["token_sparse"][rows], atol=1e-13)
+
+    def test_decode(self):
+        q = np.ones((1, 1, 1))
+        o, sc = O.decode_full(q, self.k, self.v, block=2)
+        np.testing.assert_allclose(o[0, 0], self.g["decode_o"], atol=1e-13)
+        np.testing.assert_allclose(sc[0, 0], self.g["decode_scores"], atol=1e-13)
+        idx = O.topk_decode(sc, 1, block=2)
+        assert idx[0, 0, 0] == self.g["decode_top1"][0]
+        kr = np.array([math.log(3.0)]).reshape(1, 1, 1, 1)
+        vr = np.array([4.0]).reshape(1, 1, 1, 1)
+        gate = np.zeros((1, 1, 2))
+        o = O.decode_sparse(q, self.k, self.v, idx, kr, vr, gate, block=2)
+        np.testing.assert_allclose(o[0, 0], self.g["decode_gated"], atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- library routine
+@pytest.mark.parametrize("N,D,Hq,Hkv", [(64, 64, 4, 1), (200, 128, 8, 2), (257, 64, 4, 4)])
+def test_dense_matches_torch_sdpa(N, D, Hq, Hkv):
+    rng = np.random.default_rng(N + D)
+    q, k, v = _rand(rng, 1, Hq, N, D), _rand(rng, 1, Hkv, N, D), _rand(rng, 1, Hkv, N, D)
+    o, _ = O.full_attention(q, k, v, chunk=97)
+    np.testing.assert_allclose(o[0], _sdpa(q[0], k[0], v[0]), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- closed forms
+def test_zero_queries_closed_form():
+    """Q = 0: P_{t,i} = 1/(t+1), o_t = prefix mean of V, S_{t,j} = 1/(t+1) for 64j <= t,
+    every candidate of a tile ties and TopK must return {0..k-1} (lower index wins)."""
+    N, D, G = 200, 64, 4
+    rng = np.random.default_rng(1)
+    q = np.zeros((1, G, N, D))
+    k, v = _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    o, _ = O.full_attention(q, k, v)
+    prefix_mean = np.cumsum(v[0, 0], axis=0) / np.arange(1, N + 1)[:, None]
+    for h in range(G):
+        np.testing.assert_allclose(o[0, h], prefix_mean, atol=1e-13)
+    sc = O.block_scores(q, k, "sum")
+    for I in range(sc.shape[2]):
+        rows = O.tile_rows(I, N)
+        expect = G * np.sum(1.0 / (rows + 1.0))
+        np.testing.assert_allclose(sc[0, 0, I, :I + 1], expect, rtol=1e-13)
+        assert np.all(sc[0, 0, I, I + 1:] == 0)
+    idx = O.topk_blocks(sc, 2)
+    assert idx[0, 0, 0].tolist() == [0, -1]
+    assert idx[0, 0, 3].tolist() == [0, 1]
+
+
+def test_dominant_key():
+    """One key with a huge logit for every query that can see it: o_t -> v_p for t >= p."""
+    N, D, p = 150, 64, 70
+    rng = np.random.default_rng(2)
+    u = rng.standard_normal(D)
+    u /= np.linalg.norm(u)
+    q = np.tile(u, (1, 1, N, 1))
+    k = 0.01 * _rand(rng, 1, 1, N, D)
+    k[0, 0, p] = 80.0 * math.sqrt(D) * u
+    v = _rand(rng, 1, 1, N, D)
+    o, _ = O.full_attention(q, k, v)
+    np.testing.assert_allclose(o[0, 0, p:], np.tile(v[0, 0, p], (N - p, 1)), atol=1e-12)
+    # block max: the block holding p scores ~1 for the rows after p
+    rows = np.arange(p, N)
+    pr, _, _ = O.causal_softmax(q[0, 0, p:], rows, k[0, 0])
+    s = O.block_max_probs(pr, rows)
+    np.testing.assert_allclose(s[:, p // 64], 1.0, atol=1e-12)
+
+
+def test_gate_saturation():
+    """Gate logits +-40 select one branch; 0 gives the average of both branches."""
+    rng = np.random.default_rng(3)
+    N, D = 130, 64
+    q, k, v = _rand(rng, 1, 2, N, D), _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    ks, vs = _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    idx = O.topk_blocks(O.block_scores(q, k), 1)
+    only_sp = O.sparse_attention(q, k, v, idx, ks, vs, 16, np.tile([40.0, -40.0], (1, 2, N, 1)))
+    only_sw = O.sparse_attention(q, k, v, idx, ks, vs, 16, np.tile([-40.0, 40.0], (1, 2, N, 1)))
+    half = O.sparse_attention(q, k, v, idx, ks, vs, 16, np.zeros((1, 2, N, 2)))
+    for h in range(2):
+        for I in range(3):
+            rows = O.tile_rows(I, N)
+            sp = O.sparse_branch_rows(q[0, h, rows], rows, k[0, 0], v[0, 0], idx[0, 0, I])
+            sw = O.swa_branch_rows(q[0, h, rows], rows, ks[0, 0], vs[0, 0], 16)
+            np.testing.assert_allclose(only_sp[0, h, rows], sp, atol=1e-12)
+            np.testing.assert_allclose(only_sw[0, h, rows], sw, atol=1e-12)
+            np.testing.assert_allclose(half[0, h, rows], 0.5 * (sp + sw), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- invariants
+@pytest.mark.parametrize("N,D,G", [(256, 64, 4), (200, 128, 2)])
+def test_score_invariants(N, D, G):
+    rng = np.random.default_rng(N * G)
+    q, k = _rand(rng, 1, G, N, D), _rand(rng, 1, 1, N, D)
+    rows = np.arange(N)
+    for h in range(G):
+        p, _, _ = O.causal_softmax(q[0, h], rows, k[0, 0])
+        s = O.block_max_probs(p, rows)
+        assert np.all(s >= 0) and np.all(s <= 1)
+        np.testing.assert_allclose(s.max(axis=1), p.max(axis=1), rtol=0, atol=0)
+        assert np.all(s[np.arange(s.shape[1])[None, :] * 64 > rows[:, None]] == 0)
+    smax = O.block_scores(q, k, "max")
+    assert np.all(smax <= 1.0)
+    ssum = O.block_scores(q, k, "sum")
+    assert np.all(ssum >= smax - 1e-15)
+    k_sel = 3
+    idx = O.topk_blocks(ssum, k_sel)
+    for I in range(ssum.shape[2]):
+        sel = [j for j in idx[0, 0, I] if j >= 0]
+        assert len(sel) == min(k_sel, I + 1) and len(set(sel)) == len(sel)
+        assert all(0 <= j <= I for j in sel) and sel == sorted(sel)
+        rest = [j for j in range(I + 1) if j not in sel]
+        if rest:
+            assert min(ssum[0, 0, I, sel]) >= max(ssum[0, 0, I, rest])
+
+
+def test_k_covering_all_blocks_is_dense():
+    """With every block selected the sparse branch equals dense causal attention."""
+    rng = np.random.default_rng(4)
+    N, D, Hq = 200, 64, 4
+    qs, k, v = _rand(rng, 1, Hq, N, D), _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    nb = 4
+    idx = O.topk_blocks(O.block_scores(qs, k), nb)
+    gate = np.tile([40.0, -40.0], (1, Hq, N, 1))
+    o = O.sparse_attention(qs, k, v, idx, k, v, 128, gate)
+    np.testing.assert_allclose(o[0], _sdpa(qs[0], k[0], v[0]), atol=1e-12)
+
+
+def test_window_covering_all_is_dense():
+    rng = np.random.default_rng(5)
+    N, D, Hq = 190, 64, 2
+    qs, k, v = _rand(rng, 1, Hq, N, D), _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    ks, vs = _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    idx = O.topk_blocks(O.block_scores(qs, k), 1)
+    gate = np.tile([-40.0, 40.0], (1, Hq, N, 1))
+    o = O.sparse_attention(qs, k, v, idx, ks, vs, N, gate)
+    np.testing.assert_allclose(o[0], _sdpa(qs[0], ks[0], vs[0]), atol=1e-12)
+
+
+def test_selection_order_irrelevant():
+    rng = np.random.default_rng(6)
+    N, D = 256, 64
+    q, k, v = _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    rows = O.tile_rows(3, N)
+    a = O.sparse_branch_rows(q[0, 0, rows], rows, k[0, 0], v[0, 0], [0, 2, 3])
+    b = O.sparse_branch_rows(q[0, 0, rows], rows, k[0, 0], v[0, 0], [3, -1, 0, 2])
+    np.testing.assert_allclose(a, b, atol=1e-14)
+
+
+def test_token_variant_invariants():
+    rng = np.random.default_rng(7)
+    N, D, G, forced, kt = 256, 64, 2, 16, 20
+    q, k, v = _rand(rng, 1, G, N, D), _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    for I in range(4):
+        ts = O.token_scores_tile(q[0], k[0, 0], I)
+        rows = O.tile_rows(I, N)
+        # every row's probabilities sum to 1
+        np.testing.assert_allclose(ts.sum(), G * len(rows), rtol=1e-12)
+        assert np.all(ts[rows[-1] + 1:] == 0)
+        sel = O.topk_tokens_tile(ts, I, N, kt, forced)
+        real = [i for i in sel if i >= 0]
+        assert all(i <= rows[-1] - forced for i in real)
+        assert len(real) == min(kt, O.token_candidates(I, N, forced))
+        # forced tokens are always attended: make the window keys dominant and compare
+        o = O.token_sparse_rows(q[0, 0, rows], rows, k[0, 0], v[0, 0], sel, forced)
+        o_win = O.swa_branch_rows(q[0, 0, rows], rows, k[0, 0], v[0, 0], forced)
+        if not real:
+            np.testing.assert_allclose(o, o_win, atol=1e-12)
+    # when the budget covers every candidate, each row sees every earlier token: dense
+    kt_all = N
+    I = 3
+    rows = O.tile_rows(I, N)
+    ts = O.token_scores_tile(q[0], k[0, 0], I)
+    sel = O.topk_tokens_tile(ts, I, N, kt_all, forced)
+    o = O.token_sparse_rows(q[0, 0, rows], rows, k[0, 0], v[0, 0], sel, forced)
+    np.testing.assert_allclose(o, _sdpa(q[0, :1], k[0], v[0])[0, rows], atol=1e-12)
+
+
+def test_decode_is_last_row_of_dense():
+    rng = np.random.default_rng(8)
+    L, D, Hq, Hkv = 300, 64, 4, 2
+    q, k, v = _rand(rng, 2, Hq, D), _rand(rng, 2, Hkv, L, D), _rand(rng, 2, Hkv, L, D)
+    seqlens = np.array([300, 129])
+    o, sc = O.decode_full(q, k, v, seqlens)
+    for b in range(2):
+        Lb = seqlens[b]
+        qq = np.zeros((Hq, Lb, D))
+        qq[:, -1] = q[b]
+        ref = _sdpa(qq, k[b, :, :Lb], v[b, :, :Lb])[:, -1]
+        np.testing.assert_allclose(o[b], ref, atol=1e-12)
+        assert np.all(sc[b, :, (Lb + 63) // 64:] == 0)
+    idx = O.topk_decode(sc, 4, seqlens)
+    assert all(0 <= j < 3 for j in idx[1].ravel() if j >= 0)
+    assert np.sum(idx[1] >= 0) == 2 * 3
+
+
+# ----------------------------------------------------------------------------- brute force
+@pytest.mark.parametrize("seed,N,D,G", [(0, 64, 16, 1), (1, 65, 16, 2), (2, 130, 8, 2), (3, 200, 8, 1)])
+def test_brute_force(seed, N, D, G):
+    rng = np.random.default_rng(100 + seed)
+    q, k, v = _rand(rng, 1, G, N, D), _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    ks, vs = _rand(rng, 1, 1, N, D), _rand(rng, 1, 1, N, D)
+    gate = _rand(rng, 1, G, N, 2)
+    kk, vv, kl, vl = k[0, 0].tolist(), v[0, 0].tolist(), ks[0, 0].tolist(), vs[0, 0].tolist()
+    qg = [q[0, h].tolist() for h in range(G)]
+    T = (N + 63) // 64
+    for red in ("sum", "max"):
+        sc = O.block_scores(q, k, red)
+        for I in range(T):
+            for j in range(T):
+                want = BF.block_score(qg, kk, I, j, N, 64, red) if j <= I else 0.0
+                assert abs(sc[0, 0, I, j] - want) <= 1e-12 * max(1.0, abs(want))
+    sc = O.block_scores(q, k, "sum")
+    kb = 2
+    idx = O.topk_blocks(sc, kb)
+    window = 24
+    o = O.sparse_attention(q, k, v, idx, ks, vs, window, gate)
+    for I in range(T):
+        assert idx[0, 0, I].tolist() == BF.topk(sc[0, 0, I].tolist(), I + 1, kb)
+        for t in O.tile_rows(I, N)[::7]:
+            for h in range(G):
+                want = BF.gated_row(qg[h][t], t, kk, vv, idx[0, 0, I].tolist(), kl, vl, window,
+                                    gate[0, h, t].tolist(), 64)
+                np.testing.assert_allclose(o[0, h, t], want, atol=1e-12)
+    # token variant
+    forced, kt = 8, 10
+    for I in range(T):
+        ts = O.token_scores_tile(q[0], k[0, 0], I)
+        for i in range(0, N, 5):
+            assert abs(ts[i] - BF.token_score(qg, kk, I, i, N, 64)) <= 1e-12
+        sel = O.topk_tokens_tile(ts, I, N, kt, forced)
+        rows = O.tile_rows(I, N)
+        assert sel.tolist() == BF.topk(ts.tolist(), O.token_candidates(I, N, forced), kt)
+        ot = O.token_sparse_rows(q[0, 0, rows], rows, k[0, 0], v[0, 0], sel, forced)
+        for r, t in list(enumerate(rows))[::9]:
+            np.testing.assert_allclose(ot[r], BF.token_row(qg[0][t], t, kk, vv, sel.tolist(), forced),
+                                       atol=1e-12)
+
+
+def test_brute_force_decode():
+    rng = np.random.default_rng(9)
+    L, D, G = 190, 8, 2
+    q, k, v = _rand(rng, 1, G, D), _rand(rng, 1, 1, L, D), _rand(rng, 1, 1, L, D)
+    kr, vr = _rand(rng, 1, 1, 5, D), _rand(rng, 1, 1, 5, D)
+    gate = _rand(rng, 1, G, 2)
+    o, sc = O.decode_full(q, k, v)
+    kk, vv = k[0, 0].tolist(), v[0, 0].tolist()
+    for j in range(3):
+        want = sum(max(p for i, p in BF.softmax_over(q[0, h].tolist(), list(range(L)), kk)
+                       if j * 64 <= i < (j + 1) * 64) for h in range(G))
+        assert abs(sc[0, 0, j] - want) < 1e-12
+    for h in range(G):
+        np.testing.assert_allclose(o[0, h], BF.attend(q[0, h].tolist(), list(range(L)), kk, vv), atol=1e-12)
+    idx = O.topk_decode(sc, 2)
+    assert idx[0, 0].tolist() == BF.topk(sc[0, 0].tolist(), 3, 2)
+    swa_len = np.array([3])
+    od = O.decode_sparse(q, k, v, idx, kr, vr, gate, swa_len=swa_len)
+    for h in range(G):
+        keys = [i for j in idx[0, 0] for i in range(j * 64, min(L, (j + 1) * 64))]
+        a = BF.attend(q[0, h].tolist(), keys, kk, vv)
+        b = BF.attend(q[0, h].tolist(), [0, 1, 2], kr[0, 0].tolist(), vr[0, 0].tolist())
+        g0, g1 = 1 / (1 + math.exp(-gate[0, h, 0])), 1 / (1 + math.exp(-gate[0, h, 1]))
+        np.testing.assert_allclose(od[0, h], [g0 * x + g1 * y for x, y in zip(a, b)], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- planted mistakes
+def test_pins_catch_planted_mistakes(monkeypatch):
+    """Plant plausible mistakes in the oracle and check that a pin above fails."""
+    g = _gold()
+    q = np.ones((1, 1, 4, 1))
+    k = np.array([0.0, math.log(2.0), 0.0, math.log(3.0)]).reshape(1, 1, 4, 1)
+    # 1) ties broken toward the higher index
+    monkeypatch.setattr(O.hysparse_oracle, "select_topk",
+                        lambda s, n, kk: np.concatenate([np.sort(np.lexsort((-np.arange(n), -s[:n]))[:kk]),
+                                                         -np.ones(max(0, kk - n), np.int64)]))
+    sc = np.zeros((1, 1, 4, 4))
+    idx = O.hysparse_oracle.topk_blocks(sc, 2)
+    assert idx[0, 0, 3].tolist() != [0, 1]
+    monkeypatch.undo()
+    # 2) forgetting to clip the block at t changes nothing (P is zero past t), but
+    #    dropping the 1/sqrt(d) scale breaks the SDPA pin
+    rng = np.random.default_rng(0)
+    qq, kk2, vv = _rand(rng, 1, 1, 40, 16), _rand(rng, 1, 1, 40, 16), _rand(rng, 1, 1, 40, 16)
+    o_ok, _ = O.full_attention(qq, kk2, vv)
+    o_bad, _ = O.full_attention(qq * 4.0, kk2, vv)   # == no 1/sqrt(16) scaling
+    ref = _sdpa(qq[0], kk2[0], vv[0])
+    assert np.allclose(o_ok[0], ref, atol=1e-12) and not np.allclose(o_bad[0], ref, atol=1e-6)
+    # 3) an off-by-one window ([t-w, t]) breaks the worked SWA example
+    rows = np.arange(4)
+    o_sw_bad = O.swa_branch_rows(q[0, 0], rows, k[0, 0], np.arange(1.0, 5.0)[:, None], 2)[:, 0]
+    assert not np.allclose(o_sw_bad, g["swa_branch"])
