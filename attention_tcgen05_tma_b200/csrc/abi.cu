@@ -1,0 +1,291 @@
+// C ABI of the HySparse hot path: argument validation, workspace carving and dispatch.
+// Every entry point enqueues on the caller's stream and never allocates.
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hys {
+__device__ int g_device_status = 0;
+
+int* device_status_ptr() {
+  static int* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    cached[dev] = static_cast<int*>(p);
+  }
+  return cached[dev];
+}
+}  // namespace hys
+
+using namespace hys;
+
+namespace {
+
+constexpr int kBlock = 64;
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hys_status check_prefill(const hys_shape* s, PrefillDims* d) {
+  if (!s) return HYS_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->N <= 0 || s->Hq <= 0 || s->Hkv <= 0) return HYS_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return HYS_ERR_INVALID_ARG;
+  if (s->D != 64 && s->D != 128) return HYS_ERR_INVALID_ARG;
+  if (s->block != kBlock) return HYS_ERR_INVALID_ARG;
+  if (s->N > (1 << 20)) return HYS_ERR_UNSUPPORTED;
+  if (s->Hq / s->Hkv > 64) return HYS_ERR_UNSUPPORTED;
+  d->B = s->B;
+  d->N = s->N;
+  d->Hq = s->Hq;
+  d->Hkv = s->Hkv;
+  d->D = s->D;
+  d->T = (s->N + kBlock - 1) / kBlock;
+  d->NB = d->T;
+  return HYS_OK;
+}
+
+hys_status check_decode(const hys_decode_shape* s, DecodeDims* d) {
+  if (!s) return HYS_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->L <= 0 || s->Hq <= 0 || s->Hkv <= 0) return HYS_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return HYS_ERR_INVALID_ARG;
+  if (s->D != 64 && s->D != 128) return HYS_ERR_INVALID_ARG;
+  if (s->block != kBlock) return HYS_ERR_INVALID_ARG;
+  if (s->Hq / s->Hkv > 16) return HYS_ERR_UNSUPPORTED;
+  if (s->L > (1 << 23)) return HYS_ERR_UNSUPPORTED;
+  d->B = s->B;
+  d->L = s->L;
+  d->Hq = s->Hq;
+  d->Hkv = s->Hkv;
+  d->D = s->D;
+  d->NB = (s->L + kBlock - 1) / kBlock;
+  return HYS_OK;
+}
+
+bool dtype_ok(hys_dtype dt) { return dt == HYS_F32 || dt == HYS_BF16; }
+
+hys_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HYS_OK : HYS_ERR_CUDA; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t full_ws_bytes(const PrefillDims& d, hys_dtype dt, hys_gran gran) {
+  if (gran == HYS_GRAN_TOKEN) return align256(sizeof(float) * (size_t)d.B * d.Hq * d.N);
+  if (full_attn_tc_supported(d, dt)) return full_attn_tc_workspace(d);
+  return align256(sizeof(float) * (size_t)d.B * d.Hq * d.T * d.NB);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hysparse_version(void) { return "0.1.0"; }
+
+const char* hysparse_status_string(hys_status s) {
+  switch (s) {
+    case HYS_OK: return "HYS_OK";
+    case HYS_ERR_INVALID_ARG: return "HYS_ERR_INVALID_ARG";
+    case HYS_ERR_UNSUPPORTED: return "HYS_ERR_UNSUPPORTED";
+    case HYS_ERR_CUDA: return "HYS_ERR_CUDA";
+    case HYS_ERR_TIMEOUT: return "HYS_ERR_TIMEOUT";
+    case HYS_ERR_WORKSPACE: return "HYS_ERR_WORKSPACE";
+  }
+  return "HYS_ERR_UNKNOWN";
+}
+
+hys_status hysparse_get_device_status(hys_stream_t stream, int reset, int* out) {
+  if (!out) return HYS_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return HYS_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HYS_ERR_CUDA;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return HYS_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HYS_ERR_CUDA;
+  }
+  *out = v;
+  return HYS_OK;
+}
+
+// ----------------------------------------------------------------------------- full layer
+hys_status hysparse_full_attn_select_workspace_size(const hys_shape* shape, hys_dtype dtype, hys_gran gran,
+                                                    size_t* bytes) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || !dtype_ok(dtype) || (gran != HYS_GRAN_BLOCK && gran != HYS_GRAN_TOKEN)) return HYS_ERR_INVALID_ARG;
+  *bytes = full_ws_bytes(d, dtype, gran);
+  return HYS_OK;
+}
+
+hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype dtype, const void* q, const void* k,
+                                     const void* v, void* o, float* scores, hys_gran gran, hys_reduce red,
+                                     float* lse_opt, void* workspace, size_t workspace_bytes,
+                                     hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype) || (gran != HYS_GRAN_BLOCK && gran != HYS_GRAN_TOKEN)) return HYS_ERR_INVALID_ARG;
+  if (red != HYS_REDUCE_SUM && red != HYS_REDUCE_MAX) return HYS_ERR_INVALID_ARG;
+  if (gran == HYS_GRAN_TOKEN && red != HYS_REDUCE_SUM) return HYS_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !scores) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(scores) ||
+      !aligned16(lse_opt) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  const size_t need = full_ws_bytes(d, dtype, gran);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return HYS_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (gran == HYS_GRAN_BLOCK) {
+    if (full_attn_tc_supported(d, dtype))
+      return from_cuda(launch_full_attn_tc(d, q, k, v, o, lse_opt, scores, red, true, workspace, workspace_bytes, s));
+    float* part = reinterpret_cast<float*>(workspace);
+    cudaError_t e = launch_full_attn_simt(d, dtype, q, k, v, o, lse_opt, part, true, red, s);
+    if (e != cudaSuccess) return HYS_ERR_CUDA;
+    return from_cuda(launch_head_reduce(d, part, scores, red, s));
+  }
+  float* lse = lse_opt ? lse_opt : reinterpret_cast<float*>(workspace);
+  cudaError_t e;
+  if (full_attn_tc_supported(d, dtype))
+    e = launch_full_attn_tc(d, q, k, v, o, lse, nullptr, HYS_REDUCE_SUM, false, nullptr, 0, s);
+  else
+    e = launch_full_attn_simt(d, dtype, q, k, v, o, lse, nullptr, false, HYS_REDUCE_SUM, s);
+  if (e != cudaSuccess) return HYS_ERR_CUDA;
+  return from_cuda(launch_token_scores_simt(d, dtype, q, k, lse, scores, s));
+}
+
+// ----------------------------------------------------------------------------- top-k
+hys_status hysparse_topk(const hys_shape* shape, const float* scores, int k, int* idx, hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!scores || !idx || k < 1 || k > 1024) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx)) return HYS_ERR_INVALID_ARG;
+  if (d.NB > 8192) return HYS_ERR_UNSUPPORTED;
+  return from_cuda(launch_topk_blocks(scores, idx, d.B, d.Hkv, d.T, d.NB, k, nullptr, 0, false,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_topk_tokens_workspace_size(const hys_shape* shape, int k_tokens, size_t* bytes) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || k_tokens < 1 || k_tokens > 16384) return HYS_ERR_INVALID_ARG;
+  *bytes = 0;
+  return HYS_OK;
+}
+
+hys_status hysparse_topk_tokens(const hys_shape* shape, const float* tok_scores, int k_tokens, int forced_window,
+                                int* idx, void* workspace, size_t workspace_bytes, hys_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!tok_scores || !idx || k_tokens < 1 || k_tokens > 16384 || forced_window < 0) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(tok_scores) || !aligned16(idx)) return HYS_ERR_INVALID_ARG;
+  return from_cuda(launch_topk_tokens(d, tok_scores, k_tokens, forced_window, idx,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ----------------------------------------------------------------------------- sparse layer
+hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const void* q_sparse, const void* k_shared,
+                                const void* v_shared, const int* idx, int k, const void* k_swa, const void* v_swa,
+                                int window, const float* gate_logits, const float* sinks, void* o,
+                                hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (sinks) return HYS_ERR_UNSUPPORTED;
+  if (!q_sparse || !k_shared || !v_shared || !idx || !k_swa || !v_swa || !gate_logits || !o) return HYS_ERR_INVALID_ARG;
+  if (k < 1 || k > 1024 || window < 1) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(k_swa) ||
+      !aligned16(v_swa) || !aligned16(gate_logits) || !aligned16(o))
+    return HYS_ERR_INVALID_ARG;
+  return from_cuda(launch_sparse_attn_simt(d, dtype, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,
+                                           gate_logits, o, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_sparse_attn_tokens(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                       const void* k_shared, const void* v_shared, const int* idx, int k_tokens,
+                                       int forced_window, const float* sinks, void* o, hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (sinks) return HYS_ERR_UNSUPPORTED;
+  if (!q_sparse || !k_shared || !v_shared || !idx || !o) return HYS_ERR_INVALID_ARG;
+  if (k_tokens < 1 || k_tokens > 16384 || forced_window < 1) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(o))
+    return HYS_ERR_INVALID_ARG;
+  return from_cuda(launch_sparse_tokens_simt(d, dtype, q_sparse, k_shared, v_shared, idx, k_tokens, forced_window, o,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ----------------------------------------------------------------------------- decode
+hys_status hysparse_full_attn_select_decode_workspace_size(const hys_decode_shape* shape, hys_dtype dtype,
+                                                           size_t* bytes) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || !dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  *bytes = align256(decode_full_workspace(d));
+  return HYS_OK;
+}
+
+hys_status hysparse_full_attn_select_decode(const hys_decode_shape* shape, hys_dtype dtype, const void* q,
+                                            const void* k_cache, const void* v_cache, const int* seqlens, void* o,
+                                            float* scores, hys_reduce red, void* workspace, size_t workspace_bytes,
+                                            hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype) || (red != HYS_REDUCE_SUM && red != HYS_REDUCE_MAX)) return HYS_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !o || !scores) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(scores) ||
+      !aligned16(seqlens) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  const size_t need = align256(decode_full_workspace(d));
+  if (workspace == nullptr || workspace_bytes < need) return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_decode_full(d, dtype, q, k_cache, v_cache, seqlens, o, scores, red, workspace,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_topk_decode(const hys_decode_shape* shape, const float* scores, int k, const int* seqlens,
+                                int* idx, hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!scores || !idx || k < 1 || k > 1024) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx) || !aligned16(seqlens)) return HYS_ERR_INVALID_ARG;
+  if (d.NB > 8192) return HYS_ERR_UNSUPPORTED;
+  return from_cuda(launch_topk_blocks(scores, idx, d.B, d.Hkv, 1, d.NB, k, seqlens, d.L, true,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype dtype, const void* q,
+                                       const void* k_cache, const void* v_cache, const int* seqlens, const int* idx,
+                                       int k, const void* k_swa_ring, const void* v_swa_ring, int window,
+                                       const int* swa_len, const float* gate_logits, const float* sinks, void* o,
+                                       hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (sinks) return HYS_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !idx || !k_swa_ring || !v_swa_ring || !gate_logits || !o) return HYS_ERR_INVALID_ARG;
+  if (k < 1 || k > 1024 || window < 1 || window > 1024) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seqlens) || !aligned16(idx) ||
+      !aligned16(k_swa_ring) || !aligned16(v_swa_ring) || !aligned16(swa_len) || !aligned16(gate_logits) ||
+      !aligned16(o))
+    return HYS_ERR_INVALID_ARG;
+  return from_cuda(launch_decode_sparse(d, dtype, q, k_cache, v_cache, seqlens, idx, k, k_swa_ring, v_swa_ring,
+                                        window, swa_len, gate_logits, o, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

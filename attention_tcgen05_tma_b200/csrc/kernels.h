@@ -1,0 +1,73 @@
+// Internal launchers of the HySparse kernels (C++; the public C ABI lives in abi.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/hysparse.h"
+
+namespace hys {
+
+// Device address of this device's status word (nullptr if it cannot be resolved).
+int* device_status_ptr();
+
+struct PrefillDims {
+  int B, N, Hq, Hkv, D;
+  int T;   // query tiles = ceil(N / 64)
+  int NB;  // key blocks  = ceil(N / 64)
+  __host__ __device__ int G() const { return Hq / Hkv; }
+};
+
+struct DecodeDims {
+  int B, L, Hq, Hkv, D;
+  int NB;  // ceil(L / 64)
+  __host__ __device__ int G() const { return Hq / Hkv; }
+};
+
+// ---- full layer, SIMT fp32-accumulate path (any supported dtype / D / G) -------------
+// Writes o, lse (always) and, in block mode, per-head partial block scores
+// part[B,Hq,T,NB] (reduced over the tile's rows with `red`).
+cudaError_t launch_full_attn_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
+                                  const void* v, void* o, float* lse, float* part, bool want_scores,
+                                  hys_reduce red, cudaStream_t s);
+// scores[B,Hkv,T,NB] = R over the group's heads (fixed head order) of part.
+cudaError_t launch_head_reduce(const PrefillDims& d, const float* part, float* scores, hys_reduce red,
+                               cudaStream_t s);
+// Token scores [B,Hkv,T,N] from q, k and the rows' LSE.
+cudaError_t launch_token_scores_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
+                                     const float* lse, float* scores, cudaStream_t s);
+
+// ---- full layer, tcgen05 path (bf16, D=128, even G) ----------------------------------------
+bool full_attn_tc_supported(const PrefillDims& d, hys_dtype dt);
+size_t full_attn_tc_workspace(const PrefillDims& d);
+cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v,
+                                void* o, float* lse, float* scores, hys_reduce red, bool want_scores,
+                                void* ws, size_t ws_bytes, cudaStream_t s);
+
+// ---- top-k -------------------------------------------------------------------------------
+// rows = B*Hkv*T (prefill) or B*Hkv (decode); row r has n_cand(r) candidates.
+cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, int T, int NB, int k,
+                               const int* seqlens, int L, bool decode, cudaStream_t s);
+cudaError_t launch_topk_tokens(const PrefillDims& d, const float* scores, int k_tokens, int forced,
+                               int* idx, cudaStream_t s);
+
+// ---- sparse layer ----------------------------------------------------------------------------
+cudaError_t launch_sparse_attn_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
+                                    const void* v, const int* idx, int kb, const void* ks,
+                                    const void* vs, int window, const float* gate, void* o,
+                                    cudaStream_t s);
+cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
+                                      const void* v, const int* idx, int kt, int forced, void* o,
+                                      cudaStream_t s);
+
+// ---- decode ----------------------------------------------------------------------------------
+size_t decode_full_workspace(const DecodeDims& d);
+cudaError_t launch_decode_full(const DecodeDims& d, hys_dtype dt, const void* q, const void* kc,
+                               const void* vc, const int* seqlens, void* o, float* scores,
+                               hys_reduce red, void* ws, cudaStream_t s);
+cudaError_t launch_decode_sparse(const DecodeDims& d, hys_dtype dt, const void* q, const void* kc,
+                                 const void* vc, const int* seqlens, const int* idx, int kb,
+                                 const void* kr, const void* vr, int W, const int* swa_len,
+                                 const float* gate, void* o, cudaStream_t s);
+
+}  // namespace hys

@@ -1,0 +1,323 @@
+"""Thin ctypes binding of libhysparse.so (the C ABI declared in include/hysparse.h).
+
+The ``hysparse_*`` functions mirror the C entry points one to one and take raw
+integers for pointers and the stream.  The short-named helpers below them only
+marshal torch tensors (device pointers, the current stream, output allocation); every
+step of the computation runs in the library's CUDA kernels.  There is no fallback:
+loading fails loudly when the library is missing or was not built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libhysparse.so")
+
+HYS_OK, HYS_ERR_INVALID_ARG, HYS_ERR_UNSUPPORTED, HYS_ERR_CUDA, HYS_ERR_TIMEOUT, HYS_ERR_WORKSPACE = range(6)
+HYS_F32, HYS_BF16 = 0, 1
+HYS_GRAN_BLOCK, HYS_GRAN_TOKEN = 0, 1
+HYS_REDUCE_SUM, HYS_REDUCE_MAX = 0, 1
+
+# every symbol include/hysparse.h declares
+EXPORTED = (
+    "hysparse_version", "hysparse_status_string", "hysparse_get_device_status",
+    "hysparse_full_attn_select_workspace_size", "hysparse_full_attn_select",
+    "hysparse_topk", "hysparse_topk_tokens_workspace_size", "hysparse_topk_tokens",
+    "hysparse_sparse_attn", "hysparse_sparse_attn_tokens",
+    "hysparse_full_attn_select_decode_workspace_size", "hysparse_full_attn_select_decode",
+    "hysparse_topk_decode", "hysparse_sparse_attn_decode",
+)
+
+
+class HysparseError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class hys_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("D", ctypes.c_int), ("block", ctypes.c_int)]
+
+
+class hys_decode_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("L", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("D", ctypes.c_int), ("block", ctypes.c_int)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+_SH = ctypes.POINTER(hys_shape)
+_DSH = ctypes.POINTER(hys_decode_shape)
+
+_SIGS = {
+    "hysparse_version": ([], ctypes.c_char_p),
+    "hysparse_status_string": ([_I], ctypes.c_char_p),
+    "hysparse_get_device_status": ([_P, _I, ctypes.POINTER(_I)], _I),
+    "hysparse_full_attn_select_workspace_size": ([_SH, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_full_attn_select": ([_SH, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P], _I),
+    "hysparse_topk": ([_SH, _P, _I, _P, _P], _I),
+    "hysparse_topk_tokens_workspace_size": ([_SH, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_topk_tokens": ([_SH, _P, _I, _I, _P, _P, _SZ, _P], _I),
+    "hysparse_sparse_attn": ([_SH, _I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P], _I),
+    "hysparse_sparse_attn_tokens": ([_SH, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P], _I),
+    "hysparse_full_attn_select_decode_workspace_size": ([_DSH, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_full_attn_select_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P], _I),
+    "hysparse_topk_decode": ([_DSH, _P, _I, _P, _P, _P], _I),
+    "hysparse_sparse_attn_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P], _I),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (once) and declare the signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libhysparse.so not found at {path}; build it with "
+                           "`python -m attention_tcgen05_tma_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (args, res) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def status_string(s: int) -> str:
+    return load().hysparse_status_string(int(s)).decode()
+
+
+def _check(s: int, where: str):
+    if s != HYS_OK:
+        raise HysparseError(s, where)
+
+
+# ----------------------------------------------------------------------------- raw C mirrors
+def hysparse_version() -> str:
+    return load().hysparse_version().decode()
+
+
+def hysparse_get_device_status(stream: int = 0, reset: bool = False) -> int:
+    out = _I(0)
+    _check(load().hysparse_get_device_status(stream, int(reset), ctypes.byref(out)), "hysparse_get_device_status")
+    return out.value
+
+
+def hysparse_full_attn_select_workspace_size(shape: hys_shape, dtype: int, gran: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_full_attn_select_workspace_size(ctypes.byref(shape), dtype, gran, ctypes.byref(n)),
+           "hysparse_full_attn_select_workspace_size")
+    return n.value
+
+
+def hysparse_full_attn_select(shape, dtype, q, k, v, o, scores, gran, red, lse, ws, ws_bytes, stream) -> int:
+    return load().hysparse_full_attn_select(ctypes.byref(shape), dtype, q, k, v, o, scores, gran, red, lse, ws,
+                                            ws_bytes, stream)
+
+
+def hysparse_topk(shape, scores, k, idx, stream) -> int:
+    return load().hysparse_topk(ctypes.byref(shape), scores, k, idx, stream)
+
+
+def hysparse_topk_tokens_workspace_size(shape: hys_shape, k_tokens: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_topk_tokens_workspace_size(ctypes.byref(shape), k_tokens, ctypes.byref(n)),
+           "hysparse_topk_tokens_workspace_size")
+    return n.value
+
+
+def hysparse_topk_tokens(shape, scores, k_tokens, forced, idx, ws, ws_bytes, stream) -> int:
+    return load().hysparse_topk_tokens(ctypes.byref(shape), scores, k_tokens, forced, idx, ws, ws_bytes, stream)
+
+
+def hysparse_sparse_attn(shape, dtype, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, stream) -> int:
+    return load().hysparse_sparse_attn(ctypes.byref(shape), dtype, q, k, v, idx, kb, ks, vs, window, gate, sinks,
+                                       o, stream)
+
+
+def hysparse_sparse_attn_tokens(shape, dtype, q, k, v, idx, kt, forced, sinks, o, stream) -> int:
+    return load().hysparse_sparse_attn_tokens(ctypes.byref(shape), dtype, q, k, v, idx, kt, forced, sinks, o, stream)
+
+
+def hysparse_full_attn_select_decode_workspace_size(shape: hys_decode_shape, dtype: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_full_attn_select_decode_workspace_size(ctypes.byref(shape), dtype, ctypes.byref(n)),
+           "hysparse_full_attn_select_decode_workspace_size")
+    return n.value
+
+
+def hysparse_full_attn_select_decode(shape, dtype, q, kc, vc, seqlens, o, scores, red, ws, ws_bytes, stream) -> int:
+    return load().hysparse_full_attn_select_decode(ctypes.byref(shape), dtype, q, kc, vc, seqlens, o, scores, red,
+                                                   ws, ws_bytes, stream)
+
+
+def hysparse_topk_decode(shape, scores, k, seqlens, idx, stream) -> int:
+    return load().hysparse_topk_decode(ctypes.byref(shape), scores, k, seqlens, idx, stream)
+
+
+def hysparse_sparse_attn_decode(shape, dtype, q, kc, vc, seqlens, idx, kb, kr, vr, window, swa_len, gate, sinks, o,
+                                stream) -> int:
+    return load().hysparse_sparse_attn_decode(ctypes.byref(shape), dtype, q, kc, vc, seqlens, idx, kb, kr, vr, window,
+                                              swa_len, gate, sinks, o, stream)
+
+
+# ----------------------------------------------------------------------------- torch helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _dt(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return HYS_BF16
+    if t.dtype == torch.float32:
+        return HYS_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def prefill_shape(q, k) -> hys_shape:
+    B, Hq, N, D = q.shape
+    return hys_shape(B, N, Hq, k.shape[1], D, 64)
+
+
+def decode_shape(q, k_cache) -> hys_decode_shape:
+    B, Hq, D = q.shape
+    return hys_decode_shape(B, k_cache.shape[2], Hq, k_cache.shape[1], D, 64)
+
+
+def workspace_for(nbytes: int, device):
+    torch = _torch()
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def full_attn_select(q, k, v, *, gran: str = "block", reduce: str = "sum", o=None, scores=None, lse=None,
+                     workspace=None, stream=None) -> Tuple[object, object]:
+    """Full causal GQA attention plus block (or token) importance scores. Returns (o, scores)."""
+    torch = _torch()
+    sh = prefill_shape(q, k)
+    g = HYS_GRAN_TOKEN if gran == "token" else HYS_GRAN_BLOCK
+    T = (sh.N + 63) // 64
+    if o is None:
+        o = torch.empty_like(q)
+    if scores is None:
+        cols = sh.N if g == HYS_GRAN_TOKEN else T
+        scores = torch.empty((sh.B, sh.Hkv, T, cols), dtype=torch.float32, device=q.device)
+    nws = hysparse_full_attn_select_workspace_size(sh, _dt(q), g)
+    if workspace is None and nws > 0:
+        workspace = workspace_for(nws, q.device)
+    st = hysparse_full_attn_select(sh, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(scores), g,
+                                   HYS_REDUCE_MAX if reduce == "max" else HYS_REDUCE_SUM, _ptr(lse),
+                                   _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                   _stream(stream))
+    _check(st, "hysparse_full_attn_select")
+    return o, scores
+
+
+def topk(scores, k: int, *, idx=None, stream=None):
+    torch = _torch()
+    B, Hkv, T, NB = scores.shape
+    sh = hys_shape(B, NB * 64, Hkv, Hkv, 64, 64)
+    if idx is None:
+        idx = torch.empty((B, Hkv, T, k), dtype=torch.int32, device=scores.device)
+    _check(hysparse_topk(sh, _ptr(scores), k, _ptr(idx), _stream(stream)), "hysparse_topk")
+    return idx
+
+
+def topk_tokens(scores, k_tokens: int, forced_window: int, *, idx=None, stream=None):
+    torch = _torch()
+    B, Hkv, T, N = scores.shape
+    sh = hys_shape(B, N, Hkv, Hkv, 64, 64)
+    if idx is None:
+        idx = torch.empty((B, Hkv, T, k_tokens), dtype=torch.int32, device=scores.device)
+    _check(hysparse_topk_tokens(sh, _ptr(scores), k_tokens, forced_window, _ptr(idx), None, 0, _stream(stream)),
+           "hysparse_topk_tokens")
+    return idx
+
+
+def sparse_attn(q_sparse, k, v, idx, k_swa, v_swa, window: int, gate_logits, *, o=None, stream=None):
+    torch = _torch()
+    sh = prefill_shape(q_sparse, k)
+    if o is None:
+        o = torch.empty_like(q_sparse)
+    _check(hysparse_sparse_attn(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k), _ptr(v), _ptr(idx), idx.shape[-1],
+                                _ptr(k_swa), _ptr(v_swa), window, _ptr(gate_logits), None, _ptr(o),
+                                _stream(stream)), "hysparse_sparse_attn")
+    return o
+
+
+def sparse_attn_tokens(q_sparse, k, v, idx, forced_window: int, *, o=None, stream=None):
+    torch = _torch()
+    sh = prefill_shape(q_sparse, k)
+    if o is None:
+        o = torch.empty_like(q_sparse)
+    _check(hysparse_sparse_attn_tokens(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k), _ptr(v), _ptr(idx),
+                                       idx.shape[-1], forced_window, None, _ptr(o), _stream(stream)),
+           "hysparse_sparse_attn_tokens")
+    return o
+
+
+def full_attn_select_decode(q, k_cache, v_cache, *, seqlens=None, reduce: str = "sum", o=None, scores=None,
+                            workspace=None, stream=None):
+    torch = _torch()
+    sh = decode_shape(q, k_cache)
+    nb = (sh.L + 63) // 64
+    if o is None:
+        o = torch.empty_like(q)
+    if scores is None:
+        scores = torch.empty((sh.B, sh.Hkv, nb), dtype=torch.float32, device=q.device)
+    nws = hysparse_full_attn_select_decode_workspace_size(sh, _dt(q))
+    if workspace is None:
+        workspace = workspace_for(nws, q.device)
+    _check(hysparse_full_attn_select_decode(sh, _dt(q), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                                            _ptr(o), _ptr(scores), HYS_REDUCE_MAX if reduce == "max" else
+                                            HYS_REDUCE_SUM, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hysparse_full_attn_select_decode")
+    return o, scores
+
+
+def topk_decode(scores, k: int, L: int, *, seqlens=None, idx=None, stream=None):
+    torch = _torch()
+    B, Hkv, NB = scores.shape
+    sh = hys_decode_shape(B, L, Hkv, Hkv, 64, 64)
+    if idx is None:
+        idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=scores.device)
+    _check(hysparse_topk_decode(sh, _ptr(scores), k, _ptr(seqlens), _ptr(idx), _stream(stream)), "hysparse_topk_decode")
+    return idx
+
+
+def sparse_attn_decode(q, k_cache, v_cache, idx, k_ring, v_ring, gate_logits, *, seqlens=None, swa_len=None,
+                       o=None, stream=None):
+    torch = _torch()
+    sh = decode_shape(q, k_cache)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(hysparse_sparse_attn_decode(sh, _dt(q), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(idx),
+                                       idx.shape[-1], _ptr(k_ring), _ptr(v_ring), k_ring.shape[2], _ptr(swa_len),
+                                       _ptr(gate_logits), None, _ptr(o), _stream(stream)),
+           "hysparse_sparse_attn_decode")
+    return o

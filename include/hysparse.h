@@ -1,0 +1,213 @@
+/*
+ * hysparse.h -- C ABI of the HySparse hybrid-block attention hot path (B200, sm_100a).
+ *
+ * Sources of the operations (cited per entry point below):
+ *   [HS]  "HySparse: A Hybrid Sparse Attention Architecture with Oracle Token Selection
+ *         and KV Cache Sharing" (paper-graph long-form summary), section 3.4.1 (full
+ *         attention o_t, block-level max score S_t^i, two-pass rescale, GQA aggregation),
+ *         3.4.2 (TopK block selection), 3.4.3 (gather, sparse branch, SWA branch,
+ *         sigmoid gated fusion), 3.4.4 (cross-layer KV sharing).
+ *   [HS2] HySparse2 explainer (deep-reads): "Precise retrieval without a separate
+ *         indexer" (token-level selection, newest 128 tokens forced in) and "Twenty
+ *         lines of algorithmic intuition" (decode step).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless stated.
+ *     The library never allocates device memory inside a call; scratch memory comes
+ *     from a caller-provided workspace whose size the matching *_workspace_size()
+ *     query returns (a NULL workspace with size 0 is accepted when the query says 0).
+ *   - Work is enqueued asynchronously on the caller's CUDA stream; no call
+ *     synchronises the host.  Inputs must stay valid until the work completes.
+ *   - Tensors are contiguous row-major:
+ *        Q, O (prefill)            [B, Hq, N, D]
+ *        K, V, K', V' (prefill)    [B, Hkv, N, D]
+ *        gate logits (prefill)     [B, Hq, N, 2] fp32 (index 0: sparse branch, 1: SWA)
+ *        block scores              [B, Hkv, T, NB] fp32, T = NB = ceil(N / block)
+ *        token scores              [B, Hkv, T, N] fp32
+ *        block indices             [B, Hkv, T, k] int32, ascending, padded with -1
+ *        token indices             [B, Hkv, T, k_tokens] int32, ascending, padded with -1
+ *     Query head h reads KV head h / (Hq / Hkv) (grouped-query attention).
+ *   - Element type: HYS_BF16 or HYS_F32 for Q/K/V/O (outputs take the input type);
+ *     arithmetic accumulates in fp32.  Scores are always fp32.
+ *   - block must be 64; D must be 64 or 128; Hq % Hkv == 0; every pointer 16-byte
+ *     aligned.  Violations return HYS_ERR_INVALID_ARG and launch nothing.
+ *   - No exception crosses the ABI.  A CUDA launch error returns HYS_ERR_CUDA.
+ *     Kernels whose waits are bounded record HYS_ERR_TIMEOUT in a device status
+ *     word that hysparse_get_device_status() reads.
+ */
+#ifndef HYSPARSE_H_
+#define HYSPARSE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HYS_API __attribute__((visibility("default")))
+#else
+#define HYS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hys_stream_t; /* same type as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  HYS_OK = 0,
+  HYS_ERR_INVALID_ARG = 1,
+  HYS_ERR_UNSUPPORTED = 2,
+  HYS_ERR_CUDA = 3,
+  HYS_ERR_TIMEOUT = 4,
+  HYS_ERR_WORKSPACE = 5 /* workspace missing or smaller than the size query returned */
+} hys_status;
+
+typedef enum { HYS_F32 = 0, HYS_BF16 = 1 } hys_dtype;
+
+/* Granularity of the importance scores the full layer emits. */
+typedef enum { HYS_GRAN_BLOCK = 0, HYS_GRAN_TOKEN = 1 } hys_gran;
+
+/* Aggregation R over the query heads of a KV group and the rows of a 64-query tile.
+ * SUM is the default; MAX is the paper's conservative group-wise maximum. */
+typedef enum { HYS_REDUCE_SUM = 0, HYS_REDUCE_MAX = 1 } hys_reduce;
+
+typedef struct {
+  int B;     /* batch */
+  int N;     /* sequence length, >= 1 */
+  int Hq;    /* query heads */
+  int Hkv;   /* key/value heads, divides Hq */
+  int D;     /* head dim, 64 or 128 */
+  int block; /* KV block = query tile = 64 */
+} hys_shape;
+
+typedef struct {
+  int B;     /* sequences */
+  int L;     /* cache capacity per sequence (tokens), >= 1 */
+  int Hq;
+  int Hkv;
+  int D;
+  int block; /* 64 */
+} hys_decode_shape;
+
+/* Library version as "major.minor.patch". Host pointer, static storage. */
+HYS_API const char* hysparse_version(void);
+
+/* Human-readable name of a status code. Host pointer, static storage. */
+HYS_API const char* hysparse_status_string(hys_status s);
+
+/* Reads (and with reset != 0 clears) the device status word of the current device:
+ * HYS_OK, or HYS_ERR_TIMEOUT when a bounded wait inside a kernel ran out.
+ * *out is a HOST pointer. Synchronises the given stream. */
+HYS_API hys_status hysparse_get_device_status(hys_stream_t stream, int reset, int* out);
+
+/* ------------------------------------------------------------------------------------
+ * Full attention layer with fused importance scores.
+ *
+ * o_t = sum_{i<=t} softmax_i(tau q_t.k_i) v_i, tau = 1/sqrt(D)            [HS] 3.4.1, o_t
+ *
+ * gran = HYS_GRAN_BLOCK: scores [B,Hkv,T,NB] with
+ *   scores[b,g,I,j] = R_{h in g} R_{t in tile I} S^h_{t,j}   for j <= I, 0 for j > I,
+ *   S^h_{t,j} = max over keys i of block j with i <= t of the probability P^h_{t,i}
+ *   ([HS] 3.4.1, S_t^i and the two-pass rescale exp(m~ - m)/l; GQA aggregation with R
+ *   = sum (default) or max).
+ * gran = HYS_GRAN_TOKEN: scores [B,Hkv,T,N] with
+ *   scores[b,g,I,i] = sum_{h in g} sum_{t in tile I, t >= i} P^h_{t,i}   ([HS2], token
+ *   selection; red must be HYS_REDUCE_SUM).
+ * lse_opt: NULL or [B,Hq,N] fp32, receives LSE_t = log sum_i exp(tau q_t.k_i).
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_full_attn_select_workspace_size(const hys_shape* shape, hys_dtype dtype,
+                                                    hys_gran gran, size_t* bytes);
+HYS_API hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype dtype, const void* q,
+                                     const void* k, const void* v, void* o, float* scores,
+                                     hys_gran gran, hys_reduce red, float* lse_opt,
+                                     void* workspace, size_t workspace_bytes,
+                                     hys_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * TopK block selection ([HS] 3.4.2).  For each (b, g, I) the k largest of
+ * scores[b,g,I,0..I] (I+1 candidates), ties to the lower block index; fewer than k
+ * candidates selects all of them.  idx [B,Hkv,T,k] int32, ascending, padded with -1.
+ * 1 <= k <= 1024.  No workspace.
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_topk(const hys_shape* shape, const float* scores, int k, int* idx,
+                         hys_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * TopK token selection with a forced recent window ([HS2]).  Candidates of tile I are
+ * positions [0, e_I - forced_window], e_I = min(64I+63, N-1); the k_tokens largest of
+ * scores[b,g,I,i] over them, ties to the lower position; ascending, padded with -1.
+ * The forced window is not part of the budget.  1 <= k_tokens <= 16384.
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_topk_tokens_workspace_size(const hys_shape* shape, int k_tokens,
+                                               size_t* bytes);
+HYS_API hys_status hysparse_topk_tokens(const hys_shape* shape, const float* tok_scores, int k_tokens,
+                                int forced_window, int* idx, void* workspace,
+                                size_t workspace_bytes, hys_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Sparse layer: block-sparse branch + sliding-window branch + sigmoid gate
+ * ([HS] 3.4.3, the gather K~,V~ = concat of the selected blocks, o~_t, o'_t, and
+ * o_t = sigmoid(g0) o~_t + sigmoid(g1) o'_t).
+ *   Row t of tile I attends {i <= t : floor(i/64) in idx[b,g,I,:]} of the shared K, V
+ *   (the full layer's cache, [HS] 3.4.4) and [max(0, t-window+1), t] of its own K', V'.
+ *   k_swa/v_swa may alias k_shared/v_shared (the "share both" ablation).
+ *   idx entries are ascending block ids <= I or -1 (ignored); 1 <= k <= 1024.
+ *   sinks must be NULL (per-head sink biases are not implemented: HYS_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                const void* k_shared, const void* v_shared, const int* idx,
+                                int k, const void* k_swa, const void* v_swa, int window,
+                                const float* gate_logits, const float* sinks, void* o,
+                                hys_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Token-sparse layer ([HS2]): row t of tile I attends idx[b,g,I,:] (token positions,
+ * ascending, -1 padded, all <= t) united with [max(0, t-forced_window+1), t], each
+ * token once, over the shared K, V; no gate.  sinks must be NULL.
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_sparse_attn_tokens(const hys_shape* shape, hys_dtype dtype,
+                                       const void* q_sparse, const void* k_shared,
+                                       const void* v_shared, const int* idx, int k_tokens,
+                                       int forced_window, const float* sinks, void* o,
+                                       hys_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Decode, full layer ([HS2] decode step; [HS] 3.4.1).  One new token per sequence at
+ * position L_b - 1 of its cache (L_b = seqlens[b], or L when seqlens is NULL).
+ *   q [B,Hq,D]; k_cache, v_cache [B,Hkv,L,D]; o [B,Hq,D];
+ *   scores [B,Hkv,NB] fp32, NB = ceil(L/64): R_{h in g} S^h_j, 0 past the sequence end.
+ *   seqlens: NULL or [B] int32 in [1, L].
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_full_attn_select_decode_workspace_size(const hys_decode_shape* shape,
+                                                           hys_dtype dtype, size_t* bytes);
+HYS_API hys_status hysparse_full_attn_select_decode(const hys_decode_shape* shape, hys_dtype dtype,
+                                            const void* q, const void* k_cache,
+                                            const void* v_cache, const int* seqlens, void* o,
+                                            float* scores, hys_reduce red, void* workspace,
+                                            size_t workspace_bytes, hys_stream_t stream);
+
+/* TopK over the decode scores: idx [B,Hkv,k]; candidates are the blocks holding
+ * cached tokens (ceil(L_b/64)); ties to the lower index; ascending, -1 padded. */
+HYS_API hys_status hysparse_topk_decode(const hys_decode_shape* shape, const float* scores, int k,
+                                const int* seqlens, int* idx, hys_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Decode, sparse layer ([HS] 3.4.3 for one query row).  The sparse branch attends every
+ * cached token (< L_b) of the selected blocks of the shared cache; the SWA branch attends
+ * the layer's own ring k_swa_ring/v_swa_ring [B,Hkv,W,D] (swa_len[b] valid entries, or W
+ * when swa_len is NULL; order is irrelevant); gate_logits [B,Hq,2]; o [B,Hq,D].
+ * W = window, 1 <= window <= 1024.  sinks must be NULL.
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype dtype,
+                                       const void* q, const void* k_cache,
+                                       const void* v_cache, const int* seqlens,
+                                       const int* idx, int k, const void* k_swa_ring,
+                                       const void* v_swa_ring, int window, const int* swa_len,
+                                       const float* gate_logits, const float* sinks, void* o,
+                                       hys_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYSPARSE_H_ */

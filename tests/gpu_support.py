@@ -1,0 +1,53 @@
+"""Helpers of the GPU parity tests: device tensors from the seeded generator, the
+hybrid-block path through the C ABI, and the two acceptance rules.
+
+Rule 1: where the oracle's k-th and (k+1)-th scores of a tile differ by more than
+1e-3 relative, the GPU's selected set equals the oracle's.  Rule 2: elsewhere it
+equals the oracle's selection routine applied to the GPU's own emitted scores.
+Outputs are then compared with the oracle run on the GPU's indices: max-abs error
+<= 1e-4 for fp32 inputs and <= 2e-2 for bf16 inputs (fp32 accumulation)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+from attention_tcgen05_tma_b200 import hysparse as H
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+GAP = 1e-3
+
+
+def to_dev(x: np.ndarray, dtype: str, device="cuda"):
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if dtype == "bf16":
+        t = t.to(torch.bfloat16)   # exact: the generator already rounded to bf16
+    return t.to(device)
+
+
+def to_np(t) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check_selection(oracle_scores: np.ndarray, gpu_scores: np.ndarray, gpu_idx: np.ndarray, n_cand: int, k: int):
+    """Apply rules 1/2 to one tile. Returns 'rule1' or 'rule2'; raises on violation."""
+    s = oracle_scores[:n_cand]
+    order = np.lexsort((np.arange(n_cand), -s))
+    want_oracle = O.select_topk(oracle_scores, n_cand, k)
+    if n_cand <= k:
+        assert np.array_equal(gpu_idx, want_oracle), (gpu_idx, want_oracle)
+        return "rule1"
+    sk, sk1 = s[order[k - 1]], s[order[k]]
+    if sk > 0 and (sk - sk1) / sk > GAP:
+        assert np.array_equal(gpu_idx, want_oracle), (gpu_idx, want_oracle)
+        return "rule1"
+    want_gpu = O.select_topk(gpu_scores.astype(np.float64), n_cand, k)
+    assert np.array_equal(gpu_idx, want_gpu), (gpu_idx, want_gpu)
+    return "rule2"
+
+
+def score_rel_err(oracle_scores: np.ndarray, gpu_scores: np.ndarray, floor: float = 1e-6) -> float:
+    mask = np.abs(oracle_scores) > floor
+    if not mask.any():
+        return 0.0
+    return float(np.max(np.abs(gpu_scores[mask] - oracle_scores[mask]) / np.abs(oracle_scores[mask])))

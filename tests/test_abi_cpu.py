@@ -1,0 +1,77 @@
+"""Host-only checks of the C ABI library: it builds, loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_tcgen05_tma_b200 import build as B
+from attention_tcgen05_tma_b200 import hysparse as H
+
+HEADER = os.path.join(B.ROOT, "include", "hysparse.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return H.load()
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"HYS_API\s+[\w\s\*]+?\b(hysparse_\w+)\s*\(", txt)))
+
+
+def test_header_and_binding_agree():
+    assert declared_symbols() == sorted(H.EXPORTED)
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert re.match(r"^\d+\.\d+\.\d+$", H.hysparse_version())
+    assert H.status_string(H.HYS_ERR_INVALID_ARG) == "HYS_ERR_INVALID_ARG"
+    assert H.status_string(H.HYS_ERR_TIMEOUT) == "HYS_ERR_TIMEOUT"
+
+
+def test_workspace_queries_and_validation(lib):
+    good = H.hys_shape(1, 1000, 8, 2, 128, 64)
+    assert H.hysparse_full_attn_select_workspace_size(good, H.HYS_BF16, H.HYS_GRAN_BLOCK) >= 0
+    assert H.hysparse_full_attn_select_workspace_size(good, H.HYS_BF16, H.HYS_GRAN_TOKEN) >= 4 * 8 * 1000
+    for bad in (H.hys_shape(1, 1000, 8, 3, 128, 64), H.hys_shape(1, 1000, 8, 2, 96, 64),
+                H.hys_shape(1, 0, 8, 2, 128, 64), H.hys_shape(1, 1000, 8, 2, 128, 32)):
+        with pytest.raises(H.HysparseError) as e:
+            H.hysparse_full_attn_select_workspace_size(bad, H.HYS_BF16, H.HYS_GRAN_BLOCK)
+        assert e.value.status == H.HYS_ERR_INVALID_ARG
+    dsh = H.hys_decode_shape(4, 5000, 32, 4, 128, 64)
+    assert H.hysparse_full_attn_select_decode_workspace_size(dsh, H.HYS_BF16) > 0
+
+
+def test_entry_points_reject_bad_arguments_without_launching(lib):
+    sh = H.hys_shape(1, 256, 4, 1, 64, 64)
+    # null pointers / misaligned pointers / bad k are rejected on the host
+    assert H.hysparse_full_attn_select(sh, H.HYS_F32, None, None, None, None, None, 0, 0, None, None, 0, None) \
+        == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_topk(sh, 16, 0, 16, None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_topk(sh, 17, 4, 16, None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_sparse_attn(sh, H.HYS_F32, 16, 16, 16, 16, 4, 16, 16, 128, 16, 16, 16, None) \
+        == H.HYS_ERR_UNSUPPORTED   # sinks are not implemented
+    assert H.hysparse_sparse_attn_tokens(sh, H.HYS_F32, 16, 16, 16, 16, 0, 128, None, 16, None) \
+        == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_full_attn_select(sh, H.HYS_F32, 16, 16, 16, 16, 16, 0, 7, None, None, 0, None) \
+        == H.HYS_ERR_INVALID_ARG
+    # token scores with max aggregation are not defined
+    assert H.hysparse_full_attn_select(sh, H.HYS_F32, 16, 16, 16, 16, 16, H.HYS_GRAN_TOKEN, H.HYS_REDUCE_MAX,
+                                       None, 16, 1 << 20, None) == H.HYS_ERR_UNSUPPORTED
+    # workspace too small
+    assert H.hysparse_full_attn_select(sh, H.HYS_F32, 16, 16, 16, 16, 16, 0, 0, None, 16, 4, None) \
+        == H.HYS_ERR_WORKSPACE
+    dsh = H.hys_decode_shape(2, 100, 4, 1, 64, 64)
+    assert H.hysparse_sparse_attn_decode(dsh, H.HYS_F32, 16, 16, 16, None, 16, 4, 16, 16, 2000, None, 16, None,
+                                         16, None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_full_attn_select_decode(dsh, H.HYS_F32, 16, 16, 16, None, 16, 16, 0, None, 0, None) \
+        == H.HYS_ERR_WORKSPACE

@@ -1,0 +1,173 @@
+"""GPU parity of every entry point against the float64 oracle on small seeded cases
+(several tiles and a ragged tail), called through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from attention_tcgen05_tma_b200 import hysparse as H
+from attention_tcgen05_tma_b200 import inputs as I
+from tests.gpu_support import TOL, check_selection, score_rel_err, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+PREFILL_CASES = [
+    # name, dtype, B, N, Hq, Hkv, D, k, window
+    ("tiny_fp32", "f32", 1, 1024, 4, 1, 64, 4, 128),
+    ("bf16_d128_g4_ragged", "bf16", 2, 1000, 8, 2, 128, 4, 128),
+    ("bf16_d64_g8", "bf16", 1, 333, 8, 1, 64, 3, 100),
+    ("bf16_d128_g2_k_large", "bf16", 1, 700, 4, 2, 128, 16, 64),
+    ("f32_d128_g1", "f32", 1, 200, 2, 2, 128, 2, 300),
+]
+
+
+def _workload(dtype, B, N, Hq, Hkv, D, k, window, seed=11):
+    base = I.WORKLOADS["tiny"] if dtype == "f32" else I.WORKLOADS["dense7b"]
+    return I.scaled(base, B=B, N=N, Hq=Hq, Hkv=Hkv, D=D, topk=k, window=window, layers=1, seed=seed,
+                    scale_std=1.0 if dtype == "f32" else 1.0 / np.sqrt(D), n_plants=min(8, N // 64))
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=[c[0] for c in PREFILL_CASES])
+@pytest.mark.parametrize("reduce", ["sum", "max"])
+def test_hybrid_block_prefill(case, reduce):
+    name, dt, B, N, Hq, Hkv, D, k, window = case
+    w = _workload(dt, B, N, Hq, Hkv, D, k, window)
+    a = I.prefill_arrays(w, layers=1)
+    q, kk, vv = (to_dev(a[x], dt) for x in ("q", "k", "v"))
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    o, sc = H.full_attn_select(q, kk, vv, reduce=reduce, lse=lse)
+    idx = H.topk(sc, k)
+    qs, ks, vs = (to_dev(a[x][0], dt) for x in ("q_sparse", "k_swa", "v_swa"))
+    gate = to_dev(a["gate"][0], "f32")
+    osp = H.sparse_attn(qs, kk, vv, idx, ks, vs, window, gate)
+    torch.cuda.synchronize()
+
+    o_ref, lse_ref = O.full_attention(a["q"], a["k"], a["v"])
+    assert np.max(np.abs(to_np(o) - o_ref)) <= TOL[dt]
+    assert np.max(np.abs(to_np(lse) - lse_ref)) <= 1e-3
+    sc_ref = O.block_scores(a["q"], a["k"], reduce)
+    sc_gpu = to_np(sc)
+    assert score_rel_err(sc_ref, sc_gpu) <= 1e-3
+    assert np.all(sc_gpu >= 0)
+    T = sc_ref.shape[2]
+    for I_ in range(T):
+        assert np.all(sc_gpu[:, :, I_, I_ + 1:] == 0)
+    gidx = idx.cpu().numpy().astype(np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            for I_ in range(T):
+                check_selection(sc_ref[b, g, I_], sc_gpu[b, g, I_], gidx[b, g, I_], I_ + 1, k)
+    ref = O.sparse_attention(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], window,
+                             a["gate"][0])
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL[dt]
+
+
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 129])
+def test_edge_lengths(N):
+    w = _workload("bf16", 1, N, 4, 2, 128, 2, 128, seed=N)
+    a = I.prefill_arrays(w, layers=1)
+    q, kk, vv = (to_dev(a[x], "bf16") for x in ("q", "k", "v"))
+    o, sc = H.full_attn_select(q, kk, vv)
+    idx = H.topk(sc, 2)
+    qs, ks, vs = (to_dev(a[x][0], "bf16") for x in ("q_sparse", "k_swa", "v_swa"))
+    osp = H.sparse_attn(qs, kk, vv, idx, ks, vs, 128, to_dev(a["gate"][0], "f32"))
+    torch.cuda.synchronize()
+    o_ref, _ = O.full_attention(a["q"], a["k"], a["v"])
+    assert np.max(np.abs(to_np(o) - o_ref)) <= TOL["bf16"]
+    gidx = idx.cpu().numpy().astype(np.int64)
+    assert np.all(gidx[..., 0] == 0)    # block 0 is always a candidate
+    ref = O.sparse_attention(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], 128,
+                             a["gate"][0])
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL["bf16"]
+
+
+def test_share_both_ablation_aliasing():
+    """K'/V' may alias the shared K/V ("share both" ablation)."""
+    w = _workload("bf16", 1, 300, 4, 1, 64, 2, 64)
+    a = I.prefill_arrays(w, layers=1)
+    q, kk, vv = (to_dev(a[x], "bf16") for x in ("q", "k", "v"))
+    _, sc = H.full_attn_select(q, kk, vv)
+    idx = H.topk(sc, 2)
+    qs = to_dev(a["q_sparse"][0], "bf16")
+    osp = H.sparse_attn(qs, kk, vv, idx, kk, vv, 64, to_dev(a["gate"][0], "f32"))
+    torch.cuda.synchronize()
+    gidx = idx.cpu().numpy().astype(np.int64)
+    ref = O.sparse_attention(a["q_sparse"][0], a["k"], a["v"], gidx, a["k"], a["v"], 64, a["gate"][0])
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL["bf16"]
+
+
+TOKEN_CASES = [
+    ("bf16_d128", "bf16", 1, 700, 8, 2, 128, 100, 128),
+    ("bf16_d64_small_forced", "bf16", 1, 300, 4, 1, 64, 40, 16),
+    ("f32_d64", "f32", 1, 400, 4, 1, 64, 64, 128),
+]
+
+
+@pytest.mark.parametrize("case", TOKEN_CASES, ids=[c[0] for c in TOKEN_CASES])
+def test_token_variant(case):
+    name, dt, B, N, Hq, Hkv, D, kt, forced = case
+    w = _workload(dt, B, N, Hq, Hkv, D, kt, forced)
+    a = I.prefill_arrays(w, layers=1)
+    q, kk, vv = (to_dev(a[x], dt) for x in ("q", "k", "v"))
+    o, ts = H.full_attn_select(q, kk, vv, gran="token")
+    idx = H.topk_tokens(ts, kt, forced)
+    qs = to_dev(a["q_sparse"][0], dt)
+    osp = H.sparse_attn_tokens(qs, kk, vv, idx, forced)
+    torch.cuda.synchronize()
+    o_ref, _ = O.full_attention(a["q"], a["k"], a["v"])
+    assert np.max(np.abs(to_np(o) - o_ref)) <= TOL[dt]
+    ts_gpu = to_np(ts)
+    gidx = idx.cpu().numpy().astype(np.int64)
+    G = Hq // Hkv
+    T = (N + 63) // 64
+    for b in range(B):
+        for g in range(Hkv):
+            qg = a["q"][b, g * G:(g + 1) * G]
+            for I_ in range(T):
+                ref_ts = O.token_scores_tile(qg, a["k"][b, g], I_)
+                assert score_rel_err(ref_ts, ts_gpu[b, g, I_]) <= 1e-3
+                nc = O.token_candidates(I_, N, forced)
+                check_selection(ref_ts, ts_gpu[b, g, I_], gidx[b, g, I_], nc, kt)
+                rows = O.tile_rows(I_, N)
+                for h in range(g * G, (g + 1) * G):
+                    ref = O.token_sparse_rows(a["q_sparse"][0][b, h, rows], rows, a["k"][b, g], a["v"][b, g],
+                                              gidx[b, g, I_], forced)
+                    assert np.max(np.abs(to_np(osp[b, h, rows]) - ref)) <= TOL[dt]
+
+
+DECODE_CASES = [
+    ("bf16_d128_g8", "bf16", 3, 1500, 16, 2, 128, 4, 128, True),
+    ("bf16_d64_g4", "bf16", 2, 700, 4, 1, 64, 8, 32, False),
+    ("f32_d64_g4", "f32", 2, 300, 8, 2, 64, 2, 16, True),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=[c[0] for c in DECODE_CASES])
+def test_decode(case):
+    name, dt, B, L, Hq, Hkv, D, k, W, ragged = case
+    w = I.scaled(I.WORKLOADS["decode"], B=B, N=L, Hq=Hq, Hkv=Hkv, D=D, topk=k, window=W, layers=1, seed=5,
+                 scale_std=1.0 / np.sqrt(D))
+    a = I.decode_arrays(w, layers=1)
+    seqlens = np.array([L - 37 * b for b in range(B)], dtype=np.int32) if ragged else None
+    swa_len = np.array([W - 3 * b for b in range(B)], dtype=np.int32) if ragged else None
+    q, kc, vc = (to_dev(a[x], dt) for x in ("q", "k", "v"))
+    sl = torch.from_numpy(seqlens).cuda() if ragged else None
+    o, sc = H.full_attn_select_decode(q, kc, vc, seqlens=sl)
+    idx = H.topk_decode(sc, k, L, seqlens=sl)
+    qs, kr, vr = (to_dev(a[x][0], dt) for x in ("q_sparse", "k_swa", "v_swa"))
+    gate = to_dev(a["gate"][0], "f32")
+    swl = torch.from_numpy(swa_len).cuda() if ragged else None
+    osp = H.sparse_attn_decode(qs, kc, vc, idx, kr, vr, gate, seqlens=sl, swa_len=swl)
+    torch.cuda.synchronize()
+    o_ref, sc_ref = O.decode_full(a["q"], a["k"], a["v"], seqlens)
+    assert np.max(np.abs(to_np(o) - o_ref)) <= TOL[dt]
+    sc_gpu = to_np(sc)
+    assert score_rel_err(sc_ref, sc_gpu) <= 1e-3
+    gidx = idx.cpu().numpy().astype(np.int64)
+    for b in range(B):
+        nb = ((int(seqlens[b]) if seqlens is not None else L) + 63) // 64
+        for g in range(Hkv):
+            check_selection(sc_ref[b, g], sc_gpu[b, g], gidx[b, g], nb, k)
+    ref = O.decode_sparse(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], a["gate"][0],
+                          seqlens, swa_len)
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL[dt]
