@@ -27,7 +27,7 @@ EXPORTED = (
     "hysparse_topk", "hysparse_topk_tokens_workspace_size", "hysparse_topk_tokens",
     "hysparse_sparse_attn", "hysparse_sparse_attn_tokens",
     "hysparse_full_attn_select_decode_workspace_size", "hysparse_full_attn_select_decode",
-    "hysparse_topk_decode", "hysparse_sparse_attn_decode",
+    "hysparse_topk_decode", "hysparse_sparse_attn_decode", "hysparse_full_attn_select_decode_noalloc",
 )
 
 
@@ -67,6 +67,7 @@ _SIGS = {
     "hysparse_full_attn_select_decode_workspace_size": ([_DSH, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_full_attn_select_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P], _I),
     "hysparse_topk_decode": ([_DSH, _P, _I, _P, _P, _P], _I),
+    "hysparse_full_attn_select_decode_noalloc": ([_DSH, _I, _P, _P, _P, _P, _P, _P, _I, _P], _I),
     "hysparse_sparse_attn_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P], _I),
 }
 
@@ -156,6 +157,13 @@ def hysparse_full_attn_select_decode_workspace_size(shape: hys_decode_shape, dty
 def hysparse_full_attn_select_decode(shape, dtype, q, kc, vc, seqlens, o, scores, red, ws, ws_bytes, stream) -> int:
     return load().hysparse_full_attn_select_decode(ctypes.byref(shape), dtype, q, kc, vc, seqlens, o, scores, red,
                                                    ws, ws_bytes, stream)
+
+
+def hysparse_full_attn_select_decode_noalloc(shape, dtype, q, kc, vc, seqlens, o, scores, red, stream) -> int:
+    """Decode full layer without a workspace (scratch in a fixed 16 MiB array inside the
+    library); for callers that cannot allocate device memory during a decode step."""
+    return load().hysparse_full_attn_select_decode_noalloc(ctypes.byref(shape), dtype, q, kc, vc, seqlens, o,
+                                                           scores, red, stream)
 
 
 def hysparse_topk_decode(shape, scores, k, seqlens, idx, stream) -> int:

@@ -186,6 +186,30 @@ HYS_API hys_status hysparse_full_attn_select_decode(const hys_decode_shape* shap
                                             float* scores, hys_reduce red, void* workspace,
                                             size_t workspace_bytes, hys_stream_t stream);
 
+/* ------------------------------------------------------------------------------------
+ * Allocation-free decode full layer.  The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory when they run a decode step
+ * (an engine that plans all of its device memory up front and forbids later
+ * cudaMalloc, which may synchronise the device; a host integration with no
+ * allocator).  Same operation, arguments and layouts as
+ * hysparse_full_attn_select_decode, minus the workspace: the split-KV scratch lives in
+ * a fixed 16 MiB array inside the library, held in device memory by every GPU that
+ * loads the library until the process exits.
+ *   - Shapes whose scratch (the value hysparse_full_attn_select_decode_workspace_size
+ *     returns) exceeds 16 MiB return HYS_ERR_WORKSPACE and launch nothing.
+ *   - The call allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *   - The first call on a device resolves the array's device address with that device
+ *     current; make that first call before any stream capture.
+ *   - All calls share the one array: calls whose work overlaps on the GPU (different
+ *     streams, or different host threads on the same device) race and must be ordered
+ *     by the caller.  Nothing in the array needs clearing between calls.
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_full_attn_select_decode_noalloc(const hys_decode_shape* shape,
+                                                          hys_dtype dtype, const void* q,
+                                                          const void* k_cache, const void* v_cache,
+                                                          const int* seqlens, void* o, float* scores,
+                                                          hys_reduce red, hys_stream_t stream);
+
 /* TopK over the decode scores: idx [B,Hkv,k]; candidates are the blocks holding
  * cached tokens (ceil(L_b/64)); ties to the lower index; ascending, -1 padded. */
 HYS_API hys_status hysparse_topk_decode(const hys_decode_shape* shape, const float* scores, int k,
