@@ -73,7 +73,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t full_ws_bytes(const PrefillDims& d, hys_dtype dt, hys_gran gran) {
   if (gran == HYS_GRAN_TOKEN) return align256(sizeof(float) * (size_t)d.B * d.Hq * d.N);
-  if (full_attn_tc_supported(d, dt)) return full_attn_tc_workspace(d);
+  if (full_attn_tc_supported(d, dt, true)) return align256(full_attn_tc_workspace(d));
   return align256(sizeof(float) * (size_t)d.B * d.Hq * d.T * d.NB);
 }
 
@@ -141,7 +141,7 @@ hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype dtype, co
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return HYS_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (gran == HYS_GRAN_BLOCK) {
-    if (full_attn_tc_supported(d, dtype))
+    if (full_attn_tc_supported(d, dtype, true))
       return from_cuda(launch_full_attn_tc(d, q, k, v, o, lse_opt, scores, red, true, workspace, workspace_bytes, s));
     float* part = reinterpret_cast<float*>(workspace);
     cudaError_t e = launch_full_attn_simt(d, dtype, q, k, v, o, lse_opt, part, true, red, s);
@@ -150,7 +150,7 @@ hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype dtype, co
   }
   float* lse = lse_opt ? lse_opt : reinterpret_cast<float*>(workspace);
   cudaError_t e;
-  if (full_attn_tc_supported(d, dtype))
+  if (full_attn_tc_supported(d, dtype, false))
     e = launch_full_attn_tc(d, q, k, v, o, lse, nullptr, HYS_REDUCE_SUM, false, nullptr, 0, s);
   else
     e = launch_full_attn_simt(d, dtype, q, k, v, o, lse, nullptr, false, HYS_REDUCE_SUM, s);

@@ -1,14 +1,539 @@
 // Full attention layer with fused block scores on the 5th-generation tensor cores.
+//
+// What it computes (HySparse 3.4.1): causal GQA attention o_t, and
+//   score[b,g,I,j] = R_{h in g} R_{t in tile I} exp(m~_{t,j} - m_t) / l_t ,   j <= I,
+// where m~_{t,j} is the row max logit of 64-key block j (clipped at t), m_t and l_t the
+// final softmax max and normaliser of row t (the paper's two-pass rescale, with the
+// exp), and R = sum (default) or max over the query heads of KV group g and the rows of
+// 64-query tile I.
+//
+// How (B200-first):
+//   * Persistent CTAs (one per SM) walk work units (b, g, I) longest-first.  A unit holds
+//     the G query heads of KV group g for the 64 positions of tile I.  They are packed two
+//     heads per 128-row M-tile (rows 0-63 head 2m, rows 64-127 head 2m+1, same positions),
+//     so every K/V tile staged in shared memory serves two heads, the causal extent of all
+//     rows of an M-tile is the same, and the whole score reduction of a unit stays in the
+//     CTA (no per-head partials, no second kernel).
+//   * Two M-tiles are in flight (ping-pong): S_s = Q_s K^T (tcgen05.mma, SS, fp32 in
+//     TMEM), softmax warpgroup s turns S_s into P_s (bf16, written back into the same TMEM
+//     columns) and O_s += P_s V (tcgen05.mma with A from TMEM).  TMEM: S0 S1 O0 O1 = 512
+//     columns.  K/V tiles (128 keys) arrive by TMA (128-byte swizzle) into a 4-stage ring.
+//   * The block max logits m~ fall out of the softmax row max for free: each thread owns
+//     one row and takes the max of the two 64-column halves of the 128-key S tile.  They are
+//     stashed (fp32, L2-resident per-CTA scratch) because m_t, l_t are final only after the
+//     last key tile; the M-tile epilogue rescales them and reduces over the tile's rows
+//     into a shared-memory accumulator per slot; the unit epilogue writes the scores.
+//   * Conditional rescaling: O and l are rescaled only when the row max grows by more
+//     than 2^8 (in exp2 units); the result is exact after the final normalisation.
+//   * Every wait is a bounded mbarrier wait; on expiry the kernel records HYS_ERR_TIMEOUT,
+//     drains its own TMA loads and MMAs, frees TMEM and returns.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace hys {
 
-bool full_attn_tc_supported(const PrefillDims&, hys_dtype) { return false; }
-size_t full_attn_tc_workspace(const PrefillDims&) { return 0; }
-cudaError_t launch_full_attn_tc(const PrefillDims&, const void*, const void*, const void*, void*, float*, float*,
-                                hys_reduce, bool, void*, size_t, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kThreads = 384;      // warp 0 TMA, warp 1 MMA, warps 4-7 / 8-11 softmax slots 0 / 1
+constexpr int kStages = 4;         // K/V ring depth (one stage = one 128-key K or V tile)
+constexpr int kMaxNB = 2048;       // score accumulator capacity per slot (N <= 131072)
+constexpr int kMaxGrid = 148;      // B200 SM count; the workspace is sized for this grid
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
+  static constexpr int kQBytes = 128 * D * 2;        // one M-tile of Q
+  static constexpr int kKVBytes = 128 * D * 2;       // one K or V tile of 128 keys
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kQBytes;
+  static constexpr int kOffAcc = kOffKV + kStages * kKVBytes;
+  static constexpr int kOffRow = kOffAcc + 2 * kMaxNB * 4;
+  static constexpr int kOffBar = kOffRow + 2 * 256 * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 * 8 + 2;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
+};
+
+struct Params {
+  int B, N, Hq, Hkv, G, T, NB, NBpad;
+  int num_units;
+  __nv_bfloat16* o;
+  float* lse;     // optional [B,Hq,N]
+  float* scores;  // optional [B,Hkv,T,NB] (block scores are emitted iff non-null)
+  float* stash;   // [grid][2][128][NBpad]
+  int red_max;
+  int* status;
+  float scale_log2;  // log2(e) / sqrt(D)
+};
+
+struct Bars {
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2], wg[2], all[2];
+  uint64_t mma_drain, spare;
+};
+
+__device__ __forceinline__ void unit_coords(const Params& p, int u, int& b, int& g, int& I) {
+  const int bgc = p.B * p.Hkv;
+  I = p.T - 1 - u / bgc;
+  const int bg = u % bgc;
+  b = bg / p.Hkv;
+  g = bg % p.Hkv;
+}
+
+// Group barrier on an mbarrier (count = group size); bounded, with acquire/release at CTA scope.
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volatile int* abort) {
+  tc::mbar_arrive(bar);
+  const bool ok = tc::mbar_wait(bar, phase & 1u, abort);
+  ++phase;
+  return ok;
+}
+
+__device__ __forceinline__ void fail(volatile int* abort, int* status) {
+  *abort = 1;
+  report_status(status, HYS_ERR_TIMEOUT);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    full_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);
+  float* acc_all = reinterpret_cast<float*>(smem + C::kOffAcc);
+  float* row_all = reinterpret_cast<float*>(smem + C::kOffRow);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool scores_on = p.scores != nullptr;
+  const int MT = p.G / 2;              // M-tiles per unit
+  const int rounds = (MT + 1) / 2;     // two M-tiles (slots) per round
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&bars->kv_full[i], 1);
+      tc::mbar_init(&bars->kv_empty[i], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->q_full[s], 1);
+      tc::mbar_init(&bars->q_empty[s], 1);
+      tc::mbar_init(&bars->s_full[s], 1);
+      tc::mbar_init(&bars->p_full[s], 128);
+      tc::mbar_init(&bars->o_full[s], 1);
+      tc::mbar_init(&bars->o_empty[s], 128);
+      tc::mbar_init(&bars->wg[s], 128);
+      tc::mbar_init(&bars->all[s], 256);
+    }
+    tc::mbar_init(&bars->mma_drain, 1);
+    *abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tensormap(&tmQ);
+    tc::prefetch_tensormap(&tmK);
+    tc::prefetch_tensormap(&tmV);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 512);
+    tc::tmem_relinquish();
+  }
+  // zero the score accumulators
+  for (int i = threadIdx.x; i < 2 * kMaxNB; i += kThreads) acc_all[i] = 0.0f;
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ============================================================== TMA producer
+    if (lane == 0) {
+      uint32_t kv_it = 0, q_cnt[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        int b, g, I;
+        unit_coords(p, u, b, g, I);
+        const int nkt = I / 2 + 1;
+        for (int r = 0; r < rounds && ok; ++r) {
+          for (int s = 0; s < 2 && ok; ++s) {
+            const int mt = 2 * r + s;
+            if (mt >= MT) continue;
+            if (!(ok = tc::mbar_wait(&bars->q_empty[s], (q_cnt[s] & 1u) ^ 1u, abort))) break;
+            ++q_cnt[s];
+            tc::mbar_arrive_expect_tx(&bars->q_full[s], C::kQBytes);
+            const int h0 = g * p.G + 2 * mt;
+            uint8_t* qdst = smem + C::kOffQ + s * C::kQBytes;
+            for (int hh = 0; hh < 2; ++hh)
+              for (int c = 0; c < C::kChunks; ++c)
+                tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + c * 16384 + hh * 8192, c * 64, 64 * I,
+                                b * p.Hq + h0 + hh);
+          }
+          for (int tau = 0; tau < nkt && ok; ++tau) {
+            for (int kv = 0; kv < 2; ++kv) {
+              const uint32_t st = kv_it % kStages;
+              if (!(ok = tc::mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1u) ^ 1u, abort))) break;
+              tc::mbar_arrive_expect_tx(&bars->kv_full[st], C::kKVBytes);
+              uint8_t* dst = smem + C::kOffKV + st * C::kKVBytes;
+              for (int c = 0; c < C::kChunks; ++c)
+                tc::tma_load_3d(kv ? &tmV : &tmK, &bars->kv_full[st], dst + c * 16384, c * 64, 128 * tau,
+                                b * p.Hkv + g);
+              ++kv_it;
+            }
+          }
+        }
+      }
+      if (!ok) fail(abort, p.status);
+      // drain: the last loads issued into each stage / Q slot must land before the CTA exits
+      for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i)
+        tc::mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u, abort, 100000000ull);
+      for (int s = 0; s < 2; ++s)
+        if (q_cnt[s] > 0) tc::mbar_wait(&bars->q_full[s], (q_cnt[s] - 1) & 1u, abort, 100000000ull);
+    }
+  } else if (warp == 1) {
+    // ============================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
+      const uint32_t idO = tc::idesc_bf16_f32(128, D, true);
+      const uint32_t tS[2] = {tmem_base, tmem_base + 128};
+      const uint32_t tO[2] = {tmem_base + 256, tmem_base + 384};
+      const uint32_t qaddr = tc::smem_u32(smem + C::kOffQ);
+      const uint32_t kvaddr = tc::smem_u32(smem + C::kOffKV);
+      uint32_t kv_it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
+      bool ok = true;
+      auto issue_S = [&](int s, uint32_t st) {
+        const uint32_t qb = qaddr + s * C::kQBytes, kb = kvaddr + st * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc::mma_ss(tS[s], tc::sdesc_sw128(qb + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024), idS,
+                     kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_PV = [&](int s, uint32_t st, bool acc) {
+        const uint32_t vb = kvaddr + st * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_ts(tO[s], tS[s] + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16384, 1024), idO,
+                     (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        int b, g, I;
+        unit_coords(p, u, b, g, I);
+        const int nkt = I / 2 + 1;
+        for (int r = 0; r < rounds && ok; ++r) {
+          bool act[2];
+          for (int s = 0; s < 2; ++s) {
+            act[s] = (2 * r + s) < MT;
+            if (act[s] && ok) {
+              ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort);
+              ++q_cnt[s];
+            }
+          }
+          if (!ok) break;
+          // prologue: S_s(0) = Q_s K_0^T
+          uint32_t kst = kv_it % kStages;
+          if (!(ok = tc::mbar_wait(&bars->kv_full[kst], (kv_it / kStages) & 1u, abort))) break;
+          ++kv_it;
+          tc::fence_after_sync();
+          for (int s = 0; s < 2; ++s)
+            if (act[s]) {
+              issue_S(s, kst);
+              tc::mma_commit(&bars->s_full[s]);
+            }
+          tc::mma_commit(&bars->kv_empty[kst]);
+          for (int tau = 1; tau <= nkt && ok; ++tau) {
+            const uint32_t vst = kv_it % kStages;
+            if (!(ok = tc::mbar_wait(&bars->kv_full[vst], (kv_it / kStages) & 1u, abort))) break;
+            ++kv_it;
+            bool have_k = false;
+            for (int s = 0; s < 2 && ok; ++s) {
+              if (!act[s]) continue;
+              if (!(ok = tc::mbar_wait(&bars->p_full[s], p_cnt[s] & 1u, abort))) break;
+              ++p_cnt[s];
+              if (tau == 1) {  // the previous round's epilogue must have read O_s
+                if (!(ok = tc::mbar_wait(&bars->o_empty[s], (o_cnt[s] & 1u) ^ 1u, abort))) break;
+              }
+              tc::fence_after_sync();
+              issue_PV(s, vst, tau > 1);
+              if (tau < nkt) {
+                if (!have_k) {
+                  kst = kv_it % kStages;
+                  if (!(ok = tc::mbar_wait(&bars->kv_full[kst], (kv_it / kStages) & 1u, abort))) break;
+                  ++kv_it;
+                  have_k = true;
+                  tc::fence_after_sync();
+                }
+                issue_S(s, kst);
+                tc::mma_commit(&bars->s_full[s]);
+              } else {
+                tc::mma_commit(&bars->o_full[s]);
+                ++o_cnt[s];
+              }
+            }
+            tc::mma_commit(&bars->kv_empty[vst]);
+            if (have_k) tc::mma_commit(&bars->kv_empty[kst]);
+          }
+          for (int s = 0; s < 2; ++s)
+            if (act[s]) tc::mma_commit(&bars->q_empty[s]);
+        }
+      }
+      if (!ok) fail(abort, p.status);
+      tc::mma_commit(&bars->mma_drain);
+      tc::mbar_wait(&bars->mma_drain, 0, abort, 100000000ull);
+    }
+  } else if (warp >= 4) {
+    // ============================================================== softmax / epilogue
+    const int s = (warp - 4) >> 2;                 // slot
+    const int row = 32 * (warp & 3) + lane;        // M-tile row == TMEM lane
+    const int wtid = threadIdx.x - 128 - 128 * s;  // 0..127 within the warpgroup
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tSrow = tmem_base + 128 * s + lane_off;
+    const uint32_t tOrow = tmem_base + 256 + 128 * s + lane_off;
+    float* acc = acc_all + s * kMaxNB;
+    float* row_m = row_all + 256 * s;
+    float* row_il = row_m + 128;
+    float* stash = p.stash + ((size_t)blockIdx.x * 2 + s) * 128 * (size_t)p.NBpad;
+    const float sc = p.scale_log2;
+    uint32_t s_cnt = 0, o_cnt = 0, wg_ph = 0, all_ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      int b, g, I;
+      unit_coords(p, u, b, g, I);
+      const int nkt = I / 2 + 1;
+      for (int r = 0; r < rounds && ok; ++r) {
+        const int mt = 2 * r + s;
+        if (mt >= MT) continue;
+        const int h = g * p.G + 2 * mt + (row >> 6);
+        const int t = 64 * I + (row & 63);
+        const bool valid = t < p.N;
+        float m_used = -INFINITY, l = 0.0f;
+        for (int tau = 0; tau < nkt; ++tau) {
+          if (!(ok = tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort))) break;
+          ++s_cnt;
+          tc::fence_after_sync();
+          float sv[128];
+          {
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tc::tmem_ld32(tSrow + 0, r0);
+            tc::tmem_ld32(tSrow + 32, r1);
+            tc::tmem_ld32(tSrow + 64, r2);
+            tc::tmem_ld32(tSrow + 96, r3);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              sv[i] = __uint_as_float(r0[i]);
+              sv[32 + i] = __uint_as_float(r1[i]);
+              sv[64 + i] = __uint_as_float(r2[i]);
+              sv[96 + i] = __uint_as_float(r3[i]);
+            }
+          }
+          if (tau == nkt - 1) {  // causal diagonal: keys past the row are masked
+            const int cmax = t - 128 * tau;
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i > cmax) sv[i] = -INFINITY;
+          }
+          float mlo = sv[0], mhi = sv[64];
+#pragma unroll
+          for (int i = 1; i < 64; ++i) {
+            mlo = fmaxf(mlo, sv[i]);
+            mhi = fmaxf(mhi, sv[64 + i]);
+          }
+          if (scores_on) *reinterpret_cast<float2*>(stash + (size_t)row * p.NBpad + 2 * tau) = make_float2(mlo, mhi);
+          const float mt_ = fmaxf(mlo, mhi);
+          float alpha = 1.0f;
+          const bool rescale = (mt_ - m_used) * sc > kRescaleLog2;
+          if (rescale) {
+            alpha = exp2f((m_used - mt_) * sc);
+            l *= alpha;
+            m_used = mt_;
+          }
+          const float ms = m_used * sc;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
+              const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
+              l += p0 + p1;
+              pk[i] = tc::pack_bf16x2(p0, p1);
+            }
+            tc::tmem_st16(tSrow + 16 * c, pk);
+          }
+          if (rescale && tau > 0) {
+            // O_s holds the sum over the earlier key tiles; its last PV is complete because
+            // S_s(tau), committed after it, is.  PV_s(tau) waits for p_full below.
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              tc::tmem_ld32(tOrow + 32 * c, ov);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tc::tmem_st32(tOrow + 32 * c, ov);
+            }
+          }
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bars->p_full[s]);
+        }
+        if (!ok) break;
+        // ---- M-tile epilogue: O / l -> global, LSE, block-score contribution
+        if (!(ok = tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort))) break;
+        ++o_cnt;
+        tc::fence_after_sync();
+        const float il = 1.0f / l;
+        __nv_bfloat16* orow = p.o + (((size_t)b * p.Hq + h) * p.N + t) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tc::tmem_ld32(tOrow + 32 * c, ov);
+          tc::tmem_wait_ld();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = tc::pack_bf16x2(__uint_as_float(ov[2 * i]) * il, __uint_as_float(ov[2 * i + 1]) * il);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&bars->o_empty[s]);
+        if (p.lse != nullptr && valid) p.lse[((size_t)b * p.Hq + h) * p.N + t] = (m_used * sc + log2f(l)) * 0.69314718055994531f;
+        if (scores_on) {
+          row_m[row] = m_used;
+          row_il[row] = valid ? il : 0.0f;
+          if (!(ok = group_sync(&bars->wg[s], wg_ph, abort))) break;
+          for (int j = wtid; j <= I; j += 128) {
+            float a = 0.0f;
+            for (int rr = 0; rr < 128; ++rr) {
+              const float x = exp2f((stash[(size_t)rr * p.NBpad + j] - row_m[rr]) * sc) * row_il[rr];
+              a = p.red_max ? fmaxf(a, x) : a + x;
+            }
+            acc[j] = p.red_max ? fmaxf(acc[j], a) : acc[j] + a;
+          }
+          if (!(ok = group_sync(&bars->wg[s], wg_ph, abort))) break;
+        }
+      }
+      if (!ok) break;
+      if (scores_on) {
+        // ---- unit epilogue: both slots' accumulators -> scores[b,g,I,:]
+        if (!(ok = group_sync(&bars->all[0], all_ph, abort))) break;
+        float* out = p.scores + (((size_t)b * p.Hkv + g) * p.T + I) * p.NB;
+        const int tid2 = wtid + 128 * s;
+        for (int j = tid2; j < p.NB; j += 256) {
+          float v = 0.0f;
+          if (j <= I) v = p.red_max ? fmaxf(acc_all[j], acc_all[kMaxNB + j]) : acc_all[j] + acc_all[kMaxNB + j];
+          out[j] = v;
+        }
+        if (!(ok = group_sync(&bars->all[0], all_ph, abort))) break;
+        for (int j = wtid; j <= I; j += 128) acc[j] = 0.0f;
+      }
+    }
+    if (!ok) fail(abort, p.status);
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [heads][rows][D] bf16, box = 64 columns x box_rows rows x 1 head, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, int D, int rows, int heads, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int nb_pad(int NB) { return (NB + 2 + 3) & ~3; }
+int num_units(const PrefillDims& d) { return d.B * d.Hkv * d.T; }
+int grid_size(const PrefillDims& d) { return num_units(d) < kMaxGrid ? num_units(d) : kMaxGrid; }
+
+template <int D>
+cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, const void* v, void* o, float* lse,
+                         float* scores, hys_reduce red, void* ws, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, d.N, d.B * d.Hq, 64) || !make_map(&mk, k, D, d.N, d.B * d.Hkv, 128) ||
+      !make_map(&mv, v, D, d.N, d.B * d.Hkv, 128))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.B = d.B;
+  p.N = d.N;
+  p.Hq = d.Hq;
+  p.Hkv = d.Hkv;
+  p.G = d.G();
+  p.T = d.T;
+  p.NB = d.NB;
+  p.NBpad = nb_pad(d.NB);
+  p.num_units = num_units(d);
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.scores = scores;
+  p.stash = reinterpret_cast<float*>(ws);
+  p.red_max = red == HYS_REDUCE_MAX;
+  p.status = device_status_ptr();
+  p.scale_log2 = kLog2e / sqrtf((float)D);
+  const int smem = Cfg<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(full_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  full_attn_tc_kernel<D><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool full_attn_tc_supported(const PrefillDims& d, hys_dtype dt, bool want_scores) {
+  if (dt != HYS_BF16 || (d.D != 64 && d.D != 128)) return false;
+  if (d.G() % 2 != 0) return false;
+  if (want_scores && d.NB > kMaxNB) return false;
+  return true;
+}
+
+size_t full_attn_tc_workspace(const PrefillDims& d) {
+  return sizeof(float) * (size_t)grid_size(d) * 2 * 128 * (size_t)nb_pad(d.NB);
+}
+
+cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, void* o,
+                                float* lse, float* scores, hys_reduce red, bool want_scores, void* ws, size_t ws_bytes,
+                                cudaStream_t s) {
+  if (!want_scores) scores = nullptr;
+  if (want_scores && ws_bytes < full_attn_tc_workspace(d)) return cudaErrorInvalidValue;
+  return d.D == 64 ? launch_typed<64>(d, q, k, v, o, lse, scores, red, ws, s)
+                   : launch_typed<128>(d, q, k, v, o, lse, scores, red, ws, s);
 }
 
 }  // namespace hys

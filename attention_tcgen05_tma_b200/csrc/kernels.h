@@ -38,7 +38,7 @@ cudaError_t launch_token_scores_simt(const PrefillDims& d, hys_dtype dt, const v
                                      const float* lse, float* scores, cudaStream_t s);
 
 // ---- full layer, tcgen05 path (bf16, D=128, even G) ----------------------------------------
-bool full_attn_tc_supported(const PrefillDims& d, hys_dtype dt);
+bool full_attn_tc_supported(const PrefillDims& d, hys_dtype dt, bool want_scores);
 size_t full_attn_tc_workspace(const PrefillDims& d);
 cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v,
                                 void* o, float* lse, float* scores, hys_reduce red, bool want_scores,

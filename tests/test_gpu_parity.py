@@ -18,6 +18,8 @@ PREFILL_CASES = [
     ("bf16_d64_g8", "bf16", 1, 333, 8, 1, 64, 3, 100),
     ("bf16_d128_g2_k_large", "bf16", 1, 700, 4, 2, 128, 16, 64),
     ("f32_d128_g1", "f32", 1, 200, 2, 2, 128, 2, 300),
+    ("bf16_d128_g16", "bf16", 1, 200, 16, 1, 128, 2, 128),
+    ("bf16_d128_g8_many_units", "bf16", 2, 2048, 32, 4, 128, 8, 128),
 ]
 
 
