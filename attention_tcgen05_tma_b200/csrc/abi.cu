@@ -193,10 +193,19 @@ hys_status hysparse_topk_tokens(const hys_shape* shape, const float* tok_scores,
 }
 
 // ----------------------------------------------------------------------------- sparse layer
+hys_status hysparse_sparse_attn_workspace_size(const hys_shape* shape, hys_dtype dtype, size_t* bytes) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || !dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  *bytes = sparse_attn_tc_supported(d, dtype) ? align256(sparse_attn_tc_workspace(d)) : 0;
+  return HYS_OK;
+}
+
 hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const void* q_sparse, const void* k_shared,
                                 const void* v_shared, const int* idx, int k, const void* k_swa, const void* v_swa,
-                                int window, const float* gate_logits, const float* sinks, void* o,
-                                hys_stream_t stream) {
+                                int window, const float* gate_logits, const float* sinks, void* o, void* workspace,
+                                size_t workspace_bytes, hys_stream_t stream) {
   PrefillDims d;
   hys_status st = check_prefill(shape, &d);
   if (st != HYS_OK) return st;
@@ -205,10 +214,17 @@ hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const v
   if (!q_sparse || !k_shared || !v_shared || !idx || !k_swa || !v_swa || !gate_logits || !o) return HYS_ERR_INVALID_ARG;
   if (k < 1 || k > 1024 || window < 1) return HYS_ERR_INVALID_ARG;
   if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(k_swa) ||
-      !aligned16(v_swa) || !aligned16(gate_logits) || !aligned16(o))
+      !aligned16(v_swa) || !aligned16(gate_logits) || !aligned16(o) || !aligned16(workspace))
     return HYS_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (sparse_attn_tc_supported(d, dtype)) {
+    const size_t need = align256(sparse_attn_tc_workspace(d));
+    if (workspace == nullptr || workspace_bytes < need) return HYS_ERR_WORKSPACE;
+    return from_cuda(launch_sparse_attn_tc(d, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,
+                                           gate_logits, o, workspace, workspace_bytes, s));
+  }
   return from_cuda(launch_sparse_attn_simt(d, dtype, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,
-                                           gate_logits, o, reinterpret_cast<cudaStream_t>(stream)));
+                                           gate_logits, o, s));
 }
 
 hys_status hysparse_sparse_attn_tokens(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,

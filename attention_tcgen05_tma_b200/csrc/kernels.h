@@ -60,6 +60,12 @@ cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const 
                                       const void* v, const int* idx, int kt, int forced, void* o,
                                       cudaStream_t s);
 
+bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt);
+size_t sparse_attn_tc_workspace(const PrefillDims& d);
+cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
+                                  int kb, const void* ks, const void* vs, int window, const float* gate, void* o,
+                                  void* ws, size_t ws_bytes, cudaStream_t s);
+
 // ---- decode ----------------------------------------------------------------------------------
 size_t decode_full_workspace(const DecodeDims& d);
 cudaError_t launch_decode_full(const DecodeDims& d, hys_dtype dt, const void* q, const void* kc,

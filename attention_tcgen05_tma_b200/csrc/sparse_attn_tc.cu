@@ -1,0 +1,558 @@
+// Sparse layer on the 5th-generation tensor cores: gathered block-sparse branch + SWA
+// branch + sigmoid gate (HySparse 3.4.3).
+//
+//   o~_t = softmax attention of q'_t over {i <= t : floor(i/64) in Sel_I} of the shared K, V
+//   o'_t = softmax attention of q'_t over [max(0, t-w+1), t] of the layer's own K', V'
+//   o_t  = sigmoid(g0) o~_t + sigmoid(g1) o'_t
+//
+// Structure follows the full-layer kernel: persistent CTAs over units (b, g, I), two
+// heads x 64 positions per 128-row M-tile, two M-tiles in flight, S and O in TMEM, P
+// written back over S and fed to the P.V MMA from TMEM.  What differs:
+//   * Gather: a 128-key tile holds two 64-key blocks.  Each block is one TMA box per
+//     128-byte chunk at row 64*j of K (or V), so only the selected blocks are read; K~, V~
+//     are never materialised.  A missing half (odd count, -1 padding) is loaded from a
+//     row past the end of the tensor, which TMA fills with zeros.
+//   * The tile list of a unit is the selected blocks in index order, then the window
+//     blocks of K', V'.  At the switch the softmax warpgroup reads O (the sparse branch is
+//     complete: its last P.V finished before the first window S did), stores
+//     sigmoid(g0) * O / l to an fp32 row of L2-resident scratch and restarts its online
+//     softmax; the epilogue adds sigmoid(g1) * O / l of the window branch.
+//   * Masks: per 64-key half, the visible key range is [64j, min(t, 64j+63)] for a selected
+//     block and [max(64j, t-w+1), min(t, 64j+63)] for a window block.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace hys {
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kStages = 4;
+constexpr int kMaxGrid = 148;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = 128 * D * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kQBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
+  static constexpr int kNumBars = 2 * kStages + 2 * 6 + 2;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+};
+
+struct Params {
+  int B, N, Hq, Hkv, G, T, kb, window;
+  int num_units;
+  const int* idx;      // [B,Hkv,T,kb]
+  const float* gate;   // [B,Hq,N,2]
+  __nv_bfloat16* o;
+  float* partial;      // [grid][2][128][D] fp32 scratch
+  int* status;
+  float scale_log2;
+};
+
+struct Bars {
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t mma_drain, spare;
+};
+
+struct Unit {
+  int b, g, I;
+  int nsel;    // leading selected entries
+  int n_sp;    // sparse tiles
+  int jw0;     // first window block
+  int n_sw;    // window tiles
+};
+
+__device__ __forceinline__ Unit load_unit(const Params& p, int u) {
+  Unit x;
+  const int bgc = p.B * p.Hkv;
+  x.I = p.T - 1 - u / bgc;
+  const int bg = u % bgc;
+  x.b = bg / p.Hkv;
+  x.g = bg % p.Hkv;
+  const int* sel = p.idx + (((size_t)x.b * p.Hkv + x.g) * p.T + x.I) * p.kb;
+  int n = 0;
+  while (n < p.kb && sel[n] >= 0) ++n;
+  x.nsel = n;
+  x.n_sp = (n + 1) / 2;
+  const int w_lo = 64 * x.I - p.window + 1;
+  x.jw0 = w_lo > 0 ? w_lo / 64 : 0;
+  x.n_sw = (x.I - x.jw0 + 2) / 2;
+  return x;
+}
+
+// Block of half h of tile tau (-1: empty).  is_swa tells which tensors it comes from.
+__device__ __forceinline__ int tile_block(const Params& p, const Unit& x, int tau, int h, bool& is_swa) {
+  if (tau < x.n_sp) {
+    is_swa = false;
+    const int e = 2 * tau + h;
+    if (e >= x.nsel) return -1;
+    const int j = p.idx[(((size_t)x.b * p.Hkv + x.g) * p.T + x.I) * p.kb + e];
+    return (j >= 0 && j <= x.I) ? j : -1;
+  }
+  is_swa = true;
+  const int j = x.jw0 + 2 * (tau - x.n_sp) + h;
+  return j <= x.I ? j : -1;
+}
+
+__device__ __forceinline__ void fail(volatile int* abort, int* status) {
+  *abort = 1;
+  report_status(status, HYS_ERR_TIMEOUT);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKs,
+                          const __grid_constant__ CUtensorMap tmVs, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int MT = p.G / 2;
+  const int rounds = (MT + 1) / 2;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&bars->kv_full[i], 1);
+      tc::mbar_init(&bars->kv_empty[i], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->q_full[s], 1);
+      tc::mbar_init(&bars->q_empty[s], 1);
+      tc::mbar_init(&bars->s_full[s], 1);
+      tc::mbar_init(&bars->p_full[s], 128);
+      tc::mbar_init(&bars->o_full[s], 1);
+      tc::mbar_init(&bars->o_empty[s], 128);
+    }
+    tc::mbar_init(&bars->mma_drain, 1);
+    *abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tensormap(&tmQ);
+    tc::prefetch_tensormap(&tmK);
+    tc::prefetch_tensormap(&tmV);
+    tc::prefetch_tensormap(&tmKs);
+    tc::prefetch_tensormap(&tmVs);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ============================================================== TMA producer (gather)
+    if (lane == 0) {
+      uint32_t kv_it = 0, q_cnt[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        const Unit x = load_unit(p, u);
+        const int ntiles = x.n_sp + x.n_sw;
+        for (int r = 0; r < rounds && ok; ++r) {
+          for (int s = 0; s < 2 && ok; ++s) {
+            const int mt = 2 * r + s;
+            if (mt >= MT) continue;
+            if (!(ok = tc::mbar_wait(&bars->q_empty[s], (q_cnt[s] & 1u) ^ 1u, abort))) break;
+            ++q_cnt[s];
+            tc::mbar_arrive_expect_tx(&bars->q_full[s], C::kQBytes);
+            const int h0 = x.g * p.G + 2 * mt;
+            uint8_t* qdst = smem + C::kOffQ + s * C::kQBytes;
+            for (int hh = 0; hh < 2; ++hh)
+              for (int c = 0; c < C::kChunks; ++c)
+                tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + c * 16384 + hh * 8192, c * 64, 64 * x.I,
+                                x.b * p.Hq + h0 + hh);
+          }
+          for (int tau = 0; tau < ntiles && ok; ++tau) {
+            bool swa0, swa1;
+            const int j0 = tile_block(p, x, tau, 0, swa0);
+            const int j1 = tile_block(p, x, tau, 1, swa1);
+            for (int kv = 0; kv < 2; ++kv) {
+              const uint32_t st = kv_it % kStages;
+              if (!(ok = tc::mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1u) ^ 1u, abort))) break;
+              tc::mbar_arrive_expect_tx(&bars->kv_full[st], C::kKVBytes);
+              uint8_t* dst = smem + C::kOffKV + st * C::kKVBytes;
+              const CUtensorMap* map = swa0 ? (kv ? &tmVs : &tmKs) : (kv ? &tmV : &tmK);
+              for (int hh = 0; hh < 2; ++hh) {
+                const int j = hh ? j1 : j0;
+                const int row = j >= 0 ? 64 * j : p.N;  // empty half: rows past the end read as zeros
+                for (int c = 0; c < C::kChunks; ++c)
+                  tc::tma_load_3d(map, &bars->kv_full[st], dst + c * 16384 + hh * 8192, c * 64, row,
+                                  x.b * p.Hkv + x.g);
+              }
+              ++kv_it;
+            }
+          }
+        }
+      }
+      if (!ok) fail(abort, p.status);
+      for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i)
+        tc::mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u, abort, 100000000ull);
+      for (int s = 0; s < 2; ++s)
+        if (q_cnt[s] > 0) tc::mbar_wait(&bars->q_full[s], (q_cnt[s] - 1) & 1u, abort, 100000000ull);
+    }
+  } else if (warp == 1) {
+    // ============================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
+      const uint32_t idO = tc::idesc_bf16_f32(128, D, true);
+      const uint32_t tS[2] = {tmem_base, tmem_base + 128};
+      const uint32_t tO[2] = {tmem_base + 256, tmem_base + 384};
+      const uint32_t qaddr = tc::smem_u32(smem + C::kOffQ);
+      const uint32_t kvaddr = tc::smem_u32(smem + C::kOffKV);
+      uint32_t kv_it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
+      bool ok = true;
+      auto issue_S = [&](int s, uint32_t st) {
+        const uint32_t qb = qaddr + s * C::kQBytes, kb = kvaddr + st * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc::mma_ss(tS[s], tc::sdesc_sw128(qb + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024), idS,
+                     kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_PV = [&](int s, uint32_t st, bool acc) {
+        const uint32_t vb = kvaddr + st * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_ts(tO[s], tS[s] + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16384, 1024), idO,
+                     (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        const Unit x = load_unit(p, u);
+        const int ntiles = x.n_sp + x.n_sw;
+        for (int r = 0; r < rounds && ok; ++r) {
+          bool act[2];
+          for (int s = 0; s < 2; ++s) {
+            act[s] = (2 * r + s) < MT;
+            if (act[s] && ok) {
+              ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort);
+              ++q_cnt[s];
+            }
+          }
+          if (!ok) break;
+          uint32_t kst = kv_it % kStages;
+          if (!(ok = tc::mbar_wait(&bars->kv_full[kst], (kv_it / kStages) & 1u, abort))) break;
+          ++kv_it;
+          tc::fence_after_sync();
+          for (int s = 0; s < 2; ++s)
+            if (act[s]) {
+              issue_S(s, kst);
+              tc::mma_commit(&bars->s_full[s]);
+            }
+          tc::mma_commit(&bars->kv_empty[kst]);
+          for (int tau = 1; tau <= ntiles && ok; ++tau) {
+            const uint32_t vst = kv_it % kStages;
+            if (!(ok = tc::mbar_wait(&bars->kv_full[vst], (kv_it / kStages) & 1u, abort))) break;
+            ++kv_it;
+            bool have_k = false;
+            // P.V of tile tau-1 starts a fresh accumulator at the first tile of each branch
+            const bool fresh = (tau - 1 == 0) || (tau - 1 == x.n_sp);
+            for (int s = 0; s < 2 && ok; ++s) {
+              if (!act[s]) continue;
+              if (!(ok = tc::mbar_wait(&bars->p_full[s], p_cnt[s] & 1u, abort))) break;
+              ++p_cnt[s];
+              if (tau == 1) {
+                if (!(ok = tc::mbar_wait(&bars->o_empty[s], (o_cnt[s] & 1u) ^ 1u, abort))) break;
+              }
+              tc::fence_after_sync();
+              issue_PV(s, vst, !fresh);
+              if (tau < ntiles) {
+                if (!have_k) {
+                  kst = kv_it % kStages;
+                  if (!(ok = tc::mbar_wait(&bars->kv_full[kst], (kv_it / kStages) & 1u, abort))) break;
+                  ++kv_it;
+                  have_k = true;
+                  tc::fence_after_sync();
+                }
+                issue_S(s, kst);
+                tc::mma_commit(&bars->s_full[s]);
+              } else {
+                tc::mma_commit(&bars->o_full[s]);
+                ++o_cnt[s];
+              }
+            }
+            tc::mma_commit(&bars->kv_empty[vst]);
+            if (have_k) tc::mma_commit(&bars->kv_empty[kst]);
+          }
+          for (int s = 0; s < 2; ++s)
+            if (act[s]) tc::mma_commit(&bars->q_empty[s]);
+        }
+      }
+      if (!ok) fail(abort, p.status);
+      tc::mma_commit(&bars->mma_drain);
+      tc::mbar_wait(&bars->mma_drain, 0, abort, 100000000ull);
+    }
+  } else if (warp >= 4) {
+    // ============================================================== softmax / gate epilogue
+    const int s = (warp - 4) >> 2;
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tSrow = tmem_base + 128 * s + lane_off;
+    const uint32_t tOrow = tmem_base + 256 + 128 * s + lane_off;
+    float* part = p.partial + (((size_t)blockIdx.x * 2 + s) * 128 + row) * D;
+    const float sc = p.scale_log2;
+    uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      const Unit x = load_unit(p, u);
+      const int ntiles = x.n_sp + x.n_sw;
+      for (int r = 0; r < rounds && ok; ++r) {
+        const int mt = 2 * r + s;
+        if (mt >= MT) continue;
+        const int h = x.g * p.G + 2 * mt + (row >> 6);
+        const int t = 64 * x.I + (row & 63);
+        const bool valid = t < p.N;
+        float g0 = 0.0f, g1 = 0.0f;
+        if (valid) {
+          const float2 gl = *reinterpret_cast<const float2*>(p.gate + (((size_t)x.b * p.Hq + h) * p.N + t) * 2);
+          g0 = sigmoidf_(gl.x);
+          g1 = sigmoidf_(gl.y);
+        }
+        float m_used = -INFINITY, l = 0.0f;
+        for (int tau = 0; tau < ntiles; ++tau) {
+          if (!(ok = tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort))) break;
+          ++s_cnt;
+          tc::fence_after_sync();
+          if (tau == x.n_sp && x.n_sp > 0) {
+            // branch switch: the sparse branch is complete in O; keep sigmoid(g0) * O / l
+            const float f = l > 0.0f ? g0 / l : 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              tc::tmem_ld32(tOrow + 32 * c, ov);
+              tc::tmem_wait_ld();
+              float4* dst = reinterpret_cast<float4*>(part + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(ov[4 * i]) * f, __uint_as_float(ov[4 * i + 1]) * f,
+                                     __uint_as_float(ov[4 * i + 2]) * f, __uint_as_float(ov[4 * i + 3]) * f);
+            }
+            m_used = -INFINITY;
+            l = 0.0f;
+          }
+          float sv[128];
+          {
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tc::tmem_ld32(tSrow + 0, r0);
+            tc::tmem_ld32(tSrow + 32, r1);
+            tc::tmem_ld32(tSrow + 64, r2);
+            tc::tmem_ld32(tSrow + 96, r3);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              sv[i] = __uint_as_float(r0[i]);
+              sv[32 + i] = __uint_as_float(r1[i]);
+              sv[64 + i] = __uint_as_float(r2[i]);
+              sv[96 + i] = __uint_as_float(r3[i]);
+            }
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            bool swa;
+            const int j = tile_block(p, x, tau, hh, swa);
+            int clo = 64, chi = -1;  // visible columns of this half (empty by default)
+            if (j >= 0) {
+              const int lo = swa ? max(64 * j, t - p.window + 1) : 64 * j;
+              const int hi = min(t, 64 * j + 63);
+              clo = lo - 64 * j;
+              chi = hi - 64 * j;
+            }
+            if (clo > 0 || chi < 63) {
+#pragma unroll
+              for (int i = 0; i < 64; ++i)
+                if (i < clo || i > chi) sv[64 * hh + i] = -INFINITY;
+            }
+          }
+          float mx = sv[0];
+#pragma unroll
+          for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+          float alpha = 1.0f;
+          bool rescale = false;
+          if (mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2) {
+            rescale = true;
+            alpha = exp2f((m_used - mx) * sc);
+            l *= alpha;
+            m_used = mx;
+          }
+          const float ms = m_used == -INFINITY ? 0.0f : m_used * sc;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
+              const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
+              l += p0 + p1;
+              pk[i] = tc::pack_bf16x2(p0, p1);
+            }
+            tc::tmem_st16(tSrow + 16 * c, pk);
+          }
+          const bool branch_start = (tau == 0) || (tau == x.n_sp);
+          if (rescale && !branch_start) {
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              tc::tmem_ld32(tOrow + 32 * c, ov);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tc::tmem_st32(tOrow + 32 * c, ov);
+            }
+          }
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bars->p_full[s]);
+        }
+        if (!ok) break;
+        if (!(ok = tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort))) break;
+        ++o_cnt;
+        tc::fence_after_sync();
+        const float f1 = l > 0.0f ? g1 / l : 0.0f;
+        const bool have_sp = x.n_sp > 0;
+        __nv_bfloat16* orow = p.o + (((size_t)x.b * p.Hq + h) * p.N + t) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tc::tmem_ld32(tOrow + 32 * c, ov);
+          tc::tmem_wait_ld();
+          if (valid) {
+            float add[32];
+            if (have_sp) {
+              const float4* src = reinterpret_cast<const float4*>(part + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 a = src[i];
+                add[4 * i] = a.x;
+                add[4 * i + 1] = a.y;
+                add[4 * i + 2] = a.z;
+                add[4 * i + 3] = a.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) add[i] = 0.0f;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = tc::pack_bf16x2(fmaf(__uint_as_float(ov[2 * i]), f1, add[2 * i]),
+                                      fmaf(__uint_as_float(ov[2 * i + 1]), f1, add[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&bars->o_empty[s]);
+      }
+    }
+    if (!ok) fail(abort, p.status);
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int D, int rows, int heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_units(const PrefillDims& d) { return d.B * d.Hkv * d.T; }
+int grid_size(const PrefillDims& d) { return num_units(d) < kMaxGrid ? num_units(d) : kMaxGrid; }
+
+template <int D>
+cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx, int kb,
+                         const void* ks, const void* vs, int window, const float* gate, void* o, void* ws,
+                         cudaStream_t s) {
+  CUtensorMap mq, mk, mv, mks, mvs;
+  if (!make_map(&mq, q, D, d.N, d.B * d.Hq) || !make_map(&mk, k, D, d.N, d.B * d.Hkv) ||
+      !make_map(&mv, v, D, d.N, d.B * d.Hkv) || !make_map(&mks, ks, D, d.N, d.B * d.Hkv) ||
+      !make_map(&mvs, vs, D, d.N, d.B * d.Hkv))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.B = d.B;
+  p.N = d.N;
+  p.Hq = d.Hq;
+  p.Hkv = d.Hkv;
+  p.G = d.G();
+  p.T = d.T;
+  p.kb = kb;
+  p.window = window;
+  p.num_units = num_units(d);
+  p.idx = idx;
+  p.gate = gate;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.partial = reinterpret_cast<float*>(ws);
+  p.status = device_status_ptr();
+  p.scale_log2 = kLog2e / sqrtf((float)D);
+  const int smem = Cfg<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  sparse_attn_tc_kernel<D><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, mks, mvs, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt) {
+  return dt == HYS_BF16 && (d.D == 64 || d.D == 128) && d.G() % 2 == 0;
+}
+
+size_t sparse_attn_tc_workspace(const PrefillDims& d) {
+  return sizeof(float) * (size_t)grid_size(d) * 2 * 128 * d.D;
+}
+
+cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
+                                  int kb, const void* ks, const void* vs, int window, const float* gate, void* o,
+                                  void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (ws_bytes < sparse_attn_tc_workspace(d)) return cudaErrorInvalidValue;
+  return d.D == 64 ? launch_typed<64>(d, q, k, v, idx, kb, ks, vs, window, gate, o, ws, s)
+                   : launch_typed<128>(d, q, k, v, idx, kb, ks, vs, window, gate, o, ws, s);
+}
+
+}  // namespace hys

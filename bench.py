@@ -178,6 +178,7 @@ class PrefillStep:
         sh = H.prefill_shape(x["q"], x["k"])
         nws = H.hysparse_full_attn_select_workspace_size(sh, H.HYS_BF16, H.HYS_GRAN_BLOCK)
         self.ws = H.workspace_for(nws, dev)
+        self.ws_sp = H.workspace_for(H.hysparse_sparse_attn_workspace_size(sh, H.HYS_BF16), dev)
         self.events = None
 
     def run(self, timing=None):
@@ -193,7 +194,7 @@ class PrefillStep:
             ev["topk"][1].record()
         for l in range(w.layers):
             H.sparse_attn(x["q_sparse"][l], x["k"], x["v"], self.idx, x["k_swa"][l], x["v_swa"][l], w.window,
-                          x["gate"][l], o=self.o_sp)
+                          x["gate"][l], o=self.o_sp, workspace=self.ws_sp)
         if ev is not None:
             ev["sparse"][1].record()
 

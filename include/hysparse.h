@@ -153,12 +153,16 @@ HYS_API hys_status hysparse_topk_tokens(const hys_shape* shape, const float* tok
  *   k_swa/v_swa may alias k_shared/v_shared (the "share both" ablation).
  *   idx entries are ascending block ids <= I or -1 (ignored); 1 <= k <= 1024.
  *   sinks must be NULL (per-head sink biases are not implemented: HYS_ERR_UNSUPPORTED).
+ *   workspace: at least hysparse_sparse_attn_workspace_size() bytes (fp32 scratch that
+ *   holds the gated sparse-branch rows while the window branch runs).
  * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_sparse_attn_workspace_size(const hys_shape* shape, hys_dtype dtype,
+                                                     size_t* bytes);
 HYS_API hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
                                 const void* k_shared, const void* v_shared, const int* idx,
                                 int k, const void* k_swa, const void* v_swa, int window,
                                 const float* gate_logits, const float* sinks, void* o,
-                                hys_stream_t stream);
+                                void* workspace, size_t workspace_bytes, hys_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Token-sparse layer ([HS2]): row t of tile I attends idx[b,g,I,:] (token positions,
