@@ -250,7 +250,7 @@ hys_status hysparse_full_attn_select_decode_workspace_size(const hys_decode_shap
   hys_status st = check_decode(shape, &d);
   if (st != HYS_OK) return st;
   if (!bytes || !dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
-  *bytes = align256(decode_full_workspace(d));
+  *bytes = align256(decode_mma_supported(d, dtype) ? decode_mma_full_workspace(d) : decode_full_workspace(d));
   return HYS_OK;
 }
 
@@ -266,10 +266,12 @@ hys_status hysparse_full_attn_select_decode(const hys_decode_shape* shape, hys_d
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(scores) ||
       !aligned16(seqlens) || !aligned16(workspace))
     return HYS_ERR_INVALID_ARG;
-  const size_t need = align256(decode_full_workspace(d));
+  const bool mma = decode_mma_supported(d, dtype);
+  const size_t need = align256(mma ? decode_mma_full_workspace(d) : decode_full_workspace(d));
   if (workspace == nullptr || workspace_bytes < need) return HYS_ERR_WORKSPACE;
-  return from_cuda(launch_decode_full(d, dtype, q, k_cache, v_cache, seqlens, o, scores, red, workspace,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (mma) return from_cuda(launch_decode_full_mma(d, q, k_cache, v_cache, seqlens, o, scores, red, workspace, s));
+  return from_cuda(launch_decode_full(d, dtype, q, k_cache, v_cache, seqlens, o, scores, red, workspace, s));
 }
 
 hys_status hysparse_topk_decode(const hys_decode_shape* shape, const float* scores, int k, const int* seqlens,
@@ -284,11 +286,21 @@ hys_status hysparse_topk_decode(const hys_decode_shape* shape, const float* scor
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+hys_status hysparse_sparse_attn_decode_workspace_size(const hys_decode_shape* shape, hys_dtype dtype, int k,
+                                                      size_t* bytes) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || !dtype_ok(dtype) || k < 1 || k > 1024) return HYS_ERR_INVALID_ARG;
+  *bytes = decode_mma_supported(d, dtype) ? align256(decode_mma_sparse_workspace(d, k)) : 0;
+  return HYS_OK;
+}
+
 hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype dtype, const void* q,
                                        const void* k_cache, const void* v_cache, const int* seqlens, const int* idx,
                                        int k, const void* k_swa_ring, const void* v_swa_ring, int window,
                                        const int* swa_len, const float* gate_logits, const float* sinks, void* o,
-                                       hys_stream_t stream) {
+                                       void* workspace, size_t workspace_bytes, hys_stream_t stream) {
   DecodeDims d;
   hys_status st = check_decode(shape, &d);
   if (st != HYS_OK) return st;
@@ -298,10 +310,16 @@ hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype 
   if (k < 1 || k > 1024 || window < 1 || window > 1024) return HYS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seqlens) || !aligned16(idx) ||
       !aligned16(k_swa_ring) || !aligned16(v_swa_ring) || !aligned16(swa_len) || !aligned16(gate_logits) ||
-      !aligned16(o))
+      !aligned16(o) || !aligned16(workspace))
     return HYS_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (decode_mma_supported(d, dtype)) {
+    if (workspace == nullptr || workspace_bytes < align256(decode_mma_sparse_workspace(d, k))) return HYS_ERR_WORKSPACE;
+    return from_cuda(launch_decode_sparse_mma(d, q, k_cache, v_cache, seqlens, idx, k, k_swa_ring, v_swa_ring, window,
+                                              swa_len, gate_logits, o, workspace, s));
+  }
   return from_cuda(launch_decode_sparse(d, dtype, q, k_cache, v_cache, seqlens, idx, k, k_swa_ring, v_swa_ring,
-                                        window, swa_len, gate_logits, o, reinterpret_cast<cudaStream_t>(stream)));
+                                        window, swa_len, gate_logits, o, s));
 }
 
 }  // extern "C"

@@ -1,0 +1,506 @@
+// Single-token decode, bf16: split-KV kernels that stream the cache at HBM speed.
+// (HySparse2 explainer, "Twenty lines of algorithmic intuition": scores of the new query
+// against the cache, top-k of the old blocks, then the sparse followers; HySparse 3.4.1
+// block scores and 3.4.3 sparse/SWA/gate for one query row.)
+//
+// One CTA = (split, KV group g, sequence b): 4 consumer warps + 1 TMA producer warp.  The
+// producer streams 64-key blocks of K and V (two 128-byte-swizzled TMA boxes each per
+// tensor, 32 KB per block) through a 5-stage ring; consumer warp w takes blocks w, w+4, ...
+// of the split, so the max logit of a block (HySparse's m~) is a warp-local reduction.
+// The G <= 16 query heads of the group form the 16 rows of mma.sync.m16n8k16 tiles
+// (zero-padded): S = Q K^T (64 mma per block), online softmax in registers, O += P V (64
+// mma per block).  The four warps' partial (m, l, O) are merged in shared memory and the
+// split's partial goes to the workspace; a combine kernel merges the splits, writes o and
+// (full layer) the block scores exp(m~ - m)/l aggregated over the group's heads, or
+// (sparse layer) the gated sum of the sparse-branch and SWA-ring branches.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace hys {
+
+namespace {
+
+constexpr int kConsumers = 4;
+constexpr int kThreads = 32 * (kConsumers + 1);
+constexpr int kStages = 5;
+constexpr int kStageBytes = 2 * 64 * 128 * 2;   // K + V of one 64-key block, D = 128
+constexpr int kMaxList = 72;                     // blocks per split (incl. padding)
+constexpr int kPartBytes = kConsumers * 16 * (128 + 2) * 4;
+constexpr int kSmemBytes = kStages * kStageBytes + kPartBytes + kMaxList * 16 + 256 + 1024;
+constexpr int kTargetCtas = 4 * 148;
+
+struct Params {
+  int B, L, Hq, Hkv, G, NB;
+  const int* seqlens;
+  int mode;         // 0: full layer (contiguous blocks), 1: sparse layer (selected blocks + ring)
+  int bps;          // blocks per split
+  int nsplit;       // splits per (b, g)
+  int nsp;          // sparse-mode splits over the selected list (the ring is split nsp)
+  const int* idx;   // [B,Hkv,kb] (mode 1)
+  int kb;
+  int W;            // ring capacity (mode 1)
+  const int* swa_len;
+  const __nv_bfloat16* q;  // [B,Hq,D]
+  float* pm;        // [B,Hq,nsplit]
+  float* pl;
+  float* po;        // [B,Hq,nsplit,D]
+  float* bmax;      // [B,Hq,NB] raw max logit of each block (mode 0)
+  int* status;
+  float scale_log2;
+};
+
+struct Entry {  // 16 bytes
+  int row;    // first key row in its tensor
+  int valid;  // valid keys (1..64)
+  int src;    // 0: shared cache, 1: SWA ring
+  int blk;    // block id (for the block max)
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// byte offset of (row, 16-byte unit) inside a [64 rows][128 B] 128-byte-swizzled box
+__device__ __forceinline__ uint32_t sw128(int row, int unit) { return row * 128 + ((unit ^ (row & 7)) << 4); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
+                        const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* part = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  Entry* list = reinterpret_cast<Entry*>(smem + kStages * kStageBytes + kPartBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kPartBytes + kMaxList * 16);
+  uint64_t* empty = full + kStages;
+  int* s_nlist = reinterpret_cast<int*>(empty + kStages);
+  volatile int* abort = s_nlist + 1;
+
+  const int sp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Lb = p.seqlens ? max(1, min(p.seqlens[b], p.L)) : p.L;
+
+  if (threadIdx.x == 0) {
+    // this split's block list
+    int n = 0;
+    if (p.mode == 0) {
+      const int nb = (Lb + 63) / 64;
+      for (int j = sp * p.bps; j < min(nb, (sp + 1) * p.bps); ++j) list[n++] = Entry{64 * j, min(64, Lb - 64 * j), 0, j};
+    } else if (sp < p.nsp) {
+      const int nb = (Lb + 63) / 64;
+      const int* sel = p.idx + ((size_t)b * p.Hkv + g) * p.kb;
+      for (int e = sp * p.bps; e < min(p.kb, (sp + 1) * p.bps); ++e) {
+        const int j = sel[e];
+        if (j >= 0 && j < nb) list[n++] = Entry{64 * j, min(64, Lb - 64 * j), 0, j};
+      }
+    } else {
+      const int nring = p.swa_len ? max(0, min(p.swa_len[b], p.W)) : p.W;
+      for (int j = 0; 64 * j < nring; ++j) list[n++] = Entry{64 * j, min(64, nring - 64 * j), 1, j};
+    }
+    *s_nlist = n;
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&full[i], 1);
+      tc::mbar_init(&empty[i], 1);
+    }
+    *abort = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  const int nlist = *s_nlist;
+  const float sc = p.scale_log2;
+
+  if (warp == kConsumers) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nlist; ++i) {
+        const int st = i % kStages;
+        if (!(ok = tc::mbar_wait(&empty[st], ((i / kStages) & 1) ^ 1, abort))) break;
+        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
+        uint8_t* dst = smem + st * kStageBytes;
+        const Entry e = list[i];
+        const CUtensorMap* mk = e.src ? &tmKr : &tmK;
+        const CUtensorMap* mv = e.src ? &tmVr : &tmV;
+        const int head = b * p.Hkv + g;
+        tc::tma_load_3d(mk, &full[st], dst, 0, e.row, head);
+        tc::tma_load_3d(mk, &full[st], dst + 8192, 64, e.row, head);
+        tc::tma_load_3d(mv, &full[st], dst + 16384, 0, e.row, head);
+        tc::tma_load_3d(mv, &full[st], dst + 24576, 64, e.row, head);
+      }
+      if (!ok) {
+        *abort = 1;
+        report_status(p.status, HYS_ERR_TIMEOUT);
+      }
+      for (int i = max(0, nlist - kStages); i < nlist; ++i)
+        tc::mbar_wait(&full[i % kStages], (i / kStages) & 1, abort, 100000000ull);
+    }
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int r = lane >> 2, cq = lane & 3;
+    const int h_lo = r, h_hi = r + 8;
+    // Q as A fragments (rows = heads, zero past G)
+    uint32_t qa[8][4];
+    const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + g * p.G) * 128;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int c0 = 16 * ks + 2 * cq;
+      qa[ks][0] = h_lo < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_lo * 128 + c0) : 0u;
+      qa[ks][1] = h_hi < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_hi * 128 + c0) : 0u;
+      qa[ks][2] = h_lo < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_lo * 128 + c0 + 8) : 0u;
+      qa[ks][3] = h_hi < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_hi * 128 + c0 + 8) : 0u;
+    }
+    float o[16][4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.0f, l_hi = 0.0f;
+    bool ok = true;
+    const uint32_t sbase = tc::smem_u32(smem);
+    for (int i = warp; i < nlist; i += kConsumers) {
+      const int st = i % kStages;
+      if (!(ok = tc::mbar_wait(&full[st], (i / kStages) & 1, abort))) break;
+      const Entry e = list[i];
+      const uint32_t kb = sbase + st * kStageBytes, vb = kb + 16384;
+      // ---- S = Q K^T : 8 key tiles x 8 dim steps
+      float s[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+        const int key = 8 * nt + (lane & 7);
+        const int mtx = lane >> 3;
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {  // pairs of 16-dim steps
+          const int ks = 2 * kp;
+          const int chunk = ks >> 2;
+          const int unit = 2 * (ks & 3) + mtx;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kb + chunk * 8192 + sw128(key, unit), b0, b1, b2, b3);
+          mma16816(s[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+          mma16816(s[nt], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], b2, b3);
+        }
+      }
+      // ---- mask keys past the valid count, block max, online softmax
+      float bm_lo = -INFINITY, bm_hi = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int key = 8 * nt + 2 * cq + c;
+          if (key >= e.valid) {
+            s[nt][c] = -INFINITY;
+            s[nt][2 + c] = -INFINITY;
+          }
+          bm_lo = fmaxf(bm_lo, s[nt][c]);
+          bm_hi = fmaxf(bm_hi, s[nt][2 + c]);
+        }
+      }
+      bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 1));
+      bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 2));
+      bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 1));
+      bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 2));
+      if (p.mode == 0 && cq == 0) {
+        if (h_lo < p.G) p.bmax[((size_t)b * p.Hq + g * p.G + h_lo) * p.NB + e.blk] = bm_lo;
+        if (h_hi < p.G) p.bmax[((size_t)b * p.Hq + g * p.G + h_hi) * p.NB + e.blk] = bm_hi;
+      }
+      const float mn_lo = fmaxf(m_lo, bm_lo), mn_hi = fmaxf(m_hi, bm_hi);
+      const float a_lo = exp2f((m_lo - mn_lo) * sc), a_hi = exp2f((m_hi - mn_hi) * sc);
+      m_lo = mn_lo;
+      m_hi = mn_hi;
+      l_lo *= a_lo;
+      l_hi *= a_hi;
+#pragma unroll
+      for (int dt = 0; dt < 16; ++dt) {
+        o[dt][0] *= a_lo;
+        o[dt][1] *= a_lo;
+        o[dt][2] *= a_hi;
+        o[dt][3] *= a_hi;
+      }
+      const float ms_lo = m_lo * sc, ms_hi = m_hi * sc;
+      uint32_t pa[8][2];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const float p0 = exp2f(fmaf(s[nt][0], sc, -ms_lo));
+        const float p1 = exp2f(fmaf(s[nt][1], sc, -ms_lo));
+        const float p2 = h_hi < p.G ? exp2f(fmaf(s[nt][2], sc, -ms_hi)) : 0.0f;
+        const float p3 = h_hi < p.G ? exp2f(fmaf(s[nt][3], sc, -ms_hi)) : 0.0f;
+        l_lo += p0 + p1;
+        l_hi += p2 + p3;
+        pa[nt][0] = tc::pack_bf16x2(p0, p1);
+        pa[nt][1] = tc::pack_bf16x2(p2, p3);
+      }
+      // ---- O += P V : 4 key steps x 16 dim tiles
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int mtx = lane >> 3;
+        const int key = 16 * kk + 8 * (mtx & 1) + (lane & 7);
+#pragma unroll
+        for (int dp = 0; dp < 8; ++dp) {  // pairs of 8-dim tiles
+          const int dt = 2 * dp + (mtx >> 1);
+          const int chunk = dt >> 3;
+          const int unit = dt & 7;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vb + chunk * 8192 + sw128(key, unit), b0, b1, b2, b3);
+          mma16816(o[2 * dp], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
+          mma16816(o[2 * dp + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[st]);
+    }
+    if (!ok) {
+      *abort = 1;
+      report_status(p.status, HYS_ERR_TIMEOUT);
+    }
+    // ---- this warp's partial (m, l, O) -> shared memory
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+    float* wp = part + warp * 16 * 130;  // [16 heads][m, l, O[128]]
+    if (cq == 0) {
+      wp[h_lo * 130 + 0] = m_lo;
+      wp[h_lo * 130 + 1] = l_lo;
+      wp[h_hi * 130 + 0] = m_hi;
+      wp[h_hi * 130 + 1] = l_hi;
+    }
+#pragma unroll
+    for (int dt = 0; dt < 16; ++dt) {
+      const int d0 = 8 * dt + 2 * cq;
+      wp[h_lo * 130 + 2 + d0] = o[dt][0];
+      wp[h_lo * 130 + 2 + d0 + 1] = o[dt][1];
+      wp[h_hi * 130 + 2 + d0] = o[dt][2];
+      wp[h_hi * 130 + 2 + d0 + 1] = o[dt][3];
+    }
+  }
+  __syncthreads();
+  // ---- merge the warps' partials into the split's partial
+  for (int e = threadIdx.x; e < p.G * 128; e += kThreads) {
+    const int hh = e >> 7, d = e & 127;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, part[(w * 16 + hh) * 130]);
+    float lsum = 0.0f, acc = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kConsumers; ++w) {
+      const float mw = part[(w * 16 + hh) * 130];
+      const float f = mw == -INFINITY ? 0.0f : exp2f((mw - M) * sc);
+      lsum += part[(w * 16 + hh) * 130 + 1] * f;
+      acc += part[(w * 16 + hh) * 130 + 2 + d] * f;
+    }
+    const size_t ph = ((size_t)b * p.Hq + g * p.G + hh) * p.nsplit + sp;
+    p.po[ph * 128 + d] = acc;
+    if (d == 0) {
+      p.pm[ph] = M;
+      p.pl[ph] = lsum;
+    }
+  }
+}
+
+// Merge the splits of one (b, g).  mode 0: o and block scores; mode 1: gated two-branch output.
+__global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const float* __restrict__ gate,
+                                                           __nv_bfloat16* __restrict__ o, float* __restrict__ scores,
+                                                           int red_max) {
+  __shared__ float sM[2][16], sInv[2][16];
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int Lb = p.seqlens ? max(1, min(p.seqlens[b], p.L)) : p.L;
+  const float sc = p.scale_log2;
+  const int nbr = p.mode == 0 ? 1 : 2;
+  if (threadIdx.x < p.G * nbr) {
+    const int hh = threadIdx.x % p.G, br = threadIdx.x / p.G;
+    const int s0 = p.mode == 0 ? 0 : (br == 0 ? 0 : p.nsp);
+    const int s1 = p.mode == 0 ? p.nsplit : (br == 0 ? p.nsp : p.nsplit);
+    const size_t ph = ((size_t)b * p.Hq + g * p.G + hh) * p.nsplit;
+    float M = -INFINITY;
+    for (int s = s0; s < s1; ++s) M = fmaxf(M, p.pm[ph + s]);
+    float L = 0.0f;
+    for (int s = s0; s < s1; ++s)
+      if (p.pm[ph + s] != -INFINITY) L += p.pl[ph + s] * exp2f((p.pm[ph + s] - M) * sc);
+    sM[br][hh] = M;
+    sInv[br][hh] = L > 0.0f ? 1.0f / L : 0.0f;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < p.G * 128; e += blockDim.x) {
+    const int hh = e >> 7, d = e & 127;
+    const size_t ph = ((size_t)b * p.Hq + g * p.G + hh) * p.nsplit;
+    float out = 0.0f;
+    for (int br = 0; br < nbr; ++br) {
+      const int s0 = p.mode == 0 ? 0 : (br == 0 ? 0 : p.nsp);
+      const int s1 = p.mode == 0 ? p.nsplit : (br == 0 ? p.nsp : p.nsplit);
+      float acc = 0.0f;
+      for (int s = s0; s < s1; ++s) {
+        const float m = p.pm[ph + s];
+        if (m != -INFINITY) acc = fmaf(p.po[(ph + s) * 128 + d], exp2f((m - sM[br][hh]) * sc), acc);
+      }
+      float w = sInv[br][hh];
+      if (p.mode == 1) w *= sigmoidf_(gate[((size_t)b * p.Hq + g * p.G + hh) * 2 + br]);
+      out = fmaf(acc, w, out);
+    }
+    o[((size_t)b * p.Hq + g * p.G + hh) * 128 + d] = __float2bfloat16_rn(out);
+  }
+  if (p.mode == 0) {
+    const int nb = (Lb + 63) / 64;
+    for (int j = threadIdx.x; j < p.NB; j += blockDim.x) {
+      float a = 0.0f;
+      if (j < nb) {
+        for (int hh = 0; hh < p.G; ++hh) {
+          const float x = exp2f((p.bmax[((size_t)b * p.Hq + g * p.G + hh) * p.NB + j] - sM[0][hh]) * sc) * sInv[0][hh];
+          a = hh == 0 ? x : (red_max ? fmaxf(a, x) : a + x);
+        }
+      }
+      scores[((size_t)b * p.Hkv + g) * p.NB + j] = a;
+    }
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int rows, int heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {256, (cuuint64_t)rows * 256};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int full_bps(const DecodeDims& d) {
+  const long long work = (long long)d.NB * d.B * d.Hkv;
+  long long bps = (work + kTargetCtas - 1) / kTargetCtas;
+  if (bps < 4) bps = 4;
+  if (bps > 64) bps = 64;
+  return (int)bps;
+}
+
+void fill_common(Params& p, const DecodeDims& d, const void* q, const int* seqlens, void* ws, int nsplit) {
+  p.B = d.B;
+  p.L = d.L;
+  p.Hq = d.Hq;
+  p.Hkv = d.Hkv;
+  p.G = d.G();
+  p.NB = d.NB;
+  p.seqlens = seqlens;
+  p.nsplit = nsplit;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  float* w = reinterpret_cast<float*>(ws);
+  const size_t np = (size_t)d.B * d.Hq * nsplit;
+  p.pm = w;
+  p.pl = w + np;
+  p.po = w + 2 * np;
+  p.bmax = w + 2 * np + np * 128;
+  p.status = device_status_ptr();
+  p.scale_log2 = kLog2e / sqrtf(128.0f);
+  p.idx = nullptr;
+  p.kb = 0;
+  p.W = 0;
+  p.swa_len = nullptr;
+  p.nsp = 0;
+}
+
+cudaError_t set_smem() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
+}  // namespace
+
+bool decode_mma_supported(const DecodeDims& d, hys_dtype dt) { return dt == HYS_BF16 && d.D == 128 && d.G() <= 16; }
+
+size_t decode_mma_full_workspace(const DecodeDims& d) {
+  const size_t nsplit = (d.NB + full_bps(d) - 1) / full_bps(d);
+  const size_t np = (size_t)d.B * d.Hq * nsplit;
+  return sizeof(float) * (np * (2 + 128) + (size_t)d.B * d.Hq * d.NB);
+}
+
+int decode_sparse_splits(int kb) { return (kb + 7) / 8; }
+
+size_t decode_mma_sparse_workspace(const DecodeDims& d, int kb) {
+  const size_t nsplit = decode_sparse_splits(kb) + 1;
+  return sizeof(float) * ((size_t)d.B * d.Hq * nsplit * (2 + 128));
+}
+
+cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                   const int* seqlens, void* o, float* scores, hys_reduce red, void* ws,
+                                   cudaStream_t s) {
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv)) return cudaErrorInvalidValue;
+  cudaError_t e = set_smem();
+  if (e != cudaSuccess) return e;
+  Params p;
+  const int bps = full_bps(d);
+  const int nsplit = (d.NB + bps - 1) / bps;
+  fill_common(p, d, q, seqlens, ws, nsplit);
+  p.mode = 0;
+  p.bps = bps;
+  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), scores,
+                                                      red == HYS_REDUCE_MAX);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                     const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
+                                     const int* swa_len, const float* gate, void* o, void* ws, cudaStream_t s) {
+  CUtensorMap mk, mv, mkr, mvr;
+  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv) ||
+      !make_map(&mkr, kr, W, d.B * d.Hkv) || !make_map(&mvr, vr, W, d.B * d.Hkv))
+    return cudaErrorInvalidValue;
+  cudaError_t e = set_smem();
+  if (e != cudaSuccess) return e;
+  Params p;
+  const int nsp = decode_sparse_splits(kb);
+  fill_common(p, d, q, seqlens, ws, nsp + 1);
+  p.mode = 1;
+  p.bps = 8;
+  p.nsp = nsp;
+  p.idx = idx;
+  p.kb = kb;
+  p.W = W;
+  p.swa_len = swa_len;
+  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, gate, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
+  return cudaGetLastError();
+}
+
+}  // namespace hys

@@ -76,4 +76,15 @@ cudaError_t launch_decode_sparse(const DecodeDims& d, hys_dtype dt, const void* 
                                  const void* kr, const void* vr, int W, const int* swa_len,
                                  const float* gate, void* o, cudaStream_t s);
 
+// bf16, D = 128, G <= 16: tensor-core split-KV kernels
+bool decode_mma_supported(const DecodeDims& d, hys_dtype dt);
+size_t decode_mma_full_workspace(const DecodeDims& d);
+size_t decode_mma_sparse_workspace(const DecodeDims& d, int kb);
+cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                   const int* seqlens, void* o, float* scores, hys_reduce red, void* ws,
+                                   cudaStream_t s);
+cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                     const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
+                                     const int* swa_len, const float* gate, void* o, void* ws, cudaStream_t s);
+
 }  // namespace hys

@@ -27,7 +27,7 @@ EXPORTED = (
     "hysparse_topk", "hysparse_topk_tokens_workspace_size", "hysparse_topk_tokens",
     "hysparse_sparse_attn_workspace_size", "hysparse_sparse_attn", "hysparse_sparse_attn_tokens",
     "hysparse_full_attn_select_decode_workspace_size", "hysparse_full_attn_select_decode",
-    "hysparse_topk_decode", "hysparse_sparse_attn_decode", "hysparse_full_attn_select_decode_noalloc",
+    "hysparse_topk_decode", "hysparse_sparse_attn_decode_workspace_size", "hysparse_sparse_attn_decode", "hysparse_full_attn_select_decode_noalloc",
 )
 
 
@@ -69,7 +69,9 @@ _SIGS = {
     "hysparse_full_attn_select_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P], _I),
     "hysparse_topk_decode": ([_DSH, _P, _I, _P, _P, _P], _I),
     "hysparse_full_attn_select_decode_noalloc": ([_DSH, _I, _P, _P, _P, _P, _P, _P, _I, _P], _I),
-    "hysparse_sparse_attn_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P], _I),
+    "hysparse_sparse_attn_decode_workspace_size": ([_DSH, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_sparse_attn_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
+                                    _I),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -179,10 +181,17 @@ def hysparse_topk_decode(shape, scores, k, seqlens, idx, stream) -> int:
     return load().hysparse_topk_decode(ctypes.byref(shape), scores, k, seqlens, idx, stream)
 
 
+def hysparse_sparse_attn_decode_workspace_size(shape: hys_decode_shape, dtype: int, k: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_sparse_attn_decode_workspace_size(ctypes.byref(shape), dtype, k, ctypes.byref(n)),
+           "hysparse_sparse_attn_decode_workspace_size")
+    return n.value
+
+
 def hysparse_sparse_attn_decode(shape, dtype, q, kc, vc, seqlens, idx, kb, kr, vr, window, swa_len, gate, sinks, o,
-                                stream) -> int:
+                                ws, ws_bytes, stream) -> int:
     return load().hysparse_sparse_attn_decode(ctypes.byref(shape), dtype, q, kc, vc, seqlens, idx, kb, kr, vr, window,
-                                              swa_len, gate, sinks, o, stream)
+                                              swa_len, gate, sinks, o, ws, ws_bytes, stream)
 
 
 # ----------------------------------------------------------------------------- torch helpers
@@ -331,13 +340,16 @@ def topk_decode(scores, k: int, L: int, *, seqlens=None, idx=None, stream=None):
 
 
 def sparse_attn_decode(q, k_cache, v_cache, idx, k_ring, v_ring, gate_logits, *, seqlens=None, swa_len=None,
-                       o=None, stream=None):
+                       o=None, workspace=None, stream=None):
     torch = _torch()
     sh = decode_shape(q, k_cache)
     if o is None:
         o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(hysparse_sparse_attn_decode_workspace_size(sh, _dt(q), idx.shape[-1]), q.device)
     _check(hysparse_sparse_attn_decode(sh, _dt(q), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(idx),
                                        idx.shape[-1], _ptr(k_ring), _ptr(v_ring), k_ring.shape[2], _ptr(swa_len),
-                                       _ptr(gate_logits), None, _ptr(o), _stream(stream)),
+                                       _ptr(gate_logits), None, _ptr(o), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)),
            "hysparse_sparse_attn_decode")
     return o

@@ -326,6 +326,7 @@ def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
     osp = torch.empty_like(x["q"])
     sh = H.decode_shape(x["q"], x["k"])
     ws = H.workspace_for(H.hysparse_full_attn_select_decode_workspace_size(sh, H.HYS_BF16), dev)
+    ws_sp = H.workspace_for(H.hysparse_sparse_attn_decode_workspace_size(sh, H.HYS_BF16, w.topk), dev)
 
     def step(ev=None):
         if ev:
@@ -338,7 +339,7 @@ def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
             ev[2].record()
         for l in range(w.layers):
             H.sparse_attn_decode(x["q_sparse"][l], x["k"], x["v"], idx, x["k_swa"][l], x["v_swa"][l], x["gate"][l],
-                                 o=osp)
+                                 o=osp, workspace=ws_sp)
         if ev:
             ev[3].record()
 

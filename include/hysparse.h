@@ -224,15 +224,18 @@ HYS_API hys_status hysparse_topk_decode(const hys_decode_shape* shape, const flo
  * cached token (< L_b) of the selected blocks of the shared cache; the SWA branch attends
  * the layer's own ring k_swa_ring/v_swa_ring [B,Hkv,W,D] (swa_len[b] valid entries, or W
  * when swa_len is NULL; order is irrelevant); gate_logits [B,Hq,2]; o [B,Hq,D].
- * W = window, 1 <= window <= 1024.  sinks must be NULL.
+ * W = window, 1 <= window <= 1024.  sinks must be NULL.  workspace: at least
+ * hysparse_sparse_attn_decode_workspace_size() bytes (per-split partial softmax states).
  * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_sparse_attn_decode_workspace_size(const hys_decode_shape* shape,
+                                                            hys_dtype dtype, int k, size_t* bytes);
 HYS_API hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype dtype,
                                        const void* q, const void* k_cache,
                                        const void* v_cache, const int* seqlens,
                                        const int* idx, int k, const void* k_swa_ring,
                                        const void* v_swa_ring, int window, const int* swa_len,
                                        const float* gate_logits, const float* sinks, void* o,
-                                       hys_stream_t stream);
+                                       void* workspace, size_t workspace_bytes, hys_stream_t stream);
 
 #ifdef __cplusplus
 }

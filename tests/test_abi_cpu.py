@@ -76,6 +76,10 @@ def test_entry_points_reject_bad_arguments_without_launching(lib):
         == H.HYS_ERR_WORKSPACE
     dsh = H.hys_decode_shape(2, 100, 4, 1, 64, 64)
     assert H.hysparse_sparse_attn_decode(dsh, H.HYS_F32, 16, 16, 16, None, 16, 4, 16, 16, 2000, None, 16, None,
-                                         16, None) == H.HYS_ERR_INVALID_ARG
+                                         16, None, 0, None) == H.HYS_ERR_INVALID_ARG
+    bdsh = H.hys_decode_shape(2, 1000, 16, 2, 128, 64)
+    assert H.hysparse_sparse_attn_decode_workspace_size(bdsh, H.HYS_BF16, 32) > 0
+    assert H.hysparse_sparse_attn_decode(bdsh, H.HYS_BF16, 16, 16, 16, None, 16, 32, 16, 16, 128, None, 16, None,
+                                         16, None, 0, None) == H.HYS_ERR_WORKSPACE
     assert H.hysparse_full_attn_select_decode(dsh, H.HYS_F32, 16, 16, 16, None, 16, 16, 0, None, 0, None) \
         == H.HYS_ERR_WORKSPACE

@@ -141,6 +141,8 @@ DECODE_CASES = [
     ("bf16_d128_g8", "bf16", 3, 1500, 16, 2, 128, 4, 128, True),
     ("bf16_d64_g4", "bf16", 2, 700, 4, 1, 64, 8, 32, False),
     ("f32_d64_g4", "f32", 2, 300, 8, 2, 64, 2, 16, True),
+    ("bf16_d128_g16_long", "bf16", 2, 9000, 16, 1, 128, 8, 128, True),
+    ("bf16_d128_g4_ring100", "bf16", 2, 3000, 8, 2, 128, 4, 100, False),
 ]
 
 
