@@ -3,13 +3,15 @@
 // against the cache, top-k of the old blocks, then the sparse followers; HySparse 3.4.1
 // block scores and 3.4.3 sparse/SWA/gate for one query row.)
 //
-// One CTA = (split, KV group g, sequence b): 4 consumer warps + 1 TMA producer warp.  The
+// One CTA = (split, KV group g, sequence b): 6 consumer warps + 1 TMA producer warp.  The
 // producer streams 64-key blocks of K and V (two 128-byte-swizzled TMA boxes each per
-// tensor, 32 KB per block) through a 5-stage ring; consumer warp w takes blocks w, w+4, ...
-// of the split, so the max logit of a block (HySparse's m~) is a warp-local reduction.
+// tensor, 32 KB per block) into 6 stages; consumer warp w owns stage w and takes blocks
+// w, w+6, ... of the split, so every stage's barrier phases are consumed by one warp in
+// order (a parity wait cannot be fooled by a phase two ahead) and the max logit of a
+// block (HySparse's m~) is a warp-local reduction.
 // The G <= 16 query heads of the group form the 16 rows of mma.sync.m16n8k16 tiles
 // (zero-padded): S = Q K^T (64 mma per block), online softmax in registers, O += P V (64
-// mma per block).  The four warps' partial (m, l, O) are merged in shared memory and the
+// mma per block).  The warps' partial (m, l, O) are merged in shared memory (reusing the stages) and the
 // split's partial goes to the workspace; a combine kernel merges the splits, writes o and
 // (full layer) the block scores exp(m~ - m)/l aggregated over the group's heads, or
 // (sparse layer) the gated sum of the sparse-branch and SWA-ring branches.
@@ -24,13 +26,14 @@ namespace hys {
 
 namespace {
 
-constexpr int kConsumers = 4;
+constexpr int kConsumers = 6;
 constexpr int kThreads = 32 * (kConsumers + 1);
-constexpr int kStages = 5;
+constexpr int kStages = kConsumers;              // stage w belongs to consumer warp w
 constexpr int kStageBytes = 2 * 64 * 128 * 2;   // K + V of one 64-key block, D = 128
 constexpr int kMaxList = 72;                     // blocks per split (incl. padding)
 constexpr int kPartBytes = kConsumers * 16 * (128 + 2) * 4;
-constexpr int kSmemBytes = kStages * kStageBytes + kPartBytes + kMaxList * 16 + 256 + 1024;
+static_assert(kPartBytes <= kStages * kStageBytes, "partials reuse the stage buffers");
+constexpr int kSmemBytes = kStages * kStageBytes + kMaxList * 16 + 256 + 1024;
 constexpr int kTargetCtas = 4 * 148;
 
 struct Params {
@@ -88,9 +91,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* part = reinterpret_cast<float*>(smem + kStages * kStageBytes);
-  Entry* list = reinterpret_cast<Entry*>(smem + kStages * kStageBytes + kPartBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kPartBytes + kMaxList * 16);
+  float* part = reinterpret_cast<float*>(smem);  // after the pipeline has drained
+  Entry* list = reinterpret_cast<Entry*>(smem + kStages * kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kMaxList * 16);
   uint64_t* empty = full + kStages;
   int* s_nlist = reinterpret_cast<int*>(empty + kStages);
   volatile int* abort = s_nlist + 1;
@@ -153,6 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = max(0, nlist - kStages); i < nlist; ++i)
         tc::mbar_wait(&full[i % kStages], (i / kStages) & 1, abort, 100000000ull);
     }
+    __syncwarp();
+    tc::named_bar_sync(1, kThreads);
   } else {
     // ---------------------------------------------------------------- consumers
     const int r = lane >> 2, cq = lane & 3;
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     const uint32_t sbase = tc::smem_u32(smem);
     for (int i = warp; i < nlist; i += kConsumers) {
-      const int st = i % kStages;
+      const int st = warp;  // == i % kStages
       if (!(ok = tc::mbar_wait(&full[st], (i / kStages) & 1, abort))) break;
       const Entry e = list[i];
       const uint32_t kb = sbase + st * kStageBytes, vb = kb + 16384;
@@ -269,7 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       *abort = 1;
       report_status(p.status, HYS_ERR_TIMEOUT);
     }
-    // ---- this warp's partial (m, l, O) -> shared memory
+    // ---- this warp's partial (m, l, O) -> shared memory, once no warp reads a stage
+    //      any more and the producer has drained its loads (all consumer + producer warps)
+    tc::named_bar_sync(1, kThreads);
     l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
     l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
     l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);

@@ -143,6 +143,7 @@ DECODE_CASES = [
     ("f32_d64_g4", "f32", 2, 300, 8, 2, 64, 2, 16, True),
     ("bf16_d128_g16_long", "bf16", 2, 9000, 16, 1, 128, 8, 128, True),
     ("bf16_d128_g4_ring100", "bf16", 2, 3000, 8, 2, 128, 4, 100, False),
+    ("bf16_d128_g8_stage_reuse", "bf16", 64, 40000, 8, 1, 128, 32, 128, True),
 ]
 
 
