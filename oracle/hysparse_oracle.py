@@ -324,7 +324,8 @@ def decode_sparse(q: np.ndarray, k_cache, v_cache, idx, k_ring, v_ring, gate, se
     """One sparse layer for the new token: selected blocks of the shared cache (all keys
     of a selected block that hold cached tokens) plus the layer's own SWA ring of
     swa_len[b] tokens (ring order does not matter: softmax is permutation invariant),
-    merged by the sigmoid gate [B,Hq,2]."""
+    merged by the sigmoid gate [B,Hq,2].  A branch with no keys (an empty ring, or no
+    selected block holding cached tokens) contributes zero."""
     B, Hq, D = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
     G = Hq // Hkv
@@ -341,8 +342,8 @@ def decode_sparse(q: np.ndarray, k_cache, v_cache, idx, k_ring, v_ring, gate, se
             vr = np.asarray(v_ring[b, g, :nring], np.float64)
             for h in range(g * G, (g + 1) * G):
                 qq = np.asarray(q[b, h], np.float64)[None, :]
-                o_sp, _ = attention_rows(qq, np.array([len(keys)]), ks, vs)
-                o_sw, _ = attention_rows(qq, np.array([nring]), kr, vr)
+                o_sp = attention_rows(qq, np.array([len(keys)]), ks, vs)[0] if len(keys) else np.zeros((1, D))
+                o_sw = attention_rows(qq, np.array([nring]), kr, vr)[0] if nring else np.zeros((1, D))
                 gg = sigmoid(gate[b, h])
                 o[b, h] = gg[0] * o_sp[0] + gg[1] * o_sw[0]
     return o

@@ -154,7 +154,8 @@ def test_decode(case):
                  scale_std=1.0 / np.sqrt(D))
     a = I.decode_arrays(w, layers=1)
     seqlens = np.array([L - 37 * b for b in range(B)], dtype=np.int32) if ragged else None
-    swa_len = np.array([W - 3 * b for b in range(B)], dtype=np.int32) if ragged else None
+    # ragged rings, including an empty one (a sequence with no window tokens yet)
+    swa_len = np.array([(W - 3 * b) % (W + 1) for b in range(B)], dtype=np.int32) if ragged else None
     q, kc, vc = (to_dev(a[x], dt) for x in ("q", "k", "v"))
     sl = torch.from_numpy(seqlens).cuda() if ragged else None
     o, sc = H.full_attn_select_decode(q, kc, vc, seqlens=sl)

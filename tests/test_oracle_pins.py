@@ -289,6 +289,21 @@ def test_decode_is_last_row_of_dense():
     assert np.sum(idx[1] >= 0) == 2 * 3
 
 
+def test_decode_empty_branch_contributes_zero():
+    """An empty SWA ring (swa_len 0) leaves only the gated sparse branch."""
+    rng = np.random.default_rng(10)
+    L, D, G = 200, 8, 2
+    q, k, v = _rand(rng, 1, G, D), _rand(rng, 1, 1, L, D), _rand(rng, 1, 1, L, D)
+    kr, vr, gate = _rand(rng, 1, 1, 4, D), _rand(rng, 1, 1, 4, D), _rand(rng, 1, G, 2)
+    idx = np.array([[[0, 2]]])
+    o = O.decode_sparse(q, k, v, idx, kr, vr, gate, swa_len=np.array([0]))
+    keys = list(range(0, 64)) + list(range(128, 192))
+    for h in range(G):
+        want = BF.attend(q[0, h].tolist(), keys, k[0, 0].tolist(), v[0, 0].tolist())
+        g0 = 1 / (1 + math.exp(-gate[0, h, 0]))
+        np.testing.assert_allclose(o[0, h], [g0 * x for x in want], atol=1e-12)
+
+
 # ----------------------------------------------------------------------------- brute force
 @pytest.mark.parametrize("seed,N,D,G", [(0, 64, 16, 1), (1, 65, 16, 2), (2, 130, 8, 2), (3, 200, 8, 1)])
 def test_brute_force(seed, N, D, G):
