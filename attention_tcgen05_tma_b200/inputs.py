@@ -85,6 +85,9 @@ WORKLOADS: Dict[str, Workload] = {
                        seed=3, scale_std=1.0 / math.sqrt(128)),
     "token": Workload("token", "prefill_token", "bf16", 1, 131072, 32, 4, 128, 3, 2048, 128,
                       seed=4, scale_std=1.0 / math.sqrt(128), plant="blocks", n_plants=64),
+    # smaller decode batch with the same per-sequence shape (profiling captures: 2 GiB of cache)
+    "decode_small": Workload("decode_small", "decode", "bf16", 8, 131072, 32, 4, 128, 11, 32, 128,
+                             seed=5, scale_std=1.0 / math.sqrt(128)),
 }
 
 

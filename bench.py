@@ -318,7 +318,7 @@ def _uses_tc(H, w):
 def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
     from attention_tcgen05_tma_b200 import hysparse as H
     from attention_tcgen05_tma_b200 import inputs as I
-    w = I.WORKLOADS["decode"]
+    w = I.WORKLOADS[args.decode_workload]
     x = make_decode_inputs(w, torch, dev, w.layers, seed_offset=1000 * rank)
     o = torch.empty_like(x["q"])
     sc = torch.empty((w.B, w.Hkv, w.NB), dtype=torch.float32, device=dev)
@@ -532,7 +532,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="moe80b")
+    ap.add_argument("--workload", default="moe80b", help="prefill workload (moe80b, dense7b, ...)")
+    ap.add_argument("--decode-workload", default="decode", help="decode workload (decode, decode_small)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
