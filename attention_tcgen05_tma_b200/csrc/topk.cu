@@ -5,6 +5,11 @@
 // runs on an order-preserving uint32 image of the fp32 score, so the selection is a
 // deterministic function of the emitted scores.  Output indices are ascending and padded
 // with -1.
+//
+// One CTA per candidate row.  Radix select finds the k-th largest key in four 8-bit passes
+// (per-warp histograms in shared memory, then a suffix scan over the 256 bins); one
+// index-ordered sweep then takes every key above it plus the lowest-index ties, and a
+// block-wide scan places them in ascending order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -12,9 +17,7 @@ namespace hys {
 
 namespace {
 
-constexpr int kTopkThreads = 256;
-
-// Block-wide exclusive scan of one int per thread (blockDim.x == 256 or 1024).
+// Block-wide exclusive scan of one int per thread (NT threads, NT % 32 == 0, NT <= 1024).
 template <int NT>
 __device__ __forceinline__ int block_exclusive_scan(int x, int* total, int* sbuf /* >= NT/32 + 1 */) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -44,14 +47,74 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* total, int* sbuf
   return res;
 }
 
-// One CTA per (b, g, I) row of candidates.  Candidates live in shared memory as keys;
-// the rank of candidate c is the number of candidates that beat it.
-__global__ void __launch_bounds__(kTopkThreads) topk_blocks_kernel(const float* __restrict__ scores,
-                                                                   int* __restrict__ idx, int Hkv, int T, int NB,
-                                                                   int k, const int* __restrict__ seqlens, int L,
-                                                                   int decode) {
+template <int NW>
+struct RadixSmem {
+  int hist[NW][256];  // per-warp histograms
+  int sbuf[33];
+  uint32_t prefix;
+  int need;
+};
+
+// Select the k largest of n keys (key(c) for c in [0, n)), ties to the lower index, and write
+// their indices ascending to out[0..k) (n > k is required).  NT threads, NT >= 256.
+template <int NT, typename KeyFn>
+__device__ void radix_topk(KeyFn key, int n, int k, int* out, RadixSmem<NT / 32>& sm) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t prefix = 0, pmask = 0;
+  int need = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < NW * 256; i += NT) (&sm.hist[0][0])[i] = 0;
+    __syncthreads();
+    for (int c = tid; c < n; c += NT) {
+      const uint32_t kc = key(c);
+      if ((kc & pmask) == prefix) atomicAdd(&sm.hist[warp][(kc >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    // bin counts in descending bin order: thread t < 256 owns bin 255 - t
+    int cnt = 0;
+    if (tid < 256) {
+      const int bin = 255 - tid;
+      for (int w = 0; w < NW; ++w) cnt += sm.hist[w][bin];
+    }
+    int total;
+    const int above = block_exclusive_scan<NT>(tid < 256 ? cnt : 0, &total, sm.sbuf);  // keys in higher bins
+    if (tid < 256 && above < need && above + cnt >= need) {
+      sm.prefix = prefix | ((uint32_t)(255 - tid) << shift);
+      sm.need = need - above;
+    }
+    __syncthreads();
+    prefix = sm.prefix;
+    need = sm.need;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  (void)lane;
+  // prefix is the k-th largest key: take the greater keys and the `need` lowest-index ties
+  const uint32_t kth = prefix;
+  int ties_before = 0, written = 0;
+  for (int base = 0; base < n; base += NT) {
+    const int c = base + tid;
+    const uint32_t kc = c < n ? key(c) : 0u;
+    const int is_tie = (c < n && kc == kth) ? 1 : 0;
+    int tie_total;
+    const int tie_rank = ties_before + block_exclusive_scan<NT>(is_tie, &tie_total, sm.sbuf);
+    ties_before += tie_total;
+    const int sel = (c < n) && (kc > kth || (is_tie && tie_rank < need));
+    int sel_total;
+    const int pos = written + block_exclusive_scan<NT>(sel, &sel_total, sm.sbuf);
+    if (sel) out[pos] = c;
+    written += sel_total;
+  }
+}
+
+constexpr int kBlkThreads = 256;
+
+__global__ void __launch_bounds__(kBlkThreads) topk_blocks_kernel(const float* __restrict__ scores,
+                                                                  int* __restrict__ idx, int Hkv, int T, int NB, int k,
+                                                                  const int* __restrict__ seqlens, int L, int decode) {
   extern __shared__ uint32_t skey[];  // NB keys
-  __shared__ int sbuf[kTopkThreads / 32 + 1];
+  __shared__ RadixSmem<kBlkThreads / 32> sm;
   const int row = blockIdx.x;
   int n;
   if (decode) {
@@ -61,101 +124,35 @@ __global__ void __launch_bounds__(kTopkThreads) topk_blocks_kernel(const float* 
   } else {
     n = min(NB, row % T + 1);
   }
-  const float* srow = scores + (size_t)row * NB;
-  for (int c = threadIdx.x; c < n; c += kTopkThreads) skey[c] = order_key(srow[c]);
-  __syncthreads();
-  // contiguous segment per thread so that a scan gives ascending output positions
-  const int seg = (n + kTopkThreads - 1) / kTopkThreads;
-  const int c0 = min(n, threadIdx.x * seg), c1 = min(n, c0 + seg);
-  uint32_t selmask = 0;  // seg <= 32 (n <= 8192)
-  int cnt = 0;
-  for (int c = c0; c < c1; ++c) {
-    const uint32_t kc = skey[c];
-    int rank = 0;
-    for (int j = 0; j < n && rank < k; ++j) {
-      const uint32_t kj = skey[j];
-      rank += (kj > kc) || (kj == kc && j < c);
-    }
-    if (rank < k) {
-      selmask |= 1u << (c - c0);
-      ++cnt;
-    }
-  }
-  int total;
-  int pos = block_exclusive_scan<kTopkThreads>(cnt, &total, sbuf);
   int* out = idx + (size_t)row * k;
-  for (int c = c0; c < c1; ++c)
-    if (selmask & (1u << (c - c0))) out[pos++] = c;
-  for (int p = total + threadIdx.x; p < k; p += kTopkThreads) out[p] = -1;
+  if (n <= k) {
+    for (int c = threadIdx.x; c < k; c += kBlkThreads) out[c] = c < n ? c : -1;
+    return;
+  }
+  const float* srow = scores + (size_t)row * NB;
+  for (int c = threadIdx.x; c < n; c += kBlkThreads) skey[c] = order_key(srow[c]);
+  __syncthreads();
+  radix_topk<kBlkThreads>([&](int c) { return skey[c]; }, n, k, out, sm);
 }
 
-// ------------------------------------------------------------------ token top-k
 constexpr int kTokThreads = 1024;
 
-// One CTA per (b, g, I).  Radix select (4 passes of 8 bits) finds the k-th largest key;
-// then one ordered sweep takes every key above it plus the lowest-index ties.
+// Token candidates of tile I are positions [0, e_I - forced], e_I = min(64I+63, N-1).
 __global__ void __launch_bounds__(kTokThreads) topk_tokens_kernel(const float* __restrict__ scores,
                                                                   int* __restrict__ idx, int T, int N, int k,
                                                                   int forced) {
-  __shared__ int hist[256];
-  __shared__ int sbuf[kTokThreads / 32 + 1];
-  __shared__ uint32_t s_prefix, s_need;
+  __shared__ RadixSmem<kTokThreads / 32> sm;
   const int row = blockIdx.x;
   const int I = row % T;
   const int e = min(N, (I + 1) * 64) - 1;
   const int n = max(0, e - forced + 1);
   const float* srow = scores + (size_t)row * N;
   int* out = idx + (size_t)row * k;
-  const int tid = threadIdx.x;
-
   if (n <= k) {
-    for (int c = tid; c < k; c += kTokThreads) out[c] = c < n ? c : -1;
+    for (int c = threadIdx.x; c < k; c += kTokThreads) out[c] = c < n ? c : -1;
     return;
   }
-  // radix select of the k-th largest key
-  uint32_t prefix = 0, pmask = 0;
-  int need = k;  // how many to take among keys matching the prefix
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int c = tid; c < 256; c += kTokThreads) hist[c] = 0;
-    __syncthreads();
-    for (int c = tid; c < n; c += kTokThreads) {
-      const uint32_t key = order_key(srow[c]);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      int acc = 0, bin = 255;
-      for (; bin > 0; --bin) {
-        if (acc + hist[bin] >= need) break;
-        acc += hist[bin];
-      }
-      s_prefix = prefix | ((uint32_t)bin << shift);
-      s_need = (uint32_t)(need - acc);
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    need = (int)s_need;
-    pmask |= 255u << shift;
-    __syncthreads();
-  }
-  // prefix is now the k-th largest key; take all greater keys and the `need` lowest-index ties
-  const uint32_t kth = prefix;
-  int ties_before = 0, written = 0;
-  for (int base = 0; base < n; base += kTokThreads) {
-    const int c = base + tid;
-    uint32_t key = 0;
-    if (c < n) key = order_key(srow[c]);
-    const int is_tie = (c < n && key == kth) ? 1 : 0;
-    int tie_total;
-    const int tie_rank = ties_before + block_exclusive_scan<kTokThreads>(is_tie, &tie_total, sbuf);
-    ties_before += tie_total;
-    const int sel = (c < n) && (key > kth || (is_tie && tie_rank < need));
-    int sel_total;
-    const int pos = written + block_exclusive_scan<kTokThreads>(sel, &sel_total, sbuf);
-    if (sel) out[pos] = c;
-    written += sel_total;
-  }
-  for (int p = written + tid; p < k; p += kTokThreads) out[p] = -1;
+  radix_topk<kTokThreads>([&](int c) { return order_key(srow[c]); }, n, k, out, sm);
 }
 
 }  // namespace
@@ -164,12 +161,13 @@ cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, in
                                const int* seqlens, int L, bool decode, cudaStream_t s) {
   const int rows = decode ? B * Hkv : B * Hkv * T;
   const size_t smem = (size_t)NB * sizeof(uint32_t);
-  if (smem > 48 * 1024) {
+  const size_t static_smem = sizeof(RadixSmem<kBlkThreads / 32>);
+  if (smem + static_smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(topk_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  topk_blocks_kernel<<<rows, kTopkThreads, smem, s>>>(scores, idx, Hkv, T, NB, k, seqlens, L, decode ? 1 : 0);
+  topk_blocks_kernel<<<rows, kBlkThreads, smem, s>>>(scores, idx, Hkv, T, NB, k, seqlens, L, decode ? 1 : 0);
   return cudaGetLastError();
 }
 

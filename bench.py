@@ -29,6 +29,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from attention_tcgen05_tma_b200.distributed import max_over_ranks  # noqa: E402
+
 METRIC = "hybrid-block prefill tokens/s @32K and decode µs/token; % of tensor/HBM roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -256,11 +258,7 @@ def run_ours(args, torch, dist, rank, world, dev):
     clk = clocks.stop()
     ms_total = t0.elapsed_time(t1)
     per = {k: sum(e[k][0].elapsed_time(e[k][1]) for e in evs) / args.steps for k in ("full", "topk", "sparse")}
-    ms_step = ms_total / args.steps
-    if dist is not None:
-        tt = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step = float(tt.item())
+    ms_step = max_over_ranks(ms_total / args.steps, dist, dev)
     tokens_job = w.B * w.N * world
     value = tokens_job / (ms_step / 1e3)
 
@@ -298,7 +296,7 @@ def run_ours(args, torch, dist, rank, world, dev):
                       "l2": "inputs larger than L2 (Q 512 MiB per layer)"},
            "kernels": kernels, "roofline": roof, "clocks": clk, "gpu_launches": launches}
     if not args.no_e2e:
-        res["e2e"] = run_e2e(args, torch, dist, world, w, x, step)
+        res["e2e"] = run_e2e(args, torch, dist, world, w, x, step, dev)
     del x, step
     torch.cuda.empty_cache()
 
@@ -356,11 +354,7 @@ def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
     full_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     topk_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     sp_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-    ms_step = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
-    if dist is not None:
-        tt = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step = float(tt.item())
+    ms_step = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps, dist, dev)
     full_bytes = 2.0 * w.B * w.Hkv * w.N * w.D * 2
     sp_bytes = 2.0 * w.B * w.Hkv * (w.topk * 64 + w.window) * w.D * 2
     hbm = peaks["hbm_gbs"]
@@ -381,7 +375,7 @@ def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
     return res
 
 
-def run_e2e(args, torch, dist, world, w, x, step):
+def run_e2e(args, torch, dist, world, w, x, step, dev=None):
     """Same step through the public API with the inputs in pinned HOST memory: every step
     copies its inputs host->device and reads the last layer's output back."""
     host = {k: (v.cpu().pin_memory() if not isinstance(v, list) else [t.cpu().pin_memory() for t in v])
@@ -412,11 +406,7 @@ def run_e2e(args, torch, dist, world, w, x, step):
         one()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    if dist is not None:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
     del host
     return {"value": round(w.B * w.N * world / (ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3), "steps": steps}
