@@ -71,9 +71,13 @@ hys_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HYS_OK : HYS_ERR
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace of hysparse_full_attn_select.  Block scores: the tensor-core kernel's counter and
+// m~ stash, or the SIMT path's per-head partial scores.  Token scores: the tensor-core
+// kernel's counter (256 B) followed by room for the LSE of every row (used when the caller
+// passes no lse buffer).
 size_t full_ws_bytes(const PrefillDims& d, hys_dtype dt, hys_gran gran) {
-  if (gran == HYS_GRAN_TOKEN) return align256(sizeof(float) * (size_t)d.B * d.Hq * d.N);
-  if (full_attn_tc_supported(d, dt, true)) return align256(full_attn_tc_workspace(d));
+  if (gran == HYS_GRAN_TOKEN) return 256 + align256(sizeof(float) * (size_t)d.B * d.Hq * d.N);
+  if (full_attn_tc_supported(d, dt, true)) return align256(full_attn_tc_workspace(d, true));
   return align256(sizeof(float) * (size_t)d.B * d.Hq * d.T * d.NB);
 }
 
@@ -148,10 +152,10 @@ hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype dtype, co
     if (e != cudaSuccess) return HYS_ERR_CUDA;
     return from_cuda(launch_head_reduce(d, part, scores, red, s));
   }
-  float* lse = lse_opt ? lse_opt : reinterpret_cast<float*>(workspace);
+  float* lse = lse_opt ? lse_opt : reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + 256);
   cudaError_t e;
   if (full_attn_tc_supported(d, dtype, false))
-    e = launch_full_attn_tc(d, q, k, v, o, lse, nullptr, HYS_REDUCE_SUM, false, nullptr, 0, s);
+    e = launch_full_attn_tc(d, q, k, v, o, lse, nullptr, HYS_REDUCE_SUM, false, workspace, 256, s);
   else
     e = launch_full_attn_simt(d, dtype, q, k, v, o, lse, nullptr, false, HYS_REDUCE_SUM, s);
   if (e != cudaSuccess) return HYS_ERR_CUDA;

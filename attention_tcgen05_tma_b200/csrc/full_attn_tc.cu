@@ -43,6 +43,27 @@ constexpr int kMaxNB = 2048;       // score accumulator capacity per slot (N <= 
 constexpr int kMaxGrid = 148;      // B200 SM count; the workspace is sized for this grid
 constexpr float kRescaleLog2 = 8.0f;
 
+
+struct Params {
+  int B, N, Hq, Hkv, G, T, NB, NBpad;
+  int num_units;
+  __nv_bfloat16* o;
+  float* lse;     // optional [B,Hq,N]
+  float* scores;  // optional [B,Hkv,T,NB] (block scores are emitted iff non-null)
+  float* stash;   // [grid][2][128][NBpad]
+  int* counter;   // work-unit counter (zeroed before the launch)
+  int red_max;
+  int* status;
+  float scale_log2;  // log2(e) / sqrt(D)
+};
+
+struct Bars {
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2], wg[2], all[2];
+  uint64_t mma_drain, spare;
+  tc::UnitQueue queue;
+};
+
 template <int D>
 struct Cfg {
   static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
@@ -53,33 +74,16 @@ struct Cfg {
   static constexpr int kOffAcc = kOffKV + kStages * kKVBytes;
   static constexpr int kOffRow = kOffAcc + 2 * kMaxNB * 4;
   static constexpr int kOffBar = kOffRow + 2 * 256 * 4;
-  static constexpr int kNumBars = 2 * kStages + 2 * 8 + 2;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
 };
 
-struct Params {
-  int B, N, Hq, Hkv, G, T, NB, NBpad;
-  int num_units;
-  __nv_bfloat16* o;
-  float* lse;     // optional [B,Hq,N]
-  float* scores;  // optional [B,Hkv,T,NB] (block scores are emitted iff non-null)
-  float* stash;   // [grid][2][128][NBpad]
-  int red_max;
-  int* status;
-  float scale_log2;  // log2(e) / sqrt(D)
-};
-
-struct Bars {
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2], wg[2], all[2];
-  uint64_t mma_drain, spare;
-};
-
+// Units are drawn from a counter in KV-group-major order, longest query tile first within a
+// group: co-running CTAs then stream the same group's K/V (L2-resident), and the dynamic draw
+// balances the causal lengths and leaves the shortest units for the tail.
 __device__ __forceinline__ void unit_coords(const Params& p, int u, int& b, int& g, int& I) {
-  const int bgc = p.B * p.Hkv;
-  I = p.T - 1 - u / bgc;
-  const int bg = u % bgc;
+  const int bg = u / p.T;
+  I = p.T - 1 - u % p.T;
   b = bg / p.Hkv;
   g = bg % p.Hkv;
 }
@@ -131,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->all[s], 256);
     }
     tc::mbar_init(&bars->mma_drain, 1);
+    tc::queue_init(&bars->queue, 1 + 256);  // MMA thread + both softmax warpgroups
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -155,7 +160,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kv_it = 0, q_cnt[2] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      for (uint32_t n = 0; ok; ++n) {
+        const int c = atomicAdd(p.counter, 1);
+        const int u = c < p.num_units ? c : -1;
+        if (!(ok = tc::queue_push(&bars->queue, n, u, abort))) break;
+        if (u < 0) break;
         int b, g, I;
         unit_coords(p, u, b, g, I);
         const int nkt = I / 2 + 1;
@@ -221,7 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mma_ts(tO[s], tS[s] + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16384, 1024), idO,
                      (acc || kk > 0) ? 1u : 0u);
       };
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      for (uint32_t n = 0; ok; ++n) {
+        const int u = tc::queue_pop(&bars->queue, n, abort, ok);
+        if (u < 0) break;
         int b, g, I;
         unit_coords(p, u, b, g, I);
         const int nkt = I / 2 + 1;
@@ -301,7 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sc = p.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0, wg_ph = 0, all_ph = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    for (uint32_t n = 0; ok; ++n) {
+      const int u = tc::queue_pop(&bars->queue, n, abort, ok);
+      if (u < 0) break;
       int b, g, I;
       unit_coords(p, u, b, g, I);
       const int nkt = I / 2 + 1;
@@ -338,11 +351,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 128; ++i)
               if (i > cmax) sv[i] = -INFINITY;
           }
-          float mlo = sv[0], mhi = sv[64];
+          float mlo, mhi;
+          {
+            float a[8], bb[8];
 #pragma unroll
-          for (int i = 1; i < 64; ++i) {
-            mlo = fmaxf(mlo, sv[i]);
-            mhi = fmaxf(mhi, sv[64 + i]);
+            for (int i = 0; i < 8; ++i) {
+              a[i] = sv[i];
+              bb[i] = sv[64 + i];
+            }
+#pragma unroll
+            for (int i = 8; i < 64; i += 8)
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                a[j] = fmaxf(a[j], sv[i + j]);
+                bb[j] = fmaxf(bb[j], sv[64 + i + j]);
+              }
+#pragma unroll
+            for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+              for (int j = 0; j < w; ++j) {
+                a[j] = fmaxf(a[j], a[j + w]);
+                bb[j] = fmaxf(bb[j], bb[j + w]);
+              }
+            mlo = a[0];
+            mhi = bb[0];
           }
           if (scores_on) *reinterpret_cast<float2*>(stash + (size_t)row * p.NBpad + 2 * tau) = make_float2(mlo, mhi);
           const float mt_ = fmaxf(mlo, mhi);
@@ -354,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_used = mt_;
           }
           const float ms = m_used * sc;
+          float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[16];
@@ -361,11 +394,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) {
               const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
               const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
-              l += p0 + p1;
+              ls[i & 3] += p0 + p1;
               pk[i] = tc::pack_bf16x2(p0, p1);
             }
             tc::tmem_st16(tSrow + 16 * c, pk);
           }
+          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
           if (rescale && tau > 0) {
             // O_s holds the sum over the earlier key tiles; its last PV is complete because
             // S_s(tau), committed after it, is.  PV_s(tau) waits for p_full below.
@@ -503,12 +537,15 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.scores = scores;
-  p.stash = reinterpret_cast<float*>(ws);
+  p.counter = reinterpret_cast<int*>(ws);
+  p.stash = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
   p.red_max = red == HYS_REDUCE_MAX;
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(full_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   full_attn_tc_kernel<D><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, p);
   return cudaGetLastError();
@@ -523,15 +560,15 @@ bool full_attn_tc_supported(const PrefillDims& d, hys_dtype dt, bool want_scores
   return true;
 }
 
-size_t full_attn_tc_workspace(const PrefillDims& d) {
-  return sizeof(float) * (size_t)grid_size(d) * 2 * 128 * (size_t)nb_pad(d.NB);
+size_t full_attn_tc_workspace(const PrefillDims& d, bool want_scores) {
+  return 256 + (want_scores ? sizeof(float) * (size_t)grid_size(d) * 2 * 128 * (size_t)nb_pad(d.NB) : 0);
 }
 
 cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, void* o,
                                 float* lse, float* scores, hys_reduce red, bool want_scores, void* ws, size_t ws_bytes,
                                 cudaStream_t s) {
   if (!want_scores) scores = nullptr;
-  if (want_scores && ws_bytes < full_attn_tc_workspace(d)) return cudaErrorInvalidValue;
+  if (ws == nullptr || ws_bytes < full_attn_tc_workspace(d, want_scores)) return cudaErrorInvalidValue;
   return d.D == 64 ? launch_typed<64>(d, q, k, v, o, lse, scores, red, ws, s)
                    : launch_typed<128>(d, q, k, v, o, lse, scores, red, ws, s);
 }

@@ -39,7 +39,7 @@ cudaError_t launch_token_scores_simt(const PrefillDims& d, hys_dtype dt, const v
 
 // ---- full layer, tcgen05 path (bf16, D=128, even G) ----------------------------------------
 bool full_attn_tc_supported(const PrefillDims& d, hys_dtype dt, bool want_scores);
-size_t full_attn_tc_workspace(const PrefillDims& d);
+size_t full_attn_tc_workspace(const PrefillDims& d, bool want_scores);
 cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v,
                                 void* o, float* lse, float* scores, hys_reduce red, bool want_scores,
                                 void* ws, size_t ws_bytes, cudaStream_t s);

@@ -34,18 +34,6 @@ constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;
 constexpr float kRescaleLog2 = 8.0f;
 
-template <int D>
-struct Cfg {
-  static constexpr int kChunks = D / 64;
-  static constexpr int kQBytes = 128 * D * 2;
-  static constexpr int kKVBytes = 128 * D * 2;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = 2 * kQBytes;
-  static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
-  static constexpr int kNumBars = 2 * kStages + 2 * 6 + 2;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
-};
 
 struct Params {
   int B, N, Hq, Hkv, G, T, kb, window;
@@ -54,6 +42,7 @@ struct Params {
   const float* gate;   // [B,Hq,N,2]
   __nv_bfloat16* o;
   float* partial;      // [grid][2][128][D] fp32 scratch
+  int* counter;        // work-unit counter (zeroed before the launch)
   int* status;
   float scale_log2;
 };
@@ -62,6 +51,19 @@ struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_drain, spare;
+  tc::UnitQueue queue;
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = 128 * D * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kQBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
+  static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 };
 
 struct Unit {
@@ -72,11 +74,12 @@ struct Unit {
   int n_sw;    // window tiles
 };
 
+// Units come from a counter in KV-group-major order, so co-running CTAs gather from the same
+// group's K/V (L2-resident); within a group the order is longest-first.
 __device__ __forceinline__ Unit load_unit(const Params& p, int u) {
   Unit x;
-  const int bgc = p.B * p.Hkv;
-  x.I = p.T - 1 - u / bgc;
-  const int bg = u % bgc;
+  const int bg = u / p.T;
+  x.I = p.T - 1 - u % p.T;
   x.b = bg / p.Hkv;
   x.g = bg % p.Hkv;
   const int* sel = p.idx + (((size_t)x.b * p.Hkv + x.g) * p.T + x.I) * p.kb;
@@ -139,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->o_empty[s], 128);
     }
     tc::mbar_init(&bars->mma_drain, 1);
+    tc::queue_init(&bars->queue, 1 + 256);
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -163,7 +167,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kv_it = 0, q_cnt[2] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      for (uint32_t n = 0; ok; ++n) {
+        const int c = atomicAdd(p.counter, 1);
+        const int u = c < p.num_units ? c : -1;
+        if (!(ok = tc::queue_push(&bars->queue, n, u, abort))) break;
+        if (u < 0) break;
         const Unit x = load_unit(p, u);
         const int ntiles = x.n_sp + x.n_sw;
         for (int r = 0; r < rounds && ok; ++r) {
@@ -235,7 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mma_ts(tO[s], tS[s] + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16384, 1024), idO,
                      (acc || kk > 0) ? 1u : 0u);
       };
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      for (uint32_t n = 0; ok; ++n) {
+        const int u = tc::queue_pop(&bars->queue, n, abort, ok);
+        if (u < 0) break;
         const Unit x = load_unit(p, u);
         const int ntiles = x.n_sp + x.n_sw;
         for (int r = 0; r < rounds && ok; ++r) {
@@ -311,7 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sc = p.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    for (uint32_t n = 0; ok; ++n) {
+      const int u = tc::queue_pop(&bars->queue, n, abort, ok);
+      if (u < 0) break;
       const Unit x = load_unit(p, u);
       const int ntiles = x.n_sp + x.n_sw;
       for (int r = 0; r < rounds && ok; ++r) {
@@ -381,9 +393,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (i < clo || i > chi) sv[64 * hh + i] = -INFINITY;
             }
           }
-          float mx = sv[0];
+          float mx;
+          {
+            float a[8];
 #pragma unroll
-          for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+            for (int j = 0; j < 8; ++j) a[j] = sv[j];
+#pragma unroll
+            for (int i = 8; i < 128; i += 8)
+#pragma unroll
+              for (int j = 0; j < 8; ++j) a[j] = fmaxf(a[j], sv[i + j]);
+#pragma unroll
+            for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+              for (int j = 0; j < w; ++j) a[j] = fmaxf(a[j], a[j + w]);
+            mx = a[0];
+          }
           float alpha = 1.0f;
           bool rescale = false;
           if (mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2) {
@@ -393,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_used = mx;
           }
           const float ms = m_used == -INFINITY ? 0.0f : m_used * sc;
+          float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[16];
@@ -400,11 +425,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) {
               const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
               const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
-              l += p0 + p1;
+              ls[i & 3] += p0 + p1;
               pk[i] = tc::pack_bf16x2(p0, p1);
             }
             tc::tmem_st16(tSrow + 16 * c, pk);
           }
+          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
           const bool branch_start = (tau == 0) || (tau == x.n_sp);
           if (rescale && !branch_start) {
 #pragma unroll 1
@@ -527,11 +553,14 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.idx = idx;
   p.gate = gate;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
-  p.partial = reinterpret_cast<float*>(ws);
+  p.counter = reinterpret_cast<int*>(ws);
+  p.partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   sparse_attn_tc_kernel<D><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, mks, mvs, p);
   return cudaGetLastError();
@@ -544,7 +573,7 @@ bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt) {
 }
 
 size_t sparse_attn_tc_workspace(const PrefillDims& d) {
-  return sizeof(float) * (size_t)grid_size(d) * 2 * 128 * d.D;
+  return 256 + sizeof(float) * (size_t)grid_size(d) * 2 * 128 * d.D;
 }
 
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,

@@ -197,3 +197,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 }  // namespace tc
 }  // namespace hys
+
+namespace hys {
+namespace tc {
+
+// ------------------------------------------------------------------ dynamic unit queue
+// The TMA-producer thread draws work-unit ids from a global counter (atomicAdd) and
+// publishes them through a small shared-memory ring; every other role pops them in the
+// same order.  A published id < 0 ends the sequence.  `consumers` = number of threads that
+// pop each id (they all arrive on the slot's empty barrier).
+constexpr int kQueueSlots = 4;
+
+struct UnitQueue {
+  uint64_t full[kQueueSlots], empty[kQueueSlots];
+  int unit[kQueueSlots];
+};
+
+__device__ __forceinline__ void queue_init(UnitQueue* q, uint32_t consumers) {
+  for (int i = 0; i < kQueueSlots; ++i) {
+    mbar_init(&q->full[i], 1);
+    mbar_init(&q->empty[i], consumers);
+  }
+}
+
+// producer side: publish the n-th id; returns false on timeout
+__device__ __forceinline__ bool queue_push(UnitQueue* q, uint32_t n, int unit, volatile int* abort) {
+  const uint32_t s = n % kQueueSlots;
+  if (!mbar_wait(&q->empty[s], ((n / kQueueSlots) & 1u) ^ 1u, abort)) return false;
+  q->unit[s] = unit;
+  mbar_arrive(&q->full[s]);  // release: the id is visible to threads that observe the phase
+  return true;
+}
+
+// consumer side: pop the n-th id (or -1 on timeout / abort)
+__device__ __forceinline__ int queue_pop(UnitQueue* q, uint32_t n, volatile int* abort, bool& ok) {
+  const uint32_t s = n % kQueueSlots;
+  if (!mbar_wait(&q->full[s], (n / kQueueSlots) & 1u, abort)) {
+    ok = false;
+    return -1;
+  }
+  const int u = *reinterpret_cast<volatile int*>(&q->unit[s]);
+  mbar_arrive(&q->empty[s]);
+  return u;
+}
+
+}  // namespace tc
+}  // namespace hys
