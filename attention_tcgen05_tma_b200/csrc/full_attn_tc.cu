@@ -42,6 +42,7 @@ constexpr int kStages = 4;         // K/V ring depth (one stage = one 128-key K 
 constexpr int kMaxNB = 2048;       // score accumulator capacity per slot (N <= 131072)
 constexpr int kMaxGrid = 148;      // B200 SM count; the workspace is sized for this grid
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kPolyCols = 32;      // softmax columns (of 128) whose exp2 runs on the FMA pipe
 
 
 struct Params {
@@ -392,8 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
-              const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
+              // the first kPolyCols columns of each row use the FMA-pipe exp2, the rest MUFU
+              const float x0 = fmaf(sv[32 * c + 2 * i], sc, -ms);
+              const float x1 = fmaf(sv[32 * c + 2 * i + 1], sc, -ms);
+              const bool poly = 32 * c + 2 * i < kPolyCols;
+              const float p0 = poly ? tc::exp2_poly3(x0) : exp2f(x0);
+              const float p1 = poly ? tc::exp2_poly3(x1) : exp2f(x1);
               ls[i & 3] += p0 + p1;
               pk[i] = tc::pack_bf16x2(p0, p1);
             }

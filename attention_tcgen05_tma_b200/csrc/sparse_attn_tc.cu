@@ -32,7 +32,9 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;
+constexpr int kMaxKb = 1024;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kPolyCols = 32;      // softmax columns (of 128) whose exp2 runs on the FMA pipe
 
 
 struct Params {
@@ -61,50 +63,37 @@ struct Cfg {
   static constexpr int kKVBytes = 128 * D * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kQBytes;
-  static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
+  static constexpr int kOffList = kOffKV + kStages * kKVBytes;   // producer's copy of a unit's indices
+  static constexpr int kOffBar = kOffList + kMaxKb * 4;
   static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 };
 
 struct Unit {
   int b, g, I;
-  int nsel;    // leading selected entries
+  int nsel;    // leading valid selected entries (0 <= j <= I); later entries are ignored
+  int diag;    // entry holding block I (causally masked per row), or -1
   int n_sp;    // sparse tiles
   int jw0;     // first window block
   int n_sw;    // window tiles
 };
 
 // Units come from a counter in KV-group-major order, so co-running CTAs gather from the same
-// group's K/V (L2-resident); within a group the order is longest-first.
-__device__ __forceinline__ Unit load_unit(const Params& p, int u) {
+// group's K/V (L2-resident); within a group the order is longest-first.  nsel and diag are
+// found once by the producer warp and published with the unit id.
+__device__ __forceinline__ Unit make_unit(const Params& p, int u, int nsel, int diag) {
   Unit x;
   const int bg = u / p.T;
   x.I = p.T - 1 - u % p.T;
   x.b = bg / p.Hkv;
   x.g = bg % p.Hkv;
-  const int* sel = p.idx + (((size_t)x.b * p.Hkv + x.g) * p.T + x.I) * p.kb;
-  int n = 0;
-  while (n < p.kb && sel[n] >= 0) ++n;
-  x.nsel = n;
-  x.n_sp = (n + 1) / 2;
+  x.nsel = nsel;
+  x.diag = diag;
+  x.n_sp = (nsel + 1) / 2;
   const int w_lo = 64 * x.I - p.window + 1;
   x.jw0 = w_lo > 0 ? w_lo / 64 : 0;
   x.n_sw = (x.I - x.jw0 + 2) / 2;
   return x;
-}
-
-// Block of half h of tile tau (-1: empty).  is_swa tells which tensors it comes from.
-__device__ __forceinline__ int tile_block(const Params& p, const Unit& x, int tau, int h, bool& is_swa) {
-  if (tau < x.n_sp) {
-    is_swa = false;
-    const int e = 2 * tau + h;
-    if (e >= x.nsel) return -1;
-    const int j = p.idx[(((size_t)x.b * p.Hkv + x.g) * p.T + x.I) * p.kb + e];
-    return (j >= 0 && j <= x.I) ? j : -1;
-  }
-  is_swa = true;
-  const int j = x.jw0 + 2 * (tau - x.n_sp) + h;
-  return j <= x.I ? j : -1;
 }
 
 __device__ __forceinline__ void fail(volatile int* abort, int* status) {
@@ -164,15 +153,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ============================================================== TMA producer (gather)
-    if (lane == 0) {
-      uint32_t kv_it = 0, q_cnt[2] = {0, 0};
-      bool ok = true;
-      for (uint32_t n = 0; ok; ++n) {
+    // The whole warp reads a unit's index row (32 entries per step) and finds the leading
+    // valid entries with a ballot; lane 0 then issues the Q and gathered K/V loads.
+    int* plist = reinterpret_cast<int*>(smem + C::kOffList);
+    uint32_t kv_it = 0, q_cnt[2] = {0, 0};
+    bool ok = true;
+    for (uint32_t n = 0; ok; ++n) {
+      int u = 0;
+      if (lane == 0) {
         const int c = atomicAdd(p.counter, 1);
-        const int u = c < p.num_units ? c : -1;
-        if (!(ok = tc::queue_push(&bars->queue, n, u, abort))) break;
-        if (u < 0) break;
-        const Unit x = load_unit(p, u);
+        u = c < p.num_units ? c : -1;
+      }
+      u = __shfl_sync(0xffffffffu, u, 0);
+      int nsel = 0, diag = -1;
+      if (u >= 0) {
+        const Unit x0 = make_unit(p, u, 0, -1);
+        const int* sel = p.idx + (((size_t)x0.b * p.Hkv + x0.g) * p.T + x0.I) * p.kb;
+        nsel = p.kb;
+        for (int e0 = 0; e0 < p.kb; e0 += 32) {
+          const int e = e0 + lane;
+          const int j = e < p.kb ? sel[e] : -1;
+          if (e < p.kb) plist[e] = j;
+          const unsigned bad = __ballot_sync(0xffffffffu, e < p.kb && (j < 0 || j > x0.I));
+          const unsigned dg = __ballot_sync(0xffffffffu, e < p.kb && j == x0.I);
+          const int first_bad = bad ? e0 + __ffs(bad) - 1 : p.kb;
+          if (diag < 0 && dg) {
+            const int first_dg = e0 + __ffs(dg) - 1;
+            if (first_dg < first_bad) diag = first_dg;
+          }
+          if (bad) {
+            nsel = first_bad;
+            break;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) ok = tc::queue_push(&bars->queue, n, u, abort, nsel, diag);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok || u < 0) break;
+      if (lane == 0) {
+        const Unit x = make_unit(p, u, nsel, diag);
         const int ntiles = x.n_sp + x.n_sw;
         for (int r = 0; r < rounds && ok; ++r) {
           for (int s = 0; s < 2 && ok; ++s) {
@@ -184,25 +204,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int h0 = x.g * p.G + 2 * mt;
             uint8_t* qdst = smem + C::kOffQ + s * C::kQBytes;
             for (int hh = 0; hh < 2; ++hh)
-              for (int c = 0; c < C::kChunks; ++c)
-                tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + c * 16384 + hh * 8192, c * 64, 64 * x.I,
+              for (int ch = 0; ch < C::kChunks; ++ch)
+                tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + ch * 16384 + hh * 8192, ch * 64, 64 * x.I,
                                 x.b * p.Hq + h0 + hh);
           }
           for (int tau = 0; tau < ntiles && ok; ++tau) {
-            bool swa0, swa1;
-            const int j0 = tile_block(p, x, tau, 0, swa0);
-            const int j1 = tile_block(p, x, tau, 1, swa1);
+            const bool swa = tau >= x.n_sp;
+            int jj[2];
+            for (int hh = 0; hh < 2; ++hh) {
+              if (!swa) {
+                const int e = 2 * tau + hh;
+                jj[hh] = e < x.nsel ? plist[e] : -1;
+              } else {
+                const int j = x.jw0 + 2 * (tau - x.n_sp) + hh;
+                jj[hh] = j <= x.I ? j : -1;
+              }
+            }
             for (int kv = 0; kv < 2; ++kv) {
               const uint32_t st = kv_it % kStages;
               if (!(ok = tc::mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1u) ^ 1u, abort))) break;
               tc::mbar_arrive_expect_tx(&bars->kv_full[st], C::kKVBytes);
               uint8_t* dst = smem + C::kOffKV + st * C::kKVBytes;
-              const CUtensorMap* map = swa0 ? (kv ? &tmVs : &tmKs) : (kv ? &tmV : &tmK);
+              const CUtensorMap* map = swa ? (kv ? &tmVs : &tmKs) : (kv ? &tmV : &tmK);
               for (int hh = 0; hh < 2; ++hh) {
-                const int j = hh ? j1 : j0;
-                const int row = j >= 0 ? 64 * j : p.N;  // empty half: rows past the end read as zeros
-                for (int c = 0; c < C::kChunks; ++c)
-                  tc::tma_load_3d(map, &bars->kv_full[st], dst + c * 16384 + hh * 8192, c * 64, row,
+                const int row = jj[hh] >= 0 ? 64 * jj[hh] : p.N;  // empty half: rows past the end read as zeros
+                for (int ch = 0; ch < C::kChunks; ++ch)
+                  tc::tma_load_3d(map, &bars->kv_full[st], dst + ch * 16384 + hh * 8192, ch * 64, row,
                                   x.b * p.Hkv + x.g);
               }
               ++kv_it;
@@ -210,6 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0) {
       if (!ok) fail(abort, p.status);
       for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i)
         tc::mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u, abort, 100000000ull);
@@ -244,9 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                      (acc || kk > 0) ? 1u : 0u);
       };
       for (uint32_t n = 0; ok; ++n) {
-        const int u = tc::queue_pop(&bars->queue, n, abort, ok);
+        int nsel = 0, diag = -1;
+        const int u = tc::queue_pop(&bars->queue, n, abort, ok, &nsel, &diag);
         if (u < 0) break;
-        const Unit x = load_unit(p, u);
+        const Unit x = make_unit(p, u, nsel, diag);
         const int ntiles = x.n_sp + x.n_sw;
         for (int r = 0; r < rounds && ok; ++r) {
           bool act[2];
@@ -322,9 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
     for (uint32_t n = 0; ok; ++n) {
-      const int u = tc::queue_pop(&bars->queue, n, abort, ok);
+      int nsel = 0, diag = -1;
+      const int u = tc::queue_pop(&bars->queue, n, abort, ok, &nsel, &diag);
       if (u < 0) break;
-      const Unit x = load_unit(p, u);
+      const Unit x = make_unit(p, u, nsel, diag);
       const int ntiles = x.n_sp + x.n_sw;
       for (int r = 0; r < rounds && ok; ++r) {
         const int mt = 2 * r + s;
@@ -378,14 +410,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            bool swa;
-            const int j = tile_block(p, x, tau, hh, swa);
             int clo = 64, chi = -1;  // visible columns of this half (empty by default)
-            if (j >= 0) {
-              const int lo = swa ? max(64 * j, t - p.window + 1) : 64 * j;
-              const int hi = min(t, 64 * j + 63);
-              clo = lo - 64 * j;
-              chi = hi - 64 * j;
+            if (tau < x.n_sp) {
+              const int e = 2 * tau + hh;
+              if (e < x.nsel) {
+                clo = 0;
+                chi = (e == x.diag) ? t - 64 * x.I : 63;  // only block I crosses the causal line
+              }
+            } else {
+              const int j = x.jw0 + 2 * (tau - x.n_sp) + hh;
+              if (j <= x.I) {
+                clo = max(64 * j, t - p.window + 1) - 64 * j;
+                chi = min(t, 64 * j + 63) - 64 * j;
+              }
             }
             if (clo > 0 || chi < 63) {
 #pragma unroll
@@ -423,8 +460,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
-              const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
+              // the first kPolyCols columns of each row use the FMA-pipe exp2, the rest MUFU
+              const float x0 = fmaf(sv[32 * c + 2 * i], sc, -ms);
+              const float x1 = fmaf(sv[32 * c + 2 * i + 1], sc, -ms);
+              const bool poly = 32 * c + 2 * i < kPolyCols;
+              const float p0 = poly ? tc::exp2_poly3(x0) : exp2f(x0);
+              const float p1 = poly ? tc::exp2_poly3(x1) : exp2f(x1);
               ls[i & 3] += p0 + p1;
               pk[i] = tc::pack_bf16x2(p0, p1);
             }

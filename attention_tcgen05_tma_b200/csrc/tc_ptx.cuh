@@ -190,6 +190,23 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// 2^x on the FMA/ALU pipes, to take part of the softmax exponentials off the MUFU unit.
+// x = n + f with n = rint(x) (adding and subtracting 1.5 * 2^23 rounds to an integer, which
+// also sits in the low mantissa bits of the sum), f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial fitted here by the Remez exchange algorithm on relative error (max 7.5e-5 in
+// fp32 Horner form); 2^n is added to the exponent field.  x is clamped to >= -125 so the
+// exponent field never underflows: inputs below (masked logits included) give tiny positive
+// values under 2^-124, which only feed bf16 probabilities.
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = __fadd_rn(x, 12582912.0f);
+  const float f = __fadd_rn(x, -__fadd_rn(t, -12582912.0f));
+  float p = fmaf(0.0551716685f, f, 0.2426111251f);
+  p = fmaf(p, f, 0.6932609677f);
+  p = fmaf(p, f, 0.9999280572f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -211,6 +228,7 @@ constexpr int kQueueSlots = 4;
 struct UnitQueue {
   uint64_t full[kQueueSlots], empty[kQueueSlots];
   int unit[kQueueSlots];
+  int info[kQueueSlots][2];  // per-unit facts the producer publishes with the id
 };
 
 __device__ __forceinline__ void queue_init(UnitQueue* q, uint32_t consumers) {
@@ -220,23 +238,29 @@ __device__ __forceinline__ void queue_init(UnitQueue* q, uint32_t consumers) {
   }
 }
 
-// producer side: publish the n-th id; returns false on timeout
-__device__ __forceinline__ bool queue_push(UnitQueue* q, uint32_t n, int unit, volatile int* abort) {
+// producer side: publish the n-th id (with two ints of unit facts); false on timeout
+__device__ __forceinline__ bool queue_push(UnitQueue* q, uint32_t n, int unit, volatile int* abort, int info0 = 0,
+                                           int info1 = 0) {
   const uint32_t s = n % kQueueSlots;
   if (!mbar_wait(&q->empty[s], ((n / kQueueSlots) & 1u) ^ 1u, abort)) return false;
   q->unit[s] = unit;
+  q->info[s][0] = info0;
+  q->info[s][1] = info1;
   mbar_arrive(&q->full[s]);  // release: the id is visible to threads that observe the phase
   return true;
 }
 
-// consumer side: pop the n-th id (or -1 on timeout / abort)
-__device__ __forceinline__ int queue_pop(UnitQueue* q, uint32_t n, volatile int* abort, bool& ok) {
+// consumer side: pop the n-th id (or -1 on timeout / abort) and its unit facts
+__device__ __forceinline__ int queue_pop(UnitQueue* q, uint32_t n, volatile int* abort, bool& ok, int* info0 = nullptr,
+                                         int* info1 = nullptr) {
   const uint32_t s = n % kQueueSlots;
   if (!mbar_wait(&q->full[s], (n / kQueueSlots) & 1u, abort)) {
     ok = false;
     return -1;
   }
   const int u = *reinterpret_cast<volatile int*>(&q->unit[s]);
+  if (info0) *info0 = *reinterpret_cast<volatile int*>(&q->info[s][0]);
+  if (info1) *info1 = *reinterpret_cast<volatile int*>(&q->info[s][1]);
   mbar_arrive(&q->empty[s]);
   return u;
 }
