@@ -159,6 +159,7 @@ hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype dtype, co
   else
     e = launch_full_attn_simt(d, dtype, q, k, v, o, lse, nullptr, false, HYS_REDUCE_SUM, s);
   if (e != cudaSuccess) return HYS_ERR_CUDA;
+  if (token_scores_tc_supported(d, dtype)) return from_cuda(launch_token_scores_tc(d, q, k, lse, scores, workspace, s));
   return from_cuda(launch_token_scores_simt(d, dtype, q, k, lse, scores, s));
 }
 

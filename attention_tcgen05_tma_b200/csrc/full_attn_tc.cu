@@ -42,7 +42,10 @@ constexpr int kStages = 4;         // K/V ring depth (one stage = one 128-key K 
 constexpr int kMaxNB = 2048;       // score accumulator capacity per slot (N <= 131072)
 constexpr int kMaxGrid = 148;      // B200 SM count; the workspace is sized for this grid
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kPolyCols = 32;      // softmax columns (of 128) whose exp2 runs on the FMA pipe
+#ifndef HYS_POLY_COLS
+#define HYS_POLY_COLS 0
+#endif
+constexpr int kPolyCols = HYS_POLY_COLS;  // softmax columns (of 128) whose exp2 runs on the FMA pipe
 
 
 struct Params {

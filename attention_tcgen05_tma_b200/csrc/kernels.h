@@ -44,6 +44,11 @@ cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void*
                                 void* o, float* lse, float* scores, hys_reduce red, bool want_scores,
                                 void* ws, size_t ws_bytes, cudaStream_t s);
 
+// Token scores (second pass) on the tensor cores; ws holds the 256-byte unit counter.
+bool token_scores_tc_supported(const PrefillDims& d, hys_dtype dt);
+cudaError_t launch_token_scores_tc(const PrefillDims& d, const void* q, const void* k, const float* lse,
+                                   float* scores, void* ws, cudaStream_t s);
+
 // ---- top-k -------------------------------------------------------------------------------
 // rows = B*Hkv*T (prefill) or B*Hkv (decode); row r has n_cand(r) candidates.
 cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, int T, int NB, int k,

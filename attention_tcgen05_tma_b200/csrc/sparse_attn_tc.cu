@@ -34,7 +34,10 @@ constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;
 constexpr int kMaxKb = 1024;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kPolyCols = 32;      // softmax columns (of 128) whose exp2 runs on the FMA pipe
+#ifndef HYS_POLY_COLS
+#define HYS_POLY_COLS 0
+#endif
+constexpr int kPolyCols = HYS_POLY_COLS;  // softmax columns (of 128) whose exp2 runs on the FMA pipe
 
 
 struct Params {

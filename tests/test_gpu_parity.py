@@ -102,6 +102,7 @@ TOKEN_CASES = [
     ("bf16_d128", "bf16", 1, 700, 8, 2, 128, 100, 128),
     ("bf16_d64_small_forced", "bf16", 1, 300, 4, 1, 64, 40, 16),
     ("f32_d64", "f32", 1, 400, 4, 1, 64, 64, 128),
+    ("bf16_d128_g8_rounds", "bf16", 1, 1500, 16, 2, 128, 300, 128),
 ]
 
 
