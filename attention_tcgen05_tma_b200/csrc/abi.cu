@@ -232,9 +232,20 @@ hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const v
                                            gate_logits, o, s));
 }
 
+hys_status hysparse_sparse_attn_tokens_workspace_size(const hys_shape* shape, hys_dtype dtype, int forced_window,
+                                                      size_t* bytes) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || !dtype_ok(dtype) || forced_window < 1) return HYS_ERR_INVALID_ARG;
+  *bytes = token_sparse_tc_supported(d, dtype, forced_window) ? align256(token_sparse_tc_workspace()) : 0;
+  return HYS_OK;
+}
+
 hys_status hysparse_sparse_attn_tokens(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
                                        const void* k_shared, const void* v_shared, const int* idx, int k_tokens,
-                                       int forced_window, const float* sinks, void* o, hys_stream_t stream) {
+                                       int forced_window, const float* sinks, void* o, void* workspace,
+                                       size_t workspace_bytes, hys_stream_t stream) {
   PrefillDims d;
   hys_status st = check_prefill(shape, &d);
   if (st != HYS_OK) return st;
@@ -242,10 +253,17 @@ hys_status hysparse_sparse_attn_tokens(const hys_shape* shape, hys_dtype dtype, 
   if (sinks) return HYS_ERR_UNSUPPORTED;
   if (!q_sparse || !k_shared || !v_shared || !idx || !o) return HYS_ERR_INVALID_ARG;
   if (k_tokens < 1 || k_tokens > 16384 || forced_window < 1) return HYS_ERR_INVALID_ARG;
-  if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(o))
+  if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(o) ||
+      !aligned16(workspace))
     return HYS_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (token_sparse_tc_supported(d, dtype, forced_window)) {
+    if (workspace == nullptr || workspace_bytes < align256(token_sparse_tc_workspace())) return HYS_ERR_WORKSPACE;
+    return from_cuda(launch_token_sparse_tc(d, q_sparse, k_shared, v_shared, idx, k_tokens, forced_window, o,
+                                            workspace, s));
+  }
   return from_cuda(launch_sparse_tokens_simt(d, dtype, q_sparse, k_shared, v_shared, idx, k_tokens, forced_window, o,
-                                             reinterpret_cast<cudaStream_t>(stream)));
+                                             s));
 }
 
 // ----------------------------------------------------------------------------- decode

@@ -49,6 +49,12 @@ bool token_scores_tc_supported(const PrefillDims& d, hys_dtype dt);
 cudaError_t launch_token_scores_tc(const PrefillDims& d, const void* q, const void* k, const float* lse,
                                    float* scores, void* ws, cudaStream_t s);
 
+// Token-sparse layer on the tensor cores; ws holds the 256-byte unit counter.
+bool token_sparse_tc_supported(const PrefillDims& d, hys_dtype dt, int forced);
+size_t token_sparse_tc_workspace();
+cudaError_t launch_token_sparse_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
+                                   int kt, int forced, void* o, void* ws, cudaStream_t s);
+
 // ---- top-k -------------------------------------------------------------------------------
 // rows = B*Hkv*T (prefill) or B*Hkv (decode); row r has n_cand(r) candidates.
 cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, int T, int NB, int k,

@@ -267,3 +267,36 @@ __device__ __forceinline__ int queue_pop(UnitQueue* q, uint32_t n, volatile int*
 
 }  // namespace tc
 }  // namespace hys
+
+namespace hys {
+namespace tc {
+
+// Two-step pop for consumers that keep using data published alongside the id (for example a
+// per-slot array the producer filled): peek waits for the id; release frees the slot, and the
+// producer may overwrite it only after every consumer released it.
+__device__ __forceinline__ int queue_peek(UnitQueue* q, uint32_t n, volatile int* abort, bool& ok, int* info0,
+                                          int* info1) {
+  const uint32_t s = n % kQueueSlots;
+  if (!mbar_wait(&q->full[s], (n / kQueueSlots) & 1u, abort)) {
+    ok = false;
+    return -1;
+  }
+  *info0 = *reinterpret_cast<volatile int*>(&q->info[s][0]);
+  *info1 = *reinterpret_cast<volatile int*>(&q->info[s][1]);
+  return *reinterpret_cast<volatile int*>(&q->unit[s]);
+}
+__device__ __forceinline__ void queue_release(UnitQueue* q, uint32_t n) { mbar_arrive(&q->empty[n % kQueueSlots]); }
+
+// TMA gather of four rows (one 2-D box row each) of a [rows][cols] tensor into shared memory,
+// completing on an mbarrier.  The tensor map's box must be one row high.
+__device__ __forceinline__ void tma_gather4(const CUtensorMap* map, uint64_t* bar, void* dst, int col, int r0, int r1,
+                                            int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
+}  // namespace tc
+}  // namespace hys

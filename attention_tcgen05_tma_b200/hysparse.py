@@ -25,7 +25,8 @@ EXPORTED = (
     "hysparse_version", "hysparse_status_string", "hysparse_get_device_status",
     "hysparse_full_attn_select_workspace_size", "hysparse_full_attn_select",
     "hysparse_topk", "hysparse_topk_tokens_workspace_size", "hysparse_topk_tokens",
-    "hysparse_sparse_attn_workspace_size", "hysparse_sparse_attn", "hysparse_sparse_attn_tokens",
+    "hysparse_sparse_attn_workspace_size", "hysparse_sparse_attn",
+    "hysparse_sparse_attn_tokens_workspace_size", "hysparse_sparse_attn_tokens",
     "hysparse_full_attn_select_decode_workspace_size", "hysparse_full_attn_select_decode",
     "hysparse_topk_decode", "hysparse_sparse_attn_decode_workspace_size", "hysparse_sparse_attn_decode", "hysparse_full_attn_select_decode_noalloc",
 )
@@ -64,7 +65,8 @@ _SIGS = {
     "hysparse_topk_tokens": ([_SH, _P, _I, _I, _P, _P, _SZ, _P], _I),
     "hysparse_sparse_attn_workspace_size": ([_SH, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_sparse_attn": ([_SH, _I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
-    "hysparse_sparse_attn_tokens": ([_SH, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P], _I),
+    "hysparse_sparse_attn_tokens_workspace_size": ([_SH, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_sparse_attn_tokens": ([_SH, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "hysparse_full_attn_select_decode_workspace_size": ([_DSH, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_full_attn_select_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P], _I),
     "hysparse_topk_decode": ([_DSH, _P, _I, _P, _P, _P], _I),
@@ -154,8 +156,16 @@ def hysparse_sparse_attn(shape, dtype, q, k, v, idx, kb, ks, vs, window, gate, s
                                        o, ws, ws_bytes, stream)
 
 
-def hysparse_sparse_attn_tokens(shape, dtype, q, k, v, idx, kt, forced, sinks, o, stream) -> int:
-    return load().hysparse_sparse_attn_tokens(ctypes.byref(shape), dtype, q, k, v, idx, kt, forced, sinks, o, stream)
+def hysparse_sparse_attn_tokens_workspace_size(shape: hys_shape, dtype: int, forced: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_sparse_attn_tokens_workspace_size(ctypes.byref(shape), dtype, forced, ctypes.byref(n)),
+           "hysparse_sparse_attn_tokens_workspace_size")
+    return n.value
+
+
+def hysparse_sparse_attn_tokens(shape, dtype, q, k, v, idx, kt, forced, sinks, o, ws, ws_bytes, stream) -> int:
+    return load().hysparse_sparse_attn_tokens(ctypes.byref(shape), dtype, q, k, v, idx, kt, forced, sinks, o, ws,
+                                              ws_bytes, stream)
 
 
 def hysparse_full_attn_select_decode_workspace_size(shape: hys_decode_shape, dtype: int) -> int:
@@ -299,13 +309,17 @@ def sparse_attn(q_sparse, k, v, idx, k_swa, v_swa, window: int, gate_logits, *, 
     return o
 
 
-def sparse_attn_tokens(q_sparse, k, v, idx, forced_window: int, *, o=None, stream=None):
+def sparse_attn_tokens(q_sparse, k, v, idx, forced_window: int, *, o=None, workspace=None, stream=None):
     torch = _torch()
     sh = prefill_shape(q_sparse, k)
     if o is None:
         o = torch.empty_like(q_sparse)
+    if workspace is None:
+        workspace = workspace_for(hysparse_sparse_attn_tokens_workspace_size(sh, _dt(q_sparse), forced_window),
+                                  q_sparse.device)
     _check(hysparse_sparse_attn_tokens(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k), _ptr(v), _ptr(idx),
-                                       idx.shape[-1], forced_window, None, _ptr(o), _stream(stream)),
+                                       idx.shape[-1], forced_window, None, _ptr(o), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)),
            "hysparse_sparse_attn_tokens")
     return o
 

@@ -167,13 +167,16 @@ HYS_API hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype,
 /* ------------------------------------------------------------------------------------
  * Token-sparse layer ([HS2]): row t of tile I attends idx[b,g,I,:] (token positions,
  * ascending, -1 padded, all <= t) united with [max(0, t-forced_window+1), t], each
- * token once, over the shared K, V; no gate.  sinks must be NULL.
+ * token once, over the shared K, V; no gate.  sinks must be NULL.  workspace: at least
+ * hysparse_sparse_attn_tokens_workspace_size() bytes.
  * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_sparse_attn_tokens_workspace_size(const hys_shape* shape, hys_dtype dtype,
+                                                            int forced_window, size_t* bytes);
 HYS_API hys_status hysparse_sparse_attn_tokens(const hys_shape* shape, hys_dtype dtype,
                                        const void* q_sparse, const void* k_shared,
                                        const void* v_shared, const int* idx, int k_tokens,
                                        int forced_window, const float* sinks, void* o,
-                                       hys_stream_t stream);
+                                       void* workspace, size_t workspace_bytes, hys_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Decode, full layer ([HS2] decode step; [HS] 3.4.1).  One new token per sequence at

@@ -64,8 +64,12 @@ def test_entry_points_reject_bad_arguments_without_launching(lib):
     assert H.hysparse_sparse_attn_workspace_size(bsh, H.HYS_BF16) > 0
     assert H.hysparse_sparse_attn(bsh, H.HYS_BF16, 16, 16, 16, 16, 4, 16, 16, 128, 16, None, 16, None, 0, None) \
         == H.HYS_ERR_WORKSPACE
-    assert H.hysparse_sparse_attn_tokens(sh, H.HYS_F32, 16, 16, 16, 16, 0, 128, None, 16, None) \
+    assert H.hysparse_sparse_attn_tokens(sh, H.HYS_F32, 16, 16, 16, 16, 0, 128, None, 16, None, 0, None) \
         == H.HYS_ERR_INVALID_ARG
+    tsh = H.hys_shape(1, 512, 8, 2, 128, 64)
+    assert H.hysparse_sparse_attn_tokens_workspace_size(tsh, H.HYS_BF16, 128) > 0
+    assert H.hysparse_sparse_attn_tokens(tsh, H.HYS_BF16, 16, 16, 16, 16, 64, 128, None, 16, None, 0, None) \
+        == H.HYS_ERR_WORKSPACE
     assert H.hysparse_full_attn_select(sh, H.HYS_F32, 16, 16, 16, 16, 16, 0, 7, None, None, 0, None) \
         == H.HYS_ERR_INVALID_ARG
     # token scores with max aggregation are not defined
