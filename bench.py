@@ -302,6 +302,8 @@ def run_ours(args, torch, dist, rank, world, dev):
 
     if not args.no_decode:
         res["decode"] = run_decode(args, torch, dist, rank, world, dev, peaks, peak_src)
+    if not args.no_token:
+        res["token"] = run_token(args, torch, dist, rank, world, dev, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     return res
@@ -371,6 +373,91 @@ def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
            "sparse_roofline": {"bound": "hbm", "achieved": round(sp_gbs, 1), "peak": hbm, "unit": "GB/s",
                                "frac": round(sp_gbs / hbm, 4)}}
     del x
+    torch.cuda.empty_cache()
+    return res
+
+
+def token_sparse_flops(idx_np, N, G, D, W, block=64):
+    """Algorithmic flops of one token-sparse layer: 4*D per (row, head, attended key), the
+    attended set being the tile's selected tokens (all before the row's window) plus the
+    row's newest W tokens."""
+    B, Hkv, T, k = idx_np.shape
+    nsel = (idx_np >= 0).sum(-1)                                  # [B, Hkv, T]
+    rows = np.arange(N)
+    win = np.minimum(rows + 1, W)
+    per_tile_rows = np.array([min(N, (I + 1) * block) - I * block for I in range(T)])
+    win_tile = np.add.reduceat(win, np.arange(0, N, block))
+    total = int((nsel * per_tile_rows[None, None, :]).sum()) * G + int(win_tile.sum()) * B * Hkv * G
+    return 4.0 * D * total
+
+
+def run_token(args, torch, dist, rank, world, dev, peaks, peak_src):
+    """Token-granularity variant: full layer with token scores (two passes), top-k tokens with
+    the forced newest window, and its token-sparse layers."""
+    from attention_tcgen05_tma_b200 import hysparse as H
+    from attention_tcgen05_tma_b200 import inputs as I
+    w = I.WORKLOADS[args.token_workload]
+    x = make_prefill_inputs(w, torch, dev, w.layers, seed_offset=1000 * rank)
+    for key in ("k_swa", "v_swa", "gate"):
+        x[key] = []   # the token variant has no SWA branch and no gate
+    torch.cuda.empty_cache()
+    T = w.T
+    sh = H.prefill_shape(x["q"], x["k"])
+    ws = H.workspace_for(H.hysparse_full_attn_select_workspace_size(sh, H.HYS_BF16, H.HYS_GRAN_TOKEN), dev)
+    wst = H.workspace_for(H.hysparse_sparse_attn_tokens_workspace_size(sh, H.HYS_BF16, w.window), dev)
+    o = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    ts = torch.empty((w.B, w.Hkv, T, w.N), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.Hkv, T, w.topk), dtype=torch.int32, device=dev)
+    osp = torch.empty_like(x["q"])
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        H.full_attn_select(x["q"], x["k"], x["v"], gran="token", o=o, scores=ts, lse=lse, workspace=ws)
+        if ev:
+            ev[1].record()
+        H.topk_tokens(ts, w.topk, w.window, idx=idx)
+        if ev:
+            ev[2].record()
+        for l in range(w.layers):
+            H.sparse_attn_tokens(x["q_sparse"][l], x["k"], x["v"], idx, w.window, o=osp, workspace=wst)
+        if ev:
+            ev[3].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    full_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    topk_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    sp_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / steps / w.layers
+    ms_step = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / steps, dist, dev)
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    full_alg = 4.0 * w.D * w.Hq * w.B * w.N * (w.N + 1) / 2
+    full_exec = 2.0 * full_alg      # pass 2 recomputes QK^T and adds the column-sum MMA
+    sp_fl = token_sparse_flops(idx.cpu().numpy(), w.N, w.G, w.D, w.window)
+    res = {"tokens_per_s": round(w.B * w.N * world / (ms_step / 1e3), 1), "ms_per_step": round(ms_step, 3),
+           "steps": steps,
+           "config": f"B={w.B} N={w.N} Hq={w.Hq} Hkv={w.Hkv} D={w.D}: full layer + token scores, top-{w.topk} "
+                     f"tokens + forced newest {w.window}, {w.layers} token-sparse layers",
+           "full_token_ms": round(full_ms, 3),
+           "full_token_alg_tflops": round(full_alg / full_ms / 1e9, 1),
+           "full_token_exec_tflops": round(full_exec / full_ms / 1e9, 1),
+           "full_token_frac_exec": round(full_exec / full_ms / 1e9 / peak_tf, 4),
+           "topk_tokens_ms": round(topk_ms, 3),
+           "sparse_tokens_ms_per_layer": round(sp_ms, 3),
+           "sparse_tokens_tflops": round(sp_fl / sp_ms / 1e9, 1),
+           "sparse_tokens_frac": round(sp_fl / sp_ms / 1e9 / peak_tf, 4),
+           "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    del x, o, lse, ts, idx, osp, ws, wst
     torch.cuda.empty_cache()
     return res
 
@@ -527,6 +614,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-token", action="store_true")
+    ap.add_argument("--token-workload", default="token", help="token-variant workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
