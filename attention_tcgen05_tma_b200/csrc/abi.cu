@@ -222,7 +222,7 @@ hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const v
       !aligned16(v_swa) || !aligned16(gate_logits) || !aligned16(o) || !aligned16(workspace))
     return HYS_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (sparse_attn_tc_supported(d, dtype)) {
+  if (sparse_attn_tc_supported(d, dtype) && k <= 256) {
     const size_t need = align256(sparse_attn_tc_workspace(d));
     if (workspace == nullptr || workspace_bytes < need) return HYS_ERR_WORKSPACE;
     return from_cuda(launch_sparse_attn_tc(d, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,

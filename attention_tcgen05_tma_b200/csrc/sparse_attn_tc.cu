@@ -30,9 +30,9 @@ namespace hys {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kStages = 4;
+constexpr int kStages = 3;         // K/V ring (one stage = one 128-key K or V tile)
 constexpr int kMaxGrid = 148;
-constexpr int kMaxKb = 1024;
+constexpr int kMaxKb = 256;        // selected blocks per tile on this path
 constexpr float kRescaleLog2 = 8.0f;
 #ifndef HYS_POLY_COLS
 #define HYS_POLY_COLS 0
@@ -54,7 +54,8 @@ struct Params {
 
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t q_full[2][2], q_empty[2][2];  // [slot][buffer]: Q is double-buffered per slot
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_drain, spare;
   tc::UnitQueue queue;
 };
@@ -65,7 +66,7 @@ struct Cfg {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 128 * D * 2;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = 2 * kQBytes;
+  static constexpr int kOffKV = 4 * kQBytes;   // Q: [slot][buffer]
   static constexpr int kOffList = kOffKV + kStages * kKVBytes;   // producer's copy of a unit's indices
   static constexpr int kOffBar = kOffList + kMaxKb * 4;
   static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
@@ -126,8 +127,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->kv_empty[i], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->q_full[s], 1);
-      tc::mbar_init(&bars->q_empty[s], 1);
+      for (int qb = 0; qb < 2; ++qb) {
+        tc::mbar_init(&bars->q_full[s][qb], 1);
+        tc::mbar_init(&bars->q_empty[s][qb], 1);
+      }
       tc::mbar_init(&bars->s_full[s], 1);
       tc::mbar_init(&bars->p_full[s], 128);
       tc::mbar_init(&bars->o_full[s], 1);
@@ -201,14 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int s = 0; s < 2 && ok; ++s) {
             const int mt = 2 * r + s;
             if (mt >= MT) continue;
-            if (!(ok = tc::mbar_wait(&bars->q_empty[s], (q_cnt[s] & 1u) ^ 1u, abort))) break;
+            const uint32_t qb = q_cnt[s] & 1u;
+            if (!(ok = tc::mbar_wait(&bars->q_empty[s][qb], ((q_cnt[s] >> 1) & 1u) ^ 1u, abort))) break;
             ++q_cnt[s];
-            tc::mbar_arrive_expect_tx(&bars->q_full[s], C::kQBytes);
+            tc::mbar_arrive_expect_tx(&bars->q_full[s][qb], C::kQBytes);
             const int h0 = x.g * p.G + 2 * mt;
-            uint8_t* qdst = smem + C::kOffQ + s * C::kQBytes;
+            uint8_t* qdst = smem + C::kOffQ + (2 * s + qb) * C::kQBytes;
             for (int hh = 0; hh < 2; ++hh)
               for (int ch = 0; ch < C::kChunks; ++ch)
-                tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + ch * 16384 + hh * 8192, ch * 64, 64 * x.I,
+                tc::tma_load_3d(&tmQ, &bars->q_full[s][qb], qdst + ch * 16384 + hh * 8192, ch * 64, 64 * x.I,
                                 x.b * p.Hq + h0 + hh);
           }
           for (int tau = 0; tau < ntiles && ok; ++tau) {
@@ -247,7 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i)
         tc::mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u, abort, 100000000ull);
       for (int s = 0; s < 2; ++s)
-        if (q_cnt[s] > 0) tc::mbar_wait(&bars->q_full[s], (q_cnt[s] - 1) & 1u, abort, 100000000ull);
+        for (uint32_t i = (q_cnt[s] > 2 ? q_cnt[s] - 2 : 0); i < q_cnt[s]; ++i)
+          tc::mbar_wait(&bars->q_full[s][i & 1u], (i >> 1) & 1u, abort, 100000000ull);
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
@@ -260,8 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t kvaddr = tc::smem_u32(smem + C::kOffKV);
       uint32_t kv_it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
       bool ok = true;
+      uint32_t qbuf[2] = {0, 0};
       auto issue_S = [&](int s, uint32_t st) {
-        const uint32_t qb = qaddr + s * C::kQBytes, kb = kvaddr + st * C::kKVBytes;
+        const uint32_t qb = qaddr + (2 * s + qbuf[s]) * C::kQBytes, kb = kvaddr + st * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -287,7 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int s = 0; s < 2; ++s) {
             act[s] = (2 * r + s) < MT;
             if (act[s] && ok) {
-              ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort);
+              qbuf[s] = q_cnt[s] & 1u;
+              ok = tc::mbar_wait(&bars->q_full[s][qbuf[s]], (q_cnt[s] >> 1) & 1u, abort);
               ++q_cnt[s];
             }
           }
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (have_k) tc::mma_commit(&bars->kv_empty[kst]);
           }
           for (int s = 0; s < 2; ++s)
-            if (act[s]) tc::mma_commit(&bars->q_empty[s]);
+            if (act[s]) tc::mma_commit(&bars->q_empty[s][qbuf[s]]);
         }
       }
       if (!ok) fail(abort, p.status);
@@ -381,16 +388,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tau == x.n_sp && x.n_sp > 0) {
             // branch switch: the sparse branch is complete in O; keep sigmoid(g0) * O / l
             const float f = l > 0.0f ? g0 / l : 0.0f;
-#pragma unroll 1
+            uint32_t ov[D / 32][32];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, ov[c]);
+            tc::tmem_wait_ld();
+#pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tc::tmem_ld32(tOrow + 32 * c, ov);
-              tc::tmem_wait_ld();
               float4* dst = reinterpret_cast<float4*>(part + 32 * c);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(ov[4 * i]) * f, __uint_as_float(ov[4 * i + 1]) * f,
-                                     __uint_as_float(ov[4 * i + 2]) * f, __uint_as_float(ov[4 * i + 3]) * f);
+                dst[i] = make_float4(__uint_as_float(ov[c][4 * i]) * f, __uint_as_float(ov[c][4 * i + 1]) * f,
+                                     __uint_as_float(ov[c][4 * i + 2]) * f, __uint_as_float(ov[c][4 * i + 3]) * f);
             }
             m_used = -INFINITY;
             l = 0.0f;
@@ -498,12 +506,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float f1 = l > 0.0f ? g1 / l : 0.0f;
         const bool have_sp = x.n_sp > 0;
         __nv_bfloat16* orow = p.o + (((size_t)x.b * p.Hq + h) * p.N + t) * D;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tc::tmem_ld32(tOrow + 32 * c, ov);
-          tc::tmem_wait_ld();
-          if (valid) {
+        uint32_t ov[D / 32][32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, ov[c]);
+        tc::tmem_wait_ld();
+        tc::fence_before_sync();
+        tc::mbar_arrive(&bars->o_empty[s]);  // O may be overwritten by the next round from here on
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
             float add[32];
             if (have_sp) {
               const float4* src = reinterpret_cast<const float4*>(part + 32 * c);
@@ -522,15 +533,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              pk[i] = tc::pack_bf16x2(fmaf(__uint_as_float(ov[2 * i]), f1, add[2 * i]),
-                                      fmaf(__uint_as_float(ov[2 * i + 1]), f1, add[2 * i + 1]));
+              pk[i] = tc::pack_bf16x2(fmaf(__uint_as_float(ov[c][2 * i]), f1, add[2 * i]),
+                                      fmaf(__uint_as_float(ov[c][2 * i + 1]), f1, add[2 * i + 1]));
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
-        tc::fence_before_sync();
-        tc::mbar_arrive(&bars->o_empty[s]);
       }
     }
     if (!ok) fail(abort, p.status);
