@@ -12,11 +12,12 @@
 //     128-byte chunk at row 64*j of K (or V), so only the selected blocks are read; K~, V~
 //     are never materialised.  A missing half (odd count, -1 padding) is loaded from a
 //     row past the end of the tensor, which TMA fills with zeros.
-//   * The tile list of a unit is the selected blocks in index order, then the window
-//     blocks of K', V'.  At the switch the softmax warpgroup reads O (the sparse branch is
-//     complete: its last P.V finished before the first window S did), stores
-//     sigmoid(g0) * O / l to an fp32 row of L2-resident scratch and restarts its online
-//     softmax; the epilogue adds sigmoid(g1) * O / l of the window branch.
+//   * Both branches accumulate into the same O, with no scratch memory.  The tiles of a
+//     round are: the selected blocks (online softmax into O); then the window tiles twice.
+//     Before the first window pass the softmax warpgroup scales O in TMEM by sigmoid(g0)/l
+//     (O becomes sigmoid(g0) o~, exactly); the first window pass only computes the window
+//     branch's row max m' and sum l'; the second recomputes S and adds
+//     P' = exp(s - m') * sigmoid(g1) / l' times V' to O, which then holds o_t.
 //   * Masks: per 64-key half, the visible key range is [64j, min(t, 64j+63)] for a selected
 //     block and [max(64j, t-w+1), min(t, 64j+63)] for a window block.
 #include <cuda.h>
@@ -30,14 +31,10 @@ namespace hys {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kStages = 3;         // K/V ring (one stage = one 128-key K or V tile)
+constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;
-constexpr int kMaxKb = 256;        // selected blocks per tile on this path
+constexpr int kMaxKb = 1024;
 constexpr float kRescaleLog2 = 8.0f;
-#ifndef HYS_POLY_COLS
-#define HYS_POLY_COLS 0
-#endif
-constexpr int kPolyCols = HYS_POLY_COLS;  // softmax columns (of 128) whose exp2 runs on the FMA pipe
 
 
 struct Params {
@@ -46,7 +43,6 @@ struct Params {
   const int* idx;      // [B,Hkv,T,kb]
   const float* gate;   // [B,Hq,N,2]
   __nv_bfloat16* o;
-  float* partial;      // [grid][2][128][D] fp32 scratch
   int* counter;        // work-unit counter (zeroed before the launch)
   int* status;
   float scale_log2;
@@ -54,8 +50,7 @@ struct Params {
 
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t q_full[2][2], q_empty[2][2];  // [slot][buffer]: Q is double-buffered per slot
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_drain, spare;
   tc::UnitQueue queue;
 };
@@ -66,7 +61,7 @@ struct Cfg {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 128 * D * 2;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = 4 * kQBytes;   // Q: [slot][buffer]
+  static constexpr int kOffKV = 2 * kQBytes;
   static constexpr int kOffList = kOffKV + kStages * kKVBytes;   // producer's copy of a unit's indices
   static constexpr int kOffBar = kOffList + kMaxKb * 4;
   static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
@@ -79,8 +74,16 @@ struct Unit {
   int diag;    // entry holding block I (causally masked per row), or -1
   int n_sp;    // sparse tiles
   int jw0;     // first window block
-  int n_sw;    // window tiles
+  int n_sw;    // window tiles (each appears twice: statistics pass, then P.V pass)
 };
+
+// tile kinds of a round: selected blocks, window statistics pass, window P.V pass
+enum TileKind { kSparse = 0, kWinStats = 1, kWinPV = 2 };
+
+__device__ __forceinline__ int tile_kind(const Unit& x, int tau) {
+  return tau < x.n_sp ? kSparse : (tau < x.n_sp + x.n_sw ? kWinStats : kWinPV);
+}
+__device__ __forceinline__ int num_tiles(const Unit& x) { return x.n_sp + 2 * x.n_sw; }
 
 // Units come from a counter in KV-group-major order, so co-running CTAs gather from the same
 // group's K/V (L2-resident); within a group the order is longest-first.  nsel and diag are
@@ -127,10 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->kv_empty[i], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      for (int qb = 0; qb < 2; ++qb) {
-        tc::mbar_init(&bars->q_full[s][qb], 1);
-        tc::mbar_init(&bars->q_empty[s][qb], 1);
-      }
+      tc::mbar_init(&bars->q_full[s], 1);
+      tc::mbar_init(&bars->q_empty[s], 1);
       tc::mbar_init(&bars->s_full[s], 1);
       tc::mbar_init(&bars->p_full[s], 128);
       tc::mbar_init(&bars->o_full[s], 1);
@@ -199,35 +200,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok || u < 0) break;
       if (lane == 0) {
         const Unit x = make_unit(p, u, nsel, diag);
-        const int ntiles = x.n_sp + x.n_sw;
+        const int ntiles = num_tiles(x);
         for (int r = 0; r < rounds && ok; ++r) {
           for (int s = 0; s < 2 && ok; ++s) {
             const int mt = 2 * r + s;
             if (mt >= MT) continue;
-            const uint32_t qb = q_cnt[s] & 1u;
-            if (!(ok = tc::mbar_wait(&bars->q_empty[s][qb], ((q_cnt[s] >> 1) & 1u) ^ 1u, abort))) break;
+            if (!(ok = tc::mbar_wait(&bars->q_empty[s], (q_cnt[s] & 1u) ^ 1u, abort))) break;
             ++q_cnt[s];
-            tc::mbar_arrive_expect_tx(&bars->q_full[s][qb], C::kQBytes);
+            tc::mbar_arrive_expect_tx(&bars->q_full[s], C::kQBytes);
             const int h0 = x.g * p.G + 2 * mt;
-            uint8_t* qdst = smem + C::kOffQ + (2 * s + qb) * C::kQBytes;
+            uint8_t* qdst = smem + C::kOffQ + s * C::kQBytes;
             for (int hh = 0; hh < 2; ++hh)
               for (int ch = 0; ch < C::kChunks; ++ch)
-                tc::tma_load_3d(&tmQ, &bars->q_full[s][qb], qdst + ch * 16384 + hh * 8192, ch * 64, 64 * x.I,
+                tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + ch * 16384 + hh * 8192, ch * 64, 64 * x.I,
                                 x.b * p.Hq + h0 + hh);
           }
           for (int tau = 0; tau < ntiles && ok; ++tau) {
-            const bool swa = tau >= x.n_sp;
+            const int kind = tile_kind(x, tau);
+            const bool swa = kind != kSparse;
+            const int wi = kind == kWinStats ? tau - x.n_sp : tau - x.n_sp - x.n_sw;  // window pair
             int jj[2];
             for (int hh = 0; hh < 2; ++hh) {
               if (!swa) {
                 const int e = 2 * tau + hh;
                 jj[hh] = e < x.nsel ? plist[e] : -1;
               } else {
-                const int j = x.jw0 + 2 * (tau - x.n_sp) + hh;
+                const int j = x.jw0 + 2 * wi + hh;
                 jj[hh] = j <= x.I ? j : -1;
               }
             }
-            for (int kv = 0; kv < 2; ++kv) {
+            for (int kv = 0; kv < (kind == kWinStats ? 1 : 2); ++kv) {
               const uint32_t st = kv_it % kStages;
               if (!(ok = tc::mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1u) ^ 1u, abort))) break;
               tc::mbar_arrive_expect_tx(&bars->kv_full[st], C::kKVBytes);
@@ -251,8 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i)
         tc::mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u, abort, 100000000ull);
       for (int s = 0; s < 2; ++s)
-        for (uint32_t i = (q_cnt[s] > 2 ? q_cnt[s] - 2 : 0); i < q_cnt[s]; ++i)
-          tc::mbar_wait(&bars->q_full[s][i & 1u], (i >> 1) & 1u, abort, 100000000ull);
+        if (q_cnt[s] > 0) tc::mbar_wait(&bars->q_full[s], (q_cnt[s] - 1) & 1u, abort, 100000000ull);
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
@@ -265,9 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t kvaddr = tc::smem_u32(smem + C::kOffKV);
       uint32_t kv_it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0}, o_cnt[2] = {0, 0};
       bool ok = true;
-      uint32_t qbuf[2] = {0, 0};
       auto issue_S = [&](int s, uint32_t st) {
-        const uint32_t qb = qaddr + (2 * s + qbuf[s]) * C::kQBytes, kb = kvaddr + st * C::kKVBytes;
+        const uint32_t qb = qaddr + s * C::kQBytes, kb = kvaddr + st * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -287,14 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = tc::queue_pop(&bars->queue, n, abort, ok, &nsel, &diag);
         if (u < 0) break;
         const Unit x = make_unit(p, u, nsel, diag);
-        const int ntiles = x.n_sp + x.n_sw;
+        const int ntiles = num_tiles(x);
         for (int r = 0; r < rounds && ok; ++r) {
           bool act[2];
           for (int s = 0; s < 2; ++s) {
             act[s] = (2 * r + s) < MT;
             if (act[s] && ok) {
-              qbuf[s] = q_cnt[s] & 1u;
-              ok = tc::mbar_wait(&bars->q_full[s][qbuf[s]], (q_cnt[s] >> 1) & 1u, abort);
+              ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort);
               ++q_cnt[s];
             }
           }
@@ -309,22 +308,28 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc::mma_commit(&bars->s_full[s]);
             }
           tc::mma_commit(&bars->kv_empty[kst]);
+          bool pv_started = false;  // O of this round already holds a P.V product
           for (int tau = 1; tau <= ntiles && ok; ++tau) {
-            const uint32_t vst = kv_it % kStages;
-            if (!(ok = tc::mbar_wait(&bars->kv_full[vst], (kv_it / kStages) & 1u, abort))) break;
-            ++kv_it;
+            const bool prev_pv = tile_kind(x, tau - 1) != kWinStats;
+            uint32_t vst = 0;
+            if (prev_pv) {
+              vst = kv_it % kStages;
+              if (!(ok = tc::mbar_wait(&bars->kv_full[vst], (kv_it / kStages) & 1u, abort))) break;
+              ++kv_it;
+            }
             bool have_k = false;
-            // P.V of tile tau-1 starts a fresh accumulator at the first tile of each branch
-            const bool fresh = (tau - 1 == 0) || (tau - 1 == x.n_sp);
             for (int s = 0; s < 2 && ok; ++s) {
               if (!act[s]) continue;
+              // p_full: the softmax is done with S_s(tau-1) (and wrote P unless it was a statistics tile)
               if (!(ok = tc::mbar_wait(&bars->p_full[s], p_cnt[s] & 1u, abort))) break;
               ++p_cnt[s];
-              if (tau == 1) {
-                if (!(ok = tc::mbar_wait(&bars->o_empty[s], (o_cnt[s] & 1u) ^ 1u, abort))) break;
+              if (prev_pv) {
+                if (!pv_started) {  // the previous round's epilogue must have read O_s
+                  if (!(ok = tc::mbar_wait(&bars->o_empty[s], (o_cnt[s] & 1u) ^ 1u, abort))) break;
+                }
+                tc::fence_after_sync();
+                issue_PV(s, vst, pv_started);
               }
-              tc::fence_after_sync();
-              issue_PV(s, vst, !fresh);
               if (tau < ntiles) {
                 if (!have_k) {
                   kst = kv_it % kStages;
@@ -340,11 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++o_cnt[s];
               }
             }
-            tc::mma_commit(&bars->kv_empty[vst]);
+            if (prev_pv) {
+              pv_started = true;
+              tc::mma_commit(&bars->kv_empty[vst]);
+            }
             if (have_k) tc::mma_commit(&bars->kv_empty[kst]);
           }
           for (int s = 0; s < 2; ++s)
-            if (act[s]) tc::mma_commit(&bars->q_empty[s][qbuf[s]]);
+            if (act[s]) tc::mma_commit(&bars->q_empty[s]);
         }
       }
       if (!ok) fail(abort, p.status);
@@ -358,7 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tSrow = tmem_base + 128 * s + lane_off;
     const uint32_t tOrow = tmem_base + 256 + 128 * s + lane_off;
-    float* part = p.partial + (((size_t)blockIdx.x * 2 + s) * 128 + row) * D;
     const float sc = p.scale_log2;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
@@ -367,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int u = tc::queue_pop(&bars->queue, n, abort, ok, &nsel, &diag);
       if (u < 0) break;
       const Unit x = make_unit(p, u, nsel, diag);
-      const int ntiles = x.n_sp + x.n_sw;
+      const int ntiles = num_tiles(x);
       for (int r = 0; r < rounds && ok; ++r) {
         const int mt = 2 * r + s;
         if (mt >= MT) continue;
@@ -380,28 +387,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           g0 = sigmoidf_(gl.x);
           g1 = sigmoidf_(gl.y);
         }
-        float m_used = -INFINITY, l = 0.0f;
+        float m_used = -INFINITY, l = 0.0f;   // online state of the sparse branch
+        float mw = -INFINITY, lw = 0.0f;      // window branch statistics
+        float pw = 0.0f;                      // sigmoid(g1) / l' for the window P.V pass
         for (int tau = 0; tau < ntiles; ++tau) {
+          const int kind = tile_kind(x, tau);
           if (!(ok = tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort))) break;
           ++s_cnt;
           tc::fence_after_sync();
           if (tau == x.n_sp && x.n_sp > 0) {
-            // branch switch: the sparse branch is complete in O; keep sigmoid(g0) * O / l
+            // the sparse branch is complete in O (its last P.V finished before this S did):
+            // scale O in place to sigmoid(g0) * o~
             const float f = l > 0.0f ? g0 / l : 0.0f;
-            uint32_t ov[D / 32][32];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, ov[c]);
-            tc::tmem_wait_ld();
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
-              float4* dst = reinterpret_cast<float4*>(part + 32 * c);
+              uint32_t ov[32];
+              tc::tmem_ld32(tOrow + 32 * c, ov);
+              tc::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(ov[c][4 * i]) * f, __uint_as_float(ov[c][4 * i + 1]) * f,
-                                     __uint_as_float(ov[c][4 * i + 2]) * f, __uint_as_float(ov[c][4 * i + 3]) * f);
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+              tc::tmem_st32(tOrow + 32 * c, ov);
             }
-            m_used = -INFINITY;
-            l = 0.0f;
           }
           float sv[128];
           {
@@ -419,17 +425,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               sv[96 + i] = __uint_as_float(r3[i]);
             }
           }
+          const int wi = kind == kWinStats ? tau - x.n_sp : tau - x.n_sp - x.n_sw;
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             int clo = 64, chi = -1;  // visible columns of this half (empty by default)
-            if (tau < x.n_sp) {
+            if (kind == kSparse) {
               const int e = 2 * tau + hh;
               if (e < x.nsel) {
                 clo = 0;
                 chi = (e == x.diag) ? t - 64 * x.I : 63;  // only block I crosses the causal line
               }
             } else {
-              const int j = x.jw0 + 2 * (tau - x.n_sp) + hh;
+              const int j = x.jw0 + 2 * wi + hh;
               if (j <= x.I) {
                 clo = max(64 * j, t - p.window + 1) - 64 * j;
                 chi = min(t, 64 * j + 63) - 64 * j;
@@ -456,43 +463,66 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int j = 0; j < w; ++j) a[j] = fmaxf(a[j], a[j + w]);
             mx = a[0];
           }
-          float alpha = 1.0f;
-          bool rescale = false;
-          if (mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2) {
-            rescale = true;
-            alpha = exp2f((m_used - mx) * sc);
-            l *= alpha;
-            m_used = mx;
-          }
-          const float ms = m_used == -INFINITY ? 0.0f : m_used * sc;
-          float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              // the first kPolyCols columns of each row use the FMA-pipe exp2, the rest MUFU
-              const float x0 = fmaf(sv[32 * c + 2 * i], sc, -ms);
-              const float x1 = fmaf(sv[32 * c + 2 * i + 1], sc, -ms);
-              const bool poly = 32 * c + 2 * i < kPolyCols;
-              const float p0 = poly ? tc::exp2_poly3(x0) : exp2f(x0);
-              const float p1 = poly ? tc::exp2_poly3(x1) : exp2f(x1);
-              ls[i & 3] += p0 + p1;
-              pk[i] = tc::pack_bf16x2(p0, p1);
+          if (kind == kWinStats) {
+            // window statistics only: running max and sum, no P, no P.V
+            if (mx > mw) {
+              lw = (mw == -INFINITY) ? 0.0f : lw * exp2f((mw - mx) * sc);
+              mw = mx;
             }
-            tc::tmem_st16(tSrow + 16 * c, pk);
-          }
-          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-          const bool branch_start = (tau == 0) || (tau == x.n_sp);
-          if (rescale && !branch_start) {
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tc::tmem_ld32(tOrow + 32 * c, ov);
-              tc::tmem_wait_ld();
+            const float ms = mw == -INFINITY ? 0.0f : mw * sc;
+            float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tc::tmem_st32(tOrow + 32 * c, ov);
+            for (int i = 0; i < 128; ++i) ls[i & 3] += exp2f(fmaf(sv[i], sc, -ms));
+            lw += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            if (tau == x.n_sp + x.n_sw - 1) pw = lw > 0.0f ? g1 / lw : 0.0f;
+          } else if (kind == kWinPV) {
+            // window P.V pass with the final statistics: P' = exp(s - m') * sigmoid(g1) / l'
+            const float ms = mw == -INFINITY ? 0.0f : mw * sc;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms)) * pw;
+                const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms)) * pw;
+                pk[i] = tc::pack_bf16x2(p0, p1);
+              }
+              tc::tmem_st16(tSrow + 16 * c, pk);
+            }
+          } else {
+            float alpha = 1.0f;
+            bool rescale = false;
+            if (mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2) {
+              rescale = true;
+              alpha = exp2f((m_used - mx) * sc);
+              l *= alpha;
+              m_used = mx;
+            }
+            const float ms = m_used == -INFINITY ? 0.0f : m_used * sc;
+            float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
+                const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
+                ls[i & 3] += p0 + p1;
+                pk[i] = tc::pack_bf16x2(p0, p1);
+              }
+              tc::tmem_st16(tSrow + 16 * c, pk);
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            if (rescale && tau > 0) {
+#pragma unroll 1
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t ov[32];
+                tc::tmem_ld32(tOrow + 32 * c, ov);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                tc::tmem_st32(tOrow + 32 * c, ov);
+              }
             }
           }
           tc::tmem_wait_st();
@@ -500,46 +530,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mbar_arrive(&bars->p_full[s]);
         }
         if (!ok) break;
+        // ---- epilogue: O already holds sigmoid(g0) o~ + sigmoid(g1) o'
         if (!(ok = tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort))) break;
         ++o_cnt;
         tc::fence_after_sync();
-        const float f1 = l > 0.0f ? g1 / l : 0.0f;
-        const bool have_sp = x.n_sp > 0;
         __nv_bfloat16* orow = p.o + (((size_t)x.b * p.Hq + h) * p.N + t) * D;
-        uint32_t ov[D / 32][32];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, ov[c]);
-        tc::tmem_wait_ld();
-        tc::fence_before_sync();
-        tc::mbar_arrive(&bars->o_empty[s]);  // O may be overwritten by the next round from here on
-        if (valid) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float add[32];
-            if (have_sp) {
-              const float4* src = reinterpret_cast<const float4*>(part + 32 * c);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float4 a = src[i];
-                add[4 * i] = a.x;
-                add[4 * i + 1] = a.y;
-                add[4 * i + 2] = a.z;
-                add[4 * i + 3] = a.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) add[i] = 0.0f;
-            }
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tc::tmem_ld32(tOrow + 32 * c, ov);
+          tc::tmem_wait_ld();
+          if (valid) {
             uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = tc::pack_bf16x2(fmaf(__uint_as_float(ov[c][2 * i]), f1, add[2 * i]),
-                                      fmaf(__uint_as_float(ov[c][2 * i + 1]), f1, add[2 * i + 1]));
+            for (int i = 0; i < 16; ++i) pk[i] = tc::pack_bf16x2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1]));
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&bars->o_empty[s]);
       }
     }
     if (!ok) fail(abort, p.status);
@@ -607,7 +618,6 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.gate = gate;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.counter = reinterpret_cast<int*>(ws);
-  p.partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
@@ -625,9 +635,7 @@ bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt) {
   return dt == HYS_BF16 && (d.D == 64 || d.D == 128) && d.G() % 2 == 0;
 }
 
-size_t sparse_attn_tc_workspace(const PrefillDims& d) {
-  return 256 + sizeof(float) * (size_t)grid_size(d) * 2 * 128 * d.D;
-}
+size_t sparse_attn_tc_workspace(const PrefillDims&) { return 256; }
 
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
                                   int kb, const void* ks, const void* vs, int window, const float* gate, void* o,
