@@ -399,70 +399,76 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the sparse branch is complete in O (its last P.V finished before this S did):
             // scale O in place to sigmoid(g0) * o~
             const float f = l > 0.0f ? g0 / l : 0.0f;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tc::tmem_ld32(tOrow + 32 * c, ov);
-              tc::tmem_wait_ld();
+            uint32_t ov[D];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-              tc::tmem_st32(tOrow + 32 * c, ov);
-            }
-          }
-          float sv[128];
-          {
-            uint32_t r0[32], r1[32], r2[32], r3[32];
-            tc::tmem_ld32(tSrow + 0, r0);
-            tc::tmem_ld32(tSrow + 32, r1);
-            tc::tmem_ld32(tSrow + 64, r2);
-            tc::tmem_ld32(tSrow + 96, r3);
+            for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              sv[i] = __uint_as_float(r0[i]);
-              sv[32 + i] = __uint_as_float(r1[i]);
-              sv[64 + i] = __uint_as_float(r2[i]);
-              sv[96 + i] = __uint_as_float(r3[i]);
+            for (int i = 0; i < D; i += 2) {
+              const float2 v = tc::fmul2(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(f, f));
+              ov[i] = __float_as_uint(v.x);
+              ov[i + 1] = __float_as_uint(v.y);
             }
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tc::tmem_st32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
           }
+          // visible columns of the two 64-key halves of this tile (empty by default)
           const int wi = kind == kWinStats ? tau - x.n_sp : tau - x.n_sp - x.n_sw;
+          int clo[2], chi[2];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            int clo = 64, chi = -1;  // visible columns of this half (empty by default)
+            clo[hh] = 64;
+            chi[hh] = -1;
             if (kind == kSparse) {
               const int e = 2 * tau + hh;
               if (e < x.nsel) {
-                clo = 0;
-                chi = (e == x.diag) ? t - 64 * x.I : 63;  // only block I crosses the causal line
+                clo[hh] = 0;
+                chi[hh] = (e == x.diag) ? t - 64 * x.I : 63;  // only block I crosses the causal line
               }
             } else {
               const int j = x.jw0 + 2 * wi + hh;
               if (j <= x.I) {
-                clo = max(64 * j, t - p.window + 1) - 64 * j;
-                chi = min(t, 64 * j + 63) - 64 * j;
+                clo[hh] = max(64 * j, t - p.window + 1) - 64 * j;
+                chi[hh] = min(t, 64 * j + 63) - 64 * j;
               }
             }
-            if (clo > 0 || chi < 63) {
-#pragma unroll
-              for (int i = 0; i < 64; ++i)
-                if (i < clo || i > chi) sv[64 * hh + i] = -INFINITY;
-            }
           }
+          // S row from TMEM in two batches: the first half is masked and reduced while the
+          // second is in flight
+          float sv[128];
           float mx;
           {
-            float a[8];
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tc::tmem_ld32(tSrow + 0, r0);
+            tc::tmem_ld32(tSrow + 32, r1);
+            tc::tmem_wait_ld();
+            tc::tmem_ld32(tSrow + 64, r2);
+            tc::tmem_ld32(tSrow + 96, r3);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) a[j] = sv[j];
+            for (int i = 0; i < 32; ++i) {
+              sv[i] = __uint_as_float(r0[i]);
+              sv[32 + i] = __uint_as_float(r1[i]);
+            }
+            if (clo[0] > 0 || chi[0] < 63) {
 #pragma unroll
-            for (int i = 8; i < 128; i += 8)
+              for (int i = 0; i < 64; ++i)
+                if (i < clo[0] || i > chi[0]) sv[i] = -INFINITY;
+            }
+            const float m0 = tc::max64(sv);
+            tc::tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 8; ++j) a[j] = fmaxf(a[j], sv[i + j]);
+            for (int i = 0; i < 32; ++i) {
+              sv[64 + i] = __uint_as_float(r2[i]);
+              sv[96 + i] = __uint_as_float(r3[i]);
+            }
+            if (clo[1] > 0 || chi[1] < 63) {
 #pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-              for (int j = 0; j < w; ++j) a[j] = fmaxf(a[j], a[j + w]);
-            mx = a[0];
+              for (int i = 0; i < 64; ++i)
+                if (i < clo[1] || i > chi[1]) sv[64 + i] = -INFINITY;
+            }
+            mx = fmaxf(m0, tc::max64(sv + 64));
           }
+          const float2 sc2 = make_float2(sc, sc);
           if (kind == kWinStats) {
             // window statistics only: running max and sum, no P, no P.V
             if (mx > mw) {
@@ -470,22 +476,30 @@ __global__ void __launch_bounds__(kThreads, 1)
               mw = mx;
             }
             const float ms = mw == -INFINITY ? 0.0f : mw * sc;
-            float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const float2 nm2 = make_float2(-ms, -ms);
+            float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-            for (int i = 0; i < 128; ++i) ls[i & 3] += exp2f(fmaf(sv[i], sc, -ms));
-            lw += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            if (tau == x.n_sp + x.n_sw - 1) pw = lw > 0.0f ? g1 / lw : 0.0f;
+            for (int i = 0; i < 64; ++i) {
+              const float2 xv = tc::ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
+              acc[i & 1] = tc::fadd2(acc[i & 1], make_float2(exp2f(xv.x), exp2f(xv.y)));
+            }
+            const float2 a = tc::fadd2(acc[0], acc[1]);
+            lw += a.x + a.y;
+            if (tau == x.n_sp + x.n_sw - 1) {
+              // P' = exp2((s - m') sc) * sigmoid(g1) / l' = exp2(s sc - (m' sc - log2(sigmoid(g1) / l')))
+              pw = lw > 0.0f ? g1 / lw : 0.0f;
+              pw = (mw == -INFINITY ? 0.0f : mw * sc) - __log2f(pw);
+            }
           } else if (kind == kWinPV) {
-            // window P.V pass with the final statistics: P' = exp(s - m') * sigmoid(g1) / l'
-            const float ms = mw == -INFINITY ? 0.0f : mw * sc;
+            // window P.V pass with the final statistics; pw holds the combined exponent offset
+            const float2 nm2 = make_float2(-pw, -pw);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t pk[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms)) * pw;
-                const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms)) * pw;
-                pk[i] = tc::pack_bf16x2(p0, p1);
+                const float2 xv = tc::ffma2(make_float2(sv[32 * c + 2 * i], sv[32 * c + 2 * i + 1]), sc2, nm2);
+                pk[i] = tc::pack_bf16x2(exp2f(xv.x), exp2f(xv.y));
               }
               tc::tmem_st16(tSrow + 16 * c, pk);
             }
@@ -499,30 +513,35 @@ __global__ void __launch_bounds__(kThreads, 1)
               m_used = mx;
             }
             const float ms = m_used == -INFINITY ? 0.0f : m_used * sc;
-            float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const float2 nm2 = make_float2(-ms, -ms);
+            float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t pk[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
-                const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
-                ls[i & 3] += p0 + p1;
-                pk[i] = tc::pack_bf16x2(p0, p1);
+                const float2 xv = tc::ffma2(make_float2(sv[32 * c + 2 * i], sv[32 * c + 2 * i + 1]), sc2, nm2);
+                const float2 pv = make_float2(exp2f(xv.x), exp2f(xv.y));
+                acc[i & 1] = tc::fadd2(acc[i & 1], pv);
+                pk[i] = tc::pack_bf16x2(pv.x, pv.y);
               }
               tc::tmem_st16(tSrow + 16 * c, pk);
             }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            const float2 a = tc::fadd2(acc[0], acc[1]);
+            l += a.x + a.y;
             if (rescale && tau > 0) {
-#pragma unroll 1
-              for (int c = 0; c < D / 32; ++c) {
-                uint32_t ov[32];
-                tc::tmem_ld32(tOrow + 32 * c, ov);
-                tc::tmem_wait_ld();
+              uint32_t ov[D];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                tc::tmem_st32(tOrow + 32 * c, ov);
+              for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < D; i += 2) {
+                const float2 v = tc::fmul2(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(alpha, alpha));
+                ov[i] = __float_as_uint(v.x);
+                ov[i + 1] = __float_as_uint(v.y);
               }
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) tc::tmem_st32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
             }
           }
           tc::tmem_wait_st();
@@ -535,22 +554,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++o_cnt;
         tc::fence_after_sync();
         __nv_bfloat16* orow = p.o + (((size_t)x.b * p.Hq + h) * p.N + t) * D;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tc::tmem_ld32(tOrow + 32 * c, ov);
+        uint32_t pk[D / 2];
+        {
+          uint32_t ov[D];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
           tc::tmem_wait_ld();
-          if (valid) {
-            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = tc::pack_bf16x2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
+          for (int i = 0; i < D / 2; ++i) pk[i] = tc::pack_bf16x2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1]));
         }
         tc::fence_before_sync();
-        tc::mbar_arrive(&bars->o_empty[s]);
+        tc::mbar_arrive(&bars->o_empty[s]);  // O may be overwritten by the next round from here on
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
       }
     }
     if (!ok) fail(abort, p.status);

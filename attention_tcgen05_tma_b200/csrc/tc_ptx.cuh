@@ -212,6 +212,61 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ------------------------------------------------------------------ sm_100 fp32 pair / 3-input ops
+// The FMA pipe of sm_100 executes fp32 pairs (fma/add/mul .f32x2) in one instruction, and max
+// takes three operands; softmax rows use them to halve their FMA-pipe instruction count.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t f2_pack(float x, float y) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+
+__device__ __forceinline__ float2 f2_unpack(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+
+// a * b + c on both lanes
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)), "l"(f2_pack(c.x, c.y)));
+  return f2_unpack(d);
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)));
+  return f2_unpack(d);
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a.x, a.y)), "l"(f2_pack(b.x, b.y)));
+  return f2_unpack(d);
+}
+
+// max of 64 consecutive values (four independent chains of three-input max)
+__device__ __forceinline__ float max64(const float* v) {
+  float a0 = v[0], a1 = v[1], a2 = v[2], a3 = v[3];
+#pragma unroll
+  for (int i = 4; i + 8 <= 64; i += 8) {
+    a0 = fmax3(a0, v[i], v[i + 4]);
+    a1 = fmax3(a1, v[i + 1], v[i + 5]);
+    a2 = fmax3(a2, v[i + 2], v[i + 6]);
+    a3 = fmax3(a3, v[i + 3], v[i + 7]);
+  }
+  a0 = fmax3(a0, v[60], v[61]);
+  a1 = fmax3(a1, v[62], v[63]);
+  return fmax3(fmaxf(a0, a1), a2, a3);
+}
+
 }  // namespace tc
 }  // namespace hys
 

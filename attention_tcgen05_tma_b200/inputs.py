@@ -17,6 +17,7 @@ the token-level variant and the forced newest-128 window):
 * ``tiny``     fp32, B1 N1024, 4 query heads / 1 KV head, D64, k=4 blocks, 3 sparse layers
 * ``dense7b``  bf16, B1 N8192, 32/8, D128, k=16 blocks, 3 sparse layers
 * ``moe80b``   bf16, B2 N32768, 32/4, D128, k=32 blocks, 11 sparse layers
+* ``moe80b_small``  the same per-unit shape at B1 N16384 with 2 sparse layers (profiling)
 * ``decode``   bf16, B64, L131072 cached tokens, 32/4, D128, k=32 blocks, 11 sparse layers
 * ``token``    bf16, B1 N131072, 32/4, D128, top-2048 tokens + forced 128, 3 sparse layers
 """
@@ -85,6 +86,9 @@ WORKLOADS: Dict[str, Workload] = {
                        seed=3, scale_std=1.0 / math.sqrt(128)),
     "token": Workload("token", "prefill_token", "bf16", 1, 131072, 32, 4, 128, 3, 2048, 128,
                       seed=4, scale_std=1.0 / math.sqrt(128), plant="blocks", n_plants=64),
+    # the moe80b per-unit shape (G=8, k=32) at one sequence of 16K (profiling captures, < 1 GiB)
+    "moe80b_small": Workload("moe80b_small", "prefill_block", "bf16", 1, 16384, 32, 4, 128, 2, 32, 128,
+                             seed=6, scale_std=1.0 / math.sqrt(128), plant="blocks", n_plants=64),
     # smaller decode batch with the same per-sequence shape (profiling captures: 2 GiB of cache)
     "decode_small": Workload("decode_small", "decode", "bf16", 8, 131072, 32, 4, 128, 11, 32, 128,
                              seed=5, scale_std=1.0 / math.sqrt(128)),
