@@ -42,10 +42,22 @@ constexpr int kStages = 4;         // K/V ring depth (one stage = one 128-key K 
 constexpr int kMaxNB = 2048;       // score accumulator capacity per slot (N <= 131072)
 constexpr int kMaxGrid = 148;      // B200 SM count; the workspace is sized for this grid
 constexpr float kRescaleLog2 = 8.0f;
-#ifndef HYS_POLY_COLS
-#define HYS_POLY_COLS 0
+#ifndef HYS_FULL_POLY_PAIRS
+#define HYS_FULL_POLY_PAIRS 8
 #endif
-constexpr int kPolyCols = HYS_POLY_COLS;  // softmax columns (of 128) whose exp2 runs on the FMA pipe
+// column pairs (of the 64 in a 128-key row) whose exp2 runs on the FMA pipe instead of MUFU
+constexpr int kPolyPairs = HYS_FULL_POLY_PAIRS;
+// Register split between the warpgroups (setmaxnreg): the launch gives every thread
+// kLaunchRegs; the producer/MMA warpgroup drops to kLowRegs and each softmax warpgroup rises to
+// kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
+// the host checks the compiled register count before every launch.
+constexpr int kLaunchRegs = 168, kLowRegs = 88, kHighRegs = 208;
+static_assert(kLowRegs + 2 * kHighRegs == 3 * kLaunchRegs, "register split must match the launch allocation");
+
+__device__ __forceinline__ float2 exp2_pair(float2 x, int i) {
+  if ((i * kPolyPairs) % 64 < kPolyPairs) return tc::exp2_poly3_x2(x);
+  return make_float2(exp2f(x.x), exp2f(x.y));
+}
 
 
 struct Params {
@@ -161,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ============================================================== TMA producer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     if (lane == 0) {
       uint32_t kv_it = 0, q_cnt[2] = {0, 0};
       bool ok = true;
@@ -209,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
       const uint32_t idO = tc::idesc_bf16_f32(128, D, true);
@@ -301,8 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mma_commit(&bars->mma_drain);
       tc::mbar_wait(&bars->mma_drain, 0, abort, 100000000ull);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+  } else {
     // ============================================================== softmax / epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     const int s = (warp - 4) >> 2;                 // slot
     const int row = 32 * (warp & 3) + lane;        // M-tile row == TMEM lane
     const int wtid = threadIdx.x - 128 - 128 * s;  // 0..127 within the warpgroup
@@ -318,7 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (uint32_t n = 0; ok; ++n) {
       const int u = tc::queue_pop(&bars->queue, n, abort, ok);
-      if (u < 0) break;
+      // warp-uniform outcomes: the warp-collective TMEM accesses must not diverge
+      ok = __all_sync(0xffffffffu, ok);
+      if (__any_sync(0xffffffffu, u < 0)) break;
       int b, g, I;
       unit_coords(p, u, b, g, I);
       const int nkt = I / 2 + 1;
@@ -330,9 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = t < p.N;
         float m_used = -INFINITY, l = 0.0f;
         for (int tau = 0; tau < nkt; ++tau) {
-          if (!(ok = tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort))) break;
+          if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort)))) break;
           ++s_cnt;
           tc::fence_after_sync();
+          // S row from TMEM; keys past the row are masked on the causal diagonal
+          const bool diag = tau == nkt - 1;
+          const int cmax = t - 128 * tau;
           float sv[128];
           {
             uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -348,112 +370,110 @@ __global__ void __launch_bounds__(kThreads, 1)
               sv[64 + i] = __uint_as_float(r2[i]);
               sv[96 + i] = __uint_as_float(r3[i]);
             }
-          }
-          if (tau == nkt - 1) {  // causal diagonal: keys past the row are masked
-            const int cmax = t - 128 * tau;
+            if (diag) {
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (i > cmax) sv[i] = -INFINITY;
-          }
-          float mlo, mhi;
-          {
-            float a[8], bb[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              a[i] = sv[i];
-              bb[i] = sv[64 + i];
+              for (int i = 0; i < 128; ++i)
+                if (i > cmax) sv[i] = -INFINITY;
             }
-#pragma unroll
-            for (int i = 8; i < 64; i += 8)
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                a[j] = fmaxf(a[j], sv[i + j]);
-                bb[j] = fmaxf(bb[j], sv[64 + i + j]);
-              }
-#pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-              for (int j = 0; j < w; ++j) {
-                a[j] = fmaxf(a[j], a[j + w]);
-                bb[j] = fmaxf(bb[j], bb[j + w]);
-              }
-            mlo = a[0];
-            mhi = bb[0];
           }
+          const float2 sc2 = make_float2(sc, sc);
+          // P = exp2(s sc - ms) written to TMEM as bf16 over S; returns the row sum and (three-
+          // input max chains on the ALU, beside the MUFU work) the maxima of the two 64-key
+          // halves, which are the block maxima of blocks 2 tau and 2 tau + 1
+          auto emit_p = [&](float ms, float& mlo, float& mhi) -> float {
+            const float2 nm2 = make_float2(-ms, -ms);
+            float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+            float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float s0 = sv[32 * c + 2 * i], s1 = sv[32 * c + 2 * i + 1];
+                mk[2 * (c >> 1) + (i & 1)] = tc::fmax3(mk[2 * (c >> 1) + (i & 1)], s0, s1);
+                const float2 pv = exp2_pair(tc::ffma2(make_float2(s0, s1), sc2, nm2), 16 * c + i);
+                acc[i & 1] = tc::fadd2(acc[i & 1], pv);
+                pk[i] = tc::pack_bf16x2(pv.x, pv.y);
+              }
+              tc::tmem_st16(tSrow + 16 * c, pk);
+            }
+            mlo = fmaxf(mk[0], mk[1]);
+            mhi = fmaxf(mk[2], mk[3]);
+            const float2 a = tc::fadd2(acc[0], acc[1]);
+            return a.x + a.y;
+          };
+          // The row max is needed first only while the row has none: later tiles compute P
+          // with the running max m_used straight away and find the tile maxima beside it; a row
+          // whose max rose by more than 2^kRescaleLog2 redoes the tile with the new max (rare),
+          // and O is rescaled.  Warp-uniform branches only: TMEM loads and stores are
+          // warp-collective.
+          if (m_used == -INFINITY) m_used = fmaxf(tc::max64(sv), tc::max64(sv + 64));
+          float mlo, mhi;
+          float lt = emit_p(m_used == -INFINITY ? 0.0f : m_used * sc, mlo, mhi);
           if (scores_on) *reinterpret_cast<float2*>(stash + (size_t)row * p.NBpad + 2 * tau) = make_float2(mlo, mhi);
           const float mt_ = fmaxf(mlo, mhi);
           float alpha = 1.0f;
           const bool rescale = (mt_ - m_used) * sc > kRescaleLog2;
-          if (rescale) {
-            alpha = exp2f((m_used - mt_) * sc);
-            l *= alpha;
-            m_used = mt_;
-          }
-          const float ms = m_used * sc;
-          float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              // the first kPolyCols columns of each row use the FMA-pipe exp2, the rest MUFU
-              const float x0 = fmaf(sv[32 * c + 2 * i], sc, -ms);
-              const float x1 = fmaf(sv[32 * c + 2 * i + 1], sc, -ms);
-              const bool poly = 32 * c + 2 * i < kPolyCols;
-              const float p0 = poly ? tc::exp2_poly3(x0) : exp2f(x0);
-              const float p1 = poly ? tc::exp2_poly3(x1) : exp2f(x1);
-              ls[i & 3] += p0 + p1;
-              pk[i] = tc::pack_bf16x2(p0, p1);
+          if (__any_sync(0xffffffffu, rescale)) {
+            if (rescale) {
+              alpha = exp2f((m_used - mt_) * sc);
+              m_used = mt_;
             }
-            tc::tmem_st16(tSrow + 16 * c, pk);
-          }
-          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-          if (rescale && tau > 0) {
-            // O_s holds the sum over the earlier key tiles; its last PV is complete because
-            // S_s(tau), committed after it, is.  PV_s(tau) waits for p_full below.
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tc::tmem_ld32(tOrow + 32 * c, ov);
+            float u0, u1;
+            lt = emit_p(m_used * sc, u0, u1);   // unchanged rows write the same P again
+            if (tau > 0) {
+              // O_s holds the sum over the earlier key tiles; its last PV is complete because
+              // S_s(tau), committed after it, is.  PV_s(tau) waits for p_full below.
+              uint32_t ov[D];
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
               tc::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tc::tmem_st32(tOrow + 32 * c, ov);
+              for (int i = 0; i < D; i += 2) {
+                const float2 v = tc::fmul2(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(alpha, alpha));
+                ov[i] = __float_as_uint(v.x);
+                ov[i + 1] = __float_as_uint(v.y);
+              }
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) tc::tmem_st32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
             }
           }
+          l = l * alpha + lt;
           tc::tmem_wait_st();
           tc::fence_before_sync();
           tc::mbar_arrive(&bars->p_full[s]);
         }
         if (!ok) break;
         // ---- M-tile epilogue: O / l -> global, LSE, block-score contribution
-        if (!(ok = tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort))) break;
+        if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort)))) break;
         ++o_cnt;
         tc::fence_after_sync();
         const float il = 1.0f / l;
         __nv_bfloat16* orow = p.o + (((size_t)b * p.Hq + h) * p.N + t) * D;
+        uint32_t pk[D / 2];
+        {
+          uint32_t ov[D];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tc::tmem_ld32(tOrow + 32 * c, ov);
+          for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
           tc::tmem_wait_ld();
-          if (valid) {
-            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = tc::pack_bf16x2(__uint_as_float(ov[2 * i]) * il, __uint_as_float(ov[2 * i + 1]) * il);
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < D / 2; ++i) {
+            const float2 v = tc::fmul2(make_float2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1])), make_float2(il, il));
+            pk[i] = tc::pack_bf16x2(v.x, v.y);
           }
         }
         tc::fence_before_sync();
-        tc::mbar_arrive(&bars->o_empty[s]);
+        tc::mbar_arrive(&bars->o_empty[s]);  // O may be overwritten by the next round from here on
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
         if (p.lse != nullptr && valid) p.lse[((size_t)b * p.Hq + h) * p.N + t] = (m_used * sc + log2f(l)) * 0.69314718055994531f;
         if (scores_on) {
           row_m[row] = m_used;
           row_il[row] = valid ? il : 0.0f;
-          if (!(ok = group_sync(&bars->wg[s], wg_ph, abort))) break;
+          if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->wg[s], wg_ph, abort)))) break;
           for (int j = wtid; j <= I; j += 128) {
             float a = 0.0f;
             for (int rr = 0; rr < 128; ++rr) {
@@ -462,13 +482,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             acc[j] = p.red_max ? fmaxf(acc[j], a) : acc[j] + a;
           }
-          if (!(ok = group_sync(&bars->wg[s], wg_ph, abort))) break;
+          if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->wg[s], wg_ph, abort)))) break;
         }
       }
       if (!ok) break;
       if (scores_on) {
         // ---- unit epilogue: both slots' accumulators -> scores[b,g,I,:]
-        if (!(ok = group_sync(&bars->all[0], all_ph, abort))) break;
+        if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->all[0], all_ph, abort)))) break;
         float* out = p.scores + (((size_t)b * p.Hkv + g) * p.T + I) * p.NB;
         const int tid2 = wtid + 128 * s;
         for (int j = tid2; j < p.NB; j += 256) {
@@ -476,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j <= I) v = p.red_max ? fmaxf(acc_all[j], acc_all[kMaxNB + j]) : acc_all[j] + acc_all[kMaxNB + j];
           out[j] = v;
         }
-        if (!(ok = group_sync(&bars->all[0], all_ph, abort))) break;
+        if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->all[0], all_ph, abort)))) break;
         for (int j = wtid; j <= I; j += 128) acc[j] = 0.0f;
       }
     }
@@ -551,6 +571,14 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
+  static int regs = -1;   // the register split assumes exactly kLaunchRegs per thread at launch
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa, full_attn_tc_kernel<D>);
+    if (e0 != cudaSuccess) return e0;
+    regs = fa.numRegs;
+  }
+  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(full_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);

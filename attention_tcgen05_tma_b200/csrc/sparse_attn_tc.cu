@@ -31,10 +31,26 @@ namespace hys {
 namespace {
 
 constexpr int kThreads = 384;
+// Register split between the warpgroups (setmaxnreg): the launch gives every thread
+// kLaunchRegs; the producer/MMA warpgroup drops to kLowRegs and each softmax warpgroup rises to
+// kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
+// the host checks the compiled register count before every launch.
+constexpr int kLaunchRegs = 168, kLowRegs = 88, kHighRegs = 208;
+static_assert(kLowRegs + 2 * kHighRegs == 3 * kLaunchRegs, "register split must match the launch allocation");
 constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;
 constexpr int kMaxKb = 1024;
 constexpr float kRescaleLog2 = 8.0f;
+#ifndef HYS_SPARSE_POLY_PAIRS
+#define HYS_SPARSE_POLY_PAIRS 8
+#endif
+// column pairs (of the 64 in a 128-key row) whose exp2 runs on the FMA pipe instead of MUFU
+constexpr int kPolyPairs = HYS_SPARSE_POLY_PAIRS;
+
+__device__ __forceinline__ float2 exp2_pair(float2 x, int i) {
+  if ((i * kPolyPairs) % 64 < kPolyPairs) return tc::exp2_poly3_x2(x);
+  return make_float2(exp2f(x.x), exp2f(x.y));
+}
 
 
 struct Params {
@@ -160,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ============================================================== TMA producer (gather)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     // The whole warp reads a unit's index row (32 entries per step) and finds the leading
     // valid entries with a ballot; lane 0 then issues the Q and gathered K/V loads.
     int* plist = reinterpret_cast<int*>(smem + C::kOffList);
@@ -257,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
       const uint32_t idO = tc::idesc_bf16_f32(128, D, true);
@@ -359,8 +377,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mma_commit(&bars->mma_drain);
       tc::mbar_wait(&bars->mma_drain, 0, abort, 100000000ull);
     }
+  } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
   } else if (warp >= 4) {
     // ============================================================== softmax / gate epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     const int s = (warp - 4) >> 2;
     const int row = 32 * (warp & 3) + lane;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
@@ -372,7 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (uint32_t n = 0; ok; ++n) {
       int nsel = 0, diag = -1;
       const int u = tc::queue_pop(&bars->queue, n, abort, ok, &nsel, &diag);
-      if (u < 0) break;
+      // warp-uniform outcomes: the warp-collective TMEM accesses must not diverge
+      ok = __all_sync(0xffffffffu, ok);
+      if (__any_sync(0xffffffffu, u < 0)) break;
       const Unit x = make_unit(p, u, nsel, diag);
       const int ntiles = num_tiles(x);
       for (int r = 0; r < rounds && ok; ++r) {
@@ -392,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float pw = 0.0f;                      // sigmoid(g1) / l' for the window P.V pass
         for (int tau = 0; tau < ntiles; ++tau) {
           const int kind = tile_kind(x, tau);
-          if (!(ok = tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort))) break;
+          if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort)))) break;
           ++s_cnt;
           tc::fence_after_sync();
           if (tau == x.n_sp && x.n_sp > 0) {
@@ -433,44 +456,62 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          // S row from TMEM in two batches: the first half is masked and reduced while the
-          // second is in flight
+          // S row from TMEM (masked per half)
           float sv[128];
-          float mx;
           {
             uint32_t r0[32], r1[32], r2[32], r3[32];
             tc::tmem_ld32(tSrow + 0, r0);
             tc::tmem_ld32(tSrow + 32, r1);
-            tc::tmem_wait_ld();
             tc::tmem_ld32(tSrow + 64, r2);
             tc::tmem_ld32(tSrow + 96, r3);
+            tc::tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               sv[i] = __uint_as_float(r0[i]);
               sv[32 + i] = __uint_as_float(r1[i]);
-            }
-            if (clo[0] > 0 || chi[0] < 63) {
-#pragma unroll
-              for (int i = 0; i < 64; ++i)
-                if (i < clo[0] || i > chi[0]) sv[i] = -INFINITY;
-            }
-            const float m0 = tc::max64(sv);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
               sv[64 + i] = __uint_as_float(r2[i]);
               sv[96 + i] = __uint_as_float(r3[i]);
             }
-            if (clo[1] > 0 || chi[1] < 63) {
 #pragma unroll
-              for (int i = 0; i < 64; ++i)
-                if (i < clo[1] || i > chi[1]) sv[64 + i] = -INFINITY;
+            for (int hh = 0; hh < 2; ++hh) {
+              if (clo[hh] > 0 || chi[hh] < 63) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                  if (i < clo[hh] || i > chi[hh]) sv[64 * hh + i] = -INFINITY;
+              }
             }
-            mx = fmaxf(m0, tc::max64(sv + 64));
           }
           const float2 sc2 = make_float2(sc, sc);
-          if (kind == kWinStats) {
+          // P = exp2(s sc - ms) for the whole row, written to TMEM as bf16 over S; returns the
+          // row sum and (three-input max chains on the ALU, beside the MUFU work) the row max
+          auto emit_p = [&](float ms, float& rmax) -> float {
+            const float2 nm2 = make_float2(-ms, -ms);
+            float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+            float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float s0 = sv[32 * c + 2 * i], s1 = sv[32 * c + 2 * i + 1];
+                mk[i & 3] = tc::fmax3(mk[i & 3], s0, s1);
+                const float2 pv = exp2_pair(tc::ffma2(make_float2(s0, s1), sc2, nm2), 16 * c + i);
+                acc[i & 1] = tc::fadd2(acc[i & 1], pv);
+                pk[i] = tc::pack_bf16x2(pv.x, pv.y);
+              }
+              tc::tmem_st16(tSrow + 16 * c, pk);
+            }
+            rmax = tc::fmax3(fmaxf(mk[0], mk[1]), mk[2], mk[3]);
+            const float2 a = tc::fadd2(acc[0], acc[1]);
+            return a.x + a.y;
+          };
+          if (kind == kWinPV) {
+            // window P.V pass with the final statistics; pw holds the combined exponent offset
+            float unused;
+            emit_p(pw, unused);
+          } else if (kind == kWinStats) {
             // window statistics only: running max and sum, no P, no P.V
+            const float mx = fmaxf(tc::max64(sv), tc::max64(sv + 64));
             if (mx > mw) {
               lw = (mw == -INFINITY) ? 0.0f : lw * exp2f((mw - mx) * sc);
               mw = mx;
@@ -481,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
               const float2 xv = tc::ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sc2, nm2);
-              acc[i & 1] = tc::fadd2(acc[i & 1], make_float2(exp2f(xv.x), exp2f(xv.y)));
+              acc[i & 1] = tc::fadd2(acc[i & 1], exp2_pair(xv, i));
             }
             const float2 a = tc::fadd2(acc[0], acc[1]);
             lw += a.x + a.y;
@@ -490,59 +531,40 @@ __global__ void __launch_bounds__(kThreads, 1)
               pw = lw > 0.0f ? g1 / lw : 0.0f;
               pw = (mw == -INFINITY ? 0.0f : mw * sc) - __log2f(pw);
             }
-          } else if (kind == kWinPV) {
-            // window P.V pass with the final statistics; pw holds the combined exponent offset
-            const float2 nm2 = make_float2(-pw, -pw);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t pk[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float2 xv = tc::ffma2(make_float2(sv[32 * c + 2 * i], sv[32 * c + 2 * i + 1]), sc2, nm2);
-                pk[i] = tc::pack_bf16x2(exp2f(xv.x), exp2f(xv.y));
-              }
-              tc::tmem_st16(tSrow + 16 * c, pk);
-            }
           } else {
+            // Sparse tile.  The row max is needed first only while the row has none: later
+            // tiles compute P with the running max m_used straight away and find the tile max
+            // beside it; a row whose max rose by more than 2^kRescaleLog2 redoes the tile with
+            // the new max (rare), and O is rescaled.  Warp-uniform branches only: the TMEM
+            // loads and stores are warp-collective.
+            if (m_used == -INFINITY) m_used = fmaxf(tc::max64(sv), tc::max64(sv + 64));
+            float mx;
+            float lt = emit_p(m_used == -INFINITY ? 0.0f : m_used * sc, mx);
             float alpha = 1.0f;
-            bool rescale = false;
-            if (mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2) {
-              rescale = true;
-              alpha = exp2f((m_used - mx) * sc);
-              l *= alpha;
-              m_used = mx;
-            }
-            const float ms = m_used == -INFINITY ? 0.0f : m_used * sc;
-            const float2 nm2 = make_float2(-ms, -ms);
-            float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t pk[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float2 xv = tc::ffma2(make_float2(sv[32 * c + 2 * i], sv[32 * c + 2 * i + 1]), sc2, nm2);
-                const float2 pv = make_float2(exp2f(xv.x), exp2f(xv.y));
-                acc[i & 1] = tc::fadd2(acc[i & 1], pv);
-                pk[i] = tc::pack_bf16x2(pv.x, pv.y);
+            const bool rescale = mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2;
+            if (__any_sync(0xffffffffu, rescale)) {
+              if (rescale) {
+                alpha = exp2f((m_used - mx) * sc);
+                m_used = mx;
               }
-              tc::tmem_st16(tSrow + 16 * c, pk);
-            }
-            const float2 a = tc::fadd2(acc[0], acc[1]);
-            l += a.x + a.y;
-            if (rescale && tau > 0) {
-              uint32_t ov[D];
+              float unused;
+              lt = emit_p(m_used * sc, unused);   // unchanged rows write the same P again
+              if (tau > 0) {
+                uint32_t ov[D];
 #pragma unroll
-              for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
-              tc::tmem_wait_ld();
+                for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
+                tc::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < D; i += 2) {
-                const float2 v = tc::fmul2(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(alpha, alpha));
-                ov[i] = __float_as_uint(v.x);
-                ov[i + 1] = __float_as_uint(v.y);
+                for (int i = 0; i < D; i += 2) {
+                  const float2 v = tc::fmul2(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(alpha, alpha));
+                  ov[i] = __float_as_uint(v.x);
+                  ov[i + 1] = __float_as_uint(v.y);
+                }
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) tc::tmem_st32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
               }
-#pragma unroll
-              for (int c = 0; c < D / 32; ++c) tc::tmem_st32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
             }
+            l = l * alpha + lt;
           }
           tc::tmem_wait_st();
           tc::fence_before_sync();
@@ -550,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         // ---- epilogue: O already holds sigmoid(g0) o~ + sigmoid(g1) o'
-        if (!(ok = tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort))) break;
+        if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort)))) break;
         ++o_cnt;
         tc::fence_after_sync();
         __nv_bfloat16* orow = p.o + (((size_t)x.b * p.Hq + h) * p.N + t) * D;
@@ -640,6 +662,14 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
+  static int regs = -1;   // the register split assumes exactly kLaunchRegs per thread at launch
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<D>);
+    if (e0 != cudaSuccess) return e0;
+    regs = fa.numRegs;
+  }
+  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);

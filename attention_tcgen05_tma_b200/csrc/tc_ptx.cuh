@@ -252,19 +252,33 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return f2_unpack(d);
 }
 
-// max of 64 consecutive values (four independent chains of three-input max)
+// max of 64 consecutive values (eight independent chains of three-input max)
 __device__ __forceinline__ float max64(const float* v) {
-  float a0 = v[0], a1 = v[1], a2 = v[2], a3 = v[3];
+  float a[8];
 #pragma unroll
-  for (int i = 4; i + 8 <= 64; i += 8) {
-    a0 = fmax3(a0, v[i], v[i + 4]);
-    a1 = fmax3(a1, v[i + 1], v[i + 5]);
-    a2 = fmax3(a2, v[i + 2], v[i + 6]);
-    a3 = fmax3(a3, v[i + 3], v[i + 7]);
-  }
-  a0 = fmax3(a0, v[60], v[61]);
-  a1 = fmax3(a1, v[62], v[63]);
-  return fmax3(fmaxf(a0, a1), a2, a3);
+  for (int j = 0; j < 8; ++j) a[j] = v[j];
+#pragma unroll
+  for (int i = 8; i < 56; i += 16)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] = fmax3(a[j], v[i + j], v[i + 8 + j]);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = fmaxf(a[j], v[56 + j]);
+  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// 2^x for a pair on the FMA/ALU pipes (the MUFU pipe is the softmax's bottleneck): the same
+// Remez degree-3 construction as exp2_poly3, with the fp32 steps done as .f32x2 pairs.
+__device__ __forceinline__ float2 exp2_poly3_x2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(12582912.0f, 12582912.0f));        // round(x) in the low bits
+  const float2 u = fadd2(t, make_float2(-12582912.0f, -12582912.0f));      // round(x)
+  const float2 f = ffma2(u, make_float2(-1.0f, -1.0f), x);                  // x - round(x)
+  float2 q = ffma2(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111251f, 0.2426111251f));
+  q = ffma2(q, f, make_float2(0.6932609677f, 0.6932609677f));
+  q = ffma2(q, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 }  // namespace tc

@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (uint32_t n = 0; ok; ++n) {
       const int u = tc::queue_pop(&bars->queue, n, abort, ok);
-      if (u < 0) break;
+      ok = __all_sync(0xffffffffu, ok);   // warp-uniform: TMEM accesses are warp-collective
+      if (__any_sync(0xffffffffu, u < 0)) break;
       int b, g, I;
       unit_coords(p, u, b, g, I);
       const int nkt = I / 2 + 1;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < rounds && ok; ++r) {
         for (int tau = 0; tau < nkt; ++tau) {
           const uint32_t buf = d_cnt & 1u;
-          if (!(ok = tc::mbar_wait(&bars->d_full[buf], (d_cnt >> 1) & 1u, abort))) break;
+          if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->d_full[buf], (d_cnt >> 1) & 1u, abort)))) break;
           ++d_cnt;
           tc::fence_after_sync();
           uint32_t v0[32], v1[32];
@@ -325,7 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (uint32_t n = 0; ok; ++n) {
       const int u = tc::queue_pop(&bars->queue, n, abort, ok);
-      if (u < 0) break;
+      ok = __all_sync(0xffffffffu, ok);   // warp-uniform: TMEM accesses are warp-collective
+      if (__any_sync(0xffffffffu, u < 0)) break;
       int b, g, I;
       unit_coords(p, u, b, g, I);
       const int nkt = I / 2 + 1;
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // p * 2^12 = exp2(s * sc - LSE_t * log2(e) + 12); invalid rows contribute nothing
         const float bias = valid ? kPScaleLog2 - p.lse[((size_t)b * p.Hq + h) * p.N + t] * kLog2e : -INFINITY;
         for (int tau = 0; tau < nkt; ++tau) {
-          if (!(ok = tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort))) break;
+          if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort)))) break;
           ++s_cnt;
           tc::fence_after_sync();
           uint32_t r0[32], r1[32], r2[32], r3[32];

@@ -344,7 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (uint32_t n = 0; ok; ++n) {
       int nA = 0, unused = 0;
       const int u = tc::queue_peek(&bars->queue, n, abort, ok, &nA, &unused);
-      if (u < 0) break;
+      ok = __all_sync(0xffffffffu, ok);   // warp-uniform: TMEM accesses are warp-collective
+      if (__any_sync(0xffffffffu, u < 0)) break;
       const Unit x = make_unit(p, u, nA);
       const uint32_t* mask = bars->selmask[n % tc::kQueueSlots];
       const int ntiles = x.n_sp + x.n_w;
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = t < p.N;
         float m_used = -INFINITY, l = 0.0f;
         for (int tau = 0; tau < ntiles; ++tau) {
-          if (!(ok = tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort))) break;
+          if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort)))) break;
           ++s_cnt;
           tc::fence_after_sync();
           float sv[128];
@@ -436,7 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tmem_st16(tSrow + 16 * c, pk);
           }
           l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-          if (rescale && tau > 0) {
+          // warp-uniform: the TMEM loads and stores are warp-collective; rows that keep their
+          // max scale by alpha = 1
+          if (__any_sync(0xffffffffu, rescale && tau > 0)) {
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
               uint32_t ov[32];
@@ -452,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mbar_arrive(&bars->p_full[s]);
         }
         if (!ok) break;
-        if (!(ok = tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort))) break;
+        if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort)))) break;
         ++o_cnt;
         tc::fence_after_sync();
         const float il = l > 0.0f ? 1.0f / l : 0.0f;
