@@ -15,6 +15,7 @@ data-path collective); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -30,6 +31,38 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from attention_tcgen05_tma_b200.distributed import max_over_ranks  # noqa: E402
+
+# DRAM traffic of the dominant prefill kernel from one ncu capture (profiles/
+# sparse_attn_tc_moe80b_small.md): dram__bytes_read.sum + dram__bytes_write.sum of one launch on
+# the moe80b_small workload, the work units (batch, KV group, 64-query tile) that launch
+# processed, and a digest of the kernel's sources at capture time.  Every term of the traffic
+# (Q', O, gate, K'/V', the gathered blocks) grows with the units, so the bench scales the bytes
+# to its own units; it reports null once the sources differ from the captured ones.
+NCU_TRAFFIC = {
+    "sparse_attn": {"bytes": 199.251968e6 + 98.007808e6, "units": 1024,
+                    "sources": ("sparse_attn_tc.cu", "tc_ptx.cuh", "common.cuh", "kernels.h"),
+                    "sha256": "2e5052aa97cef6de7cf0c2a7ea647a36d7f1e4e63b7e69e8def3cd9a0c241c40"},
+}
+
+
+def ncu_traffic(kernel, units):
+    """Bytes per launch from the recorded capture scaled to `units`, or None when the kernel's
+    sources changed since the counters were taken."""
+    rec = NCU_TRAFFIC.get(kernel)
+    if rec is None:
+        return None
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "attention_tcgen05_tma_b200", "csrc")
+    h = hashlib.sha256()
+    try:
+        for f in rec["sources"]:
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    if h.hexdigest() != rec["sha256"]:
+        return None
+    return round(rec["bytes"] * units / rec["units"])
+
 
 METRIC = "hybrid-block prefill tokens/s @32K and decode µs/token; % of tensor/HBM roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -274,7 +307,10 @@ def run_ours(args, torch, dist, rank, world, dev):
                 "unit": "TFLOP/s", "frac": round(full_tf / peak_tf, 4), "traffic": None}
     else:
         roof = {"kernel": "sparse_attn", "bound": "tensor", "achieved": round(sp_tf, 2), "peak": peak_tf,
-                "unit": "TFLOP/s", "frac": round(sp_tf / peak_tf, 4), "traffic": None}
+                "unit": "TFLOP/s", "frac": round(sp_tf / peak_tf, 4),
+                "traffic": ncu_traffic("sparse_attn", w.B * w.Hkv * w.T)}
+        if roof["traffic"] is not None:
+            roof["traffic_source"] = "ncu dram bytes of one moe80b_small launch, scaled by work units"
     roof["peak_source"] = f"{peak_src} bf16_tflops_sustained"
     kernels = {
         "full_attn_select_ms": round(full_ms, 4), "full_attn_select_tflops": round(full_tf, 2),
