@@ -64,6 +64,7 @@ struct Params {
   int B, N, Hq, Hkv, G, T, NB, NBpad;
   int num_units;
   __nv_bfloat16* o;
+  int o_v8;       // o is 32-byte aligned (256-bit stores)
   float* lse;     // optional [B,Hq,N]
   float* scores;  // optional [B,Hkv,T,NB] (block scores are emitted iff non-null)
   float* stash;   // [grid][2][128][NBpad]
@@ -465,9 +466,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         tc::mbar_arrive(&bars->o_empty[s]);  // O may be overwritten by the next round from here on
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
+          if (p.o_v8) {  // 32-byte aligned output: 256-bit stores, full sectors
 #pragma unroll
-          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < D / 16; ++i) tc::st_global_v8(orow + 16 * i, pk + 8 * i);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
         }
         if (p.lse != nullptr && valid) p.lse[((size_t)b * p.Hq + h) * p.N + t] = (m_used * sc + log2f(l)) * 0.69314718055994531f;
         if (scores_on) {
@@ -563,6 +569,7 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.NBpad = nb_pad(d.NB);
   p.num_units = num_units(d);
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   p.lse = lse;
   p.scores = scores;
   p.counter = reinterpret_cast<int*>(ws);

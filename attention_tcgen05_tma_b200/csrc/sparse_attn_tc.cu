@@ -59,6 +59,7 @@ struct Params {
   const int* idx;      // [B,Hkv,T,kb]
   const float* gate;   // [B,Hq,N,2]
   __nv_bfloat16* o;
+  int o_v8;            // o is 32-byte aligned (256-bit stores)
   int* counter;        // work-unit counter (zeroed before the launch)
   int* status;
   float scale_log2;
@@ -404,12 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = x.g * p.G + 2 * mt + (row >> 6);
         const int t = 64 * x.I + (row & 63);
         const bool valid = t < p.N;
-        float g0 = 0.0f, g1 = 0.0f;
-        if (valid) {
-          const float2 gl = *reinterpret_cast<const float2*>(p.gate + (((size_t)x.b * p.Hq + h) * p.N + t) * 2);
-          g0 = sigmoidf_(gl.x);
-          g1 = sigmoidf_(gl.y);
-        }
+        // gate logits: loaded here, used at the branch switch and after the window statistics,
+        // so the load latency hides behind the first tiles
+        float2 gl = make_float2(-INFINITY, -INFINITY);
+        if (valid) gl = *reinterpret_cast<const float2*>(p.gate + (((size_t)x.b * p.Hq + h) * p.N + t) * 2);
         float m_used = -INFINITY, l = 0.0f;   // online state of the sparse branch
         float mw = -INFINITY, lw = 0.0f;      // window branch statistics
         float pw = 0.0f;                      // sigmoid(g1) / l' for the window P.V pass
@@ -421,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tau == x.n_sp && x.n_sp > 0) {
             // the sparse branch is complete in O (its last P.V finished before this S did):
             // scale O in place to sigmoid(g0) * o~
-            const float f = l > 0.0f ? g0 / l : 0.0f;
+            const float f = l > 0.0f ? sigmoidf_(gl.x) / l : 0.0f;
             uint32_t ov[D];
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
@@ -528,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             lw += a.x + a.y;
             if (tau == x.n_sp + x.n_sw - 1) {
               // P' = exp2((s - m') sc) * sigmoid(g1) / l' = exp2(s sc - (m' sc - log2(sigmoid(g1) / l')))
-              pw = lw > 0.0f ? g1 / lw : 0.0f;
+              pw = lw > 0.0f ? sigmoidf_(gl.y) / lw : 0.0f;
               pw = (mw == -INFINITY ? 0.0f : mw * sc) - __log2f(pw);
             }
           } else {
@@ -588,9 +587,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         tc::mbar_arrive(&bars->o_empty[s]);  // O may be overwritten by the next round from here on
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
+          if (p.o_v8) {  // 32-byte aligned output: 256-bit stores, full sectors
 #pragma unroll
-          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < D / 16; ++i) tc::st_global_v8(orow + 16 * i, pk + 8 * i);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
         }
       }
     }
@@ -658,6 +662,7 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.idx = idx;
   p.gate = gate;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   p.counter = reinterpret_cast<int*>(ws);
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);

@@ -212,6 +212,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 32 bytes to global memory in one instruction (sm_100 256-bit store); ptr 32-byte aligned
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // ------------------------------------------------------------------ sm_100 fp32 pair / 3-input ops
 // The FMA pipe of sm_100 executes fp32 pairs (fma/add/mul .f32x2) in one instruction, and max
 // takes three operands; softmax rows use them to halve their FMA-pipe instruction count.

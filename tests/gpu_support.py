@@ -25,6 +25,19 @@ def to_dev(x: np.ndarray, dtype: str, device="cuda"):
     return t.to(device)
 
 
+def device_fill(shape, fn, keys, bf16: bool = True, device="cuda"):
+    """A device tensor filled slice by slice from the seeded generator (slices drawn by a
+    thread pool), the way the benchmark builds its full-size inputs."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    out = torch.empty(shape, dtype=torch.bfloat16 if bf16 else torch.float32, device=device)
+    with ThreadPoolExecutor(min(32, os.cpu_count() or 8)) as ex:
+        for key, arr in ex.map(lambda key: (key, fn(*key)), keys):
+            t = torch.from_numpy(np.ascontiguousarray(arr))
+            out[key].copy_(t.to(torch.bfloat16) if bf16 else t)
+    return out
+
+
 def to_np(t) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 

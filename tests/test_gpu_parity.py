@@ -98,6 +98,28 @@ def test_share_both_ablation_aliasing():
     assert np.max(np.abs(to_np(osp) - ref)) <= TOL["bf16"]
 
 
+def test_output_alignment_16_bytes():
+    """Output rows at a 16-byte (not 32-byte) aligned address take the 128-bit store path of the
+    tensor-core kernels; the values match the aligned call's exactly."""
+    w = _workload("bf16", 1, 700, 8, 2, 128, 4, 128)
+    a = I.prefill_arrays(w, layers=1)
+    q, kk, vv = (to_dev(a[x], "bf16") for x in ("q", "k", "v"))
+    o_al, sc = H.full_attn_select(q, kk, vv)
+    buf = torch.empty(q.numel() + 8, dtype=q.dtype, device=q.device)
+    o_un = buf[8:].view(q.shape)                      # 16 bytes past a 256-byte aligned base
+    assert o_un.data_ptr() % 32 == 16
+    H.full_attn_select(q, kk, vv, o=o_un, scores=torch.empty_like(sc))
+    idx = H.topk(sc, 4)
+    qs, gate = to_dev(a["q_sparse"][0], "bf16"), to_dev(a["gate"][0], "f32")
+    ks, vs = to_dev(a["k_swa"][0], "bf16"), to_dev(a["v_swa"][0], "bf16")
+    s_al = H.sparse_attn(qs, kk, vv, idx, ks, vs, 128, gate)
+    buf2 = torch.empty(qs.numel() + 8, dtype=qs.dtype, device=qs.device)
+    s_un = buf2[8:].view(qs.shape)
+    H.sparse_attn(qs, kk, vv, idx, ks, vs, 128, gate, o=s_un)
+    torch.cuda.synchronize()
+    assert torch.equal(o_al, o_un) and torch.equal(s_al, s_un)
+
+
 TOKEN_CASES = [
     ("bf16_d128", "bf16", 1, 700, 8, 2, 128, 100, 128),
     ("bf16_d64_small_forced", "bf16", 1, 300, 4, 1, 64, 40, 16),
