@@ -3,12 +3,14 @@
 // against the cache, top-k of the old blocks, then the sparse followers; HySparse 3.4.1
 // block scores and 3.4.3 sparse/SWA/gate for one query row.)
 //
-// One CTA = (split, KV group g, sequence b): 6 consumer warps + 1 TMA producer warp.  The
+// One CTA = (split, KV group g, sequence b): C consumer warps + 1 TMA producer warp (C = 3,
+// so two CTAs share an SM and one's start-up and drain overlap the other's streaming).  The
 // producer streams 64-key blocks of K and V (two 128-byte-swizzled TMA boxes each per
-// tensor, 32 KB per block) into 6 stages; consumer warp w owns stage w and takes blocks
-// w, w+6, ... of the split, so every stage's barrier phases are consumed by one warp in
+// tensor, 32 KB per block) into C stages; consumer warp w owns stage w and takes blocks
+// w, w+C, ... of the split, so every stage's barrier phases are consumed by one warp in
 // order (a parity wait cannot be fooled by a phase two ahead) and the max logit of a
-// block (HySparse's m~) is a warp-local reduction.
+// block (HySparse's m~) is a warp-local reduction.  A sparse layer's split holds 16 of the
+// selected blocks; its SWA ring is a split of its own.
 // The G <= 16 query heads of the group form the 16 rows of mma.sync.m16n8k16 tiles
 // (zero-padded): S = Q K^T (64 mma per block), online softmax in registers, O += P V (64
 // mma per block).  The warps' partial (m, l, O) are merged in shared memory (reusing the stages) and the
@@ -26,7 +28,11 @@ namespace hys {
 
 namespace {
 
-constexpr int kConsumers = 6;
+#ifndef HYS_DECODE_CONSUMERS
+#define HYS_DECODE_CONSUMERS 3
+#endif
+constexpr int kConsumers = HYS_DECODE_CONSUMERS;
+constexpr int kCtasPerSm = kConsumers <= 3 ? 2 : 1;   // two CTAs share an SM when they fit
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = kConsumers;              // stage w belongs to consumer warp w
 constexpr int kStageBytes = 2 * 64 * 128 * 2;   // K + V of one 64-key block, D = 128
@@ -35,6 +41,11 @@ constexpr int kPartBytes = kConsumers * 16 * (128 + 2) * 4;
 static_assert(kPartBytes <= kStages * kStageBytes, "partials reuse the stage buffers");
 constexpr int kSmemBytes = kStages * kStageBytes + kMaxList * 16 + 256 + 1024;
 constexpr int kTargetCtas = 4 * 148;
+#ifndef HYS_DECODE_SPARSE_BPS
+#define HYS_DECODE_SPARSE_BPS 16
+#endif
+constexpr int kSparseBps = HYS_DECODE_SPARSE_BPS;   // selected blocks per sparse-layer split (<= 32)
+static_assert(kSparseBps <= 32 && kSparseBps <= kMaxList, "one warp gathers a split's entries");
 
 struct Params {
   int B, L, Hq, Hkv, G, NB;
@@ -85,7 +96,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // byte offset of (row, 16-byte unit) inside a [64 rows][128 B] 128-byte-swizzled box
 __device__ __forceinline__ uint32_t sw128(int row, int unit) { return row * 128 + ((unit ^ (row & 7)) << 4); }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
                         const Params p) {
@@ -102,24 +113,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Lb = p.seqlens ? max(1, min(p.seqlens[b], p.L)) : p.L;
 
+  if (p.mode == 1 && sp < p.nsp) {
+    // this split's selected blocks: warp 0 reads the index entries at once and keeps the
+    // valid ones in order (ballot + prefix count)
+    if (warp == 0) {
+      const int nb = (Lb + 63) / 64;
+      const int* sel = p.idx + ((size_t)b * p.Hkv + g) * p.kb;
+      const int e = sp * p.bps + lane;
+      const int j = (lane < p.bps && e < p.kb) ? sel[e] : -1;
+      const bool keep = j >= 0 && j < nb;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) list[__popc(m & ((1u << lane) - 1u))] = Entry{64 * j, min(64, Lb - 64 * j), 0, j};
+      if (lane == 0) *s_nlist = __popc(m);
+    }
+  }
   if (threadIdx.x == 0) {
     // this split's block list
     int n = 0;
     if (p.mode == 0) {
       const int nb = (Lb + 63) / 64;
       for (int j = sp * p.bps; j < min(nb, (sp + 1) * p.bps); ++j) list[n++] = Entry{64 * j, min(64, Lb - 64 * j), 0, j};
-    } else if (sp < p.nsp) {
-      const int nb = (Lb + 63) / 64;
-      const int* sel = p.idx + ((size_t)b * p.Hkv + g) * p.kb;
-      for (int e = sp * p.bps; e < min(p.kb, (sp + 1) * p.bps); ++e) {
-        const int j = sel[e];
-        if (j >= 0 && j < nb) list[n++] = Entry{64 * j, min(64, Lb - 64 * j), 0, j};
-      }
-    } else {
+      *s_nlist = n;
+    } else if (sp >= p.nsp) {
       const int nring = p.swa_len ? max(0, min(p.swa_len[b], p.W)) : p.W;
       for (int j = 0; 64 * j < nring; ++j) list[n++] = Entry{64 * j, min(64, nring - 64 * j), 1, j};
+      *s_nlist = n;
     }
-    *s_nlist = n;
+
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&full[i], 1);
       tc::mbar_init(&empty[i], 1);
@@ -456,7 +476,7 @@ size_t decode_mma_full_workspace(const DecodeDims& d) {
   return sizeof(float) * (np * (2 + 128) + (size_t)d.B * d.Hq * d.NB);
 }
 
-int decode_sparse_splits(int kb) { return (kb + 7) / 8; }
+int decode_sparse_splits(int kb) { return (kb + kSparseBps - 1) / kSparseBps; }
 
 size_t decode_mma_sparse_workspace(const DecodeDims& d, int kb) {
   const size_t nsplit = decode_sparse_splits(kb) + 1;
@@ -497,7 +517,7 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   const int nsp = decode_sparse_splits(kb);
   fill_common(p, d, q, seqlens, ws, nsp + 1);
   p.mode = 1;
-  p.bps = 8;
+  p.bps = kSparseBps;
   p.nsp = nsp;
   p.idx = idx;
   p.kb = kb;
