@@ -20,6 +20,7 @@ the token-level variant and the forced newest-128 window):
 * ``moe80b_small``  the same per-unit shape at B1 N16384 with 2 sparse layers (profiling)
 * ``decode``   bf16, B64, L131072 cached tokens, 32/4, D128, k=32 blocks, 11 sparse layers
 * ``token``    bf16, B1 N131072, 32/4, D128, top-2048 tokens + forced 128, 3 sparse layers
+* ``token_small``  the token variant at N32768 with 1 sparse layer (profiling)
 """
 from __future__ import annotations
 
@@ -89,6 +90,9 @@ WORKLOADS: Dict[str, Workload] = {
     # the moe80b per-unit shape (G=8, k=32) at one sequence of 16K (profiling captures, < 1 GiB)
     "moe80b_small": Workload("moe80b_small", "prefill_block", "bf16", 1, 16384, 32, 4, 128, 2, 32, 128,
                              seed=6, scale_std=1.0 / math.sqrt(128), plant="blocks", n_plants=64),
+    # the token variant at one sequence of 32K (profiling captures: token scores 256 MiB)
+    "token_small": Workload("token_small", "prefill_token", "bf16", 1, 32768, 32, 4, 128, 1, 2048, 128,
+                            seed=7, scale_std=1.0 / math.sqrt(128), plant="blocks", n_plants=64),
     # smaller decode batch with the same per-sequence shape (profiling captures: 2 GiB of cache)
     "decode_small": Workload("decode_small", "decode", "bf16", 8, 131072, 32, 4, 128, 11, 32, 128,
                              seed=5, scale_std=1.0 / math.sqrt(128)),
