@@ -33,6 +33,10 @@ Readings where the pages leave a step open (each is listed in the design notes):
   token once, no gate.
 * Decode: the new token sits at position L-1 of an L-token cache; it is its own
   tile; candidates are all blocks (block variant).
+* Sink biases ([HSP] §4.1, per-head learnable sinks in the sparse and SWA branches,
+  following gpt-oss): one logit per (head, branch), sinks [Hq, 2] with index 0 for
+  the sparse branch and 1 for the SWA branch; it joins the branch's softmax as an
+  extra entry with a zero value, so the denominator gains exp(sink - m).
 
 All arithmetic is float64; inputs are converted exactly (bf16 and fp32 values are
 exactly representable in float64).
@@ -51,15 +55,17 @@ NEG_INF = -np.inf
 # dense causal attention  ([HS] §3.4.1, equation for o_t)
 # -----------------------------------------------------------------------------
 def causal_softmax(q_rows: np.ndarray, t_rows: np.ndarray, k: np.ndarray,
-                   keys_visible: Optional[np.ndarray] = None
+                   keys_visible: Optional[np.ndarray] = None, sink: Optional[float] = None
                    ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Softmax attention probabilities of some query rows against the keys of one head.
 
     q_rows [R, D], t_rows [R] (absolute query positions), k [N, D].
     keys_visible, if given, is a boolean [R, N] mask of the keys each row may see
-    (it is intersected with causality i <= t).
+    (it is intersected with causality i <= t).  sink, if given, is a logit that joins
+    every row's softmax as an extra entry with a zero value.
     Returns P [R, N] (zero where a key is not visible), the row max m [R] of the
-    scaled logits and the normaliser l [R] = sum_i exp(s_i - m).
+    scaled logits (and the sink) and the normaliser l [R] = sum_i exp(s_i - m)
+    (+ exp(sink - m)).
     """
     q_rows = np.asarray(q_rows, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -71,14 +77,18 @@ def causal_softmax(q_rows: np.ndarray, t_rows: np.ndarray, k: np.ndarray,
         visible = visible & keys_visible
     s = np.where(visible, s, NEG_INF)
     m = s.max(axis=1)
+    if sink is not None:
+        m = np.maximum(m, sink)
     e = np.where(visible, np.exp(s - m[:, None]), 0.0)
     l = e.sum(axis=1)
+    if sink is not None:
+        l = l + np.exp(sink - m)
     return e / l[:, None], m, l
 
 
-def attention_rows(q_rows, t_rows, k, v, keys_visible=None):
+def attention_rows(q_rows, t_rows, k, v, keys_visible=None, sink=None):
     """o_t = sum_i P_{t,i} v_i for the given rows; also returns LSE_t = m_t + log l_t."""
-    p, m, l = causal_softmax(q_rows, t_rows, k, keys_visible)
+    p, m, l = causal_softmax(q_rows, t_rows, k, keys_visible, sink)
     o = p @ np.asarray(v, dtype=np.float64)
     return o, m + np.log(l)
 
@@ -192,38 +202,40 @@ def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-np.asarray(x, dtype=np.float64)))
 
 
-def sparse_branch_rows(q_rows, t_rows, k, v, sel_blocks: Sequence[int], block: int = 64):
+def sparse_branch_rows(q_rows, t_rows, k, v, sel_blocks: Sequence[int], block: int = 64, sink=None):
     """Sparse-branch output of rows of one tile: keys i <= t with floor(i/64) in Sel."""
     N = k.shape[0]
     in_sel = np.zeros(N, dtype=bool)
     for j in sel_blocks:
         if j >= 0:
             in_sel[j * block:min(N, (j + 1) * block)] = True
-    o, _ = attention_rows(q_rows, t_rows, k, v, np.broadcast_to(in_sel, (len(t_rows), N)))
+    o, _ = attention_rows(q_rows, t_rows, k, v, np.broadcast_to(in_sel, (len(t_rows), N)), sink)
     return o
 
 
-def swa_branch_rows(q_rows, t_rows, k_swa, v_swa, window: int):
+def swa_branch_rows(q_rows, t_rows, k_swa, v_swa, window: int, sink=None):
     """SWA-branch output: keys in [max(0, t-w+1), t] of the layer's own K', V'."""
     N = k_swa.shape[0]
     i = np.arange(N)[None, :]
     vis = i >= (np.asarray(t_rows)[:, None] - window + 1)
-    o, _ = attention_rows(q_rows, t_rows, k_swa, v_swa, vis)
+    o, _ = attention_rows(q_rows, t_rows, k_swa, v_swa, vis, sink)
     return o
 
 
 def gated_sparse_rows(q_rows, t_rows, k, v, sel_blocks, k_swa, v_swa, window, gate_rows,
-                      block: int = 64):
-    """o_t = sigmoid(g0) * o~_t + sigmoid(g1) * o'_t for rows of one tile."""
-    o_sp = sparse_branch_rows(q_rows, t_rows, k, v, sel_blocks, block)
-    o_sw = swa_branch_rows(q_rows, t_rows, k_swa, v_swa, window)
+                      block: int = 64, sinks=None):
+    """o_t = sigmoid(g0) * o~_t + sigmoid(g1) * o'_t for rows of one tile; sinks, if given,
+    is this head's (sparse-branch, SWA-branch) sink logit pair."""
+    s0, s1 = (None, None) if sinks is None else (float(sinks[0]), float(sinks[1]))
+    o_sp = sparse_branch_rows(q_rows, t_rows, k, v, sel_blocks, block, s0)
+    o_sw = swa_branch_rows(q_rows, t_rows, k_swa, v_swa, window, s1)
     g = sigmoid(gate_rows)
     return g[:, 0:1] * o_sp + g[:, 1:2] * o_sw
 
 
-def sparse_attention(q_s, k, v, idx, k_swa, v_swa, window: int, gate, block: int = 64):
+def sparse_attention(q_s, k, v, idx, k_swa, v_swa, window: int, gate, block: int = 64, sinks=None):
     """Whole sparse layer. q_s [B,Hq,N,D]; k, v, k_swa, v_swa [B,Hkv,N,D];
-    idx [B,Hkv,T,k]; gate [B,Hq,N,2].  Returns o [B,Hq,N,D]."""
+    idx [B,Hkv,T,k]; gate [B,Hq,N,2]; sinks None or [Hq,2].  Returns o [B,Hq,N,D]."""
     B, Hq, N, D = q_s.shape
     G = Hq // k.shape[1]
     T = (N + block - 1) // block
@@ -236,7 +248,8 @@ def sparse_attention(q_s, k, v, idx, k_swa, v_swa, window: int, gate, block: int
             for I in range(T):
                 rows = tile_rows(I, N, block)
                 o[b, h, rows] = gated_sparse_rows(q_s[b, h, rows], rows, kk, vv, idx[b, g, I],
-                                                  ks, vs, window, gate[b, h, rows], block)
+                                                  ks, vs, window, gate[b, h, rows], block,
+                                                  None if sinks is None else sinks[h])
     return o
 
 
@@ -320,12 +333,13 @@ def topk_decode(scores: np.ndarray, k: int, seqlens=None, L: Optional[int] = Non
 
 
 def decode_sparse(q: np.ndarray, k_cache, v_cache, idx, k_ring, v_ring, gate, seqlens=None,
-                  swa_len=None, block: int = 64):
+                  swa_len=None, block: int = 64, sinks=None):
     """One sparse layer for the new token: selected blocks of the shared cache (all keys
     of a selected block that hold cached tokens) plus the layer's own SWA ring of
     swa_len[b] tokens (ring order does not matter: softmax is permutation invariant),
     merged by the sigmoid gate [B,Hq,2].  A branch with no keys (an empty ring, or no
-    selected block holding cached tokens) contributes zero."""
+    selected block holding cached tokens) contributes zero; sinks None or [Hq,2] as in
+    gated_sparse_rows."""
     B, Hq, D = q.shape
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
     G = Hq // Hkv
@@ -342,8 +356,9 @@ def decode_sparse(q: np.ndarray, k_cache, v_cache, idx, k_ring, v_ring, gate, se
             vr = np.asarray(v_ring[b, g, :nring], np.float64)
             for h in range(g * G, (g + 1) * G):
                 qq = np.asarray(q[b, h], np.float64)[None, :]
-                o_sp = attention_rows(qq, np.array([len(keys)]), ks, vs)[0] if len(keys) else np.zeros((1, D))
-                o_sw = attention_rows(qq, np.array([nring]), kr, vr)[0] if nring else np.zeros((1, D))
+                s0, s1 = (None, None) if sinks is None else (float(sinks[h][0]), float(sinks[h][1]))
+                o_sp = attention_rows(qq, np.array([len(keys)]), ks, vs, None, s0)[0] if len(keys) else np.zeros((1, D))
+                o_sw = attention_rows(qq, np.array([nring]), kr, vr, None, s1)[0] if nring else np.zeros((1, D))
                 gg = sigmoid(gate[b, h])
                 o[b, h] = gg[0] * o_sp[0] + gg[1] * o_sw[0]
     return o

@@ -374,6 +374,63 @@ def test_brute_force_decode():
 
 
 # ----------------------------------------------------------------------------- planted mistakes
+def test_sink_closed_forms():
+    """A sink logit b joins the softmax as an extra entry with zero value ([HSP] §4.1, gpt-oss
+    sinks): one visible key gives o = v * sigmoid(s - b); n keys with equal logits give
+    o = mean(v) * n / (n + exp(b - s)); b = -inf is no sink at all."""
+    rng = np.random.default_rng(5)
+    D = 16
+    k = rng.standard_normal((4, D))
+    v = rng.standard_normal((4, D))
+    q = rng.standard_normal((1, D))
+    s0 = float(q[0] @ k[0]) / math.sqrt(D)
+    for b in (-2.0, 0.0, 1.5, 7.0):
+        o, _ = O.attention_rows(q, np.array([0]), k, v, sink=b)
+        want = v[0] / (1.0 + math.exp(b - s0))
+        np.testing.assert_allclose(o[0], want, rtol=1e-12, atol=1e-14)
+    qz = np.zeros((1, D))
+    for b in (-1.0, 0.5, 3.0):
+        o, _ = O.attention_rows(qz, np.array([3]), k, v, sink=b)
+        want = v.mean(axis=0) * 4.0 / (4.0 + math.exp(b))
+        np.testing.assert_allclose(o[0], want, rtol=1e-12, atol=1e-14)
+    o_none, _ = O.attention_rows(q, np.array([3]), k, v)
+    o_inf, _ = O.attention_rows(q, np.array([3]), k, v, sink=-np.inf)
+    np.testing.assert_array_equal(o_none, o_inf)
+
+
+def test_sink_per_branch_and_decode():
+    """sinks[h] = (sparse-branch, SWA-branch) logits: each branch's output shrinks by exactly its
+    own factor l / (l + exp(b - m)); a huge sink silences its branch; decode agrees with the
+    prefill rows of the same keys."""
+    rng = np.random.default_rng(6)
+    N, D = 128, 16
+    k, v, ks, vs = (rng.standard_normal((N, D)) for _ in range(4))
+    q = rng.standard_normal((64, D))
+    rows = np.arange(64, 128)
+    gate = rng.standard_normal((64, 2))
+    base = O.gated_sparse_rows(q, rows, k, v, [0], ks, vs, 32, gate)
+    # huge sparse-branch sink: only the SWA branch remains
+    only_swa = O.gated_sparse_rows(q, rows, k, v, [0], ks, vs, 32, gate, sinks=(1e3, -np.inf))
+    want = O.sigmoid(gate[:, 1:2]) * O.swa_branch_rows(q, rows, ks, vs, 32)
+    np.testing.assert_allclose(only_swa, want, rtol=1e-12, atol=1e-14)
+    # huge SWA sink: only the sparse branch remains
+    only_sp = O.gated_sparse_rows(q, rows, k, v, [0], ks, vs, 32, gate, sinks=(-np.inf, 1e3))
+    want = O.sigmoid(gate[:, 0:1]) * O.sparse_branch_rows(q, rows, k, v, [0])
+    np.testing.assert_allclose(only_sp, want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(O.gated_sparse_rows(q, rows, k, v, [0], ks, vs, 32, gate,
+                                                      sinks=(-np.inf, -np.inf)), base)
+    # decode: the new token at L-1 = the last prefill row, sink factors included
+    L = 128
+    kc, vc = k[None, None], v[None, None]
+    kr, vr = ks[None, None, L - 32:], vs[None, None, L - 32:]
+    qd = q[-1][None, None]
+    g = gate[-1][None, None]
+    sk = np.array([[0.7, -0.3]])
+    od = O.decode_sparse(qd, kc, vc, np.array([[[0, 1]]]), kr, vr, g, sinks=sk)
+    op = O.gated_sparse_rows(q[-1:], np.array([L - 1]), k, v, [0, 1], ks, vs, 32, gate[-1:], sinks=sk[0])
+    np.testing.assert_allclose(od[0, 0], op[0], rtol=1e-12, atol=1e-14)
+
+
 def test_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the oracle and check that a pin above fails."""
     g = _gold()
