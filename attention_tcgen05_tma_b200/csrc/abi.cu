@@ -215,8 +215,8 @@ hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const v
   hys_status st = check_prefill(shape, &d);
   if (st != HYS_OK) return st;
   if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
-  if (sinks) return HYS_ERR_UNSUPPORTED;
   if (!q_sparse || !k_shared || !v_shared || !idx || !k_swa || !v_swa || !gate_logits || !o) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(sinks)) return HYS_ERR_INVALID_ARG;
   if (k < 1 || k > 1024 || window < 1) return HYS_ERR_INVALID_ARG;
   if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(k_swa) ||
       !aligned16(v_swa) || !aligned16(gate_logits) || !aligned16(o) || !aligned16(workspace))
@@ -226,10 +226,10 @@ hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const v
     const size_t need = align256(sparse_attn_tc_workspace(d));
     if (workspace == nullptr || workspace_bytes < need) return HYS_ERR_WORKSPACE;
     return from_cuda(launch_sparse_attn_tc(d, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,
-                                           gate_logits, o, workspace, workspace_bytes, s));
+                                           gate_logits, sinks, o, workspace, workspace_bytes, s));
   }
   return from_cuda(launch_sparse_attn_simt(d, dtype, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,
-                                           gate_logits, o, s));
+                                           gate_logits, sinks, o, s));
 }
 
 hys_status hysparse_sparse_attn_tokens_workspace_size(const hys_shape* shape, hys_dtype dtype, int forced_window,
@@ -328,8 +328,8 @@ hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype 
   hys_status st = check_decode(shape, &d);
   if (st != HYS_OK) return st;
   if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
-  if (sinks) return HYS_ERR_UNSUPPORTED;
   if (!q || !k_cache || !v_cache || !idx || !k_swa_ring || !v_swa_ring || !gate_logits || !o) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(sinks)) return HYS_ERR_INVALID_ARG;
   if (k < 1 || k > 1024 || window < 1 || window > 1024) return HYS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seqlens) || !aligned16(idx) ||
       !aligned16(k_swa_ring) || !aligned16(v_swa_ring) || !aligned16(swa_len) || !aligned16(gate_logits) ||
@@ -339,10 +339,10 @@ hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype 
   if (decode_mma_supported(d, dtype)) {
     if (workspace == nullptr || workspace_bytes < align256(decode_mma_sparse_workspace(d, k))) return HYS_ERR_WORKSPACE;
     return from_cuda(launch_decode_sparse_mma(d, q, k_cache, v_cache, seqlens, idx, k, k_swa_ring, v_swa_ring, window,
-                                              swa_len, gate_logits, o, workspace, s));
+                                              swa_len, gate_logits, sinks, o, workspace, s));
   }
   return from_cuda(launch_decode_sparse(d, dtype, q, k_cache, v_cache, seqlens, idx, k, k_swa_ring, v_swa_ring,
-                                        window, swa_len, gate_logits, o, s));
+                                        window, swa_len, gate_logits, sinks, o, s));
 }
 
 }  // extern "C"

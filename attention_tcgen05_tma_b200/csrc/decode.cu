@@ -194,7 +194,8 @@ __global__ void __launch_bounds__(kThreads) decode_sparse_kernel(DecodeDims d, c
                                                                  const int* __restrict__ idx, int kb,
                                                                  const T* __restrict__ kr, const T* __restrict__ vr,
                                                                  int W, const int* __restrict__ swa_len,
-                                                                 const float* __restrict__ gate, T* __restrict__ o) {
+                                                                 const float* __restrict__ gate,
+                                                                 const float* __restrict__ sinks, T* __restrict__ o) {
   constexpr int R = kMaxG * D / kThreads;
   __shared__ DecodeSmem<D> sm;
   __shared__ int spos[kKC];
@@ -260,8 +261,11 @@ __global__ void __launch_bounds__(kThreads) decode_sparse_kernel(DecodeDims d, c
       const int h = g * G + hh;
       const float g0 = sigmoidf_(gate[((size_t)b * d.Hq + h) * 2 + 0]);
       const float g1 = sigmoidf_(gate[((size_t)b * d.Hq + h) * 2 + 1]);
-      const float a = sL1[hh] > 0.0f ? acc1[r] * (g0 / sL1[hh]) : 0.0f;
-      const float c = sm.l[hh] > 0.0f ? acc[r] * (g1 / sm.l[hh]) : 0.0f;
+      // each branch's sink logit joins its softmax as an entry with a zero value (log2 units)
+      const float l1 = sL1[hh] + (sinks ? exp2f(sinks[2 * h] * kLog2e - sM1[hh]) : 0.0f);
+      const float l2 = sm.l[hh] + (sinks ? exp2f(sinks[2 * h + 1] * kLog2e - sm.m[hh]) : 0.0f);
+      const float a = l1 > 0.0f ? acc1[r] * (g0 / l1) : 0.0f;
+      const float c = l2 > 0.0f ? acc[r] * (g1 / l2) : 0.0f;
       Elem<T>::store(o + ((size_t)b * d.Hq + h) * D + dd, a + c);
     }
   }
@@ -291,10 +295,10 @@ cudaError_t decode_full_typed(const DecodeDims& d, const void* q, const void* kc
 template <typename T, int D>
 cudaError_t decode_sparse_typed(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                 const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
-                                const int* swa_len, const float* gate, void* o, cudaStream_t s) {
+                                const int* swa_len, const float* gate, const float* sinks, void* o, cudaStream_t s) {
   dim3 grid(d.Hkv, d.B);
   decode_sparse_kernel<T, D><<<grid, kThreads, 0, s>>>(d, (const T*)q, (const T*)kc, (const T*)vc, seqlens, idx, kb,
-                                                       (const T*)kr, (const T*)vr, W, swa_len, gate, (T*)o);
+                                                       (const T*)kr, (const T*)vr, W, swa_len, gate, sinks, (T*)o);
   return cudaGetLastError();
 }
 
@@ -317,13 +321,15 @@ cudaError_t launch_decode_full(const DecodeDims& d, hys_dtype dt, const void* q,
 
 cudaError_t launch_decode_sparse(const DecodeDims& d, hys_dtype dt, const void* q, const void* kc, const void* vc,
                                  const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
-                                 const int* swa_len, const float* gate, void* o, cudaStream_t s) {
+                                 const int* swa_len, const float* gate, const float* sinks, void* o, cudaStream_t s) {
   if (dt == HYS_F32)
-    return d.D == 64 ? decode_sparse_typed<float, 64>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate, o, s)
-                     : decode_sparse_typed<float, 128>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate, o, s);
-  return d.D == 64
-             ? decode_sparse_typed<__nv_bfloat16, 64>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate, o, s)
-             : decode_sparse_typed<__nv_bfloat16, 128>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate, o, s);
+    return d.D == 64
+               ? decode_sparse_typed<float, 64>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate, sinks, o, s)
+               : decode_sparse_typed<float, 128>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate, sinks, o, s);
+  return d.D == 64 ? decode_sparse_typed<__nv_bfloat16, 64>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate,
+                                                            sinks, o, s)
+                   : decode_sparse_typed<__nv_bfloat16, 128>(d, q, kc, vc, seqlens, idx, kb, kr, vr, W, swa_len, gate,
+                                                             sinks, o, s);
 }
 
 }  // namespace hys

@@ -58,6 +58,7 @@ struct Params {
   int kb;
   int W;            // ring capacity (mode 1)
   const int* swa_len;
+  const float* sinks;      // [Hq,2] sink logits of the two branches (mode 1), or null
   const __nv_bfloat16* q;  // [B,Hq,D]
   float* pm;        // [B,Hq,nsplit]
   float* pl;
@@ -360,6 +361,8 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const
     float L = 0.0f;
     for (int s = s0; s < s1; ++s)
       if (p.pm[ph + s] != -INFINITY) L += p.pl[ph + s] * exp2f((p.pm[ph + s] - M) * sc);
+    // the branch's sink logit: a softmax entry with a zero value
+    if (p.mode == 1 && p.sinks != nullptr) L += exp2f(p.sinks[2 * (g * p.G + hh) + br] * kLog2e - M * sc);
     sM[br][hh] = M;
     sInv[br][hh] = L > 0.0f ? 1.0f / L : 0.0f;
   }
@@ -455,6 +458,7 @@ void fill_common(Params& p, const DecodeDims& d, const void* q, const int* seqle
   p.kb = 0;
   p.W = 0;
   p.swa_len = nullptr;
+  p.sinks = nullptr;
   p.nsp = 0;
 }
 
@@ -506,7 +510,8 @@ cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const voi
 
 cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                      const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
-                                     const int* swa_len, const float* gate, void* o, void* ws, cudaStream_t s) {
+                                     const int* swa_len, const float* gate, const float* sinks, void* o, void* ws,
+                                     cudaStream_t s) {
   CUtensorMap mk, mv, mkr, mvr;
   if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv) ||
       !make_map(&mkr, kr, W, d.B * d.Hkv) || !make_map(&mvr, vr, W, d.B * d.Hkv))
@@ -523,6 +528,7 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   p.kb = kb;
   p.W = W;
   p.swa_len = swa_len;
+  p.sinks = sinks;
   decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

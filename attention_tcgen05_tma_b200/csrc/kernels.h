@@ -65,7 +65,7 @@ cudaError_t launch_topk_tokens(const PrefillDims& d, const float* scores, int k_
 // ---- sparse layer ----------------------------------------------------------------------------
 cudaError_t launch_sparse_attn_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
                                     const void* v, const int* idx, int kb, const void* ks,
-                                    const void* vs, int window, const float* gate, void* o,
+                                    const void* vs, int window, const float* gate, const float* sinks, void* o,
                                     cudaStream_t s);
 cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
                                       const void* v, const int* idx, int kt, int forced, void* o,
@@ -74,8 +74,8 @@ cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const 
 bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt);
 size_t sparse_attn_tc_workspace(const PrefillDims& d);
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
-                                  int kb, const void* ks, const void* vs, int window, const float* gate, void* o,
-                                  void* ws, size_t ws_bytes, cudaStream_t s);
+                                  int kb, const void* ks, const void* vs, int window, const float* gate,
+                                  const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s);
 
 // ---- decode ----------------------------------------------------------------------------------
 size_t decode_full_workspace(const DecodeDims& d);
@@ -85,7 +85,7 @@ cudaError_t launch_decode_full(const DecodeDims& d, hys_dtype dt, const void* q,
 cudaError_t launch_decode_sparse(const DecodeDims& d, hys_dtype dt, const void* q, const void* kc,
                                  const void* vc, const int* seqlens, const int* idx, int kb,
                                  const void* kr, const void* vr, int W, const int* swa_len,
-                                 const float* gate, void* o, cudaStream_t s);
+                                 const float* gate, const float* sinks, void* o, cudaStream_t s);
 
 // bf16, D = 128, G <= 16: tensor-core split-KV kernels
 bool decode_mma_supported(const DecodeDims& d, hys_dtype dt);
@@ -96,6 +96,7 @@ cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const voi
                                    cudaStream_t s);
 cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                      const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
-                                     const int* swa_len, const float* gate, void* o, void* ws, cudaStream_t s);
+                                     const int* swa_len, const float* gate, const float* sinks, void* o, void* ws,
+                                     cudaStream_t s);
 
 }  // namespace hys

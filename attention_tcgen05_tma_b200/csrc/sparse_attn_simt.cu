@@ -70,7 +70,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) sparse_attn_simt_kernel(
     PrefillDims d, const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int* __restrict__ idx, int kb, const T* __restrict__ ks, const T* __restrict__ vs, int window,
-    const float* __restrict__ gate, T* __restrict__ o) {
+    const float* __restrict__ gate, const float* __restrict__ sinks, T* __restrict__ o) {
   constexpr int DL = D / 4;
   __shared__ float sk[kKC][D];
   __shared__ float sv[kKC][D];
@@ -128,8 +128,11 @@ __global__ void __launch_bounds__(kThreads) sparse_attn_simt_kernel(
   if (!valid) return;
   const float* gl = gate + (((size_t)b * d.Hq + h) * d.N + t) * 2;
   const float g0 = sigmoidf_(gl[0]), g1 = sigmoidf_(gl[1]);
-  const float i_sp = st_sp.l > 0.0f ? g0 / st_sp.l : 0.0f;
-  const float i_sw = st_sw.l > 0.0f ? g1 / st_sw.l : 0.0f;
+  // each branch's sink logit joins its softmax as an entry with a zero value (log2 units here)
+  const float l_sp = st_sp.l + (sinks ? exp2f(sinks[2 * h] * kLog2e - st_sp.m) : 0.0f);
+  const float l_sw = st_sw.l + (sinks ? exp2f(sinks[2 * h + 1] * kLog2e - st_sw.m) : 0.0f);
+  const float i_sp = l_sp > 0.0f ? g0 / l_sp : 0.0f;
+  const float i_sw = l_sw > 0.0f ? g1 / l_sw : 0.0f;
   T* oh = o + ((size_t)b * d.Hq + h) * d.N * D + (size_t)t * D;
 #pragma unroll
   for (int c = 0; c < DL; ++c) Elem<T>::store(oh + c * 4 + lg, a_sp[c] * i_sp + a_sw[c] * i_sw);
@@ -197,11 +200,11 @@ __global__ void __launch_bounds__(kThreads) sparse_tokens_simt_kernel(PrefillDim
 
 template <typename T, int D>
 cudaError_t launch_sparse_typed(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
-                                int kb, const void* ks, const void* vs, int window, const float* gate, void* o,
-                                cudaStream_t s) {
+                                int kb, const void* ks, const void* vs, int window, const float* gate,
+                                const float* sinks, void* o, cudaStream_t s) {
   dim3 grid(d.T, d.Hq, d.B);
   sparse_attn_simt_kernel<T, D><<<grid, kThreads, 0, s>>>(d, (const T*)q, (const T*)k, (const T*)v, idx, kb,
-                                                          (const T*)ks, (const T*)vs, window, gate, (T*)o);
+                                                          (const T*)ks, (const T*)vs, window, gate, sinks, (T*)o);
   return cudaGetLastError();
 }
 
@@ -218,12 +221,12 @@ cudaError_t launch_tokens_typed(const PrefillDims& d, const void* q, const void*
 
 cudaError_t launch_sparse_attn_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k, const void* v,
                                     const int* idx, int kb, const void* ks, const void* vs, int window,
-                                    const float* gate, void* o, cudaStream_t s) {
+                                    const float* gate, const float* sinks, void* o, cudaStream_t s) {
   if (dt == HYS_F32)
-    return d.D == 64 ? launch_sparse_typed<float, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, o, s)
-                     : launch_sparse_typed<float, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, o, s);
-  return d.D == 64 ? launch_sparse_typed<__nv_bfloat16, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, o, s)
-                   : launch_sparse_typed<__nv_bfloat16, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, o, s);
+    return d.D == 64 ? launch_sparse_typed<float, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s)
+                     : launch_sparse_typed<float, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s);
+  return d.D == 64 ? launch_sparse_typed<__nv_bfloat16, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s)
+                   : launch_sparse_typed<__nv_bfloat16, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s);
 }
 
 cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,

@@ -58,6 +58,7 @@ struct Params {
   int num_units;
   const int* idx;      // [B,Hkv,T,kb]
   const float* gate;   // [B,Hq,N,2]
+  const float* sinks;  // [Hq,2] sink logits of the two branches, or null
   __nv_bfloat16* o;
   int o_v8;            // o is 32-byte aligned (256-bit stores)
   int* counter;        // work-unit counter (zeroed before the launch)
@@ -409,6 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // so the load latency hides behind the first tiles
         float2 gl = make_float2(-INFINITY, -INFINITY);
         if (valid) gl = *reinterpret_cast<const float2*>(p.gate + (((size_t)x.b * p.Hq + h) * p.N + t) * 2);
+        // sink logits (a softmax entry with a zero value per branch), in log2 units
+        float2 sk = make_float2(-INFINITY, -INFINITY);
+        if (p.sinks != nullptr) {
+          sk = *reinterpret_cast<const float2*>(p.sinks + 2 * h);
+          sk.x *= kLog2e;
+          sk.y *= kLog2e;
+        }
         float m_used = -INFINITY, l = 0.0f;   // online state of the sparse branch
         float mw = -INFINITY, lw = 0.0f;      // window branch statistics
         float pw = 0.0f;                      // sigmoid(g1) / l' for the window P.V pass
@@ -420,7 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tau == x.n_sp && x.n_sp > 0) {
             // the sparse branch is complete in O (its last P.V finished before this S did):
             // scale O in place to sigmoid(g0) * o~
-            const float f = l > 0.0f ? sigmoidf_(gl.x) / l : 0.0f;
+            const float lt = l + exp2f(sk.x - m_used * sc);   // + the sparse branch's sink
+            const float f = lt > 0.0f ? sigmoidf_(gl.x) / lt : 0.0f;
             uint32_t ov[D];
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
@@ -527,7 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             lw += a.x + a.y;
             if (tau == x.n_sp + x.n_sw - 1) {
               // P' = exp2((s - m') sc) * sigmoid(g1) / l' = exp2(s sc - (m' sc - log2(sigmoid(g1) / l')))
-              pw = lw > 0.0f ? sigmoidf_(gl.y) / lw : 0.0f;
+              const float lwt = lw + exp2f(sk.y - (mw == -INFINITY ? 0.0f : mw * sc));   // + its sink
+              pw = lwt > 0.0f ? sigmoidf_(gl.y) / lwt : 0.0f;
               pw = (mw == -INFINITY ? 0.0f : mw * sc) - __log2f(pw);
             }
           } else {
@@ -642,8 +652,8 @@ int grid_size(const PrefillDims& d) { return num_units(d) < kMaxGrid ? num_units
 
 template <int D>
 cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx, int kb,
-                         const void* ks, const void* vs, int window, const float* gate, void* o, void* ws,
-                         cudaStream_t s) {
+                         const void* ks, const void* vs, int window, const float* gate, const float* sinks,
+                         void* o, void* ws, cudaStream_t s) {
   CUtensorMap mq, mk, mv, mks, mvs;
   if (!make_map(&mq, q, D, d.N, d.B * d.Hq) || !make_map(&mk, k, D, d.N, d.B * d.Hkv) ||
       !make_map(&mv, v, D, d.N, d.B * d.Hkv) || !make_map(&mks, ks, D, d.N, d.B * d.Hkv) ||
@@ -661,6 +671,7 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.num_units = num_units(d);
   p.idx = idx;
   p.gate = gate;
+  p.sinks = sinks;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   p.counter = reinterpret_cast<int*>(ws);
@@ -692,11 +703,11 @@ bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt) {
 size_t sparse_attn_tc_workspace(const PrefillDims&) { return 256; }
 
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
-                                  int kb, const void* ks, const void* vs, int window, const float* gate, void* o,
-                                  void* ws, size_t ws_bytes, cudaStream_t s) {
+                                  int kb, const void* ks, const void* vs, int window, const float* gate,
+                                  const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s) {
   if (ws_bytes < sparse_attn_tc_workspace(d)) return cudaErrorInvalidValue;
-  return d.D == 64 ? launch_typed<64>(d, q, k, v, idx, kb, ks, vs, window, gate, o, ws, s)
-                   : launch_typed<128>(d, q, k, v, idx, kb, ks, vs, window, gate, o, ws, s);
+  return d.D == 64 ? launch_typed<64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s)
+                   : launch_typed<128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s);
 }
 
 }  // namespace hys

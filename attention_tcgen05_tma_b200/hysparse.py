@@ -295,8 +295,8 @@ def topk_tokens(scores, k_tokens: int, forced_window: int, *, idx=None, stream=N
     return idx
 
 
-def sparse_attn(q_sparse, k, v, idx, k_swa, v_swa, window: int, gate_logits, *, o=None, workspace=None,
-                stream=None):
+def sparse_attn(q_sparse, k, v, idx, k_swa, v_swa, window: int, gate_logits, *, sinks=None, o=None,
+                workspace=None, stream=None):
     torch = _torch()
     sh = prefill_shape(q_sparse, k)
     if o is None:
@@ -304,7 +304,7 @@ def sparse_attn(q_sparse, k, v, idx, k_swa, v_swa, window: int, gate_logits, *, 
     if workspace is None:
         workspace = workspace_for(hysparse_sparse_attn_workspace_size(sh, _dt(q_sparse)), q_sparse.device)
     _check(hysparse_sparse_attn(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k), _ptr(v), _ptr(idx), idx.shape[-1],
-                                _ptr(k_swa), _ptr(v_swa), window, _ptr(gate_logits), None, _ptr(o),
+                                _ptr(k_swa), _ptr(v_swa), window, _ptr(gate_logits), _ptr(sinks), _ptr(o),
                                 _ptr(workspace), workspace.numel(), _stream(stream)), "hysparse_sparse_attn")
     return o
 
@@ -354,7 +354,7 @@ def topk_decode(scores, k: int, L: int, *, seqlens=None, idx=None, stream=None):
 
 
 def sparse_attn_decode(q, k_cache, v_cache, idx, k_ring, v_ring, gate_logits, *, seqlens=None, swa_len=None,
-                       o=None, workspace=None, stream=None):
+                       sinks=None, o=None, workspace=None, stream=None):
     torch = _torch()
     sh = decode_shape(q, k_cache)
     if o is None:
@@ -363,7 +363,7 @@ def sparse_attn_decode(q, k_cache, v_cache, idx, k_ring, v_ring, gate_logits, *,
         workspace = workspace_for(hysparse_sparse_attn_decode_workspace_size(sh, _dt(q), idx.shape[-1]), q.device)
     _check(hysparse_sparse_attn_decode(sh, _dt(q), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(idx),
                                        idx.shape[-1], _ptr(k_ring), _ptr(v_ring), k_ring.shape[2], _ptr(swa_len),
-                                       _ptr(gate_logits), None, _ptr(o), _ptr(workspace), workspace.numel(),
+                                       _ptr(gate_logits), _ptr(sinks), _ptr(o), _ptr(workspace), workspace.numel(),
                                        _stream(stream)),
            "hysparse_sparse_attn_decode")
     return o

@@ -37,7 +37,7 @@ import numpy as np
 TID_Q, TID_K, TID_V = 0, 1, 2
 TID_PLANT = 15
 _TID_LAYER0 = 16
-SPARSE_Q, SPARSE_KSWA, SPARSE_VSWA, SPARSE_GATE = 0, 1, 2, 3
+SPARSE_Q, SPARSE_KSWA, SPARSE_VSWA, SPARSE_GATE, SPARSE_SINK = 0, 1, 2, 3, 4
 
 
 def layer_tid(layer: int, which: int) -> int:
@@ -240,6 +240,13 @@ def gate_slice(w: Workload, layer: int, b: int, h: int) -> np.ndarray:
     """Gate logits (fp32, standard normal): [N, 2] for prefill, [2] for decode."""
     shape = (2,) if w.mode == "decode" else (w.N, 2)
     return normal_slice(w.seed, layer_tid(layer, SPARSE_GATE), b, h, shape, 1.0, False)
+
+
+def sink_logits(w: Workload, layer: int, std: float = 2.0) -> np.ndarray:
+    """Per-head sink logits of a sparse layer, [Hq, 2] fp32 (index 0: sparse branch, 1: SWA
+    branch); standard deviation 2 so that sinks range from negligible to dominant."""
+    return np.stack([normal_slice(w.seed, layer_tid(layer, SPARSE_SINK), 0, h, (2,), std, False)
+                     for h in range(w.Hq)]).astype(np.float32)
 
 
 # decode: the query of the new token, the shared cache and the SWA rings

@@ -152,9 +152,12 @@ HYS_API hys_status hysparse_topk_tokens(const hys_shape* shape, const float* tok
  *   (the full layer's cache, [HS] 3.4.4) and [max(0, t-window+1), t] of its own K', V'.
  *   k_swa/v_swa may alias k_shared/v_shared (the "share both" ablation).
  *   idx entries are ascending block ids <= I or -1 (ignored); 1 <= k <= 1024.
- *   sinks must be NULL (per-head sink biases are not implemented: HYS_ERR_UNSUPPORTED).
- *   workspace: at least hysparse_sparse_attn_workspace_size() bytes (fp32 scratch that
- *   holds the gated sparse-branch rows while the window branch runs).
+ *   sinks: NULL, or [Hq, 2] fp32 per-head sink logits ([HSP] 4.1: per-head learnable sink
+ *   biases in the sparse and sliding-window branches, as in gpt-oss), index 0 for the sparse
+ *   branch and 1 for the window branch, in the units of the scaled logits tau q.k: each joins
+ *   its branch's softmax as an entry with a zero value (the denominator gains exp(sink - m)).
+ *   workspace: at least hysparse_sparse_attn_workspace_size() bytes (the tensor-core kernel's
+ *   work-unit counter; no scratch rows: both branches accumulate into one output tile).
  * ------------------------------------------------------------------------------------ */
 HYS_API hys_status hysparse_sparse_attn_workspace_size(const hys_shape* shape, hys_dtype dtype,
                                                      size_t* bytes);
@@ -227,7 +230,8 @@ HYS_API hys_status hysparse_topk_decode(const hys_decode_shape* shape, const flo
  * cached token (< L_b) of the selected blocks of the shared cache; the SWA branch attends
  * the layer's own ring k_swa_ring/v_swa_ring [B,Hkv,W,D] (swa_len[b] valid entries, or W
  * when swa_len is NULL; order is irrelevant); gate_logits [B,Hq,2]; o [B,Hq,D].
- * W = window, 1 <= window <= 1024.  sinks must be NULL.  workspace: at least
+ * W = window, 1 <= window <= 1024.  sinks: NULL or [Hq, 2] fp32 sink logits, as for
+ * hysparse_sparse_attn.  workspace: at least
  * hysparse_sparse_attn_decode_workspace_size() bytes (per-split partial softmax states).
  * ------------------------------------------------------------------------------------ */
 HYS_API hys_status hysparse_sparse_attn_decode_workspace_size(const hys_decode_shape* shape,

@@ -58,8 +58,15 @@ def test_entry_points_reject_bad_arguments_without_launching(lib):
         == H.HYS_ERR_INVALID_ARG
     assert H.hysparse_topk(sh, 16, 0, 16, None) == H.HYS_ERR_INVALID_ARG
     assert H.hysparse_topk(sh, 17, 4, 16, None) == H.HYS_ERR_INVALID_ARG
-    assert H.hysparse_sparse_attn(sh, H.HYS_F32, 16, 16, 16, 16, 4, 16, 16, 128, 16, 16, 16, None, 0, None) \
-        == H.HYS_ERR_UNSUPPORTED   # sinks are not implemented
+    # sink logits are accepted, but like every pointer must be 16-byte aligned (checked before
+    # anything launches); the token variant has no sink biases
+    assert H.hysparse_sparse_attn(sh, H.HYS_F32, 16, 16, 16, 16, 4, 16, 16, 128, 16, 8, 16, None, 0, None) \
+        == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_sparse_attn_tokens(sh, H.HYS_F32, 16, 16, 16, 16, 4, 128, 16, 16, None, 0, None) \
+        == H.HYS_ERR_UNSUPPORTED
+    dsh1 = H.hys_decode_shape(2, 1000, 8, 2, 128, 64)
+    assert H.hysparse_sparse_attn_decode(dsh1, H.HYS_BF16, 16, 16, 16, None, 16, 4, 16, 16, 128, None, 16, 8, 16,
+                                         16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
     bsh = H.hys_shape(1, 256, 4, 2, 128, 64)
     assert H.hysparse_sparse_attn_workspace_size(bsh, H.HYS_BF16) > 0
     assert H.hysparse_sparse_attn(bsh, H.HYS_BF16, 16, 16, 16, 16, 4, 16, 16, 128, 16, None, 16, None, 0, None) \

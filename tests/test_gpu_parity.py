@@ -200,3 +200,58 @@ def test_decode(case):
     ref = O.decode_sparse(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], a["gate"][0],
                           seqlens, swa_len)
     assert np.max(np.abs(to_np(osp) - ref)) <= TOL[dt]
+
+
+SINK_PREFILL_CASES = [
+    # name, dtype, B, N, Hq, Hkv, D, k, window  (tensor-core path for bf16 D in {64,128}, even G)
+    ("bf16_d128_g4_tc", "bf16", 1, 700, 8, 2, 128, 4, 128),
+    ("bf16_d64_g8_tc", "bf16", 1, 333, 8, 1, 64, 3, 100),
+    ("f32_d64_g4_simt", "f32", 1, 300, 4, 1, 64, 3, 64),
+]
+
+
+@pytest.mark.parametrize("case", SINK_PREFILL_CASES, ids=[c[0] for c in SINK_PREFILL_CASES])
+def test_sparse_layer_sinks(case):
+    """Per-head sink logits of both branches ([HSP] 4.1): parity with the oracle, and sinks of
+    -inf reproduce the call without sinks exactly."""
+    name, dt, B, N, Hq, Hkv, D, k, window = case
+    w = _workload(dt, B, N, Hq, Hkv, D, k, window)
+    a = I.prefill_arrays(w, layers=1)
+    q, kk, vv = (to_dev(a[x], dt) for x in ("q", "k", "v"))
+    _, sc = H.full_attn_select(q, kk, vv)
+    idx = H.topk(sc, k)
+    qs, ks, vs = (to_dev(a[x][0], dt) for x in ("q_sparse", "k_swa", "v_swa"))
+    gate = to_dev(a["gate"][0], "f32")
+    sinks = I.sink_logits(w, 0)
+    osp = H.sparse_attn(qs, kk, vv, idx, ks, vs, window, gate, sinks=torch.from_numpy(sinks).cuda())
+    none = H.sparse_attn(qs, kk, vv, idx, ks, vs, window, gate)
+    neg = H.sparse_attn(qs, kk, vv, idx, ks, vs, window, gate,
+                        sinks=torch.full((Hq, 2), float("-inf"), device="cuda"))
+    torch.cuda.synchronize()
+    gidx = idx.cpu().numpy().astype(np.int64)
+    ref = O.sparse_attention(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], window,
+                             a["gate"][0], sinks=sinks.astype(np.float64))
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL[dt]
+    assert torch.equal(none, neg)
+
+
+@pytest.mark.parametrize("dt,D,Hq,Hkv", [("bf16", 128, 16, 2), ("f32", 64, 8, 2)], ids=["mma", "simt"])
+def test_decode_sinks(dt, D, Hq, Hkv):
+    B, L, k, W = 3, 1500, 4, 128
+    w = I.scaled(I.WORKLOADS["decode"], B=B, N=L, Hq=Hq, Hkv=Hkv, D=D, topk=k, window=W, layers=1, seed=8,
+                 scale_std=1.0 / np.sqrt(D))
+    a = I.decode_arrays(w, layers=1)
+    swa_len = np.array([W, 0, 37], dtype=np.int32)          # an empty ring: its branch gives zero
+    q, kc, vc = (to_dev(a[x], dt) for x in ("q", "k", "v"))
+    _, sc = H.full_attn_select_decode(q, kc, vc)
+    idx = H.topk_decode(sc, k, L)
+    qs, kr, vr = (to_dev(a[x][0], dt) for x in ("q_sparse", "k_swa", "v_swa"))
+    gate = to_dev(a["gate"][0], "f32")
+    sinks = I.sink_logits(w, 0)
+    osp = H.sparse_attn_decode(qs, kc, vc, idx, kr, vr, gate, swa_len=torch.from_numpy(swa_len).cuda(),
+                               sinks=torch.from_numpy(sinks).cuda())
+    torch.cuda.synchronize()
+    gidx = idx.cpu().numpy().astype(np.int64)
+    ref = O.decode_sparse(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], a["gate"][0],
+                          None, swa_len, sinks=sinks.astype(np.float64))
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL[dt]
