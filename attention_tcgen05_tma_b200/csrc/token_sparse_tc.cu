@@ -27,6 +27,7 @@ constexpr int kThreads = 384;
 constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;
 constexpr int kMaskWords = 16;     // extended window <= 512 keys  ->  W <= 449
+constexpr int kMaxList = 4096;     // selected positions kept in shared memory (larger k: read from L2)
 constexpr float kRescaleLog2 = 8.0f;
 
 struct Params {
@@ -56,7 +57,8 @@ struct Cfg {
   static constexpr int kOffKV = 2 * kQBytes;
   static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
   static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+  static constexpr int kOffList = kOffMisc + 64;   // the producer's copy of a unit's positions
+  static constexpr int kSmemBytes = kOffList + kMaxList * 4 + 1024;
 };
 
 struct Unit {
@@ -134,13 +136,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ============================================================== producer warp (gathers)
+    int* plist = reinterpret_cast<int*>(smem + C::kOffList);
     uint32_t kv_it = 0, q_cnt[2] = {0, 0};
     bool ok = true;
+    // the next unit is claimed one unit ahead, so the counter's round trip overlaps a unit's work
+    int claim = 0;
+    if (lane == 0) claim = atomicAdd(p.counter, 1);
     for (uint32_t n = 0; ok; ++n) {
       int u = 0;
       if (lane == 0) {
-        const int c = atomicAdd(p.counter, 1);
-        u = c < p.num_units ? c : -1;
+        u = claim < p.num_units ? claim : -1;
+        if (u >= 0) claim = atomicAdd(p.counter, 1);
       }
       u = __shfl_sync(0xffffffffu, u, 0);
       // wait for the queue slot before filling its mask
@@ -156,15 +162,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         sel = p.idx + (((size_t)x0.b * p.Hkv + x0.g) * p.T + x0.I) * p.kt;
         if (lane < kMaskWords) mask[lane] = 0u;
         __syncwarp();
-        for (int e0 = 0; e0 < p.kt; e0 += 32) {
-          const int e = e0 + lane;
-          const int j = e < p.kt ? sel[e] : -1;
-          const unsigned stop = __ballot_sync(0xffffffffu, j < 0);       // first -1 ends the list
-          const int first_stop = stop ? __ffs(stop) - 1 : 32;
-          const bool live = lane < first_stop;
-          nA += __popc(__ballot_sync(0xffffffffu, live && j < x0.w0));
-          if (live && j >= x0.w0 && j <= x0.eI) atomicOr(&mask[(j - x0.w0) >> 5], 1u << ((j - x0.w0) & 31));
-          if (stop) break;
+        // eight 32-entry chunks in flight per step (the list's loads do not wait on each other);
+        // the positions are kept in shared memory for the per-tile gathers
+        bool stopped = false;
+        for (int e0 = 0; e0 < p.kt && !stopped; e0 += 256) {
+          int jv[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int e = e0 + 32 * c + lane;
+            jv[c] = e < p.kt ? sel[e] : -1;
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (stopped) break;
+            const int e = e0 + 32 * c + lane;
+            const int j = jv[c];
+            const unsigned stop = __ballot_sync(0xffffffffu, j < 0);       // first -1 ends the list
+            const int first_stop = stop ? __ffs(stop) - 1 : 32;
+            const bool live = lane < first_stop;
+            nA += __popc(__ballot_sync(0xffffffffu, live && j < x0.w0));
+            if (live && j >= x0.w0 && j <= x0.eI) atomicOr(&mask[(j - x0.w0) >> 5], 1u << ((j - x0.w0) & 31));
+            if (live && e < kMaxList) plist[e] = j;
+            if (stop) stopped = true;
+          }
         }
       }
       __syncwarp();
@@ -206,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int pos;
             if (tau < x.n_sp) {
               const int e = 128 * tau + rr;
-              pos = e < x.nA ? sel[e] : 0;  // padding rows read row 0; their columns are masked
+              pos = e < x.nA ? (e < kMaxList ? plist[e] : sel[e]) : 0;  // padding rows read row 0 (masked)
             } else {
               const int i = x.w0 + 128 * (tau - x.n_sp) + rr;
               pos = i <= x.eI ? i : 0;
