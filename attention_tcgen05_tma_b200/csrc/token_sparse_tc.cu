@@ -29,12 +29,29 @@ constexpr int kMaxGrid = 148;
 constexpr int kMaskWords = 16;     // extended window <= 512 keys  ->  W <= 449
 constexpr int kMaxList = 4096;     // selected positions kept in shared memory (larger k: read from L2)
 constexpr float kRescaleLog2 = 8.0f;
+#ifndef HYS_TOKEN_POLY_PAIRS
+#define HYS_TOKEN_POLY_PAIRS 8
+#endif
+// column pairs (of the 64 in a 128-key row) whose exp2 runs on the FMA pipe instead of MUFU
+constexpr int kPolyPairs = HYS_TOKEN_POLY_PAIRS;
+// Register split between the warpgroups (setmaxnreg): the launch gives every thread
+// kLaunchRegs; the producer/MMA warpgroup drops to kLowRegs and each softmax warpgroup rises to
+// kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
+// the host checks the compiled register count before every launch.
+constexpr int kLaunchRegs = 168, kLowRegs = 88, kHighRegs = 208;
+static_assert(kLowRegs + 2 * kHighRegs == 3 * kLaunchRegs, "register split must match the launch allocation");
+
+__device__ __forceinline__ float2 exp2_pair(float2 x, int i) {
+  if ((i * kPolyPairs) % 64 < kPolyPairs) return tc::exp2_poly3_x2(x);
+  return make_float2(exp2f(x.x), exp2f(x.y));
+}
 
 struct Params {
   int B, N, Hq, Hkv, G, T, kt, W;
   int num_units;
   const int* idx;     // [B,Hkv,T,kt]
   __nv_bfloat16* o;
+  int o_v8;           // o is 32-byte aligned (256-bit stores)
   int* counter;
   int* status;
   float scale_log2;
@@ -136,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ============================================================== producer warp (gathers)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     int* plist = reinterpret_cast<int*>(smem + C::kOffList);
     uint32_t kv_it = 0, q_cnt[2] = {0, 0};
     bool ok = true;
@@ -259,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     if (lane == 0) {
       const uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
       const uint32_t idO = tc::idesc_bf16_f32(128, D, true);
@@ -351,8 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mma_commit(&bars->mma_drain);
       tc::mbar_wait(&bars->mma_drain, 0, abort, 100000000ull);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+  } else {
     // ============================================================== softmax / epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     const int s = (warp - 4) >> 2;
     const int row = 32 * (warp & 3) + lane;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
@@ -419,57 +441,62 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          float mx;
-          {
-            float a[8];
+          const float2 sc2 = make_float2(sc, sc);
+          // P = exp2(s sc - ms) written to TMEM as bf16 over S; returns the row sum and (three-
+          // input max chains on the ALU, beside the MUFU work) the row max
+          auto emit_p = [&](float ms, float& rmax) -> float {
+            const float2 nm2 = make_float2(-ms, -ms);
+            float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+            float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) a[j] = sv[j];
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
 #pragma unroll
-            for (int i = 8; i < 128; i += 8)
-#pragma unroll
-              for (int j = 0; j < 8; ++j) a[j] = fmaxf(a[j], sv[i + j]);
-#pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-              for (int j = 0; j < w; ++j) a[j] = fmaxf(a[j], a[j + w]);
-            mx = a[0];
-          }
-          float alpha = 1.0f;
-          bool rescale = false;
-          if (mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2) {
-            rescale = true;
-            alpha = exp2f((m_used - mx) * sc);
-            l *= alpha;
-            m_used = mx;
-          }
-          const float ms = m_used == -INFINITY ? 0.0f : m_used * sc;
-          float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = exp2f(fmaf(sv[32 * c + 2 * i], sc, -ms));
-              const float p1 = exp2f(fmaf(sv[32 * c + 2 * i + 1], sc, -ms));
-              ls[i & 3] += p0 + p1;
-              pk[i] = tc::pack_bf16x2(p0, p1);
+              for (int i = 0; i < 16; ++i) {
+                const float s0 = sv[32 * c + 2 * i], s1 = sv[32 * c + 2 * i + 1];
+                mk[i & 3] = tc::fmax3(mk[i & 3], s0, s1);
+                const float2 pv = exp2_pair(tc::ffma2(make_float2(s0, s1), sc2, nm2), 16 * c + i);
+                acc[i & 1] = tc::fadd2(acc[i & 1], pv);
+                pk[i] = tc::pack_bf16x2(pv.x, pv.y);
+              }
+              tc::tmem_st16(tSrow + 16 * c, pk);
             }
-            tc::tmem_st16(tSrow + 16 * c, pk);
-          }
-          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-          // warp-uniform: the TMEM loads and stores are warp-collective; rows that keep their
-          // max scale by alpha = 1
-          if (__any_sync(0xffffffffu, rescale && tau > 0)) {
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tc::tmem_ld32(tOrow + 32 * c, ov);
+            rmax = tc::fmax3(fmaxf(mk[0], mk[1]), mk[2], mk[3]);
+            const float2 a = tc::fadd2(acc[0], acc[1]);
+            return a.x + a.y;
+          };
+          // The row max is needed first only while the row has none: later tiles compute P with
+          // the running max straight away and find the tile max beside it; a row whose max rose
+          // by more than 2^kRescaleLog2 redoes the tile with the new max (rare), and O is
+          // rescaled.  Warp-uniform branches only: TMEM loads and stores are warp-collective.
+          if (m_used == -INFINITY) m_used = fmaxf(tc::max64(sv), tc::max64(sv + 64));
+          float mx;
+          float lt = emit_p(m_used == -INFINITY ? 0.0f : m_used * sc, mx);
+          float alpha = 1.0f;
+          const bool rescale = mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2;
+          if (__any_sync(0xffffffffu, rescale)) {
+            if (rescale) {
+              alpha = exp2f((m_used - mx) * sc);
+              m_used = mx;
+            }
+            float unused;
+            lt = emit_p(m_used * sc, unused);   // unchanged rows write the same P again
+            if (tau > 0) {
+              uint32_t ov[D];
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
               tc::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tc::tmem_st32(tOrow + 32 * c, ov);
+              for (int i = 0; i < D; i += 2) {
+                const float2 vv = tc::fmul2(make_float2(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1])), make_float2(alpha, alpha));
+                ov[i] = __float_as_uint(vv.x);
+                ov[i + 1] = __float_as_uint(vv.y);
+              }
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) tc::tmem_st32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
             }
           }
+          l = l * alpha + lt;
           tc::tmem_wait_st();
           tc::fence_before_sync();
           tc::mbar_arrive(&bars->p_full[s]);
@@ -480,23 +507,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_after_sync();
         const float il = l > 0.0f ? 1.0f / l : 0.0f;
         __nv_bfloat16* orow = p.o + (((size_t)x.b * p.Hq + h) * p.N + t) * D;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tc::tmem_ld32(tOrow + 32 * c, ov);
+        uint32_t pk[D / 2];
+        {
+          uint32_t ov[D];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
           tc::tmem_wait_ld();
-          if (valid) {
-            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = tc::pack_bf16x2(__uint_as_float(ov[2 * i]) * il, __uint_as_float(ov[2 * i + 1]) * il);
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < D / 2; ++i) {
+            const float2 vv = tc::fmul2(make_float2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1])), make_float2(il, il));
+            pk[i] = tc::pack_bf16x2(vv.x, vv.y);
           }
         }
         tc::fence_before_sync();
-        tc::mbar_arrive(&bars->o_empty[s]);
+        tc::mbar_arrive(&bars->o_empty[s]);  // O may be overwritten by the next round from here on
+        if (valid) {
+          if (p.o_v8) {  // 32-byte aligned output: 256-bit stores, full sectors
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) tc::st_global_v8(orow + 16 * i, pk + 8 * i);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
       }
       tc::queue_release(&bars->queue, n);
     }
@@ -576,10 +610,19 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.num_units = num_units(d);
   p.idx = idx;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   p.counter = reinterpret_cast<int*>(ws);
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
+  static int regs = -1;   // the register split assumes exactly kLaunchRegs per thread at launch
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa, token_sparse_tc_kernel<D>);
+    if (e0 != cudaSuccess) return e0;
+    regs = fa.numRegs;
+  }
+  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(token_sparse_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);
