@@ -249,6 +249,20 @@ def sparse_flops(idx_np, N, G, D, window, block=64):
     return 4.0 * D * total
 
 
+def time_call(torch, fn, n=5, warm=2):
+    """Mean device time of fn() over n calls (CUDA events on the current stream, after warm-up)."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
 def run_ours(args, torch, dist, rank, world, dev):
     from attention_tcgen05_tma_b200 import build as Bld
     from attention_tcgen05_tma_b200 import hysparse as H
@@ -322,6 +336,13 @@ def run_ours(args, torch, dist, rank, world, dev):
     }
     launches_full = 1 if step.ws.numel() <= 1 or _uses_tc(H, w) else 2
     launches = args.steps * (launches_full + 1 + w.layers)
+    # the same sparse layer with per-head sink logits of both branches (outside the timed step)
+    sinks = torch.from_numpy(I.sink_logits(w, 0)).to(dev)
+    ms_sinks = time_call(torch, lambda: H.sparse_attn(x["q_sparse"][0], x["k"], x["v"], step.idx, x["k_swa"][0],
+                                                      x["v_swa"][0], w.window, x["gate"][0], sinks=sinks,
+                                                      o=step.o_sp, workspace=step.ws_sp))
+    kernels["sparse_attn_sinks_ms"] = round(ms_sinks, 4)
+    kernels["sparse_attn_sinks_tflops"] = round(sp_flops / (ms_sinks / 1e3) / 1e12, 2)
 
     res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",

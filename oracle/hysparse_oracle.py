@@ -33,6 +33,11 @@ Readings where the pages leave a step open (each is listed in the design notes):
   token once, no gate.
 * Decode: the new token sits at position L-1 of an L-token cache; it is its own
   tile; candidates are all blocks (block variant).
+* Token-variant decode ([HS2] "Twenty lines of algorithmic intuition" with the token
+  granularity of "Precise retrieval without a separate indexer"): the new token at
+  position L-1 scores every cached token i < L by sum over the group's heads of P_i;
+  candidates are the tokens older than the forced newest W, [0, L-1-W]; row L-1
+  attends the top-k candidates united with [L-W, L-1], each token once, no gate.
 * Sink biases ([HSP] §4.1, per-head learnable sinks in the sparse and SWA branches,
   following gpt-oss): one logit per (head, branch), sinks [Hq, 2] with index 0 for
   the sparse branch and 1 for the SWA branch; it joins the branch's softmax as an
@@ -330,6 +335,60 @@ def topk_decode(scores: np.ndarray, k: int, seqlens=None, L: Optional[int] = Non
         for g in range(Hkv):
             out[b, g] = select_topk(scores[b, g], n, k)
     return out
+
+
+def decode_token_scores(q: np.ndarray, k_cache: np.ndarray, seqlens=None) -> np.ndarray:
+    """score[b,g,i] = sum_{h in g} P^h_i of the new token (at L_b - 1) over the cached tokens
+    i < L_b (0 past the sequence end).  q [B,Hq,D]; k_cache [B,Hkv,L,D] -> [B,Hkv,L]."""
+    B, Hq, D = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    G = Hq // Hkv
+    sc = np.zeros((B, Hkv, L))
+    for b in range(B):
+        Lb = L if seqlens is None else int(seqlens[b])
+        for g in range(Hkv):
+            kk = np.asarray(k_cache[b, g, :Lb], np.float64)
+            for h in range(g * G, (g + 1) * G):
+                p, _, _ = causal_softmax(np.asarray(q[b, h], np.float64)[None, :], np.array([Lb - 1]), kk)
+                sc[b, g, :Lb] += p[0]
+    return sc
+
+
+def topk_decode_tokens(scores: np.ndarray, k_tokens: int, forced: int, seqlens=None) -> np.ndarray:
+    """[B,Hkv,L] -> [B,Hkv,k_tokens]: the top k of the candidates [0, L_b - 1 - forced]
+    (the tokens older than the forced newest window), ties to the lower index, ascending,
+    padded with -1."""
+    B, Hkv, L = scores.shape
+    out = np.full((B, Hkv, k_tokens), -1, dtype=np.int64)
+    for b in range(B):
+        Lb = L if seqlens is None else int(seqlens[b])
+        n = max(0, Lb - forced)
+        for g in range(Hkv):
+            out[b, g] = select_topk(scores[b, g], n, k_tokens)
+    return out
+
+
+def decode_token_sparse(q: np.ndarray, k_cache, v_cache, idx, forced: int, seqlens=None) -> np.ndarray:
+    """Token-sparse layer for the new token: the selected cached tokens idx[b,g,:] united
+    with the forced newest window [L_b - forced, L_b - 1], each token once; no gate."""
+    B, Hq, D = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    G = Hq // Hkv
+    o = np.zeros((B, Hq, D))
+    for b in range(B):
+        Lb = L if seqlens is None else int(seqlens[b])
+        for g in range(Hkv):
+            keep = np.zeros(Lb, dtype=bool)
+            sel = np.asarray([i for i in idx[b, g] if 0 <= i < Lb], dtype=np.int64)
+            keep[sel] = True
+            keep[max(0, Lb - forced):] = True
+            keys = np.nonzero(keep)[0]
+            ks = np.asarray(k_cache[b, g, keys], np.float64)
+            vs = np.asarray(v_cache[b, g, keys], np.float64)
+            for h in range(g * G, (g + 1) * G):
+                qq = np.asarray(q[b, h], np.float64)[None, :]
+                o[b, h] = attention_rows(qq, np.array([len(keys)]), ks, vs)[0][0]
+    return o
 
 
 def decode_sparse(q: np.ndarray, k_cache, v_cache, idx, k_ring, v_ring, gate, seqlens=None,

@@ -431,6 +431,52 @@ def test_sink_per_branch_and_decode():
     np.testing.assert_allclose(od[0, 0], op[0], rtol=1e-12, atol=1e-14)
 
 
+def test_token_decode_pins():
+    """Token-variant decode: the scores are torch's float64 softmax of the new token's logits
+    summed over the group's heads (they sum to G); every candidate selected gives dense decode;
+    the layer equals the prefill token-sparse row of position L-1 with the same selection; the
+    selection never enters the forced window and breaks ties to the lower index."""
+    rng = np.random.default_rng(9)
+    B, Hq, Hkv, D, L, W = 2, 4, 2, 16, 300, 32
+    G = Hq // Hkv
+    q = rng.standard_normal((B, Hq, D))
+    kc = rng.standard_normal((B, Hkv, L, D))
+    vc = rng.standard_normal((B, Hkv, L, D))
+    seqlens = np.array([L, 211])
+    sc = O.decode_token_scores(q, kc, seqlens)
+    for b in range(B):
+        Lb = int(seqlens[b])
+        for g in range(Hkv):
+            kk = torch.from_numpy(kc[b, g, :Lb]).double()
+            want = np.zeros(L)
+            for h in range(g * G, (g + 1) * G):
+                lg = (torch.from_numpy(q[b, h]).double() @ kk.T) / math.sqrt(D)
+                want[:Lb] += torch.softmax(lg, dim=0).numpy()
+            np.testing.assert_allclose(sc[b, g], want, rtol=1e-12, atol=1e-15)
+            assert abs(sc[b, g].sum() - G) < 1e-12
+    # all candidates selected -> dense decode
+    idx_all = O.topk_decode_tokens(sc, L, W, seqlens)
+    o_all = O.decode_token_sparse(q, kc, vc, idx_all, W, seqlens)
+    o_dense, _ = O.decode_full(q, kc, vc, seqlens)
+    np.testing.assert_allclose(o_all, o_dense, rtol=1e-12, atol=1e-13)
+    # a small budget: the prefill token-sparse row of position L_b - 1 agrees
+    kt = 20
+    idx = O.topk_decode_tokens(sc, kt, W, seqlens)
+    o = O.decode_token_sparse(q, kc, vc, idx, W, seqlens)
+    for b in range(B):
+        Lb = int(seqlens[b])
+        for g in range(Hkv):
+            sel = idx[b, g]
+            assert np.all(sel[sel >= 0] <= Lb - 1 - W) and np.all(np.diff(sel[sel >= 0]) > 0)
+            for h in range(g * G, (g + 1) * G):
+                ref = O.token_sparse_rows(q[b, h][None, :], np.array([Lb - 1]), kc[b, g, :Lb], vc[b, g, :Lb], sel, W)
+                np.testing.assert_allclose(o[b, h], ref[0], rtol=1e-12, atol=1e-13)
+    # ties: equal scores pick the lowest indices
+    flat = np.zeros((1, 1, 100))
+    got = O.topk_decode_tokens(flat, 5, 10)
+    assert got[0, 0].tolist() == [0, 1, 2, 3, 4]
+
+
 def test_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the oracle and check that a pin above fails."""
     g = _gold()
