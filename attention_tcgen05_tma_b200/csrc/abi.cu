@@ -345,4 +345,77 @@ hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hys_dtype 
                                         window, swa_len, gate_logits, sinks, o, s));
 }
 
+// ----------------------------------------------------------------------------- token-variant decode
+hys_status hysparse_full_attn_select_decode_tokens_workspace_size(const hys_decode_shape* shape, hys_dtype dtype,
+                                                                  size_t* bytes) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || !dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (!decode_mma_supported(d, dtype)) return HYS_ERR_UNSUPPORTED;
+  *bytes = align256(decode_mma_full_tokens_workspace(d));
+  return HYS_OK;
+}
+
+hys_status hysparse_full_attn_select_decode_tokens(const hys_decode_shape* shape, hys_dtype dtype, const void* q,
+                                                   const void* k_cache, const void* v_cache, const int* seqlens,
+                                                   void* o, float* tok_scores, void* workspace,
+                                                   size_t workspace_bytes, hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !o || !tok_scores) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seqlens) || !aligned16(o) ||
+      !aligned16(tok_scores) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  if (!decode_mma_supported(d, dtype)) return HYS_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < align256(decode_mma_full_tokens_workspace(d))) return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_decode_full_tokens_mma(d, q, k_cache, v_cache, seqlens, o, tok_scores, workspace,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_topk_decode_tokens(const hys_decode_shape* shape, const float* tok_scores, int k_tokens,
+                                       int forced_window, const int* seqlens, int* idx, hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!tok_scores || !idx || k_tokens < 1 || k_tokens > 16384 || forced_window < 1) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(tok_scores) || !aligned16(idx) || !aligned16(seqlens)) return HYS_ERR_INVALID_ARG;
+  return from_cuda(launch_topk_decode_tokens(tok_scores, idx, d.B, d.Hkv, d.L, k_tokens, forced_window, seqlens,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_sparse_attn_decode_tokens_workspace_size(const hys_decode_shape* shape, hys_dtype dtype,
+                                                             int k_tokens, size_t* bytes) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!bytes || !dtype_ok(dtype) || k_tokens < 1 || k_tokens > 16384) return HYS_ERR_INVALID_ARG;
+  if (!decode_mma_supported(d, dtype)) return HYS_ERR_UNSUPPORTED;
+  *bytes = align256(decode_mma_sparse_tokens_workspace(d, k_tokens));
+  return HYS_OK;
+}
+
+hys_status hysparse_sparse_attn_decode_tokens(const hys_decode_shape* shape, hys_dtype dtype, const void* q,
+                                              const void* k_cache, const void* v_cache, const int* seqlens,
+                                              const int* idx, int k_tokens, int forced_window, void* o,
+                                              void* workspace, size_t workspace_bytes, hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !idx || !o) return HYS_ERR_INVALID_ARG;
+  if (k_tokens < 1 || k_tokens > 16384 || forced_window < 1 || forced_window > 4096) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seqlens) || !aligned16(idx) ||
+      !aligned16(o) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  if (!decode_mma_supported(d, dtype)) return HYS_ERR_UNSUPPORTED;
+  if ((long long)d.B * d.Hkv * d.L >= (1ll << 31)) return HYS_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < align256(decode_mma_sparse_tokens_workspace(d, k_tokens)))
+    return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_decode_sparse_tokens_mma(d, q, k_cache, v_cache, seqlens, idx, k_tokens, forced_window, o,
+                                                   workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -37,9 +37,10 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = kConsumers;              // stage w belongs to consumer warp w
 constexpr int kStageBytes = 2 * 64 * 128 * 2;   // K + V of one 64-key block, D = 128
 constexpr int kMaxList = 72;                     // blocks per split (incl. padding)
+constexpr int kTokSplit = 512;                   // selected tokens per token-sparse split (8 stages of 64)
 constexpr int kPartBytes = kConsumers * 16 * (128 + 2) * 4;
 static_assert(kPartBytes <= kStages * kStageBytes, "partials reuse the stage buffers");
-constexpr int kSmemBytes = kStages * kStageBytes + kMaxList * 16 + 256 + 1024;
+constexpr int kSmemBytes = kStages * kStageBytes + kMaxList * 16 + 256 + kTokSplit * 4 + 1024;
 constexpr int kTargetCtas = 4 * 148;
 #ifndef HYS_DECODE_SPARSE_BPS
 #define HYS_DECODE_SPARSE_BPS 16
@@ -50,7 +51,8 @@ static_assert(kSparseBps <= 32 && kSparseBps <= kMaxList, "one warp gathers a sp
 struct Params {
   int B, L, Hq, Hkv, G, NB;
   const int* seqlens;
-  int mode;         // 0: full layer (contiguous blocks), 1: sparse layer (selected blocks + ring)
+  int mode;         // 0: full layer (contiguous blocks), 1: sparse layer (selected blocks + ring),
+                    // 2: token-sparse layer (selected tokens + the newest W of the cache)
   int bps;          // blocks per split
   int nsplit;       // splits per (b, g)
   int nsp;          // sparse-mode splits over the selected list (the ring is split nsp)
@@ -59,6 +61,9 @@ struct Params {
   int W;            // ring capacity (mode 1)
   const int* swa_len;
   const float* sinks;      // [Hq,2] sink logits of the two branches (mode 1), or null
+  float* logits;           // [B,Hq,L] raw logits of every cached key (mode 0, token scores), or null
+  float* tok_scores;       // [B,Hkv,L] token scores written by the merge (mode 0), or null
+  int forced;              // newest tokens always attended (mode 2)
   const __nv_bfloat16* q;  // [B,Hq,D]
   float* pm;        // [B,Hq,nsplit]
   float* pl;
@@ -69,9 +74,9 @@ struct Params {
 };
 
 struct Entry {  // 16 bytes
-  int row;    // first key row in its tensor
+  int row;    // first key row in its tensor (src 2: first position in the split's token list)
   int valid;  // valid keys (1..64)
-  int src;    // 0: shared cache, 1: SWA ring
+  int src;    // 0: shared cache, 1: SWA ring, 2: gathered tokens of the shared cache
   int blk;    // block id (for the block max)
 };
 
@@ -100,6 +105,7 @@ __device__ __forceinline__ uint32_t sw128(int row, int unit) { return row * 128 
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
+                        const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmVg,
                         const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -109,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   uint64_t* empty = full + kStages;
   int* s_nlist = reinterpret_cast<int*>(empty + kStages);
   volatile int* abort = s_nlist + 1;
+  int* tok = reinterpret_cast<int*>(smem + kStages * kStageBytes + kMaxList * 16 + 256);   // mode 2 token rows
 
   const int sp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,6 +135,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (lane == 0) *s_nlist = __popc(m);
     }
   }
+  if (p.mode == 2 && sp < p.nsp && warp == 0) {
+    // this split's selected tokens (older than the forced window), compacted in order; stage i
+    // gathers tokens 64i .. 64i+63 of the list
+    const int lim = Lb - p.forced;
+    const int* sel = p.idx + ((size_t)b * p.Hkv + g) * p.kb;
+    int cnt = 0;
+    for (int e0 = sp * kTokSplit; e0 < min(p.kb, (sp + 1) * kTokSplit); e0 += 32) {
+      const int e = e0 + lane;
+      const int j = e < min(p.kb, (sp + 1) * kTokSplit) ? sel[e] : -1;
+      const bool keep = j >= 0 && j < lim;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) tok[cnt + __popc(m & ((1u << lane) - 1u))] = j;
+      cnt += __popc(m);
+    }
+    if (lane == 0) {
+      int n = 0;
+      for (int i = 0; 64 * i < cnt; ++i) list[n++] = Entry{64 * i, min(64, cnt - 64 * i), 2, 0};
+      *s_nlist = n;
+    }
+  }
   if (threadIdx.x == 0) {
     // this split's block list
     int n = 0;
@@ -135,9 +162,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const int nb = (Lb + 63) / 64;
       for (int j = sp * p.bps; j < min(nb, (sp + 1) * p.bps); ++j) list[n++] = Entry{64 * j, min(64, Lb - 64 * j), 0, j};
       *s_nlist = n;
-    } else if (sp >= p.nsp) {
+    } else if (p.mode == 1 && sp >= p.nsp) {
       const int nring = p.swa_len ? max(0, min(p.swa_len[b], p.W)) : p.W;
       for (int j = 0; 64 * j < nring; ++j) list[n++] = Entry{64 * j, min(64, nring - 64 * j), 1, j};
+      *s_nlist = n;
+    } else if (p.mode == 2 && sp >= p.nsp) {
+      // the forced newest tokens [L_b - forced, L_b - 1]: contiguous rows of the cache
+      const int w0 = max(0, Lb - p.forced);
+      for (int r = w0; r < Lb; r += 64) list[n++] = Entry{r, min(64, Lb - r), 0, 0};
       *s_nlist = n;
     }
 
@@ -154,22 +186,44 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   if (warp == kConsumers) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      bool ok = true;
-      for (int i = 0; i < nlist; ++i) {
-        const int st = i % kStages;
-        if (!(ok = tc::mbar_wait(&empty[st], ((i / kStages) & 1) ^ 1, abort))) break;
-        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
-        uint8_t* dst = smem + st * kStageBytes;
-        const Entry e = list[i];
+    // Lane 0 waits for the stage and issues contiguous blocks (one TMA box per 64 rows and
+    // 128-byte chunk); a stage of gathered tokens is 16 lanes x 4 rows of tile::gather4.
+    bool ok = true;
+    const int head = b * p.Hkv + g;
+    for (int i = 0; i < nlist; ++i) {
+      const int st = i % kStages;
+      if (lane == 0) {
+        ok = tc::mbar_wait(&empty[st], ((i / kStages) & 1) ^ 1, abort);
+        if (ok) tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      uint8_t* dst = smem + st * kStageBytes;
+      const Entry e = list[i];
+      if (e.src == 2) {
+        if (lane < 16) {
+          int r[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int q = 4 * lane + k;   // rows past the stage's count repeat its first token (masked)
+            r[k] = head * p.L + tok[e.row + (q < e.valid ? q : 0)];
+          }
+          const uint32_t off = 4 * lane * 128;
+          tc::tma_gather4(&tmKg, &full[st], dst + off, 0, r[0], r[1], r[2], r[3]);
+          tc::tma_gather4(&tmKg, &full[st], dst + 8192 + off, 64, r[0], r[1], r[2], r[3]);
+          tc::tma_gather4(&tmVg, &full[st], dst + 16384 + off, 0, r[0], r[1], r[2], r[3]);
+          tc::tma_gather4(&tmVg, &full[st], dst + 24576 + off, 64, r[0], r[1], r[2], r[3]);
+        }
+      } else if (lane == 0) {
         const CUtensorMap* mk = e.src ? &tmKr : &tmK;
         const CUtensorMap* mv = e.src ? &tmVr : &tmV;
-        const int head = b * p.Hkv + g;
         tc::tma_load_3d(mk, &full[st], dst, 0, e.row, head);
         tc::tma_load_3d(mk, &full[st], dst + 8192, 64, e.row, head);
         tc::tma_load_3d(mv, &full[st], dst + 16384, 0, e.row, head);
         tc::tma_load_3d(mv, &full[st], dst + 24576, 64, e.row, head);
       }
+    }
+    if (lane == 0) {
       if (!ok) {
         *abort = 1;
         report_status(p.status, HYS_ERR_TIMEOUT);
@@ -245,6 +299,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (p.mode == 0 && cq == 0) {
         if (h_lo < p.G) p.bmax[((size_t)b * p.Hq + g * p.G + h_lo) * p.NB + e.blk] = bm_lo;
         if (h_hi < p.G) p.bmax[((size_t)b * p.Hq + g * p.G + h_hi) * p.NB + e.blk] = bm_hi;
+      }
+      if (p.logits != nullptr) {
+        // token scores need every key's logit under the final max and sum: keep them
+        float* lrow_lo = p.logits + ((size_t)b * p.Hq + g * p.G + h_lo) * p.L + e.row;
+        float* lrow_hi = p.logits + ((size_t)b * p.Hq + g * p.G + h_hi) * p.L + e.row;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int key = 8 * nt + 2 * cq + c;
+            if (key < e.valid) {
+              if (h_lo < p.G) lrow_lo[key] = s[nt][c];
+              if (h_hi < p.G) lrow_hi[key] = s[nt][2 + c];
+            }
+          }
+        }
       }
       const float mn_lo = fmaxf(m_lo, bm_lo), mn_hi = fmaxf(m_hi, bm_hi);
       const float a_lo = exp2f((m_lo - mn_lo) * sc), a_hi = exp2f((m_hi - mn_hi) * sc);
@@ -350,11 +420,12 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const
   const int g = blockIdx.x, b = blockIdx.y;
   const int Lb = p.seqlens ? max(1, min(p.seqlens[b], p.L)) : p.L;
   const float sc = p.scale_log2;
-  const int nbr = p.mode == 0 ? 1 : 2;
+  const bool two = p.mode == 1;   // the sparse layer merges two branches under the gate
+  const int nbr = two ? 2 : 1;
   if (threadIdx.x < p.G * nbr) {
     const int hh = threadIdx.x % p.G, br = threadIdx.x / p.G;
-    const int s0 = p.mode == 0 ? 0 : (br == 0 ? 0 : p.nsp);
-    const int s1 = p.mode == 0 ? p.nsplit : (br == 0 ? p.nsp : p.nsplit);
+    const int s0 = !two ? 0 : (br == 0 ? 0 : p.nsp);
+    const int s1 = !two ? p.nsplit : (br == 0 ? p.nsp : p.nsplit);
     const size_t ph = ((size_t)b * p.Hq + g * p.G + hh) * p.nsplit;
     float M = -INFINITY;
     for (int s = s0; s < s1; ++s) M = fmaxf(M, p.pm[ph + s]);
@@ -372,20 +443,31 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const
     const size_t ph = ((size_t)b * p.Hq + g * p.G + hh) * p.nsplit;
     float out = 0.0f;
     for (int br = 0; br < nbr; ++br) {
-      const int s0 = p.mode == 0 ? 0 : (br == 0 ? 0 : p.nsp);
-      const int s1 = p.mode == 0 ? p.nsplit : (br == 0 ? p.nsp : p.nsplit);
+      const int s0 = !two ? 0 : (br == 0 ? 0 : p.nsp);
+      const int s1 = !two ? p.nsplit : (br == 0 ? p.nsp : p.nsplit);
       float acc = 0.0f;
       for (int s = s0; s < s1; ++s) {
         const float m = p.pm[ph + s];
         if (m != -INFINITY) acc = fmaf(p.po[(ph + s) * 128 + d], exp2f((m - sM[br][hh]) * sc), acc);
       }
       float w = sInv[br][hh];
-      if (p.mode == 1) w *= sigmoidf_(gate[((size_t)b * p.Hq + g * p.G + hh) * 2 + br]);
+      if (two) w *= sigmoidf_(gate[((size_t)b * p.Hq + g * p.G + hh) * 2 + br]);
       out = fmaf(acc, w, out);
     }
     o[((size_t)b * p.Hq + g * p.G + hh) * 128 + d] = __float2bfloat16_rn(out);
   }
-  if (p.mode == 0) {
+  if (p.mode == 0 && p.tok_scores != nullptr) {
+    // token scores: sum over the group's heads of exp(s - m) / l under the merged statistics
+    float* trow = p.tok_scores + ((size_t)b * p.Hkv + g) * p.L;
+    const float* lg = p.logits + ((size_t)b * p.Hq + g * p.G) * p.L;
+    for (int i = threadIdx.x; i < p.L; i += blockDim.x) {
+      float a = 0.0f;
+      if (i < Lb)
+        for (int hh = 0; hh < p.G; ++hh) a += exp2f((lg[(size_t)hh * p.L + i] - sM[0][hh]) * sc) * sInv[0][hh];
+      trow[i] = a;
+    }
+  }
+  if (p.mode == 0 && scores != nullptr) {
     const int nb = (Lb + 63) / 64;
     for (int j = threadIdx.x; j < p.NB; j += blockDim.x) {
       float a = 0.0f;
@@ -428,6 +510,19 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int heads) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K or V as a 2-D [B*Hkv*L][128] tensor with a one-row box (64 columns) for tile::gather4
+bool make_gather_map(CUtensorMap* m, const void* base, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int full_bps(const DecodeDims& d) {
   const long long work = (long long)d.NB * d.B * d.Hkv;
   long long bps = (work + kTargetCtas - 1) / kTargetCtas;
@@ -459,6 +554,9 @@ void fill_common(Params& p, const DecodeDims& d, const void* q, const int* seqle
   p.W = 0;
   p.swa_len = nullptr;
   p.sinks = nullptr;
+  p.logits = nullptr;
+  p.tok_scores = nullptr;
+  p.forced = 0;
   p.nsp = 0;
 }
 
@@ -500,7 +598,7 @@ cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const voi
   fill_common(p, d, q, seqlens, ws, nsplit);
   p.mode = 0;
   p.bps = bps;
-  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), scores,
@@ -529,10 +627,68 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   p.W = W;
   p.swa_len = swa_len;
   p.sinks = sinks;
-  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
+  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, gate, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
+  return cudaGetLastError();
+}
+
+size_t decode_mma_full_tokens_workspace(const DecodeDims& d) {
+  return decode_mma_full_workspace(d) + sizeof(float) * (size_t)d.B * d.Hq * d.L;
+}
+
+cudaError_t launch_decode_full_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                          const int* seqlens, void* o, float* tok_scores, void* ws, cudaStream_t s) {
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv)) return cudaErrorInvalidValue;
+  cudaError_t e = set_smem();
+  if (e != cudaSuccess) return e;
+  Params p;
+  const int bps = full_bps(d);
+  const int nsplit = (d.NB + bps - 1) / bps;
+  fill_common(p, d, q, seqlens, ws, nsplit);
+  p.mode = 0;
+  p.bps = bps;
+  p.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + decode_mma_full_workspace(d));
+  p.tok_scores = tok_scores;
+  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, mk, mv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
+  return cudaGetLastError();
+}
+
+int decode_token_splits(int kt) { return (kt + kTokSplit - 1) / kTokSplit; }
+
+size_t decode_mma_sparse_tokens_workspace(const DecodeDims& d, int kt) {
+  const size_t nsplit = decode_token_splits(kt) + 1;
+  return sizeof(float) * ((size_t)d.B * d.Hq * nsplit * (2 + 128));
+}
+
+cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                            const int* seqlens, const int* idx, int kt, int forced, void* o, void* ws,
+                                            cudaStream_t s) {
+  CUtensorMap mk, mv, mkg, mvg;
+  const long long rows = (long long)d.B * d.Hkv * d.L;
+  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv) || !make_gather_map(&mkg, kc, rows) ||
+      !make_gather_map(&mvg, vc, rows))
+    return cudaErrorInvalidValue;
+  cudaError_t e = set_smem();
+  if (e != cudaSuccess) return e;
+  Params p;
+  const int nsp = decode_token_splits(kt);
+  fill_common(p, d, q, seqlens, ws, nsp + 1);
+  p.mode = 2;
+  p.bps = kTokSplit;
+  p.nsp = nsp;
+  p.idx = idx;
+  p.kb = kt;
+  p.forced = forced;
+  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, mkg, mvg, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
   return cudaGetLastError();
 }
 

@@ -61,6 +61,8 @@ cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, in
                                const int* seqlens, int L, bool decode, cudaStream_t s);
 cudaError_t launch_topk_tokens(const PrefillDims& d, const float* scores, int k_tokens, int forced,
                                int* idx, cudaStream_t s);
+cudaError_t launch_topk_decode_tokens(const float* scores, int* idx, int B, int Hkv, int L, int k_tokens, int forced,
+                                      const int* seqlens, cudaStream_t s);
 
 // ---- sparse layer ----------------------------------------------------------------------------
 cudaError_t launch_sparse_attn_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
@@ -94,6 +96,14 @@ size_t decode_mma_sparse_workspace(const DecodeDims& d, int kb);
 cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                    const int* seqlens, void* o, float* scores, hys_reduce red, void* ws,
                                    cudaStream_t s);
+// token-variant decode (bf16, D = 128, G <= 16)
+size_t decode_mma_full_tokens_workspace(const DecodeDims& d);
+cudaError_t launch_decode_full_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                          const int* seqlens, void* o, float* tok_scores, void* ws, cudaStream_t s);
+size_t decode_mma_sparse_tokens_workspace(const DecodeDims& d, int kt);
+cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                            const int* seqlens, const int* idx, int kt, int forced, void* o, void* ws,
+                                            cudaStream_t s);
 cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                      const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
                                      const int* swa_len, const float* gate, const float* sinks, void* o, void* ws,

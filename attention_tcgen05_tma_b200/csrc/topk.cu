@@ -137,14 +137,22 @@ __global__ void __launch_bounds__(kBlkThreads) topk_blocks_kernel(const float* _
 
 constexpr int kTokThreads = 1024;
 
-// Token candidates of tile I are positions [0, e_I - forced], e_I = min(64I+63, N-1).
+// Token candidates of tile I are positions [0, e_I - forced], e_I = min(64I+63, N-1).  In decode
+// (one row per sequence and KV group, N = L) the new token is e = L_b - 1.
 __global__ void __launch_bounds__(kTokThreads) topk_tokens_kernel(const float* __restrict__ scores,
                                                                   int* __restrict__ idx, int T, int N, int k,
-                                                                  int forced) {
+                                                                  int forced, const int* __restrict__ seqlens,
+                                                                  int Hkv, int decode) {
   __shared__ RadixSmem<kTokThreads / 32> sm;
   const int row = blockIdx.x;
-  const int I = row % T;
-  const int e = min(N, (I + 1) * 64) - 1;
+  int e;
+  if (decode) {
+    const int b = row / Hkv;
+    e = (seqlens ? max(1, min(seqlens[b], N)) : N) - 1;
+  } else {
+    const int I = row % T;
+    e = min(N, (I + 1) * 64) - 1;
+  }
   const int n = max(0, e - forced + 1);
   const float* srow = scores + (size_t)row * N;
   int* out = idx + (size_t)row * k;
@@ -173,7 +181,14 @@ cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, in
 
 cudaError_t launch_topk_tokens(const PrefillDims& d, const float* scores, int k_tokens, int forced, int* idx,
                                cudaStream_t s) {
-  topk_tokens_kernel<<<d.B * d.Hkv * d.T, kTokThreads, 0, s>>>(scores, idx, d.T, d.N, k_tokens, forced);
+  topk_tokens_kernel<<<d.B * d.Hkv * d.T, kTokThreads, 0, s>>>(scores, idx, d.T, d.N, k_tokens, forced, nullptr,
+                                                                d.Hkv, 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_decode_tokens(const float* scores, int* idx, int B, int Hkv, int L, int k_tokens, int forced,
+                                      const int* seqlens, cudaStream_t s) {
+  topk_tokens_kernel<<<B * Hkv, kTokThreads, 0, s>>>(scores, idx, 1, L, k_tokens, forced, seqlens, Hkv, 1);
   return cudaGetLastError();
 }
 

@@ -28,7 +28,11 @@ EXPORTED = (
     "hysparse_sparse_attn_workspace_size", "hysparse_sparse_attn",
     "hysparse_sparse_attn_tokens_workspace_size", "hysparse_sparse_attn_tokens",
     "hysparse_full_attn_select_decode_workspace_size", "hysparse_full_attn_select_decode",
-    "hysparse_topk_decode", "hysparse_sparse_attn_decode_workspace_size", "hysparse_sparse_attn_decode", "hysparse_full_attn_select_decode_noalloc",
+    "hysparse_topk_decode", "hysparse_sparse_attn_decode_workspace_size", "hysparse_sparse_attn_decode",
+    "hysparse_full_attn_select_decode_noalloc",
+    "hysparse_full_attn_select_decode_tokens_workspace_size", "hysparse_full_attn_select_decode_tokens",
+    "hysparse_topk_decode_tokens", "hysparse_sparse_attn_decode_tokens_workspace_size",
+    "hysparse_sparse_attn_decode_tokens",
 )
 
 
@@ -74,6 +78,11 @@ _SIGS = {
     "hysparse_sparse_attn_decode_workspace_size": ([_DSH, _I, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_sparse_attn_decode": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
                                     _I),
+    "hysparse_full_attn_select_decode_tokens_workspace_size": ([_DSH, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_full_attn_select_decode_tokens": ([_DSH, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "hysparse_topk_decode_tokens": ([_DSH, _P, _I, _I, _P, _P, _P], _I),
+    "hysparse_sparse_attn_decode_tokens_workspace_size": ([_DSH, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_sparse_attn_decode_tokens": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P], _I),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -202,6 +211,37 @@ def hysparse_sparse_attn_decode(shape, dtype, q, kc, vc, seqlens, idx, kb, kr, v
                                 ws, ws_bytes, stream) -> int:
     return load().hysparse_sparse_attn_decode(ctypes.byref(shape), dtype, q, kc, vc, seqlens, idx, kb, kr, vr, window,
                                               swa_len, gate, sinks, o, ws, ws_bytes, stream)
+
+
+def hysparse_full_attn_select_decode_tokens_workspace_size(shape: hys_decode_shape, dtype: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_full_attn_select_decode_tokens_workspace_size(ctypes.byref(shape), dtype, ctypes.byref(n)),
+           "hysparse_full_attn_select_decode_tokens_workspace_size")
+    return n.value
+
+
+def hysparse_full_attn_select_decode_tokens(shape, dtype, q, kc, vc, seqlens, o, tok_scores, ws, ws_bytes,
+                                            stream) -> int:
+    return load().hysparse_full_attn_select_decode_tokens(ctypes.byref(shape), dtype, q, kc, vc, seqlens, o,
+                                                          tok_scores, ws, ws_bytes, stream)
+
+
+def hysparse_topk_decode_tokens(shape, tok_scores, k_tokens, forced, seqlens, idx, stream) -> int:
+    return load().hysparse_topk_decode_tokens(ctypes.byref(shape), tok_scores, k_tokens, forced, seqlens, idx, stream)
+
+
+def hysparse_sparse_attn_decode_tokens_workspace_size(shape: hys_decode_shape, dtype: int, k_tokens: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_sparse_attn_decode_tokens_workspace_size(ctypes.byref(shape), dtype, k_tokens,
+                                                                    ctypes.byref(n)),
+           "hysparse_sparse_attn_decode_tokens_workspace_size")
+    return n.value
+
+
+def hysparse_sparse_attn_decode_tokens(shape, dtype, q, kc, vc, seqlens, idx, k_tokens, forced, o, ws, ws_bytes,
+                                       stream) -> int:
+    return load().hysparse_sparse_attn_decode_tokens(ctypes.byref(shape), dtype, q, kc, vc, seqlens, idx, k_tokens,
+                                                     forced, o, ws, ws_bytes, stream)
 
 
 # ----------------------------------------------------------------------------- torch helpers
@@ -366,4 +406,50 @@ def sparse_attn_decode(q, k_cache, v_cache, idx, k_ring, v_ring, gate_logits, *,
                                        _ptr(gate_logits), _ptr(sinks), _ptr(o), _ptr(workspace), workspace.numel(),
                                        _stream(stream)),
            "hysparse_sparse_attn_decode")
+    return o
+
+
+def full_attn_select_decode_tokens(q, k_cache, v_cache, *, seqlens=None, o=None, tok_scores=None, workspace=None,
+                                   stream=None):
+    """Token-variant decode full layer: o [B,Hq,D] and token scores [B,Hkv,L]."""
+    torch = _torch()
+    sh = decode_shape(q, k_cache)
+    if o is None:
+        o = torch.empty_like(q)
+    if tok_scores is None:
+        tok_scores = torch.empty((sh.B, sh.Hkv, sh.L), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = workspace_for(hysparse_full_attn_select_decode_tokens_workspace_size(sh, _dt(q)), q.device)
+    _check(hysparse_full_attn_select_decode_tokens(sh, _dt(q), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                                                   _ptr(o), _ptr(tok_scores), _ptr(workspace), workspace.numel(),
+                                                   _stream(stream)),
+           "hysparse_full_attn_select_decode_tokens")
+    return o, tok_scores
+
+
+def topk_decode_tokens(tok_scores, k_tokens: int, forced_window: int, *, seqlens=None, idx=None, stream=None):
+    torch = _torch()
+    B, Hkv, L = tok_scores.shape
+    sh = hys_decode_shape(B, L, Hkv, Hkv, 64, 64)
+    if idx is None:
+        idx = torch.empty((B, Hkv, k_tokens), dtype=torch.int32, device=tok_scores.device)
+    _check(hysparse_topk_decode_tokens(sh, _ptr(tok_scores), k_tokens, forced_window, _ptr(seqlens), _ptr(idx),
+                                       _stream(stream)), "hysparse_topk_decode_tokens")
+    return idx
+
+
+def sparse_attn_decode_tokens(q, k_cache, v_cache, idx, forced_window: int, *, seqlens=None, o=None, workspace=None,
+                              stream=None):
+    """Token-variant sparse decode layer: the selected tokens plus the newest forced_window."""
+    torch = _torch()
+    sh = decode_shape(q, k_cache)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(hysparse_sparse_attn_decode_tokens_workspace_size(sh, _dt(q), idx.shape[-1]),
+                                  q.device)
+    _check(hysparse_sparse_attn_decode_tokens(sh, _dt(q), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                                              _ptr(idx), idx.shape[-1], forced_window, _ptr(o), _ptr(workspace),
+                                              workspace.numel(), _stream(stream)),
+           "hysparse_sparse_attn_decode_tokens")
     return o

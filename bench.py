@@ -40,8 +40,8 @@ from attention_tcgen05_tma_b200.distributed import max_over_ranks  # noqa: E402
 # to its own units; it reports null once the sources differ from the captured ones.
 NCU_TRAFFIC = {
     "sparse_attn": {"bytes": 199350272 + 103375360, "units": 1024,
-                    "sources": ("sparse_attn_tc.cu", "tc_ptx.cuh", "common.cuh", "kernels.h"),
-                    "sha256": "bc9cde93797a08aad9e8e31f9d8b394ae1ccd055c2a3cb95972ce9cb037d03cc"},
+                    "sources": ("sparse_attn_tc.cu", "tc_ptx.cuh", "common.cuh"),
+                    "sha256": "ffeba27b9054c45f70d67cd2a2b4d93a75f69d6b511b3d5c1dde0594ada4bd0e"},
 }
 
 
@@ -341,7 +341,11 @@ def run_ours(args, torch, dist, rank, world, dev):
     ms_sinks = time_call(torch, lambda: H.sparse_attn(x["q_sparse"][0], x["k"], x["v"], step.idx, x["k_swa"][0],
                                                       x["v_swa"][0], w.window, x["gate"][0], sinks=sinks,
                                                       o=step.o_sp, workspace=step.ws_sp))
+    ms_plain = time_call(torch, lambda: H.sparse_attn(x["q_sparse"][0], x["k"], x["v"], step.idx, x["k_swa"][0],
+                                                      x["v_swa"][0], w.window, x["gate"][0], o=step.o_sp,
+                                                      workspace=step.ws_sp))
     kernels["sparse_attn_sinks_ms"] = round(ms_sinks, 4)
+    kernels["sparse_attn_same_layer_no_sinks_ms"] = round(ms_plain, 4)   # same repeated-call timing
     kernels["sparse_attn_sinks_tflops"] = round(sp_flops / (ms_sinks / 1e3) / 1e12, 2)
 
     res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -359,6 +363,8 @@ def run_ours(args, torch, dist, rank, world, dev):
 
     if not args.no_decode:
         res["decode"] = run_decode(args, torch, dist, rank, world, dev, peaks, peak_src)
+    if not args.no_decode_tokens:
+        res["decode_tokens"] = run_decode_tokens(args, torch, dist, rank, world, dev, peaks, peak_src)
     if not args.no_token:
         res["token"] = run_token(args, torch, dist, rank, world, dev, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -370,6 +376,74 @@ def _uses_tc(H, w):
     sh = H.hys_shape(w.B, w.N, w.Hq, w.Hkv, w.D, 64)
     return H.hysparse_full_attn_select_workspace_size(sh, H.HYS_BF16, H.HYS_GRAN_BLOCK) != \
         4 * w.B * w.Hq * w.T * w.NB
+
+
+def run_decode_tokens(args, torch, dist, rank, world, dev, peaks, peak_src):
+    """Token-variant decode step on the decode workload's cache: full layer with token scores,
+    top-2048 tokens older than the forced newest 128, and the token-sparse layers."""
+    from attention_tcgen05_tma_b200 import hysparse as H
+    from attention_tcgen05_tma_b200 import inputs as I
+    w = I.WORKLOADS[args.decode_workload]
+    kt, W = 2048, 128
+    x = make_decode_inputs(w, torch, dev, w.layers, seed_offset=1000 * rank)
+    for key in ("k_swa", "v_swa", "gate"):
+        x[key] = []   # the token variant has no SWA ring and no gate
+    torch.cuda.empty_cache()
+    o = torch.empty_like(x["q"])
+    ts = torch.empty((w.B, w.Hkv, w.N), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.Hkv, kt), dtype=torch.int32, device=dev)
+    osp = torch.empty_like(x["q"])
+    sh = H.decode_shape(x["q"], x["k"])
+    ws = H.workspace_for(H.hysparse_full_attn_select_decode_tokens_workspace_size(sh, H.HYS_BF16), dev)
+    ws_sp = H.workspace_for(H.hysparse_sparse_attn_decode_tokens_workspace_size(sh, H.HYS_BF16, kt), dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        H.full_attn_select_decode_tokens(x["q"], x["k"], x["v"], o=o, tok_scores=ts, workspace=ws)
+        if ev:
+            ev[1].record()
+        H.topk_decode_tokens(ts, kt, W, idx=idx)
+        if ev:
+            ev[2].record()
+        for l in range(w.layers):
+            H.sparse_attn_decode_tokens(x["q_sparse"][l], x["k"], x["v"], idx, W, o=osp, workspace=ws_sp)
+        if ev:
+            ev[3].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    full_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    topk_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    sp_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    ms_step = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps, dist, dev)
+    # full layer: K and V once, plus every key's logit written and read back for the scores
+    full_bytes = 2.0 * w.B * w.Hkv * w.N * w.D * 2 + 2.0 * w.B * w.Hq * w.N * 4
+    sp_bytes = 2.0 * w.B * w.Hkv * (kt + W) * w.D * 2
+    hbm = peaks["hbm_gbs"]
+    full_gbs = full_bytes / (full_ms / 1e3) / 1e9
+    sp_gbs = sp_bytes / (sp_ms / w.layers / 1e3) / 1e9
+    res = {"us_per_token": round(ms_step * 1e3 / (w.B * world), 3),
+           "ms_per_step": round(ms_step, 4),
+           "config": f"B={w.B} L={w.N} Hq={w.Hq} Hkv={w.Hkv} D={w.D}, 1 full + {w.layers} token-sparse, top-{kt} "
+                     f"tokens + forced newest {W}",
+           "full_ms": round(full_ms, 4), "topk_ms": round(topk_ms, 4), "sparse_ms_per_layer": round(sp_ms / w.layers, 4),
+           "roofline": {"kernel": "full_attn_select_decode_tokens", "bound": "hbm", "achieved": round(full_gbs, 1),
+                        "peak": hbm, "unit": "GB/s", "frac": round(full_gbs / hbm, 4), "traffic": None,
+                        "peak_source": f"{peak_src} hbm_gbs"},
+           "sparse_roofline": {"bound": "hbm", "achieved": round(sp_gbs, 1), "peak": hbm, "unit": "GB/s",
+                               "frac": round(sp_gbs / hbm, 4)}}
+    del x, ts, ws, ws_sp
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
@@ -696,6 +770,7 @@ def main():
     ap.add_argument("--workload", default="moe80b", help="prefill workload (moe80b, dense7b, ...)")
     ap.add_argument("--decode-workload", default="decode", help="decode workload (decode, decode_small)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-decode-tokens", action="store_true", help="skip the token-variant decode leg")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-token", action="store_true")

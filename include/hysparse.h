@@ -244,6 +244,47 @@ HYS_API hys_status hysparse_sparse_attn_decode(const hys_decode_shape* shape, hy
                                        const float* gate_logits, const float* sinks, void* o,
                                        void* workspace, size_t workspace_bytes, hys_stream_t stream);
 
+/* ------------------------------------------------------------------------------------
+ * Token-variant decode ([HS2] "Twenty lines of algorithmic intuition", with the token
+ * granularity of "Precise retrieval without a separate indexer").  bf16, D = 128 and
+ * Hq/Hkv <= 16 (the tensor-core decode path); other shapes and types return
+ * HYS_ERR_UNSUPPORTED.
+ *
+ * hysparse_full_attn_select_decode_tokens: the full layer for the new token (position
+ *   L_b - 1 of an L_b-token cache), o [B,Hq,D], and its token scores tok_scores [B,Hkv,L]
+ *   fp32: score[b,g,i] = sum over the group's heads of the new token's attention probability
+ *   of cached token i (0 for i >= L_b).  workspace: at least
+ *   hysparse_full_attn_select_decode_tokens_workspace_size() bytes (per-split partial softmax
+ *   states and every key's logit, B*Hq*L fp32).
+ * hysparse_topk_decode_tokens: idx [B,Hkv,k_tokens] int32, the k_tokens highest scores among
+ *   the tokens older than the forced newest window, positions [0, L_b - 1 - forced_window];
+ *   ties to the lower position; ascending, padded with -1.  1 <= k_tokens <= 16384.
+ * hysparse_sparse_attn_decode_tokens: the token-sparse layer for the new token: the selected
+ *   cached tokens idx[b,g,:] (entries outside [0, L_b - 1 - forced_window] are ignored) united
+ *   with the newest forced_window tokens [L_b - forced_window, L_b - 1], each token once, over
+ *   the shared cache; no gate.  1 <= forced_window <= 4096.  workspace: at least
+ *   hysparse_sparse_attn_decode_tokens_workspace_size() bytes.
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_full_attn_select_decode_tokens_workspace_size(const hys_decode_shape* shape,
+                                                                      hys_dtype dtype, size_t* bytes);
+HYS_API hys_status hysparse_full_attn_select_decode_tokens(const hys_decode_shape* shape, hys_dtype dtype,
+                                                       const void* q, const void* k_cache,
+                                                       const void* v_cache, const int* seqlens, void* o,
+                                                       float* tok_scores, void* workspace,
+                                                       size_t workspace_bytes, hys_stream_t stream);
+HYS_API hys_status hysparse_topk_decode_tokens(const hys_decode_shape* shape, const float* tok_scores,
+                                           int k_tokens, int forced_window, const int* seqlens, int* idx,
+                                           hys_stream_t stream);
+HYS_API hys_status hysparse_sparse_attn_decode_tokens_workspace_size(const hys_decode_shape* shape,
+                                                                 hys_dtype dtype, int k_tokens,
+                                                                 size_t* bytes);
+HYS_API hys_status hysparse_sparse_attn_decode_tokens(const hys_decode_shape* shape, hys_dtype dtype,
+                                                  const void* q, const void* k_cache,
+                                                  const void* v_cache, const int* seqlens,
+                                                  const int* idx, int k_tokens, int forced_window,
+                                                  void* o, void* workspace, size_t workspace_bytes,
+                                                  hys_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -94,3 +94,23 @@ def test_entry_points_reject_bad_arguments_without_launching(lib):
                                          16, None, 0, None) == H.HYS_ERR_WORKSPACE
     assert H.hysparse_full_attn_select_decode(dsh, H.HYS_F32, 16, 16, 16, None, 16, 16, 0, None, 0, None) \
         == H.HYS_ERR_WORKSPACE
+
+
+def test_token_decode_entry_points_validate(lib):
+    dsh = H.hys_decode_shape(2, 1000, 16, 2, 128, 64)
+    assert H.hysparse_full_attn_select_decode_tokens_workspace_size(dsh, H.HYS_BF16) > 0
+    assert H.hysparse_sparse_attn_decode_tokens_workspace_size(dsh, H.HYS_BF16, 256) > 0
+    # fp32 / D = 64 have no token-variant decode path: unsupported, nothing launched
+    fsh = H.hys_decode_shape(2, 1000, 16, 2, 64, 64)
+    assert H.hysparse_full_attn_select_decode_tokens(fsh, H.HYS_F32, 16, 16, 16, None, 16, 16, 16, 1 << 20, None) \
+        == H.HYS_ERR_UNSUPPORTED
+    # null output, bad budget / window, misaligned pointers, short workspace
+    assert H.hysparse_full_attn_select_decode_tokens(dsh, H.HYS_BF16, 16, 16, 16, None, 16, None, 16, 1 << 20, None) \
+        == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_topk_decode_tokens(dsh, 16, 0, 64, None, 16, None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_topk_decode_tokens(dsh, 16, 64, 0, None, 16, None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_topk_decode_tokens(dsh, 8, 64, 64, None, 16, None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_sparse_attn_decode_tokens(dsh, H.HYS_BF16, 16, 16, 16, None, 16, 64, 5000, 16, 16, 1 << 20,
+                                                None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_sparse_attn_decode_tokens(dsh, H.HYS_BF16, 16, 16, 16, None, 16, 64, 64, 16, 16, 64,
+                                                None) == H.HYS_ERR_WORKSPACE

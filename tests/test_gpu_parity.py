@@ -255,3 +255,45 @@ def test_decode_sinks(dt, D, Hq, Hkv):
     ref = O.decode_sparse(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], a["gate"][0],
                           None, swa_len, sinks=sinks.astype(np.float64))
     assert np.max(np.abs(to_np(osp) - ref)) <= TOL[dt]
+
+
+TOKEN_DECODE_CASES = [
+    # name, B, L, Hq, Hkv, k_tokens, forced, ragged
+    ("g8_ragged", 3, 1500, 16, 2, 100, 64, True),
+    ("g16_long", 2, 5000, 16, 1, 700, 128, False),
+    ("g8_keep_all", 2, 600, 16, 2, 4096, 64, True),    # every candidate kept: dense decode
+]
+
+
+@pytest.mark.parametrize("case", TOKEN_DECODE_CASES, ids=[c[0] for c in TOKEN_DECODE_CASES])
+def test_token_decode(case):
+    name, B, L, Hq, Hkv, kt, W, ragged = case
+    D = 128
+    w = I.scaled(I.WORKLOADS["decode"], B=B, N=L, Hq=Hq, Hkv=Hkv, D=D, topk=kt, window=W, layers=1, seed=12,
+                 scale_std=1.0 / np.sqrt(D))
+    a = I.decode_arrays(w, layers=1)
+    seqlens = np.array([L - 211 * b for b in range(B)], dtype=np.int32) if ragged else None
+    q, kc, vc = (to_dev(a[x], "bf16") for x in ("q", "k", "v"))
+    sl = torch.from_numpy(seqlens).cuda() if ragged else None
+    o, ts = H.full_attn_select_decode_tokens(q, kc, vc, seqlens=sl)
+    idx = H.topk_decode_tokens(ts, kt, W, seqlens=sl)
+    qs = to_dev(a["q_sparse"][0], "bf16")
+    osp = H.sparse_attn_decode_tokens(qs, kc, vc, idx, W, seqlens=sl)
+    torch.cuda.synchronize()
+    assert H.hysparse_get_device_status() == 0
+    o_ref, _ = O.decode_full(a["q"], a["k"], a["v"], seqlens)
+    assert np.max(np.abs(to_np(o) - o_ref)) <= TOL["bf16"]
+    ts_ref = O.decode_token_scores(a["q"], a["k"], seqlens)
+    ts_gpu = to_np(ts)
+    assert score_rel_err(ts_ref, ts_gpu) <= 1e-3
+    gidx = idx.cpu().numpy().astype(np.int64)
+    for b in range(B):
+        Lb = int(seqlens[b]) if ragged else L
+        assert np.all(ts_gpu[b, :, Lb:] == 0)
+        for g in range(Hkv):
+            check_selection(ts_ref[b, g], ts_gpu[b, g], gidx[b, g], max(0, Lb - W), kt)
+    ref = O.decode_token_sparse(a["q_sparse"][0], a["k"], a["v"], gidx, W, seqlens)
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL["bf16"]
+    if name == "g8_keep_all":   # every candidate selected: the sparse layer is dense decode of q'
+        dense, _ = O.decode_full(a["q_sparse"][0], a["k"], a["v"], seqlens)
+        assert np.max(np.abs(to_np(osp) - dense)) <= TOL["bf16"]
