@@ -10,7 +10,9 @@
 // w, w+C, ... of the split, so every stage's barrier phases are consumed by one warp in
 // order (a parity wait cannot be fooled by a phase two ahead) and the max logit of a
 // block (HySparse's m~) is a warp-local reduction.  A sparse layer's split holds 16 of the
-// selected blocks; its SWA ring is a split of its own.
+// selected blocks; its SWA ring is a split of its own.  A token-sparse layer's split holds up
+// to 1024 selected tokens, copied row by row with cp.async into the same stage layout, and the
+// forced newest tokens are a split of contiguous boxes.
 // The G <= 16 query heads of the group form the 16 rows of mma.sync.m16n8k16 tiles
 // (zero-padded): S = Q K^T (64 mma per block), online softmax in registers, O += P V (64
 // mma per block).  The warps' partial (m, l, O) are merged in shared memory (reusing the stages) and the
@@ -37,7 +39,11 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = kConsumers;              // stage w belongs to consumer warp w
 constexpr int kStageBytes = 2 * 64 * 128 * 2;   // K + V of one 64-key block, D = 128
 constexpr int kMaxList = 72;                     // blocks per split (incl. padding)
-constexpr int kTokSplit = 512;                   // selected tokens per token-sparse split (8 stages of 64)
+#ifndef HYS_DECODE_TOK_SPLIT
+#define HYS_DECODE_TOK_SPLIT 1024
+#endif
+constexpr int kTokSplit = HYS_DECODE_TOK_SPLIT;  // selected tokens per token-sparse split (stages of 64)
+static_assert(kTokSplit % 32 == 0 && kTokSplit <= 1024, "a split's list is read in one pass of 32-entry chunks");
 constexpr int kPartBytes = kConsumers * 16 * (128 + 2) * 4;
 static_assert(kPartBytes <= kStages * kStageBytes, "partials reuse the stage buffers");
 constexpr int kSmemBytes = kStages * kStageBytes + kMaxList * 16 + 256 + kTokSplit * 4 + 1024;
@@ -65,6 +71,8 @@ struct Params {
   float* tok_scores;       // [B,Hkv,L] token scores written by the merge (mode 0), or null
   int forced;              // newest tokens always attended (mode 2)
   const __nv_bfloat16* q;  // [B,Hq,D]
+  const __nv_bfloat16* kc; // [B,Hkv,L,D] shared cache (mode 2 gathers rows from it)
+  const __nv_bfloat16* vc;
   float* pm;        // [B,Hq,nsplit]
   float* pl;
   float* po;        // [B,Hq,nsplit,D]
@@ -102,10 +110,20 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // byte offset of (row, 16-byte unit) inside a [64 rows][128 B] 128-byte-swizzled box
 __device__ __forceinline__ uint32_t sw128(int row, int unit) { return row * 128 + ((unit ^ (row & 7)) << 4); }
 
+// 16-byte global -> shared copy on the load/store path (kept in L2 only), and an arrival on a
+// stage barrier that fires once every earlier copy of this thread has landed (the barrier's
+// expected count is raised for it, so it adds no arrival of its own)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_bar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
-                        const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmVg,
                         const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -138,15 +156,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (p.mode == 2 && sp < p.nsp && warp == 0) {
     // this split's selected tokens (older than the forced window), compacted in order; stage i
     // gathers tokens 64i .. 64i+63 of the list
+    // (all of the split's entries are loaded before the first ballot, so their latencies overlap)
     const int lim = Lb - p.forced;
     const int* sel = p.idx + ((size_t)b * p.Hkv + g) * p.kb;
+    const int e_lo = sp * kTokSplit, e_hi = min(p.kb, e_lo + kTokSplit);
+    int jv[kTokSplit / 32];
+#pragma unroll
+    for (int c = 0; c < kTokSplit / 32; ++c) {
+      const int e = e_lo + 32 * c + lane;
+      jv[c] = e < e_hi ? sel[e] : -1;
+    }
     int cnt = 0;
-    for (int e0 = sp * kTokSplit; e0 < min(p.kb, (sp + 1) * kTokSplit); e0 += 32) {
-      const int e = e0 + lane;
-      const int j = e < min(p.kb, (sp + 1) * kTokSplit) ? sel[e] : -1;
-      const bool keep = j >= 0 && j < lim;
+#pragma unroll
+    for (int c = 0; c < kTokSplit / 32; ++c) {
+      const bool keep = jv[c] >= 0 && jv[c] < lim;
       const unsigned m = __ballot_sync(0xffffffffu, keep);
-      if (keep) tok[cnt + __popc(m & ((1u << lane) - 1u))] = j;
+      if (keep) tok[cnt + __popc(m & ((1u << lane) - 1u))] = jv[c];
       cnt += __popc(m);
     }
     if (lane == 0) {
@@ -187,36 +212,38 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (warp == kConsumers) {
     // ---------------------------------------------------------------- producer
     // Lane 0 waits for the stage and issues contiguous blocks (one TMA box per 64 rows and
-    // 128-byte chunk); a stage of gathered tokens is 16 lanes x 4 rows of tile::gather4.
+    // 128-byte chunk).  Gathered tokens go through the load/store path instead (scattered
+    // 256-byte rows are too small for TMA's per-request rate): the warp's 32 lanes copy 16-byte
+    // units, two token rows per instruction, into the same swizzled layout as the boxes.
     bool ok = true;
     const int head = b * p.Hkv + g;
     for (int i = 0; i < nlist; ++i) {
       const int st = i % kStages;
-      if (lane == 0) {
-        ok = tc::mbar_wait(&empty[st], ((i / kStages) & 1) ^ 1, abort);
-        if (ok) tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
-      }
+      if (lane == 0) ok = tc::mbar_wait(&empty[st], ((i / kStages) & 1) ^ 1, abort);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       uint8_t* dst = smem + st * kStageBytes;
       const Entry e = list[i];
       if (e.src == 2) {
-        if (lane < 16) {
-          int r[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int q = 4 * lane + k;   // rows past the stage's count repeat its first token (masked)
-            r[k] = head * p.L + tok[e.row + (q < e.valid ? q : 0)];
-          }
-          const uint32_t off = 4 * lane * 128;
-          tc::tma_gather4(&tmKg, &full[st], dst + off, 0, r[0], r[1], r[2], r[3]);
-          tc::tma_gather4(&tmKg, &full[st], dst + 8192 + off, 64, r[0], r[1], r[2], r[3]);
-          tc::tma_gather4(&tmVg, &full[st], dst + 16384 + off, 0, r[0], r[1], r[2], r[3]);
-          tc::tma_gather4(&tmVg, &full[st], dst + 24576 + off, 64, r[0], r[1], r[2], r[3]);
+        const int u = lane & 15;   // 16-byte unit of the 256-byte row: units 0-7 in the low box, 8-15 the high
+        const uint32_t sdst = tc::smem_u32(dst) + (u >> 3) * 8192;
+        const __nv_bfloat16* kh = p.kc + (size_t)head * p.L * 128 + u * 8;
+        const __nv_bfloat16* vh = p.vc + (size_t)head * p.L * 128 + u * 8;
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+          const int q = 2 * j + (lane >> 4);   // rows past the stage's count repeat its first token (masked)
+          const size_t r = (size_t)tok[e.row + (q < e.valid ? q : 0)] * 128;
+          const uint32_t so = sdst + sw128(q, u & 7);
+          cp_async16(so, kh + r);
+          cp_async16(so + 16384, vh + r);
         }
+        cp_async_bar_arrive(&full[st]);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&full[st]);
       } else if (lane == 0) {
         const CUtensorMap* mk = e.src ? &tmKr : &tmK;
         const CUtensorMap* mv = e.src ? &tmVr : &tmV;
+        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
         tc::tma_load_3d(mk, &full[st], dst, 0, e.row, head);
         tc::tma_load_3d(mk, &full[st], dst + 8192, 64, e.row, head);
         tc::tma_load_3d(mv, &full[st], dst + 16384, 0, e.row, head);
@@ -231,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       for (int i = max(0, nlist - kStages); i < nlist; ++i)
         tc::mbar_wait(&full[i % kStages], (i / kStages) & 1, abort, 100000000ull);
     }
+    cp_async_wait_all();
     __syncwarp();
     tc::named_bar_sync(1, kThreads);
   } else {
@@ -510,19 +538,6 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int heads) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// K or V as a 2-D [B*Hkv*L][128] tensor with a one-row box (64 columns) for tile::gather4
-bool make_gather_map(CUtensorMap* m, const void* base, long long rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {256};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int full_bps(const DecodeDims& d) {
   const long long work = (long long)d.NB * d.B * d.Hkv;
   long long bps = (work + kTargetCtas - 1) / kTargetCtas;
@@ -554,6 +569,7 @@ void fill_common(Params& p, const DecodeDims& d, const void* q, const int* seqle
   p.W = 0;
   p.swa_len = nullptr;
   p.sinks = nullptr;
+  p.kc = p.vc = nullptr;
   p.logits = nullptr;
   p.tok_scores = nullptr;
   p.forced = 0;
@@ -598,7 +614,7 @@ cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const voi
   fill_common(p, d, q, seqlens, ws, nsplit);
   p.mode = 0;
   p.bps = bps;
-  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, mk, mv, p);
+  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), scores,
@@ -627,7 +643,7 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   p.W = W;
   p.swa_len = swa_len;
   p.sinks = sinks;
-  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, mk, mv, p);
+  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, gate, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
@@ -652,7 +668,7 @@ cudaError_t launch_decode_full_tokens_mma(const DecodeDims& d, const void* q, co
   p.bps = bps;
   p.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + decode_mma_full_workspace(d));
   p.tok_scores = tok_scores;
-  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, mk, mv, p);
+  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
@@ -669,11 +685,8 @@ size_t decode_mma_sparse_tokens_workspace(const DecodeDims& d, int kt) {
 cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                             const int* seqlens, const int* idx, int kt, int forced, void* o, void* ws,
                                             cudaStream_t s) {
-  CUtensorMap mk, mv, mkg, mvg;
-  const long long rows = (long long)d.B * d.Hkv * d.L;
-  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv) || !make_gather_map(&mkg, kc, rows) ||
-      !make_gather_map(&mvg, vc, rows))
-    return cudaErrorInvalidValue;
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv)) return cudaErrorInvalidValue;
   cudaError_t e = set_smem();
   if (e != cudaSuccess) return e;
   Params p;
@@ -685,7 +698,9 @@ cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, 
   p.idx = idx;
   p.kb = kt;
   p.forced = forced;
-  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, mkg, mvg, p);
+  p.kc = reinterpret_cast<const __nv_bfloat16*>(kc);
+  p.vc = reinterpret_cast<const __nv_bfloat16*>(vc);
+  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
