@@ -21,6 +21,10 @@ the token-level variant and the forced newest-128 window):
 * ``decode``   bf16, B64, L131072 cached tokens, 32/4, D128, k=32 blocks, 11 sparse layers
 * ``token``    bf16, B1 N131072, 32/4, D128, top-2048 tokens + forced 128, 3 sparse layers
 * ``token_small``  the token variant at N32768 with 1 sparse layer (profiling)
+
+An FP8 cache (the token-variant decode's FP8 option) stores the same normal draws as OCP E4M3
+codes of value / scale, with one seeded scale per KV head for K and one for V (the conversion
+to E4M3 is a storage-format rounding, like the bf16 one, done by torch).
 """
 from __future__ import annotations
 
@@ -35,6 +39,7 @@ import numpy as np
 # tensor ids (stream keys).  Per sparse layer l the ids are 16 + 8*l + {0..3}.
 # ----------------------------------------------------------------------------
 TID_Q, TID_K, TID_V = 0, 1, 2
+TID_FP8_SCALE = 14
 TID_PLANT = 15
 _TID_LAYER0 = 16
 SPARSE_Q, SPARSE_KSWA, SPARSE_VSWA, SPARSE_GATE, SPARSE_SINK = 0, 1, 2, 3, 4
@@ -266,6 +271,32 @@ def decode_sparse_q_slice(w: Workload, layer: int, b: int, h: int) -> np.ndarray
     return normal_slice(w.seed, layer_tid(layer, SPARSE_Q), b, h, (w.D,), w.scale_std, True)
 
 
+# FP8 (E4M3) decode cache: codes of value / scale, one scale per KV head for K and for V
+def fp8_kv_scales(w: Workload) -> Tuple[np.ndarray, np.ndarray]:
+    """[Hkv] float32 scales for K and for V: the cache's std / 32 times a seeded factor in
+    [0.75, 1.25], so the codes stay well inside E4M3's range (|code| <= 448)."""
+    u = _stream(w.seed, TID_FP8_SCALE).uniform(0.75, 1.25, size=(2, w.Hkv))
+    base = w.scale_std / 32.0
+    return (base * u[0]).astype(np.float32), (base * u[1]).astype(np.float32)
+
+
+def e4m3_codes(x: np.ndarray) -> np.ndarray:
+    """float32 values -> OCP E4M3 ("fn") codes as uint8, rounded to nearest (torch's conversion)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def decode_k_fp8_slice(w: Workload, b: int, g: int) -> np.ndarray:
+    x = normal_slice(w.seed, TID_K, b, g, (w.N, w.D), w.scale_std, False)
+    return e4m3_codes(x / fp8_kv_scales(w)[0][g])
+
+
+def decode_v_fp8_slice(w: Workload, b: int, g: int) -> np.ndarray:
+    x = normal_slice(w.seed, TID_V, b, g, (w.N, w.D), w.scale_std, False)
+    return e4m3_codes(x / fp8_kv_scales(w)[1][g])
+
+
 # ----------------------------------------------------------------------------
 # whole tensors (small workloads, or bulk fill with threads)
 # ----------------------------------------------------------------------------
@@ -305,6 +336,21 @@ def prefill_arrays(w: Workload, layers: Optional[int] = None, threads: int = 8) 
         out["k_swa"].append(_fill((w.B, w.Hkv, w.N, w.D), lambda b, g: swa_k_slice(w, l, b, g), bk, threads))
         out["v_swa"].append(_fill((w.B, w.Hkv, w.N, w.D), lambda b, g: swa_v_slice(w, l, b, g), bk, threads))
         out["gate"].append(_fill((w.B, w.Hq, w.N, 2), lambda b, h: gate_slice(w, l, b, h), bq, threads))
+    return out
+
+
+def decode_fp8_cache(w: Workload, threads: int = 8) -> Dict[str, np.ndarray]:
+    """The FP8 decode cache: k8/v8 uint8 codes [B,Hkv,L,D] and k_scale/v_scale [Hkv] float32."""
+    bk = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    out = {"k8": np.empty((w.B, w.Hkv, w.N, w.D), np.uint8), "v8": np.empty((w.B, w.Hkv, w.N, w.D), np.uint8)}
+
+    def one(key):
+        out["k8"][key] = decode_k_fp8_slice(w, *key)
+        out["v8"][key] = decode_v_fp8_slice(w, *key)
+
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(one, bk))
+    out["k_scale"], out["v_scale"] = fp8_kv_scales(w)
     return out
 
 

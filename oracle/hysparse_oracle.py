@@ -38,6 +38,11 @@ Readings where the pages leave a step open (each is listed in the design notes):
   position L-1 scores every cached token i < L by sum over the group's heads of P_i;
   candidates are the tokens older than the forced newest W, [0, L-1-W]; row L-1
   attends the top-k candidates united with [L-W, L-1], each token once, no gate.
+* FP8 KV cache ([HS2] "What actually improved?", the KV-cache-at-1M-tokens row, which
+  sizes the cache in FP8; the pages fix neither the FP8 format nor the scaling): each
+  cached K or V element is an OCP E4M3 code (the "fn" variant: bias 7, no infinities,
+  S.1111.111 is NaN), and its value is the decoded code times a float32 scale of its
+  KV head, one scale for K and one for V.  The decode step then runs on these values.
 * Sink biases ([HSP] §4.1, per-head learnable sinks in the sparse and SWA branches,
   following gpt-oss): one logit per (head, branch), sinks [Hq, 2] with index 0 for
   the sparse branch and 1 for the SWA branch; it joins the branch's softmax as an
@@ -389,6 +394,27 @@ def decode_token_sparse(q: np.ndarray, k_cache, v_cache, idx, forced: int, seqle
                 qq = np.asarray(q[b, h], np.float64)[None, :]
                 o[b, h] = attention_rows(qq, np.array([len(keys)]), ks, vs)[0][0]
     return o
+
+
+def e4m3_to_float(codes) -> np.ndarray:
+    """OCP 8-bit floating point, E4M3 ("fn": no infinities), code -> float64 value: sign bit 7,
+    exponent bits 6..3 with bias 7, mantissa bits 2..0; exponent 0 is subnormal (m/8 * 2^-6),
+    exponent 15 with mantissa 7 is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequant_kv_fp8(codes, scale) -> np.ndarray:
+    """FP8 cache [B,Hkv,L,D] of E4M3 codes with one float32 scale per KV head [Hkv] -> the
+    float64 cache values code * scale[g] the decode step attends over."""
+    v = e4m3_to_float(codes)
+    sc = np.asarray(scale, np.float64).reshape(1, -1, 1, 1)
+    return v * sc
 
 
 def decode_sparse(q: np.ndarray, k_cache, v_cache, idx, k_ring, v_ring, gate, seqlens=None,

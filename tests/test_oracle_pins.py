@@ -477,6 +477,66 @@ def test_token_decode_pins():
     assert got[0, 0].tolist() == [0, 1, 2, 3, 4]
 
 
+def test_e4m3_decode_pins():
+    """FP8 E4M3 codes: every one of the 256 codes equals torch's float8_e4m3fn -> float64
+    conversion (NaN exactly at S.1111.111), and hand values of the format (1.0, the largest
+    finite 448, the smallest subnormal 2^-9, the smallest normal 2^-6, the largest subnormal
+    7/8 * 2^-6, -1.0, both zeros); positive codes increase strictly up to 448."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = O.e4m3_to_float(codes)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    assert np.nonzero(np.isnan(got))[0].tolist() == [0x7F, 0xFF]
+    fin = ~np.isnan(want)
+    assert np.array_equal(got[fin], want[fin])
+    hand = {0x38: 1.0, 0x7E: 448.0, 0x01: 2.0 ** -9, 0x08: 2.0 ** -6, 0x07: 7 / 8 * 2.0 ** -6, 0xB8: -1.0,
+            0x00: 0.0, 0x80: -0.0, 0x40: 2.0, 0x3C: 1.5}
+    for c, v in hand.items():
+        assert got[c] == v and math.copysign(1.0, got[c]) == math.copysign(1.0, v), hex(c)
+    assert np.all(np.diff(got[:0x7F]) > 0)
+
+
+def test_fp8_token_decode_pins():
+    """FP8 cache: each KV head's values are its codes times that head's scale (K and V scaled
+    separately); the token-variant decode on them equals torch's float64 attention over the
+    values torch decodes from the same codes, and with every candidate selected it equals dense
+    decode over those values."""
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, D, L, W = 2, 4, 2, 16, 260, 32
+    G = Hq // Hkv
+    kx = rng.standard_normal((B, Hkv, L, D)) * 40.0
+    vx = rng.standard_normal((B, Hkv, L, D)) * 40.0
+    kcode = torch.from_numpy(kx.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    vcode = torch.from_numpy(vx.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ks, vs = np.array([0.01, 0.02]), np.array([0.03, 0.005])
+    kd, vd = O.dequant_kv_fp8(kcode, ks), O.dequant_kv_fp8(vcode, vs)
+    tk = torch.from_numpy(kcode).view(torch.float8_e4m3fn).to(torch.float64)
+    tv = torch.from_numpy(vcode).view(torch.float8_e4m3fn).to(torch.float64)
+    for g in range(Hkv):
+        assert np.array_equal(kd[:, g], tk[:, g].numpy() * ks[g])
+        assert np.array_equal(vd[:, g], tv[:, g].numpy() * vs[g])
+    q = rng.standard_normal((B, Hq, D))
+    seqlens = np.array([L, 190])
+    sc = O.decode_token_scores(q, kd, seqlens)
+    idx = O.topk_decode_tokens(sc, 24, W, seqlens)
+    o = O.decode_token_sparse(q, kd, vd, idx, W, seqlens)
+    for b in range(B):
+        Lb = int(seqlens[b])
+        for g in range(Hkv):
+            sel = [int(i) for i in idx[b, g] if i >= 0]
+            keys = sorted(set(sel) | set(range(Lb - W, Lb)))
+            kk = tk[b, g, keys] * ks[g]
+            vv = tv[b, g, keys] * vs[g]
+            for h in range(g * G, (g + 1) * G):
+                qq = torch.from_numpy(q[b, h]).double()[None, None, None, :]
+                ref = torch.nn.functional.scaled_dot_product_attention(qq, kk[None, None], vv[None, None])
+                np.testing.assert_allclose(o[b, h], ref[0, 0, 0].numpy(), rtol=1e-12, atol=1e-13)
+    idx_all = O.topk_decode_tokens(sc, L, W, seqlens)
+    o_all = O.decode_token_sparse(q, kd, vd, idx_all, W, seqlens)
+    o_dense, _ = O.decode_full(q, kd, vd, seqlens)
+    np.testing.assert_allclose(o_all, o_dense, rtol=1e-12, atol=1e-13)
+
+
 def test_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the oracle and check that a pin above fails."""
     g = _gold()
