@@ -418,4 +418,49 @@ hys_status hysparse_sparse_attn_decode_tokens(const hys_decode_shape* shape, hys
                                                    workspace, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+}  // namespace
+
+hys_status hysparse_full_attn_select_decode_tokens_fp8(const hys_decode_shape* shape, const void* q,
+                                                       const void* k_cache, const void* v_cache,
+                                                       const float* k_scale, const float* v_scale,
+                                                       const int* seqlens, void* o, float* tok_scores,
+                                                       void* workspace, size_t workspace_bytes,
+                                                       hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !o || !tok_scores) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned4(k_scale) || !aligned4(v_scale) ||
+      !aligned16(seqlens) || !aligned16(o) || !aligned16(tok_scores) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  if (!decode_mma_supported(d, HYS_BF16)) return HYS_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < align256(decode_mma_full_tokens_workspace(d))) return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_decode_full_tokens_mma_fp8(d, q, k_cache, v_cache, k_scale, v_scale, seqlens, o, tok_scores,
+                                                     workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_sparse_attn_decode_tokens_fp8(const hys_decode_shape* shape, const void* q, const void* k_cache,
+                                                  const void* v_cache, const float* k_scale, const float* v_scale,
+                                                  const int* seqlens, const int* idx, int k_tokens, int forced_window,
+                                                  void* o, void* workspace, size_t workspace_bytes,
+                                                  hys_stream_t stream) {
+  DecodeDims d;
+  hys_status st = check_decode(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !idx || !o) return HYS_ERR_INVALID_ARG;
+  if (k_tokens < 1 || k_tokens > 16384 || forced_window < 1 || forced_window > 4096) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned4(k_scale) || !aligned4(v_scale) ||
+      !aligned16(seqlens) || !aligned16(idx) || !aligned16(o) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  if (!decode_mma_supported(d, HYS_BF16)) return HYS_ERR_UNSUPPORTED;
+  if ((long long)d.B * d.Hkv * d.L >= (1ll << 31)) return HYS_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < align256(decode_mma_sparse_tokens_workspace(d, k_tokens)))
+    return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_decode_sparse_tokens_mma_fp8(d, q, k_cache, v_cache, k_scale, v_scale, seqlens, idx,
+                                                       k_tokens, forced_window, o, workspace,
+                                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -20,6 +20,7 @@
 // (full layer) the block scores exp(m~ - m)/l aggregated over the group's heads, or
 // (sparse layer) the gated sum of the sparse-branch and SWA-ring branches.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -36,8 +37,19 @@ namespace {
 constexpr int kConsumers = HYS_DECODE_CONSUMERS;
 constexpr int kCtasPerSm = kConsumers <= 3 ? 2 : 1;   // two CTAs share an SM when they fit
 constexpr int kThreads = 32 * (kConsumers + 1);
-constexpr int kStages = kConsumers;              // stage w belongs to consumer warp w
-constexpr int kStageBytes = 2 * 64 * 128 * 2;   // K + V of one 64-key block, D = 128
+constexpr int kStages = kConsumers;              // bf16: stage w belongs to consumer warp w
+constexpr int kStageBytes = 2 * 64 * 128 * 2;   // K + V of one 64-key block, D = 128, bf16
+constexpr int kMaxStages = 2 * kConsumers;
+// Stage geometry per cache format.  An FP8 block is half the bytes, so the same shared memory
+// holds twice the stages: consumer warp w owns stages w and w + C (entries w, w + C, ...
+// alternate between them), so each stage's barrier phases are still consumed by one warp in order.
+template <bool F8>
+struct Stg {
+  static constexpr int kHalf = F8 ? 64 * 128 : 64 * 128 * 2;   // K at 0, V at kHalf
+  static constexpr int kBytes = 2 * kHalf;
+  static constexpr int kCount = kStages * kStageBytes / kBytes;
+  static_assert(kCount % kConsumers == 0 && kCount <= kMaxStages, "stages per consumer warp");
+};
 constexpr int kMaxList = 72;                     // blocks per split (incl. padding)
 #ifndef HYS_DECODE_TOK_SPLIT
 #define HYS_DECODE_TOK_SPLIT 1024
@@ -71,8 +83,10 @@ struct Params {
   float* tok_scores;       // [B,Hkv,L] token scores written by the merge (mode 0), or null
   int forced;              // newest tokens always attended (mode 2)
   const __nv_bfloat16* q;  // [B,Hq,D]
-  const __nv_bfloat16* kc; // [B,Hkv,L,D] shared cache (mode 2 gathers rows from it)
-  const __nv_bfloat16* vc;
+  const uint8_t* kc;       // [B,Hkv,L,D] shared cache, bf16 or FP8 (mode 2 gathers rows from it)
+  const uint8_t* vc;
+  const float* k_scale;    // [Hkv] FP8 cache scales (value = code * scale), or null for bf16
+  const float* v_scale;
   float* pm;        // [B,Hq,nsplit]
   float* pl;
   float* po;        // [B,Hq,nsplit,D]
@@ -106,6 +120,28 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// two E4M3 codes (low byte -> low half) to two f16 values; every E4M3 value is exact in f16
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
+  uint32_t r;
+  const unsigned short h = static_cast<unsigned short>(v & 0xffffu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
 
 // byte offset of (row, 16-byte unit) inside a [64 rows][128 B] 128-byte-swizzled box
 __device__ __forceinline__ uint32_t sw128(int row, int unit) { return row * 128 + ((unit ^ (row & 7)) << 4); }
@@ -121,6 +157,7 @@ __device__ __forceinline__ void cp_async_bar_arrive(uint64_t* bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
@@ -130,8 +167,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   float* part = reinterpret_cast<float*>(smem);  // after the pipeline has drained
   Entry* list = reinterpret_cast<Entry*>(smem + kStages * kStageBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kMaxList * 16);
-  uint64_t* empty = full + kStages;
-  int* s_nlist = reinterpret_cast<int*>(empty + kStages);
+  uint64_t* empty = full + kMaxStages;
+  int* s_nlist = reinterpret_cast<int*>(empty + kMaxStages);
+  constexpr int NS = Stg<F8>::kCount, SB = Stg<F8>::kBytes, HALF = Stg<F8>::kHalf;
   volatile int* abort = s_nlist + 1;
   int* tok = reinterpret_cast<int*>(smem + kStages * kStageBytes + kMaxList * 16 + 256);   // mode 2 token rows
 
@@ -198,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       *s_nlist = n;
     }
 
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < NS; ++i) {
       tc::mbar_init(&full[i], 1);
       tc::mbar_init(&empty[i], 1);
     }
@@ -207,7 +245,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
   __syncthreads();
   const int nlist = *s_nlist;
-  const float sc = p.scale_log2;
+  // FP8: logits are kept in code units (q . code); the K scale joins the softmax scale
+  const float sc = F8 ? p.scale_log2 * p.k_scale[g] : p.scale_log2;
 
   if (warp == kConsumers) {
     // ---------------------------------------------------------------- producer
@@ -218,24 +257,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     bool ok = true;
     const int head = b * p.Hkv + g;
     for (int i = 0; i < nlist; ++i) {
-      const int st = i % kStages;
-      if (lane == 0) ok = tc::mbar_wait(&empty[st], ((i / kStages) & 1) ^ 1, abort);
+      const int st = i % NS;
+      if (lane == 0) ok = tc::mbar_wait(&empty[st], ((i / NS) & 1) ^ 1, abort);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
-      uint8_t* dst = smem + st * kStageBytes;
+      uint8_t* dst = smem + st * SB;
       const Entry e = list[i];
       if (e.src == 2) {
-        const int u = lane & 15;   // 16-byte unit of the 256-byte row: units 0-7 in the low box, 8-15 the high
+        // 16-byte unit u of a row (bf16: 256-byte rows, units 0-7 in the low box, 8-15 the
+        // high one; FP8: 128-byte rows, one box)
+        constexpr int kRow = F8 ? 128 : 256, kUpr = kRow / 16, kRpi = 32 / kUpr;
+        const int u = lane % kUpr;
         const uint32_t sdst = tc::smem_u32(dst) + (u >> 3) * 8192;
-        const __nv_bfloat16* kh = p.kc + (size_t)head * p.L * 128 + u * 8;
-        const __nv_bfloat16* vh = p.vc + (size_t)head * p.L * 128 + u * 8;
+        const uint8_t* kh = p.kc + (size_t)head * p.L * kRow + u * 16;
+        const uint8_t* vh = p.vc + (size_t)head * p.L * kRow + u * 16;
 #pragma unroll 4
-        for (int j = 0; j < 32; ++j) {
-          const int q = 2 * j + (lane >> 4);   // rows past the stage's count repeat its first token (masked)
-          const size_t r = (size_t)tok[e.row + (q < e.valid ? q : 0)] * 128;
+        for (int j = 0; j < 64 / kRpi; ++j) {
+          const int q = kRpi * j + lane / kUpr;   // rows past the stage's count repeat its first token (masked)
+          const size_t r = (size_t)tok[e.row + (q < e.valid ? q : 0)] * kRow;
           const uint32_t so = sdst + sw128(q, u & 7);
           cp_async16(so, kh + r);
-          cp_async16(so + 16384, vh + r);
+          cp_async16(so + HALF, vh + r);
         }
         cp_async_bar_arrive(&full[st]);
         __syncwarp();
@@ -243,11 +285,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       } else if (lane == 0) {
         const CUtensorMap* mk = e.src ? &tmKr : &tmK;
         const CUtensorMap* mv = e.src ? &tmVr : &tmV;
-        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
-        tc::tma_load_3d(mk, &full[st], dst, 0, e.row, head);
-        tc::tma_load_3d(mk, &full[st], dst + 8192, 64, e.row, head);
-        tc::tma_load_3d(mv, &full[st], dst + 16384, 0, e.row, head);
-        tc::tma_load_3d(mv, &full[st], dst + 24576, 64, e.row, head);
+        tc::mbar_arrive_expect_tx(&full[st], SB);
+        if (F8) {
+          tc::tma_load_3d(mk, &full[st], dst, 0, e.row, head);
+          tc::tma_load_3d(mv, &full[st], dst + HALF, 0, e.row, head);
+        } else {
+          tc::tma_load_3d(mk, &full[st], dst, 0, e.row, head);
+          tc::tma_load_3d(mk, &full[st], dst + 8192, 64, e.row, head);
+          tc::tma_load_3d(mv, &full[st], dst + 16384, 0, e.row, head);
+          tc::tma_load_3d(mv, &full[st], dst + 24576, 64, e.row, head);
+        }
       }
     }
     if (lane == 0) {
@@ -255,8 +302,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         *abort = 1;
         report_status(p.status, HYS_ERR_TIMEOUT);
       }
-      for (int i = max(0, nlist - kStages); i < nlist; ++i)
-        tc::mbar_wait(&full[i % kStages], (i / kStages) & 1, abort, 100000000ull);
+      for (int i = max(0, nlist - NS); i < nlist; ++i)
+        tc::mbar_wait(&full[i % NS], (i / NS) & 1, abort, 100000000ull);
     }
     cp_async_wait_all();
     __syncwarp();
@@ -268,13 +315,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // Q as A fragments (rows = heads, zero past G)
     uint32_t qa[8][4];
     const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + g * p.G) * 128;
+    if (F8) {
+      // f16 fragments in the dim order of the FP8 K fragments below: k-step ks covers dims
+      // 16ks .. 16ks+15 and its k slots (2c, 2c+1 | 2c+8, 2c+9) hold dims 16ks + 4c + (0, 1 | 2, 3)
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int c0 = 16 * ks + 2 * cq;
-      qa[ks][0] = h_lo < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_lo * 128 + c0) : 0u;
-      qa[ks][1] = h_hi < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_hi * 128 + c0) : 0u;
-      qa[ks][2] = h_lo < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_lo * 128 + c0 + 8) : 0u;
-      qa[ks][3] = h_hi < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_hi * 128 + c0 + 8) : 0u;
+      for (int ks = 0; ks < 8; ++ks) {
+        const int d0 = 16 * ks + 4 * cq;
+        const uint2 lo = h_lo < p.G ? *reinterpret_cast<const uint2*>(qg + h_lo * 128 + d0) : make_uint2(0u, 0u);
+        const uint2 hi = h_hi < p.G ? *reinterpret_cast<const uint2*>(qg + h_hi * 128 + d0) : make_uint2(0u, 0u);
+        qa[ks][0] = bf16x2_to_f16x2(lo.x);
+        qa[ks][1] = bf16x2_to_f16x2(hi.x);
+        qa[ks][2] = bf16x2_to_f16x2(lo.y);
+        qa[ks][3] = bf16x2_to_f16x2(hi.y);
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int c0 = 16 * ks + 2 * cq;
+        qa[ks][0] = h_lo < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_lo * 128 + c0) : 0u;
+        qa[ks][1] = h_hi < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_hi * 128 + c0) : 0u;
+        qa[ks][2] = h_lo < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_lo * 128 + c0 + 8) : 0u;
+        qa[ks][3] = h_hi < p.G ? *reinterpret_cast<const uint32_t*>(qg + h_hi * 128 + c0 + 8) : 0u;
+      }
     }
     float o[16][4];
 #pragma unroll
@@ -283,10 +345,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     bool ok = true;
     const uint32_t sbase = tc::smem_u32(smem);
     for (int i = warp; i < nlist; i += kConsumers) {
-      const int st = warp;  // == i % kStages
-      if (!(ok = tc::mbar_wait(&full[st], (i / kStages) & 1, abort))) break;
+      const int st = i % NS;   // bf16: == warp; FP8: warp or warp + C
+      if (!(ok = tc::mbar_wait(&full[st], (i / NS) & 1, abort))) break;
       const Entry e = list[i];
-      const uint32_t kb = sbase + st * kStageBytes, vb = kb + 16384;
+      const uint32_t kb = sbase + st * SB, vb = kb + HALF;
       // ---- S = Q K^T : 8 key tiles x 8 dim steps
       float s[8][4];
 #pragma unroll
@@ -294,15 +356,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
         const int key = 8 * nt + (lane & 7);
         const int mtx = lane >> 3;
+        if (F8) {
+          // an 8 x 16-byte matrix of codes read as 16-bit pairs: lane gets key 8nt + lane/4 and
+          // dims 16sg + 4c .. +3 (c = lane % 4), i.e. both B registers of k-step sg
 #pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {  // pairs of 16-dim steps
-          const int ks = 2 * kp;
-          const int chunk = ks >> 2;
-          const int unit = 2 * (ks & 3) + mtx;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kb + chunk * 8192 + sw128(key, unit), b0, b1, b2, b3);
-          mma16816(s[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-          mma16816(s[nt], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], b2, b3);
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t r[4];
+            ldsm_x4(kb + sw128(key, 4 * hf + mtx), r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const int ks = 4 * hf + m;
+              mma16816_f16(s[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], e4m3x2_to_f16x2(r[m]),
+                           e4m3x2_to_f16x2(r[m] >> 16));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int kp = 0; kp < 4; ++kp) {  // pairs of 16-dim steps
+            const int ks = 2 * kp;
+            const int chunk = ks >> 2;
+            const int unit = 2 * (ks & 3) + mtx;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kb + chunk * 8192 + sw128(key, unit), b0, b1, b2, b3);
+            mma16816(s[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+            mma16816(s[nt], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], b2, b3);
+          }
         }
       }
       // ---- mask keys past the valid count, block max, online softmax
@@ -367,23 +445,43 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const float p3 = h_hi < p.G ? exp2f(fmaf(s[nt][3], sc, -ms_hi)) : 0.0f;
         l_lo += p0 + p1;
         l_hi += p2 + p3;
-        pa[nt][0] = tc::pack_bf16x2(p0, p1);
-        pa[nt][1] = tc::pack_bf16x2(p2, p3);
+        pa[nt][0] = F8 ? pack_f16x2(p0, p1) : tc::pack_bf16x2(p0, p1);
+        pa[nt][1] = F8 ? pack_f16x2(p2, p3) : tc::pack_bf16x2(p2, p3);
       }
       // ---- O += P V : 4 key steps x 16 dim tiles
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const int mtx = lane >> 3;
         const int key = 16 * kk + 8 * (mtx & 1) + (lane & 7);
+        if (F8) {
+          // transposed 8 x 8 matrices of 16-bit pairs: lane gets keys 2c, 2c+1 x dims 2n, 2n+1 of
+          // segment sg (n = lane / 4); regrouping the bytes by dim gives the B registers of
+          // output tile 2sg (dims 16sg + 2n) and 2sg+1 (dims 16sg + 2n + 1)
 #pragma unroll
-        for (int dp = 0; dp < 8; ++dp) {  // pairs of 8-dim tiles
-          const int dt = 2 * dp + (mtx >> 1);
-          const int chunk = dt >> 3;
-          const int unit = dt & 7;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vb + chunk * 8192 + sw128(key, unit), b0, b1, b2, b3);
-          mma16816(o[2 * dp], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
-          mma16816(o[2 * dp + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2, b3);
+          for (int sp = 0; sp < 4; ++sp) {
+            uint32_t r[4];
+            ldsm_x4_t(vb + sw128(key, 2 * sp + (mtx >> 1)), r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint32_t x0 = __byte_perm(r[2 * j], 0u, 0x3120), x1 = __byte_perm(r[2 * j + 1], 0u, 0x3120);
+              const int ot = 2 * (2 * sp + j);
+              mma16816_f16(o[ot], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1],
+                           e4m3x2_to_f16x2(x0), e4m3x2_to_f16x2(x1));
+              mma16816_f16(o[ot + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1],
+                           e4m3x2_to_f16x2(x0 >> 16), e4m3x2_to_f16x2(x1 >> 16));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int dp = 0; dp < 8; ++dp) {  // pairs of 8-dim tiles
+            const int dt = 2 * dp + (mtx >> 1);
+            const int chunk = dt >> 3;
+            const int unit = dt & 7;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vb + chunk * 8192 + sw128(key, unit), b0, b1, b2, b3);
+            mma16816(o[2 * dp], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b0, b1);
+            mma16816(o[2 * dp + 1], pa[2 * kk][0], pa[2 * kk][1], pa[2 * kk + 1][0], pa[2 * kk + 1][1], b2, b3);
+          }
         }
       }
       __syncwarp();
@@ -409,11 +507,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 #pragma unroll
     for (int dt = 0; dt < 16; ++dt) {
-      const int d0 = 8 * dt + 2 * cq;
+      // bf16: tile dt holds dims 8dt + (2c, 2c+1); FP8: tile 2sg+j holds dims 16sg + 4c + j + (0, 2)
+      const int d0 = F8 ? 16 * (dt >> 1) + 4 * cq + (dt & 1) : 8 * dt + 2 * cq;
+      const int d1 = F8 ? d0 + 2 : d0 + 1;
       wp[h_lo * 130 + 2 + d0] = o[dt][0];
-      wp[h_lo * 130 + 2 + d0 + 1] = o[dt][1];
+      wp[h_lo * 130 + 2 + d1] = o[dt][1];
       wp[h_hi * 130 + 2 + d0] = o[dt][2];
-      wp[h_hi * 130 + 2 + d0 + 1] = o[dt][3];
+      wp[h_hi * 130 + 2 + d1] = o[dt][3];
     }
   }
   __syncthreads();
@@ -444,10 +544,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const float* __restrict__ gate,
                                                            __nv_bfloat16* __restrict__ o, float* __restrict__ scores,
                                                            int red_max) {
-  __shared__ float sM[2][16], sInv[2][16];
+  __shared__ float sM[2][16], sInv[2][16], sVw[2][16];
   const int g = blockIdx.x, b = blockIdx.y;
   const int Lb = p.seqlens ? max(1, min(p.seqlens[b], p.L)) : p.L;
-  const float sc = p.scale_log2;
+  const float sc = p.k_scale ? p.scale_log2 * p.k_scale[g] : p.scale_log2;   // FP8: logits in code units
+  const float vsc = p.v_scale ? p.v_scale[g] : 1.0f;
   const bool two = p.mode == 1;   // the sparse layer merges two branches under the gate
   const int nbr = two ? 2 : 1;
   if (threadIdx.x < p.G * nbr) {
@@ -464,6 +565,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const
     if (p.mode == 1 && p.sinks != nullptr) L += exp2f(p.sinks[2 * (g * p.G + hh) + br] * kLog2e - M * sc);
     sM[br][hh] = M;
     sInv[br][hh] = L > 0.0f ? 1.0f / L : 0.0f;
+    sVw[br][hh] = L > 0.0f ? vsc / L : 0.0f;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < p.G * 128; e += blockDim.x) {
@@ -478,7 +580,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const
         const float m = p.pm[ph + s];
         if (m != -INFINITY) acc = fmaf(p.po[(ph + s) * 128 + d], exp2f((m - sM[br][hh]) * sc), acc);
       }
-      float w = sInv[br][hh];
+      float w = sVw[br][hh];   // 1/l, times the V scale of an FP8 cache
       if (two) w *= sigmoidf_(gate[((size_t)b * p.Hq + g * p.G + hh) * 2 + br]);
       out = fmaf(acc, w, out);
     }
@@ -538,6 +640,24 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int heads) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// FP8 codes: [heads][rows][128] bytes, box 128 bytes x 64 rows x 1 head
+bool make_map8(CUtensorMap* m, const void* base, int rows, int heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {128, (cuuint64_t)rows * 128};
+  cuuint32_t box[3] = {128, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_cache_maps(bool f8, CUtensorMap* mk, CUtensorMap* mv, const void* kc, const void* vc, const DecodeDims& d) {
+  if (f8) return make_map8(mk, kc, d.L, d.B * d.Hkv) && make_map8(mv, vc, d.L, d.B * d.Hkv);
+  return make_map(mk, kc, d.L, d.B * d.Hkv) && make_map(mv, vc, d.L, d.B * d.Hkv);
+}
+
 int full_bps(const DecodeDims& d) {
   const long long work = (long long)d.NB * d.B * d.Hkv;
   long long bps = (work + kTargetCtas - 1) / kTargetCtas;
@@ -570,16 +690,18 @@ void fill_common(Params& p, const DecodeDims& d, const void* q, const int* seqle
   p.swa_len = nullptr;
   p.sinks = nullptr;
   p.kc = p.vc = nullptr;
+  p.k_scale = p.v_scale = nullptr;
   p.logits = nullptr;
   p.tok_scores = nullptr;
   p.forced = 0;
   p.nsp = 0;
 }
 
+template <bool F8>
 cudaError_t set_smem() {
   static bool done = false;
   if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e == cudaSuccess) done = true;
   return e;
 }
@@ -606,7 +728,7 @@ cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const voi
                                    cudaStream_t s) {
   CUtensorMap mk, mv;
   if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv)) return cudaErrorInvalidValue;
-  cudaError_t e = set_smem();
+  cudaError_t e = set_smem<false>();
   if (e != cudaSuccess) return e;
   Params p;
   const int bps = full_bps(d);
@@ -614,7 +736,7 @@ cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const voi
   fill_common(p, d, q, seqlens, ws, nsplit);
   p.mode = 0;
   p.bps = bps;
-  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  decode_split_kernel<false><<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), scores,
@@ -630,7 +752,7 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv) ||
       !make_map(&mkr, kr, W, d.B * d.Hkv) || !make_map(&mvr, vr, W, d.B * d.Hkv))
     return cudaErrorInvalidValue;
-  cudaError_t e = set_smem();
+  cudaError_t e = set_smem<false>();
   if (e != cudaSuccess) return e;
   Params p;
   const int nsp = decode_sparse_splits(kb);
@@ -643,7 +765,7 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   p.W = W;
   p.swa_len = swa_len;
   p.sinks = sinks;
-  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
+  decode_split_kernel<false><<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, gate, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
@@ -654,11 +776,14 @@ size_t decode_mma_full_tokens_workspace(const DecodeDims& d) {
   return decode_mma_full_workspace(d) + sizeof(float) * (size_t)d.B * d.Hq * d.L;
 }
 
-cudaError_t launch_decode_full_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
-                                          const int* seqlens, void* o, float* tok_scores, void* ws, cudaStream_t s) {
+namespace {
+
+template <bool F8>
+cudaError_t full_tokens(const DecodeDims& d, const void* q, const void* kc, const void* vc, const float* k_scale,
+                        const float* v_scale, const int* seqlens, void* o, float* tok_scores, void* ws, cudaStream_t s) {
   CUtensorMap mk, mv;
-  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv)) return cudaErrorInvalidValue;
-  cudaError_t e = set_smem();
+  if (!make_cache_maps(F8, &mk, &mv, kc, vc, d)) return cudaErrorInvalidValue;
+  cudaError_t e = set_smem<F8>();
   if (e != cudaSuccess) return e;
   Params p;
   const int bps = full_bps(d);
@@ -666,13 +791,28 @@ cudaError_t launch_decode_full_tokens_mma(const DecodeDims& d, const void* q, co
   fill_common(p, d, q, seqlens, ws, nsplit);
   p.mode = 0;
   p.bps = bps;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   p.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + decode_mma_full_workspace(d));
   p.tok_scores = tok_scores;
-  decode_split_kernel<<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  decode_split_kernel<F8><<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_full_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                          const int* seqlens, void* o, float* tok_scores, void* ws, cudaStream_t s) {
+  return full_tokens<false>(d, q, kc, vc, nullptr, nullptr, seqlens, o, tok_scores, ws, s);
+}
+
+cudaError_t launch_decode_full_tokens_mma_fp8(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                              const float* k_scale, const float* v_scale, const int* seqlens, void* o,
+                                              float* tok_scores, void* ws, cudaStream_t s) {
+  return full_tokens<true>(d, q, kc, vc, k_scale, v_scale, seqlens, o, tok_scores, ws, s);
 }
 
 int decode_token_splits(int kt) { return (kt + kTokSplit - 1) / kTokSplit; }
@@ -682,12 +822,15 @@ size_t decode_mma_sparse_tokens_workspace(const DecodeDims& d, int kt) {
   return sizeof(float) * ((size_t)d.B * d.Hq * nsplit * (2 + 128));
 }
 
-cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
-                                            const int* seqlens, const int* idx, int kt, int forced, void* o, void* ws,
-                                            cudaStream_t s) {
+namespace {
+
+template <bool F8>
+cudaError_t sparse_tokens(const DecodeDims& d, const void* q, const void* kc, const void* vc, const float* k_scale,
+                          const float* v_scale, const int* seqlens, const int* idx, int kt, int forced, void* o,
+                          void* ws, cudaStream_t s) {
   CUtensorMap mk, mv;
-  if (!make_map(&mk, kc, d.L, d.B * d.Hkv) || !make_map(&mv, vc, d.L, d.B * d.Hkv)) return cudaErrorInvalidValue;
-  cudaError_t e = set_smem();
+  if (!make_cache_maps(F8, &mk, &mv, kc, vc, d)) return cudaErrorInvalidValue;
+  cudaError_t e = set_smem<F8>();
   if (e != cudaSuccess) return e;
   Params p;
   const int nsp = decode_token_splits(kt);
@@ -698,13 +841,29 @@ cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, 
   p.idx = idx;
   p.kb = kt;
   p.forced = forced;
-  p.kc = reinterpret_cast<const __nv_bfloat16*>(kc);
-  p.vc = reinterpret_cast<const __nv_bfloat16*>(vc);
-  decode_split_kernel<<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  p.kc = reinterpret_cast<const uint8_t*>(kc);
+  p.vc = reinterpret_cast<const uint8_t*>(vc);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  decode_split_kernel<F8><<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                            const int* seqlens, const int* idx, int kt, int forced, void* o, void* ws,
+                                            cudaStream_t s) {
+  return sparse_tokens<false>(d, q, kc, vc, nullptr, nullptr, seqlens, idx, kt, forced, o, ws, s);
+}
+
+cudaError_t launch_decode_sparse_tokens_mma_fp8(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                                const float* k_scale, const float* v_scale, const int* seqlens,
+                                                const int* idx, int kt, int forced, void* o, void* ws, cudaStream_t s) {
+  return sparse_tokens<true>(d, q, kc, vc, k_scale, v_scale, seqlens, idx, kt, forced, o, ws, s);
 }
 
 }  // namespace hys

@@ -104,6 +104,14 @@ size_t decode_mma_sparse_tokens_workspace(const DecodeDims& d, int kt);
 cudaError_t launch_decode_sparse_tokens_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                             const int* seqlens, const int* idx, int kt, int forced, void* o, void* ws,
                                             cudaStream_t s);
+// FP8 (E4M3) cache variants of the token-variant decode: k_cache/v_cache hold codes, value =
+// code * scale[g] with k_scale/v_scale [Hkv]; workspaces as for the bf16 calls
+cudaError_t launch_decode_full_tokens_mma_fp8(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                              const float* k_scale, const float* v_scale, const int* seqlens, void* o,
+                                              float* tok_scores, void* ws, cudaStream_t s);
+cudaError_t launch_decode_sparse_tokens_mma_fp8(const DecodeDims& d, const void* q, const void* kc, const void* vc,
+                                                const float* k_scale, const float* v_scale, const int* seqlens,
+                                                const int* idx, int kt, int forced, void* o, void* ws, cudaStream_t s);
 cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const void* kc, const void* vc,
                                      const int* seqlens, const int* idx, int kb, const void* kr, const void* vr, int W,
                                      const int* swa_len, const float* gate, const float* sinks, void* o, void* ws,

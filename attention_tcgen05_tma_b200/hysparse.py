@@ -33,6 +33,7 @@ EXPORTED = (
     "hysparse_full_attn_select_decode_tokens_workspace_size", "hysparse_full_attn_select_decode_tokens",
     "hysparse_topk_decode_tokens", "hysparse_sparse_attn_decode_tokens_workspace_size",
     "hysparse_sparse_attn_decode_tokens",
+    "hysparse_full_attn_select_decode_tokens_fp8", "hysparse_sparse_attn_decode_tokens_fp8",
 )
 
 
@@ -83,6 +84,8 @@ _SIGS = {
     "hysparse_topk_decode_tokens": ([_DSH, _P, _I, _I, _P, _P, _P], _I),
     "hysparse_sparse_attn_decode_tokens_workspace_size": ([_DSH, _I, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_sparse_attn_decode_tokens": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P], _I),
+    "hysparse_full_attn_select_decode_tokens_fp8": ([_DSH, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "hysparse_sparse_attn_decode_tokens_fp8": ([_DSH, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P], _I),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -242,6 +245,18 @@ def hysparse_sparse_attn_decode_tokens(shape, dtype, q, kc, vc, seqlens, idx, k_
                                        stream) -> int:
     return load().hysparse_sparse_attn_decode_tokens(ctypes.byref(shape), dtype, q, kc, vc, seqlens, idx, k_tokens,
                                                      forced, o, ws, ws_bytes, stream)
+
+
+def hysparse_full_attn_select_decode_tokens_fp8(shape, q, kc, vc, k_scale, v_scale, seqlens, o, tok_scores, ws,
+                                                ws_bytes, stream) -> int:
+    return load().hysparse_full_attn_select_decode_tokens_fp8(ctypes.byref(shape), q, kc, vc, k_scale, v_scale,
+                                                              seqlens, o, tok_scores, ws, ws_bytes, stream)
+
+
+def hysparse_sparse_attn_decode_tokens_fp8(shape, q, kc, vc, k_scale, v_scale, seqlens, idx, k_tokens, forced, o, ws,
+                                           ws_bytes, stream) -> int:
+    return load().hysparse_sparse_attn_decode_tokens_fp8(ctypes.byref(shape), q, kc, vc, k_scale, v_scale, seqlens,
+                                                         idx, k_tokens, forced, o, ws, ws_bytes, stream)
 
 
 # ----------------------------------------------------------------------------- torch helpers
@@ -452,4 +467,54 @@ def sparse_attn_decode_tokens(q, k_cache, v_cache, idx, forced_window: int, *, s
                                               _ptr(idx), idx.shape[-1], forced_window, _ptr(o), _ptr(workspace),
                                               workspace.numel(), _stream(stream)),
            "hysparse_sparse_attn_decode_tokens")
+    return o
+
+
+def _fp8_cache_ok(q, k_cache, v_cache, k_scale, v_scale):
+    torch = _torch()
+    for t in (k_cache, v_cache):
+        if t.element_size() != 1:
+            raise TypeError("the FP8 cache holds one-byte E4M3 codes (torch.uint8 or torch.float8_e4m3fn)")
+    for t in (k_scale, v_scale):
+        if t.dtype != torch.float32 or t.numel() != k_cache.shape[1]:
+            raise TypeError("k_scale / v_scale are float32 [Hkv]")
+
+
+def full_attn_select_decode_tokens_fp8(q, k_cache, v_cache, k_scale, v_scale, *, seqlens=None, o=None,
+                                       tok_scores=None, workspace=None, stream=None):
+    """Token-variant decode full layer over an E4M3 cache (value = code * scale[g]):
+    o [B,Hq,D] bf16 and token scores [B,Hkv,L]."""
+    torch = _torch()
+    _fp8_cache_ok(q, k_cache, v_cache, k_scale, v_scale)
+    sh = decode_shape(q, k_cache)
+    if o is None:
+        o = torch.empty_like(q)
+    if tok_scores is None:
+        tok_scores = torch.empty((sh.B, sh.Hkv, sh.L), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = workspace_for(hysparse_full_attn_select_decode_tokens_workspace_size(sh, HYS_BF16), q.device)
+    _check(hysparse_full_attn_select_decode_tokens_fp8(sh, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                                                       _ptr(v_scale), _ptr(seqlens), _ptr(o), _ptr(tok_scores),
+                                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hysparse_full_attn_select_decode_tokens_fp8")
+    return o, tok_scores
+
+
+def sparse_attn_decode_tokens_fp8(q, k_cache, v_cache, k_scale, v_scale, idx, forced_window: int, *, seqlens=None,
+                                  o=None, workspace=None, stream=None):
+    """Token-variant sparse decode layer over an E4M3 cache: the selected tokens plus the newest
+    forced_window."""
+    torch = _torch()
+    _fp8_cache_ok(q, k_cache, v_cache, k_scale, v_scale)
+    sh = decode_shape(q, k_cache)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(hysparse_sparse_attn_decode_tokens_workspace_size(sh, HYS_BF16, idx.shape[-1]),
+                                  q.device)
+    _check(hysparse_sparse_attn_decode_tokens_fp8(sh, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                                                  _ptr(v_scale), _ptr(seqlens), _ptr(idx), idx.shape[-1],
+                                                  forced_window, _ptr(o), _ptr(workspace), workspace.numel(),
+                                                  _stream(stream)),
+           "hysparse_sparse_attn_decode_tokens_fp8")
     return o

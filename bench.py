@@ -380,7 +380,8 @@ def _uses_tc(H, w):
 
 def run_decode_tokens(args, torch, dist, rank, world, dev, peaks, peak_src):
     """Token-variant decode step on the decode workload's cache: full layer with token scores,
-    top-2048 tokens older than the forced newest 128, and the token-sparse layers."""
+    top-2048 tokens older than the forced newest 128, and the token-sparse layers; timed over the
+    bf16 cache and again over its FP8 (E4M3, per-KV-head scales) copy."""
     from attention_tcgen05_tma_b200 import hysparse as H
     from attention_tcgen05_tma_b200 import inputs as I
     w = I.WORKLOADS[args.decode_workload]
@@ -396,52 +397,74 @@ def run_decode_tokens(args, torch, dist, rank, world, dev, peaks, peak_src):
     sh = H.decode_shape(x["q"], x["k"])
     ws = H.workspace_for(H.hysparse_full_attn_select_decode_tokens_workspace_size(sh, H.HYS_BF16), dev)
     ws_sp = H.workspace_for(H.hysparse_sparse_attn_decode_tokens_workspace_size(sh, H.HYS_BF16, kt), dev)
-
-    def step(ev=None):
-        if ev:
-            ev[0].record()
-        H.full_attn_select_decode_tokens(x["q"], x["k"], x["v"], o=o, tok_scores=ts, workspace=ws)
-        if ev:
-            ev[1].record()
-        H.topk_decode_tokens(ts, kt, W, idx=idx)
-        if ev:
-            ev[2].record()
-        for l in range(w.layers):
-            H.sparse_attn_decode_tokens(x["q_sparse"][l], x["k"], x["v"], idx, W, o=osp, workspace=ws_sp)
-        if ev:
-            ev[3].record()
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        step(evs[i])
-    torch.cuda.synchronize()
-    full_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    topk_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    sp_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-    ms_step = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps, dist, dev)
-    # full layer: K and V once, plus every key's logit written and read back for the scores
-    full_bytes = 2.0 * w.B * w.Hkv * w.N * w.D * 2 + 2.0 * w.B * w.Hq * w.N * 4
-    sp_bytes = 2.0 * w.B * w.Hkv * (kt + W) * w.D * 2
     hbm = peaks["hbm_gbs"]
-    full_gbs = full_bytes / (full_ms / 1e3) / 1e9
-    sp_gbs = sp_bytes / (sp_ms / w.layers / 1e3) / 1e9
-    res = {"us_per_token": round(ms_step * 1e3 / (w.B * world), 3),
-           "ms_per_step": round(ms_step, 4),
-           "config": f"B={w.B} L={w.N} Hq={w.Hq} Hkv={w.Hkv} D={w.D}, 1 full + {w.layers} token-sparse, top-{kt} "
-                     f"tokens + forced newest {W}",
-           "full_ms": round(full_ms, 4), "topk_ms": round(topk_ms, 4), "sparse_ms_per_layer": round(sp_ms / w.layers, 4),
-           "roofline": {"kernel": "full_attn_select_decode_tokens", "bound": "hbm", "achieved": round(full_gbs, 1),
-                        "peak": hbm, "unit": "GB/s", "frac": round(full_gbs / hbm, 4), "traffic": None,
-                        "peak_source": f"{peak_src} hbm_gbs"},
-           "sparse_roofline": {"bound": "hbm", "achieved": round(sp_gbs, 1), "peak": hbm, "unit": "GB/s",
-                               "frac": round(sp_gbs / hbm, 4)}}
-    del x, ts, ws, ws_sp
+
+    def timed(full, sparse, elem_bytes):
+        def step(ev=None):
+            if ev:
+                ev[0].record()
+            full()
+            if ev:
+                ev[1].record()
+            H.topk_decode_tokens(ts, kt, W, idx=idx)
+            if ev:
+                ev[2].record()
+            for l in range(w.layers):
+                sparse(l)
+            if ev:
+                ev[3].record()
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+        full_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        topk_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+        sp_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+        ms_step = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps, dist, dev)
+        # full layer: K and V once, plus every key's logit written and read back for the scores
+        full_bytes = 2.0 * w.B * w.Hkv * w.N * w.D * elem_bytes + 2.0 * w.B * w.Hq * w.N * 4
+        sp_bytes = 2.0 * w.B * w.Hkv * (kt + W) * w.D * elem_bytes
+        full_gbs = full_bytes / (full_ms / 1e3) / 1e9
+        sp_gbs = sp_bytes / (sp_ms / w.layers / 1e3) / 1e9
+        return {"us_per_token": round(ms_step * 1e3 / (w.B * world), 3),
+                "ms_per_step": round(ms_step, 4),
+                "full_ms": round(full_ms, 4), "topk_ms": round(topk_ms, 4),
+                "sparse_ms_per_layer": round(sp_ms / w.layers, 4),
+                "roofline": {"kernel": "full_attn_select_decode_tokens", "bound": "hbm", "achieved": round(full_gbs, 1),
+                             "peak": hbm, "unit": "GB/s", "frac": round(full_gbs / hbm, 4), "traffic": None,
+                             "peak_source": f"{peak_src} hbm_gbs"},
+                "sparse_roofline": {"bound": "hbm", "achieved": round(sp_gbs, 1), "peak": hbm, "unit": "GB/s",
+                                    "frac": round(sp_gbs / hbm, 4)}}
+
+    res = timed(lambda: H.full_attn_select_decode_tokens(x["q"], x["k"], x["v"], o=o, tok_scores=ts, workspace=ws),
+                lambda l: H.sparse_attn_decode_tokens(x["q_sparse"][l], x["k"], x["v"], idx, W, o=osp,
+                                                      workspace=ws_sp), 2)
+    res["config"] = (f"B={w.B} L={w.N} Hq={w.Hq} Hkv={w.Hkv} D={w.D}, 1 full + {w.layers} token-sparse, top-{kt} "
+                     f"tokens + forced newest {W}")
+    # the same cache as E4M3 codes of value / scale (one scale per KV head for K and for V),
+    # converted on the device a sequence at a time
+    ks_np, vs_np = I.fp8_kv_scales(w)
+    ks, vs = torch.from_numpy(ks_np).to(dev), torch.from_numpy(vs_np).to(dev)
+    k8 = torch.empty(x["k"].shape, dtype=torch.uint8, device=dev)
+    v8 = torch.empty(x["v"].shape, dtype=torch.uint8, device=dev)
+    for b in range(w.B):
+        k8[b] = (x["k"][b].float() / ks[:, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        v8[b] = (x["v"][b].float() / vs[:, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    del x["k"], x["v"]
+    torch.cuda.empty_cache()
+    res["fp8"] = timed(lambda: H.full_attn_select_decode_tokens_fp8(x["q"], k8, v8, ks, vs, o=o, tok_scores=ts,
+                                                                    workspace=ws),
+                       lambda l: H.sparse_attn_decode_tokens_fp8(x["q_sparse"][l], k8, v8, ks, vs, idx, W, o=osp,
+                                                                 workspace=ws_sp), 1)
+    res["fp8"]["cache"] = "E4M3 codes, per-KV-head K and V scales"
+    del x, ts, ws, ws_sp, k8, v8
     torch.cuda.empty_cache()
     return res
 

@@ -285,6 +285,38 @@ HYS_API hys_status hysparse_sparse_attn_decode_tokens(const hys_decode_shape* sh
                                                   void* o, void* workspace, size_t workspace_bytes,
                                                   hys_stream_t stream);
 
+
+/* ------------------------------------------------------------------------------------
+ * Token-variant decode over an FP8 KV cache (HySparse2 explainer, "What actually improved?":
+ * the cache is sized in FP8).  The pages fix neither the FP8 format nor its scaling; these
+ * calls take OCP E4M3 codes ("fn" variant: bias 7, no infinities) with one float32 scale per
+ * KV head for K and one for V: the cached value is code * scale[g].
+ *
+ * Same operations, layouts, limits and errors as hysparse_full_attn_select_decode_tokens and
+ * hysparse_sparse_attn_decode_tokens, with:
+ *   q, o         [B,Hq,128] bf16 (D = 128 and G <= 16 only; other shapes: HYS_ERR_UNSUPPORTED);
+ *   k_cache,
+ *   v_cache      [B,Hkv,L,128] E4M3 codes, one byte each, 16-byte aligned;
+ *   k_scale,
+ *   v_scale      [Hkv] float32 device arrays, 4-byte aligned, finite and positive;
+ *   workspace    sized by the bf16 queries (hysparse_full_attn_select_decode_tokens_workspace_size
+ *                / hysparse_sparse_attn_decode_tokens_workspace_size with HYS_BF16).
+ * Token scores are the probabilities under the scaled logits, exactly as for a bf16 cache
+ * holding the decoded values; hysparse_topk_decode_tokens selects from them unchanged.
+ * ------------------------------------------------------------------------------------ */
+HYS_API hys_status hysparse_full_attn_select_decode_tokens_fp8(const hys_decode_shape* shape, const void* q,
+                                                           const void* k_cache, const void* v_cache,
+                                                           const float* k_scale, const float* v_scale,
+                                                           const int* seqlens, void* o, float* tok_scores,
+                                                           void* workspace, size_t workspace_bytes,
+                                                           hys_stream_t stream);
+HYS_API hys_status hysparse_sparse_attn_decode_tokens_fp8(const hys_decode_shape* shape, const void* q,
+                                                      const void* k_cache, const void* v_cache,
+                                                      const float* k_scale, const float* v_scale,
+                                                      const int* seqlens, const int* idx, int k_tokens,
+                                                      int forced_window, void* o, void* workspace,
+                                                      size_t workspace_bytes, hys_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

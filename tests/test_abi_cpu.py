@@ -114,3 +114,24 @@ def test_token_decode_entry_points_validate(lib):
                                                 None) == H.HYS_ERR_INVALID_ARG
     assert H.hysparse_sparse_attn_decode_tokens(dsh, H.HYS_BF16, 16, 16, 16, None, 16, 64, 64, 16, 16, 64,
                                                 None) == H.HYS_ERR_WORKSPACE
+
+
+def test_fp8_token_decode_entry_points_validate(lib):
+    """FP8-cache token decode: the scales are required (4-byte aligned), D must be 128, and the
+    workspace is the bf16 call's; every check fails before a launch."""
+    dsh = H.hys_decode_shape(2, 1000, 16, 2, 128, 64)
+    full = H.hysparse_full_attn_select_decode_tokens_fp8
+    sparse = H.hysparse_sparse_attn_decode_tokens_fp8
+    # missing scales / output, misaligned scale
+    assert full(dsh, 16, 16, 16, None, 16, None, 16, 16, 16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
+    assert full(dsh, 16, 16, 16, 16, 16, None, None, 16, 16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
+    assert full(dsh, 16, 16, 16, 18, 16, None, 16, 16, 16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
+    # D = 64: no FP8 path
+    d64 = H.hys_decode_shape(2, 1000, 16, 2, 64, 64)
+    assert full(d64, 16, 16, 16, 16, 16, None, 16, 16, 16, 1 << 20, None) == H.HYS_ERR_UNSUPPORTED
+    # short workspace
+    need = H.hysparse_full_attn_select_decode_tokens_workspace_size(dsh, H.HYS_BF16)
+    assert full(dsh, 16, 16, 16, 16, 16, None, 16, 16, 16, need - 256, None) == H.HYS_ERR_WORKSPACE
+    assert sparse(dsh, 16, 16, 16, 16, None, None, 16, 64, 64, 16, 16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
+    assert sparse(dsh, 16, 16, 16, 16, 16, None, 16, 64, 5000, 16, 16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
+    assert sparse(dsh, 16, 16, 16, 16, 16, None, 16, 64, 64, 16, 16, 64, None) == H.HYS_ERR_WORKSPACE

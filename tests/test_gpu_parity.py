@@ -297,3 +297,42 @@ def test_token_decode(case):
     if name == "g8_keep_all":   # every candidate selected: the sparse layer is dense decode of q'
         dense, _ = O.decode_full(a["q_sparse"][0], a["k"], a["v"], seqlens)
         assert np.max(np.abs(to_np(osp) - dense)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("case", TOKEN_DECODE_CASES, ids=[c[0] for c in TOKEN_DECODE_CASES])
+def test_token_decode_fp8(case):
+    """Token-variant decode over an E4M3 cache with per-KV-head K and V scales, against the
+    oracle run on the decoded cache values."""
+    name, B, L, Hq, Hkv, kt, W, ragged = case
+    D = 128
+    w = I.scaled(I.WORKLOADS["decode"], B=B, N=L, Hq=Hq, Hkv=Hkv, D=D, topk=kt, window=W, layers=1, seed=13,
+                 scale_std=1.0 / np.sqrt(D))
+    a = I.decode_arrays(w, layers=1)
+    c = I.decode_fp8_cache(w)
+    kd, vd = O.dequant_kv_fp8(c["k8"], c["k_scale"]), O.dequant_kv_fp8(c["v8"], c["v_scale"])
+    seqlens = np.array([L - 211 * b for b in range(B)], dtype=np.int32) if ragged else None
+    q, qs = to_dev(a["q"], "bf16"), to_dev(a["q_sparse"][0], "bf16")
+    k8, v8 = torch.from_numpy(c["k8"]).cuda(), torch.from_numpy(c["v8"]).cuda()
+    ks, vs = torch.from_numpy(c["k_scale"]).cuda(), torch.from_numpy(c["v_scale"]).cuda()
+    sl = torch.from_numpy(seqlens).cuda() if ragged else None
+    o, ts = H.full_attn_select_decode_tokens_fp8(q, k8, v8, ks, vs, seqlens=sl)
+    idx = H.topk_decode_tokens(ts, kt, W, seqlens=sl)
+    osp = H.sparse_attn_decode_tokens_fp8(qs, k8, v8, ks, vs, idx, W, seqlens=sl)
+    torch.cuda.synchronize()
+    assert H.hysparse_get_device_status() == 0
+    o_ref, _ = O.decode_full(a["q"], kd, vd, seqlens)
+    assert np.max(np.abs(to_np(o) - o_ref)) <= TOL["bf16"]
+    ts_ref = O.decode_token_scores(a["q"], kd, seqlens)
+    ts_gpu = to_np(ts)
+    assert score_rel_err(ts_ref, ts_gpu) <= 1e-3
+    gidx = idx.cpu().numpy().astype(np.int64)
+    for b in range(B):
+        Lb = int(seqlens[b]) if ragged else L
+        assert np.all(ts_gpu[b, :, Lb:] == 0)
+        for g in range(Hkv):
+            check_selection(ts_ref[b, g], ts_gpu[b, g], gidx[b, g], max(0, Lb - W), kt)
+    ref = O.decode_token_sparse(a["q_sparse"][0], kd, vd, gidx, W, seqlens)
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL["bf16"]
+    if name == "g8_keep_all":
+        dense, _ = O.decode_full(a["q_sparse"][0], kd, vd, seqlens)
+        assert np.max(np.abs(to_np(osp) - dense)) <= TOL["bf16"]
