@@ -25,6 +25,9 @@ Readings where the pages leave a step open (each is listed in the design notes):
   probability (the rescale step is exp(m~ - m)/l; the printed formula lost the exp).
 * TopK: candidates j in [0, I]; order by (score descending, index ascending);
   fewer than k candidates -> all of them; emitted ascending, padded with -1.
+* Per-position selection ([HS] §3.4.1-§3.4.2 as printed): S_g[t, j] = max over the
+  group's heads of S^h_{t,j}; row t selects the top k of its floor(t/64) + 1 blocks and its
+  sparse branch attends {i <= t : floor(i/64) in Sel_t}.
 * Sparse row t of tile I attends {i <= t : floor(i/64) in Sel_I}; the SWA branch
   attends [max(0, t-w+1), t]; o = sigmoid(g0) * o_sparse + sigmoid(g1) * o_swa.
 * Token variant: token score = sum over the group's heads and the tile's rows
@@ -180,6 +183,29 @@ def block_scores(q: np.ndarray, k: np.ndarray, reduce: str = "sum", block: int =
     return out
 
 
+def block_scores_rows(q: np.ndarray, k: np.ndarray, block: int = 64) -> np.ndarray:
+    """Per-position group scores ([HS] §3.4.1 group-wise maximum over the group's heads, taken
+    per (query position, key block) entry; §3.4.2 selection per query position):
+    S_g[t, j] = max_h S^h_{t,j}, with S^h_{t,j} the largest probability of row t inside block j
+    (keys <= t); 0 for blocks that start after t.  Returns [B, Hkv, N, NB]."""
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    nb = (N + block - 1) // block
+    out = np.zeros((B, Hkv, N, nb))
+    for b in range(B):
+        for g in range(Hkv):
+            kk = np.asarray(k[b, g], dtype=np.float64)
+            for I in range(nb):
+                rows = tile_rows(I, N, block)
+                acc = np.zeros((len(rows), nb))
+                for h in range(g * G, (g + 1) * G):
+                    p, _, _ = causal_softmax(np.asarray(q[b, h, rows], np.float64), rows, kk)
+                    acc = np.maximum(acc, block_max_probs(p, rows, block))
+                out[b, g, rows] = acc
+    return out
+
+
 # -----------------------------------------------------------------------------
 # TopK  ([HS] §3.4.2; tie and padding rules are the reading above)
 # -----------------------------------------------------------------------------
@@ -202,6 +228,19 @@ def topk_blocks(scores: np.ndarray, k: int) -> np.ndarray:
         for g in range(Hkv):
             for I in range(T):
                 out[b, g, I] = select_topk(scores[b, g, I], min(I + 1, NB), k)
+    return out
+
+
+def topk_blocks_rows(scores: np.ndarray, k: int, block: int = 64) -> np.ndarray:
+    """[B, Hkv, N, NB] per-position scores -> [B, Hkv, N, k] block indices ([HS] §3.4.2: for each
+    query position t and group, the k highest of the floor(t/64) + 1 blocks holding keys <= t);
+    ties to the lower index, ascending, padded with -1."""
+    B, Hkv, N, NB = scores.shape
+    out = np.full((B, Hkv, N, k), -1, dtype=np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(N):
+                out[b, g, t] = select_topk(scores[b, g, t], min(t // block + 1, NB), k)
     return out
 
 
@@ -260,6 +299,25 @@ def sparse_attention(q_s, k, v, idx, k_swa, v_swa, window: int, gate, block: int
                 o[b, h, rows] = gated_sparse_rows(q_s[b, h, rows], rows, kk, vv, idx[b, g, I],
                                                   ks, vs, window, gate[b, h, rows], block,
                                                   None if sinks is None else sinks[h])
+    return o
+
+
+def sparse_attention_rows(q_s, k, v, idx_rows, k_swa, v_swa, window: int, gate, block: int = 64, sinks=None):
+    """Whole sparse layer with per-position selection ([HS] §3.4.2 'computed per query position';
+    §3.4.3 branches and gate): row t's sparse branch attends {i <= t : floor(i/64) in Sel_t} with
+    Sel_t = idx_rows[b, g, t].  idx_rows [B,Hkv,N,k]; other arguments as sparse_attention."""
+    B, Hq, N, D = q_s.shape
+    G = Hq // k.shape[1]
+    o = np.zeros((B, Hq, N, D))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            kk, vv = np.asarray(k[b, g], np.float64), np.asarray(v[b, g], np.float64)
+            ks, vs = np.asarray(k_swa[b, g], np.float64), np.asarray(v_swa[b, g], np.float64)
+            for t in range(N):
+                rows = np.array([t])
+                o[b, h, t] = gated_sparse_rows(q_s[b, h, rows], rows, kk, vv, idx_rows[b, g, t], ks, vs, window,
+                                               gate[b, h, rows], block, None if sinks is None else sinks[h])[0]
     return o
 
 

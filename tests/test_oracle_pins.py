@@ -537,6 +537,72 @@ def test_fp8_token_decode_pins():
     np.testing.assert_allclose(o_all, o_dense, rtol=1e-12, atol=1e-13)
 
 
+def test_per_position_selection_pins():
+    """Per-position selection: the scores equal a torch float64 causal softmax, reshaped into
+    64-key blocks and maxed over the block and the group's heads; the top k of row t never
+    passes block floor(t/64), breaks ties low and matches the brute-force selection; each row's
+    sparse branch equals torch attention under a mask built from that row's own blocks; rows
+    that share one selection reproduce the per-tile layer; k covering every block is dense."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, N, D, k, win = 1, 4, 2, 300, 16, 2, 20
+    G = Hq // Hkv
+    q = rng.standard_normal((B, Hq, N, D))
+    kk = rng.standard_normal((B, Hkv, N, D))
+    vv = rng.standard_normal((B, Hkv, N, D))
+    sc = O.block_scores_rows(q, kk)
+    nb = (N + 63) // 64
+    causal = torch.ones(N, N, dtype=torch.bool).tril()
+    for g in range(Hkv):
+        want = torch.zeros(N, nb, dtype=torch.float64)
+        for h in range(g * G, (g + 1) * G):
+            lg = (torch.from_numpy(q[0, h]) @ torch.from_numpy(kk[0, g]).T) / math.sqrt(D)
+            p = torch.softmax(lg.masked_fill(~causal, float("-inf")), dim=1)
+            pad = torch.zeros(N, nb * 64, dtype=torch.float64)
+            pad[:, :N] = p
+            want = torch.maximum(want, pad.view(N, nb, 64).amax(dim=2))
+        np.testing.assert_allclose(sc[0, g], want.numpy(), rtol=1e-12, atol=1e-15)
+    idx = O.topk_blocks_rows(sc, k)
+    for g in range(Hkv):
+        for t in range(N):
+            sel = idx[0, g, t]
+            assert sel.tolist() == BF.topk(sc[0, g, t].tolist(), t // 64 + 1, k)
+            assert np.all(sel[sel >= 0] <= t // 64)
+    ties = O.topk_blocks_rows(np.zeros((1, 1, 200, 4)), 2)
+    assert ties[0, 0, 199].tolist() == [0, 1] and ties[0, 0, 10].tolist() == [0, -1]
+    # sparse branch of each row vs torch under the row's own mask (gate saturated to the sparse branch)
+    gate = np.zeros((B, Hq, N, 2))
+    gate[..., 0], gate[..., 1] = 60.0, -60.0
+    ks, vs = rng.standard_normal((B, Hkv, N, D)), rng.standard_normal((B, Hkv, N, D))
+    o = O.sparse_attention_rows(q, kk, vv, idx, ks, vs, win, gate)
+    for h in range(Hq):
+        g = h // G
+        mask = torch.zeros(N, N, dtype=torch.bool)
+        for t in range(N):
+            for j in idx[0, g, t]:
+                if j >= 0:
+                    mask[t, 64 * j:min(N, 64 * j + 64)] = True
+        mask &= causal
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[0, h])[None, None], torch.from_numpy(kk[0, g])[None, None],
+            torch.from_numpy(vv[0, g])[None, None], attn_mask=mask[None, None])
+        np.testing.assert_allclose(o[0, h], ref[0, 0].numpy(), rtol=1e-9, atol=1e-12)
+    # one selection per tile -> the per-tile layer
+    tile_idx = O.topk_blocks(O.block_scores(q, kk, "max"), k)
+    rows_idx = np.repeat(tile_idx, 64, axis=2)[:, :, :N]
+    gate2 = rng.standard_normal((B, Hq, N, 2))
+    np.testing.assert_allclose(O.sparse_attention_rows(q, kk, vv, rows_idx, ks, vs, win, gate2),
+                               O.sparse_attention(q, kk, vv, tile_idx, ks, vs, win, gate2), rtol=1e-12, atol=1e-13)
+    # k covering every block: dense causal attention
+    full_idx = O.topk_blocks_rows(sc, nb)
+    o_all = O.sparse_attention_rows(q, kk, vv, full_idx, ks, vs, win, gate)
+    for h in range(Hq):
+        g = h // G
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[0, h])[None, None], torch.from_numpy(kk[0, g])[None, None],
+            torch.from_numpy(vv[0, g])[None, None], is_causal=True)
+        np.testing.assert_allclose(o_all[0, h], ref[0, 0].numpy(), rtol=1e-9, atol=1e-12)
+
+
 def test_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the oracle and check that a pin above fails."""
     g = _gold()
