@@ -122,8 +122,9 @@ hys_status hysparse_full_attn_select_workspace_size(const hys_shape* shape, hys_
   PrefillDims d;
   hys_status st = check_prefill(shape, &d);
   if (st != HYS_OK) return st;
-  if (!bytes || !dtype_ok(dtype) || (gran != HYS_GRAN_BLOCK && gran != HYS_GRAN_TOKEN)) return HYS_ERR_INVALID_ARG;
-  *bytes = full_ws_bytes(d, dtype, gran);
+  if (!bytes || !dtype_ok(dtype) || (gran != HYS_GRAN_BLOCK && gran != HYS_GRAN_TOKEN && gran != HYS_GRAN_BLOCK_ROW))
+    return HYS_ERR_INVALID_ARG;
+  *bytes = full_ws_bytes(d, dtype, gran == HYS_GRAN_BLOCK_ROW ? HYS_GRAN_BLOCK : gran);
   return HYS_OK;
 }
 
@@ -134,16 +135,22 @@ hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype dtype, co
   PrefillDims d;
   hys_status st = check_prefill(shape, &d);
   if (st != HYS_OK) return st;
-  if (!dtype_ok(dtype) || (gran != HYS_GRAN_BLOCK && gran != HYS_GRAN_TOKEN)) return HYS_ERR_INVALID_ARG;
+  if (!dtype_ok(dtype) || (gran != HYS_GRAN_BLOCK && gran != HYS_GRAN_TOKEN && gran != HYS_GRAN_BLOCK_ROW))
+    return HYS_ERR_INVALID_ARG;
   if (red != HYS_REDUCE_SUM && red != HYS_REDUCE_MAX) return HYS_ERR_INVALID_ARG;
   if (gran == HYS_GRAN_TOKEN && red != HYS_REDUCE_SUM) return HYS_ERR_UNSUPPORTED;
+  if (gran == HYS_GRAN_BLOCK_ROW && (red != HYS_REDUCE_MAX || !full_attn_tc_supported(d, dtype, true)))
+    return HYS_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !scores) return HYS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(scores) ||
       !aligned16(lse_opt) || !aligned16(workspace))
     return HYS_ERR_INVALID_ARG;
-  const size_t need = full_ws_bytes(d, dtype, gran);
+  const size_t need = full_ws_bytes(d, dtype, gran == HYS_GRAN_BLOCK_ROW ? HYS_GRAN_BLOCK : gran);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return HYS_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (gran == HYS_GRAN_BLOCK_ROW)
+    return from_cuda(launch_full_attn_tc(d, q, k, v, o, lse_opt, scores, red, true, workspace, workspace_bytes, s,
+                                         true));
   if (gran == HYS_GRAN_BLOCK) {
     if (full_attn_tc_supported(d, dtype, true))
       return from_cuda(launch_full_attn_tc(d, q, k, v, o, lse_opt, scores, red, true, workspace, workspace_bytes, s));
@@ -173,6 +180,18 @@ hys_status hysparse_topk(const hys_shape* shape, const float* scores, int k, int
   if (d.NB > 8192) return HYS_ERR_UNSUPPORTED;
   return from_cuda(launch_topk_blocks(scores, idx, d.B, d.Hkv, d.T, d.NB, k, nullptr, 0, false,
                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_topk_rows(const hys_shape* shape, const float* scores, int k, int* idx, hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!scores || !idx || k < 1 || k > 1024) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx)) return HYS_ERR_INVALID_ARG;
+  if (d.NB > 8192) return HYS_ERR_UNSUPPORTED;
+  if ((long long)d.B * d.Hkv * d.N >= (1ll << 31)) return HYS_ERR_UNSUPPORTED;
+  return from_cuda(launch_topk_blocks_rows(scores, idx, d.B, d.Hkv, d.N, d.NB, k,
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hys_status hysparse_topk_tokens_workspace_size(const hys_shape* shape, int k_tokens, size_t* bytes) {
@@ -230,6 +249,27 @@ hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const v
   }
   return from_cuda(launch_sparse_attn_simt(d, dtype, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,
                                            gate_logits, sinks, o, s));
+}
+
+hys_status hysparse_sparse_attn_rows(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                     const void* k_shared, const void* v_shared, const int* idx, int k,
+                                     const void* k_swa, const void* v_swa, int window, const float* gate_logits,
+                                     const float* sinks, void* o, void* workspace, size_t workspace_bytes,
+                                     hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (!q_sparse || !k_shared || !v_shared || !idx || !k_swa || !v_swa || !gate_logits || !o) return HYS_ERR_INVALID_ARG;
+  if (k < 1 || k > 1024 || window < 1) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(k_swa) ||
+      !aligned16(v_swa) || !aligned16(gate_logits) || !aligned16(sinks) || !aligned16(o) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  if (!sparse_attn_rows_tc_supported(d, dtype) || k > 256) return HYS_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < align256(sparse_attn_tc_workspace(d))) return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_sparse_attn_tc(d, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window, gate_logits,
+                                         sinks, o, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream),
+                                         true));
 }
 
 hys_status hysparse_sparse_attn_tokens_workspace_size(const hys_shape* shape, hys_dtype dtype, int forced_window,

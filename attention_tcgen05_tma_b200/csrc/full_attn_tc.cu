@@ -66,7 +66,8 @@ struct Params {
   __nv_bfloat16* o;
   int o_v8;       // o is 32-byte aligned (256-bit stores)
   float* lse;     // optional [B,Hq,N]
-  float* scores;  // optional [B,Hkv,T,NB] (block scores are emitted iff non-null)
+  float* scores;  // optional [B,Hkv,T,NB], or [B,Hkv,N,NB] per position (emitted iff non-null)
+  int per_row;    // per-position scores: group max per (position, block), zeroed before the launch
   float* stash;   // [grid][2][128][NBpad]
   int* counter;   // work-unit counter (zeroed before the launch)
   int red_max;
@@ -476,7 +477,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (p.lse != nullptr && valid) p.lse[((size_t)b * p.Hq + h) * p.N + t] = (m_used * sc + log2f(l)) * 0.69314718055994531f;
-        if (scores_on) {
+        if (scores_on && p.per_row) {
+          // per-position scores: rows r and r + 64 are the M-tile's two heads at one position;
+          // their maximum joins the other heads' through an atomic max on the float bits (all
+          // values are >= 0, so the bit patterns order like the floats; any order gives one result)
+          row_m[row] = m_used;
+          row_il[row] = valid ? il : 0.0f;
+          if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->wg[s], wg_ph, abort)))) break;
+          const int nj = I + 1;
+          unsigned int* out = reinterpret_cast<unsigned int*>(p.scores) + (((size_t)b * p.Hkv + g) * p.N + 64 * I) * p.NB;
+          for (int e = wtid; e < 64 * nj; e += 128) {
+            const int pos = e / nj, j = e - pos * nj;
+            if (64 * I + pos >= p.N) break;
+            const float x0 = exp2f((stash[(size_t)pos * p.NBpad + j] - row_m[pos]) * sc) * row_il[pos];
+            const float x1 = exp2f((stash[(size_t)(pos + 64) * p.NBpad + j] - row_m[pos + 64]) * sc) * row_il[pos + 64];
+            atomicMax(out + (size_t)pos * p.NB + j, __float_as_uint(fmaxf(x0, x1)));
+          }
+          if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->wg[s], wg_ph, abort)))) break;
+        } else if (scores_on) {
           row_m[row] = m_used;
           row_il[row] = valid ? il : 0.0f;
           if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->wg[s], wg_ph, abort)))) break;
@@ -492,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      if (scores_on) {
+      if (scores_on && !p.per_row) {
         // ---- unit epilogue: both slots' accumulators -> scores[b,g,I,:]
         if (!(ok = __all_sync(0xffffffffu, group_sync(&bars->all[0], all_ph, abort)))) break;
         float* out = p.scores + (((size_t)b * p.Hkv + g) * p.T + I) * p.NB;
@@ -553,7 +571,7 @@ int grid_size(const PrefillDims& d) { return num_units(d) < kMaxGrid ? num_units
 
 template <int D>
 cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, const void* v, void* o, float* lse,
-                         float* scores, hys_reduce red, void* ws, cudaStream_t s) {
+                         float* scores, hys_reduce red, bool per_row, void* ws, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, d.N, d.B * d.Hq, 64) || !make_map(&mk, k, D, d.N, d.B * d.Hkv, 128) ||
       !make_map(&mv, v, D, d.N, d.B * d.Hkv, 128))
@@ -572,6 +590,7 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   p.lse = lse;
   p.scores = scores;
+  p.per_row = per_row ? 1 : 0;
   p.counter = reinterpret_cast<int*>(ws);
   p.stash = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + 256);
   p.red_max = red == HYS_REDUCE_MAX;
@@ -590,6 +609,10 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
+  if (per_row && scores != nullptr) {
+    e = cudaMemsetAsync(scores, 0, sizeof(float) * (size_t)d.B * d.Hkv * d.N * d.NB, s);
+    if (e != cudaSuccess) return e;
+  }
   full_attn_tc_kernel<D><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
@@ -609,11 +632,11 @@ size_t full_attn_tc_workspace(const PrefillDims& d, bool want_scores) {
 
 cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, void* o,
                                 float* lse, float* scores, hys_reduce red, bool want_scores, void* ws, size_t ws_bytes,
-                                cudaStream_t s) {
+                                cudaStream_t s, bool per_row) {
   if (!want_scores) scores = nullptr;
   if (ws == nullptr || ws_bytes < full_attn_tc_workspace(d, want_scores)) return cudaErrorInvalidValue;
-  return d.D == 64 ? launch_typed<64>(d, q, k, v, o, lse, scores, red, ws, s)
-                   : launch_typed<128>(d, q, k, v, o, lse, scores, red, ws, s);
+  return d.D == 64 ? launch_typed<64>(d, q, k, v, o, lse, scores, red, per_row, ws, s)
+                   : launch_typed<128>(d, q, k, v, o, lse, scores, red, per_row, ws, s);
 }
 
 }  // namespace hys

@@ -40,9 +40,10 @@ cudaError_t launch_token_scores_simt(const PrefillDims& d, hys_dtype dt, const v
 // ---- full layer, tcgen05 path (bf16, D=128, even G) ----------------------------------------
 bool full_attn_tc_supported(const PrefillDims& d, hys_dtype dt, bool want_scores);
 size_t full_attn_tc_workspace(const PrefillDims& d, bool want_scores);
+// per_row: scores [B,Hkv,N,NB] per position, the group max (zeroed by the launch)
 cudaError_t launch_full_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v,
                                 void* o, float* lse, float* scores, hys_reduce red, bool want_scores,
-                                void* ws, size_t ws_bytes, cudaStream_t s);
+                                void* ws, size_t ws_bytes, cudaStream_t s, bool per_row = false);
 
 // Token scores (second pass) on the tensor cores; ws holds the 256-byte unit counter.
 bool token_scores_tc_supported(const PrefillDims& d, hys_dtype dt);
@@ -59,6 +60,9 @@ cudaError_t launch_token_sparse_tc(const PrefillDims& d, const void* q, const vo
 // rows = B*Hkv*T (prefill) or B*Hkv (decode); row r has n_cand(r) candidates.
 cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, int T, int NB, int k,
                                const int* seqlens, int L, bool decode, cudaStream_t s);
+// per-position rows: B*Hkv*N rows of NB scores; row (b, g, t) has floor(t/64) + 1 candidates
+cudaError_t launch_topk_blocks_rows(const float* scores, int* idx, int B, int Hkv, int N, int NB, int k,
+                                    cudaStream_t s);
 cudaError_t launch_topk_tokens(const PrefillDims& d, const float* scores, int k_tokens, int forced,
                                int* idx, cudaStream_t s);
 cudaError_t launch_topk_decode_tokens(const float* scores, int* idx, int B, int Hkv, int L, int k_tokens, int forced,
@@ -75,9 +79,12 @@ cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const 
 
 bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt);
 size_t sparse_attn_tc_workspace(const PrefillDims& d);
+// per_row: idx is [B,Hkv,N,kb], one block list per query position (NB <= 512)
+bool sparse_attn_rows_tc_supported(const PrefillDims& d, hys_dtype dt);
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
                                   int kb, const void* ks, const void* vs, int window, const float* gate,
-                                  const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s);
+                                  const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s,
+                                  bool per_row = false);
 
 // ---- decode ----------------------------------------------------------------------------------
 size_t decode_full_workspace(const DecodeDims& d);

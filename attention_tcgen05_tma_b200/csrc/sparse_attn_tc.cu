@@ -53,10 +53,12 @@ __device__ __forceinline__ float2 exp2_pair(float2 x, int i) {
 }
 
 
+constexpr int kRowWords = 16;   // per-position mode: union entries < 512 (N <= 32768)
+
 struct Params {
   int B, N, Hq, Hkv, G, T, kb, window;
   int num_units;
-  const int* idx;      // [B,Hkv,T,kb]
+  const int* idx;      // [B,Hkv,T,kb], or [B,Hkv,N,kb] per position
   const float* gate;   // [B,Hq,N,2]
   const float* sinks;  // [Hq,2] sink logits of the two branches, or null
   __nv_bfloat16* o;
@@ -83,7 +85,11 @@ struct Cfg {
   static constexpr int kOffList = kOffKV + kStages * kKVBytes;   // producer's copy of a unit's indices
   static constexpr int kOffBar = kOffList + kMaxKb * 4;
   static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+  // per-position mode: for each queue slot and each of the tile's 64 positions, the union
+  // entries that position selected (bit e of row r), and the producer's union bitmap
+  static constexpr int kOffRows = kOffMisc + 64;
+  static constexpr int kOffUnion = kOffRows + tc::kQueueSlots * 64 * kRowWords * 4;
+  static constexpr int kSmemBytes = kOffUnion + kRowWords * 4 + 1024;
 };
 
 struct Unit {
@@ -121,12 +127,82 @@ __device__ __forceinline__ Unit make_unit(const Params& p, int u, int nsel, int 
   return x;
 }
 
+// Per-position selection of a unit (warp-wide): the union of the 64 rows' blocks, in ascending
+// order, goes to plist (nsel entries; diag = the entry of block I or -1); bit e of rb[r] is set
+// when row r selected union entry e.  Blocks past I are never candidates of the tile's rows and,
+// like padding entries (-1), are ignored.
+__device__ __noinline__ void per_row_lists(const int* __restrict__ idx, int N, int Hkv, int kb, int b, int g, int I,
+                                           int* plist, uint32_t* rb, uint32_t* ubits, int lane, int* out) {
+  const int nw = (I >> 5) + 1;
+  if (lane < kRowWords) ubits[lane] = 0u;
+  for (int i = lane; i < 64 * kRowWords; i += 32) rb[i] = 0u;
+  __syncwarp();
+  const int rows = min(64, N - 64 * I);
+  const int* base = idx + (((size_t)b * Hkv + g) * N + 64 * I) * kb;
+  const int total = rows * kb;
+  // pass 1: the union (eight 32-entry chunks in flight per step)
+  for (int e0 = 0; e0 < total; e0 += 256) {
+    int jv[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int e = e0 + 32 * c + lane;
+      jv[c] = e < total ? base[e] : -1;
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (jv[c] >= 0 && jv[c] <= I) atomicOr(&ubits[jv[c] >> 5], 1u << (jv[c] & 31));
+  }
+  __syncwarp();
+  // lane w owns bitmap word w: its entries start at the exclusive prefix of the popcounts
+  const uint32_t wv = lane < nw ? ubits[lane] : 0u;
+  const int cnt = __popc(wv);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int excl = incl - cnt;
+  const int nsel = __shfl_sync(0xffffffffu, incl, 31);
+  {
+    int pos = excl;
+    for (uint32_t w = wv; w != 0u; w &= w - 1u) plist[pos++] = 32 * lane + __ffs(w) - 1;
+  }
+  const uint32_t wI = __shfl_sync(0xffffffffu, wv, I >> 5);
+  const int xI = __shfl_sync(0xffffffffu, excl, I >> 5);
+  const int diag = ((wI >> (I & 31)) & 1u) ? xI + __popc(wI & ((1u << (I & 31)) - 1u)) : -1;
+  // pass 2: each row's selected blocks as union entries
+  for (int e0 = 0; e0 < total; e0 += 256) {
+    int jv[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int e = e0 + 32 * c + lane;
+      jv[c] = e < total ? base[e] : -1;
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int j = jv[c];
+      const bool in = j >= 0 && j <= I;
+      const int w = in ? j >> 5 : 0;
+      const int wp = __shfl_sync(0xffffffffu, excl, w);
+      const uint32_t ww = __shfl_sync(0xffffffffu, wv, w);
+      if (in) {
+        const int ent = wp + __popc(ww & ((1u << (j & 31)) - 1u));
+        const int r = (e0 + 32 * c + lane) / kb;
+        atomicOr(&rb[r * kRowWords + (ent >> 5)], 1u << (ent & 31));
+      }
+    }
+  }
+  out[0] = nsel;
+  out[1] = diag;
+}
+
 __device__ __forceinline__ void fail(volatile int* abort, int* status) {
   *abort = 1;
   report_status(status, HYS_ERR_TIMEOUT);
 }
 
-template <int D>
+template <int D, bool PR>   // PR: per-position selection (idx [B,Hkv,N,kb])
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKs,
@@ -192,7 +268,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       u = __shfl_sync(0xffffffffu, u, 0);
       int nsel = 0, diag = -1;
-      if (u >= 0) {
+      if (PR) {
+        // the slot's row masks may be rewritten only after every consumer released the slot
+        const uint32_t sl = n % tc::kQueueSlots;
+        if (lane == 0) ok = tc::mbar_wait(&bars->queue.empty[sl], ((n / tc::kQueueSlots) & 1u) ^ 1u, abort);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (u >= 0) {
+          const Unit x0 = make_unit(p, u, 0, -1);
+          int nd[2];
+          per_row_lists(p.idx, p.N, p.Hkv, p.kb, x0.b, x0.g, x0.I, plist,
+                        reinterpret_cast<uint32_t*>(smem + C::kOffRows) + sl * 64 * kRowWords,
+                        reinterpret_cast<uint32_t*>(smem + C::kOffUnion), lane, nd);
+          nsel = nd[0];
+          diag = nd[1];
+        }
+        __syncwarp();
+        __threadfence_block();
+        if (lane == 0) {
+          bars->queue.unit[sl] = u;
+          bars->queue.info[sl][0] = nsel;
+          bars->queue.info[sl][1] = diag;
+          tc::mbar_arrive(&bars->queue.full[sl]);
+        }
+      } else if (u >= 0) {
         const Unit x0 = make_unit(p, u, 0, -1);
         const int* sel = p.idx + (((size_t)x0.b * p.Hkv + x0.g) * p.T + x0.I) * p.kb;
         nsel = p.kb;
@@ -214,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      if (lane == 0) ok = tc::queue_push(&bars->queue, n, u, abort, nsel, diag);
+      if (lane == 0 && !PR) ok = tc::queue_push(&bars->queue, n, u, abort, nsel, diag);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok || u < 0) break;
       if (lane == 0) {
@@ -394,7 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (uint32_t n = 0; ok; ++n) {
       int nsel = 0, diag = -1;
-      const int u = tc::queue_pop(&bars->queue, n, abort, ok, &nsel, &diag);
+      // the slot stays held until the unit is done: per-position masks live beside its id
+      const int u = tc::queue_peek(&bars->queue, n, abort, ok, &nsel, &diag);
       // warp-uniform outcomes: the warp-collective TMEM accesses must not diverge
       ok = __all_sync(0xffffffffu, ok);
       if (__any_sync(0xffffffffu, u < 0)) break;
@@ -452,7 +552,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             chi[hh] = -1;
             if (kind == kSparse) {
               const int e = 2 * tau + hh;
-              if (e < x.nsel) {
+              bool sel = e < x.nsel;
+              if (PR && sel) {   // this position's own blocks among the unit's union
+                const uint32_t* rbits = reinterpret_cast<const uint32_t*>(smem + C::kOffRows) +
+                                        ((n % tc::kQueueSlots) * 64 + (row & 63)) * kRowWords;
+                sel = (rbits[e >> 5] >> (e & 31)) & 1u;
+              }
+              if (sel) {
                 clo[hh] = 0;
                 chi[hh] = (e == x.diag) ? t - 64 * x.I : 63;  // only block I crosses the causal line
               }
@@ -607,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      tc::queue_release(&bars->queue, n);
     }
     if (!ok) fail(abort, p.status);
   }
@@ -650,7 +757,7 @@ bool make_map(CUtensorMap* m, const void* base, int D, int rows, int heads) {
 int num_units(const PrefillDims& d) { return d.B * d.Hkv * d.T; }
 int grid_size(const PrefillDims& d) { return num_units(d) < kMaxGrid ? num_units(d) : kMaxGrid; }
 
-template <int D>
+template <int D, bool PR>
 cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx, int kb,
                          const void* ks, const void* vs, int window, const float* gate, const float* sinks,
                          void* o, void* ws, cudaStream_t s) {
@@ -677,20 +784,20 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.counter = reinterpret_cast<int*>(ws);
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
-  const int smem = Cfg<D>::kSmemBytes;
+  const int smem = PR ? Cfg<D>::kSmemBytes : Cfg<D>::kOffRows + 1024;   // per-position masks only when used
   static int regs = -1;   // the register split assumes exactly kLaunchRegs per thread at launch
   if (regs < 0) {
     cudaFuncAttributes fa;
-    cudaError_t e0 = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<D>);
+    cudaError_t e0 = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<D, PR>);
     if (e0 != cudaSuccess) return e0;
     regs = fa.numRegs;
   }
   if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D, PR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
-  sparse_attn_tc_kernel<D><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, mks, mvs, p);
+  sparse_attn_tc_kernel<D, PR><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, mks, mvs, p);
   return cudaGetLastError();
 }
 
@@ -702,12 +809,21 @@ bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt) {
 
 size_t sparse_attn_tc_workspace(const PrefillDims&) { return 256; }
 
+bool sparse_attn_rows_tc_supported(const PrefillDims& d, hys_dtype dt) {
+  return sparse_attn_tc_supported(d, dt) && d.NB <= 32 * kRowWords;
+}
+
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
                                   int kb, const void* ks, const void* vs, int window, const float* gate,
-                                  const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s) {
+                                  const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s,
+                                  bool per_row) {
   if (ws_bytes < sparse_attn_tc_workspace(d)) return cudaErrorInvalidValue;
-  return d.D == 64 ? launch_typed<64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s)
-                   : launch_typed<128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s);
+  if (per_row && d.NB > 32 * kRowWords) return cudaErrorInvalidValue;
+  if (per_row)
+    return d.D == 64 ? launch_typed<64, true>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s)
+                     : launch_typed<128, true>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s);
+  return d.D == 64 ? launch_typed<64, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s)
+                   : launch_typed<128, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s);
 }
 
 }  // namespace hys

@@ -117,7 +117,9 @@ __global__ void __launch_bounds__(kBlkThreads) topk_blocks_kernel(const float* _
   __shared__ RadixSmem<kBlkThreads / 32> sm;
   const int row = blockIdx.x;
   int n;
-  if (decode) {
+  if (decode == 2) {   // per-position rows (L = N): row t has blocks 0 .. floor(t/64)
+    n = min(NB, (row % L) / 64 + 1);
+  } else if (decode) {
     const int b = row / Hkv;
     const int Lb = seqlens ? max(1, min(seqlens[b], L)) : L;
     n = min(NB, (Lb + 63) / 64);
@@ -176,6 +178,20 @@ cudaError_t launch_topk_blocks(const float* scores, int* idx, int B, int Hkv, in
     if (e != cudaSuccess) return e;
   }
   topk_blocks_kernel<<<rows, kBlkThreads, smem, s>>>(scores, idx, Hkv, T, NB, k, seqlens, L, decode ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_blocks_rows(const float* scores, int* idx, int B, int Hkv, int N, int NB, int k,
+                                    cudaStream_t s) {
+  const size_t smem = (size_t)NB * sizeof(uint32_t);
+  const size_t static_smem = sizeof(RadixSmem<kBlkThreads / 32>);
+  if (smem + static_smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(topk_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  topk_blocks_kernel<<<(unsigned)((size_t)B * Hkv * N), kBlkThreads, smem, s>>>(scores, idx, Hkv, 1, NB, k, nullptr,
+                                                                                N, 2);
   return cudaGetLastError();
 }
 

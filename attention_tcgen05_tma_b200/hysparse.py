@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(PKG, "libhysparse.so")
 
 HYS_OK, HYS_ERR_INVALID_ARG, HYS_ERR_UNSUPPORTED, HYS_ERR_CUDA, HYS_ERR_TIMEOUT, HYS_ERR_WORKSPACE = range(6)
 HYS_F32, HYS_BF16 = 0, 1
-HYS_GRAN_BLOCK, HYS_GRAN_TOKEN = 0, 1
+HYS_GRAN_BLOCK, HYS_GRAN_TOKEN, HYS_GRAN_BLOCK_ROW = 0, 1, 2
 HYS_REDUCE_SUM, HYS_REDUCE_MAX = 0, 1
 
 # every symbol include/hysparse.h declares
@@ -34,6 +34,7 @@ EXPORTED = (
     "hysparse_topk_decode_tokens", "hysparse_sparse_attn_decode_tokens_workspace_size",
     "hysparse_sparse_attn_decode_tokens",
     "hysparse_full_attn_select_decode_tokens_fp8", "hysparse_sparse_attn_decode_tokens_fp8",
+    "hysparse_topk_rows", "hysparse_sparse_attn_rows",
 )
 
 
@@ -66,10 +67,12 @@ _SIGS = {
     "hysparse_full_attn_select_workspace_size": ([_SH, _I, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_full_attn_select": ([_SH, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P], _I),
     "hysparse_topk": ([_SH, _P, _I, _P, _P], _I),
+    "hysparse_topk_rows": ([_SH, _P, _I, _P, _P], _I),
     "hysparse_topk_tokens_workspace_size": ([_SH, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_topk_tokens": ([_SH, _P, _I, _I, _P, _P, _SZ, _P], _I),
     "hysparse_sparse_attn_workspace_size": ([_SH, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_sparse_attn": ([_SH, _I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
+    "hysparse_sparse_attn_rows": ([_SH, _I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
     "hysparse_sparse_attn_tokens_workspace_size": ([_SH, _I, _I, ctypes.POINTER(_SZ)], _I),
     "hysparse_sparse_attn_tokens": ([_SH, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "hysparse_full_attn_select_decode_workspace_size": ([_DSH, _I, ctypes.POINTER(_SZ)], _I),
@@ -144,6 +147,10 @@ def hysparse_topk(shape, scores, k, idx, stream) -> int:
     return load().hysparse_topk(ctypes.byref(shape), scores, k, idx, stream)
 
 
+def hysparse_topk_rows(shape, scores, k, idx, stream) -> int:
+    return load().hysparse_topk_rows(ctypes.byref(shape), scores, k, idx, stream)
+
+
 def hysparse_topk_tokens_workspace_size(shape: hys_shape, k_tokens: int) -> int:
     n = _SZ(0)
     _check(load().hysparse_topk_tokens_workspace_size(ctypes.byref(shape), k_tokens, ctypes.byref(n)),
@@ -166,6 +173,12 @@ def hysparse_sparse_attn(shape, dtype, q, k, v, idx, kb, ks, vs, window, gate, s
                          stream) -> int:
     return load().hysparse_sparse_attn(ctypes.byref(shape), dtype, q, k, v, idx, kb, ks, vs, window, gate, sinks,
                                        o, ws, ws_bytes, stream)
+
+
+def hysparse_sparse_attn_rows(shape, dtype, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, ws_bytes,
+                              stream) -> int:
+    return load().hysparse_sparse_attn_rows(ctypes.byref(shape), dtype, q, k, v, idx, kb, ks, vs, window, gate,
+                                            sinks, o, ws, ws_bytes, stream)
 
 
 def hysparse_sparse_attn_tokens_workspace_size(shape: hys_shape, dtype: int, forced: int) -> int:
@@ -308,16 +321,20 @@ def workspace_for(nbytes: int, device):
 
 def full_attn_select(q, k, v, *, gran: str = "block", reduce: str = "sum", o=None, scores=None, lse=None,
                      workspace=None, stream=None) -> Tuple[object, object]:
-    """Full causal GQA attention plus block (or token) importance scores. Returns (o, scores)."""
+    """Full causal GQA attention plus importance scores. Returns (o, scores).
+
+    gran "block": [B,Hkv,T,NB] per 64-query tile; "token": [B,Hkv,T,N]; "block_row":
+    [B,Hkv,N,NB] per query position (group maximum, reduce must be "max")."""
     torch = _torch()
     sh = prefill_shape(q, k)
-    g = HYS_GRAN_TOKEN if gran == "token" else HYS_GRAN_BLOCK
+    g = {"token": HYS_GRAN_TOKEN, "block_row": HYS_GRAN_BLOCK_ROW}.get(gran, HYS_GRAN_BLOCK)
     T = (sh.N + 63) // 64
     if o is None:
         o = torch.empty_like(q)
     if scores is None:
+        rows = sh.N if g == HYS_GRAN_BLOCK_ROW else T
         cols = sh.N if g == HYS_GRAN_TOKEN else T
-        scores = torch.empty((sh.B, sh.Hkv, T, cols), dtype=torch.float32, device=q.device)
+        scores = torch.empty((sh.B, sh.Hkv, rows, cols), dtype=torch.float32, device=q.device)
     nws = hysparse_full_attn_select_workspace_size(sh, _dt(q), g)
     if workspace is None and nws > 0:
         workspace = workspace_for(nws, q.device)
@@ -361,6 +378,32 @@ def sparse_attn(q_sparse, k, v, idx, k_swa, v_swa, window: int, gate_logits, *, 
     _check(hysparse_sparse_attn(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k), _ptr(v), _ptr(idx), idx.shape[-1],
                                 _ptr(k_swa), _ptr(v_swa), window, _ptr(gate_logits), _ptr(sinks), _ptr(o),
                                 _ptr(workspace), workspace.numel(), _stream(stream)), "hysparse_sparse_attn")
+    return o
+
+
+def topk_rows(scores, k: int, *, idx=None, stream=None):
+    """Per-position top-k of [B,Hkv,N,NB] scores -> idx [B,Hkv,N,k]."""
+    torch = _torch()
+    B, Hkv, N, NB = scores.shape
+    sh = hys_shape(B, N, Hkv, Hkv, 64, 64)
+    if idx is None:
+        idx = torch.empty((B, Hkv, N, k), dtype=torch.int32, device=scores.device)
+    _check(hysparse_topk_rows(sh, _ptr(scores), k, _ptr(idx), _stream(stream)), "hysparse_topk_rows")
+    return idx
+
+
+def sparse_attn_rows(q_sparse, k, v, idx, k_swa, v_swa, window: int, gate_logits, *, sinks=None, o=None,
+                     workspace=None, stream=None):
+    """The sparse layer with per-position selection (idx [B,Hkv,N,k])."""
+    torch = _torch()
+    sh = prefill_shape(q_sparse, k)
+    if o is None:
+        o = torch.empty_like(q_sparse)
+    if workspace is None:
+        workspace = workspace_for(hysparse_sparse_attn_workspace_size(sh, _dt(q_sparse)), q_sparse.device)
+    _check(hysparse_sparse_attn_rows(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k), _ptr(v), _ptr(idx), idx.shape[-1],
+                                     _ptr(k_swa), _ptr(v_swa), window, _ptr(gate_logits), _ptr(sinks), _ptr(o),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)), "hysparse_sparse_attn_rows")
     return o
 
 

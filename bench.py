@@ -39,9 +39,9 @@ from attention_tcgen05_tma_b200.distributed import max_over_ranks  # noqa: E402
 # (Q', O, gate, K'/V', the gathered blocks) grows with the units, so the bench scales the bytes
 # to its own units; it reports null once the sources differ from the captured ones.
 NCU_TRAFFIC = {
-    "sparse_attn": {"bytes": 199350272 + 103375360, "units": 1024,
+    "sparse_attn": {"bytes": 199693824 + 101788160, "units": 1024,
                     "sources": ("sparse_attn_tc.cu", "tc_ptx.cuh", "common.cuh"),
-                    "sha256": "ffeba27b9054c45f70d67cd2a2b4d93a75f69d6b511b3d5c1dde0594ada4bd0e"},
+                    "sha256": "a65e9526106b3c1952049c84e2b7fb2ccc3e04179ab09c30b8b4d23a1daf9fd9"},
 }
 
 
@@ -347,6 +347,7 @@ def run_ours(args, torch, dist, rank, world, dev):
     kernels["sparse_attn_sinks_ms"] = round(ms_sinks, 4)
     kernels["sparse_attn_same_layer_no_sinks_ms"] = round(ms_plain, 4)   # same repeated-call timing
     kernels["sparse_attn_sinks_tflops"] = round(sp_flops / (ms_sinks / 1e3) / 1e12, 2)
+    rows = None if args.no_rows else run_rows(torch, H, w, x, step, peak_tf)
 
     res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -356,6 +357,8 @@ def run_ours(args, torch, dist, rank, world, dev):
                       "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas x{world}",
                       "l2": "inputs larger than L2 (Q 512 MiB per layer)"},
            "kernels": kernels, "roofline": roof, "clocks": clk, "gpu_launches": launches}
+    if rows is not None:
+        res["rows"] = rows
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, torch, dist, world, w, x, step, dev)
     del x, step
@@ -369,6 +372,41 @@ def run_ours(args, torch, dist, rank, world, dev):
         res["token"] = run_token(args, torch, dist, rank, world, dev, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    return res
+
+
+def run_rows(torch, H, w, x, step, peak_tf):
+    """Per-position selection ([HS] 3.4.2 per query position, group max) on the same inputs, one
+    sparse layer, each call timed on its own: full layer with [B,Hkv,N,NB] scores, per-row top-k,
+    and the sparse layer over each tile's union of its rows' blocks (every row masked to its own)."""
+    o = torch.empty_like(x["q"])
+    sc = torch.empty((w.B, w.Hkv, w.N, w.NB), dtype=torch.float32, device=x["q"].device)
+    idx = torch.empty((w.B, w.Hkv, w.N, w.topk), dtype=torch.int32, device=x["q"].device)
+    full = lambda: H.full_attn_select(x["q"], x["k"], x["v"], gran="block_row", reduce="max", o=o, scores=sc,
+                                      workspace=step.ws)
+    topk = lambda: H.topk_rows(sc, w.topk, idx=idx)
+    sparse = lambda: H.sparse_attn_rows(x["q_sparse"][0], x["k"], x["v"], idx, x["k_swa"][0], x["v_swa"][0],
+                                        w.window, x["gate"][0], o=step.o_sp, workspace=step.ws_sp)
+    ms_full = time_call(torch, full, n=3, warm=1)
+    ms_topk = time_call(torch, topk, n=3, warm=1)
+    ms_sparse = time_call(torch, sparse, n=3, warm=1)
+    # attended keys per row (selected blocks up to t, then the window) and the tiles' union sizes
+    t = torch.arange(w.N, device=idx.device)
+    jt = (t // 64).view(1, 1, w.N, 1)
+    valid = (idx >= 0) & (idx <= jt)
+    keys = torch.where(idx < jt, 64, (t % 64 + 1).view(1, 1, w.N, 1)) * valid
+    attended = keys.sum(dim=3).double() + torch.clamp(t + 1, max=w.window).double().view(1, 1, w.N)
+    alg_flops = 4.0 * w.D * (w.Hq // w.Hkv) * attended.sum().item()
+    tiles = idx.view(w.B, w.Hkv, w.T, 64 * w.topk).sort(dim=3).values
+    distinct = ((tiles[..., 1:] != tiles[..., :-1]) & (tiles[..., 1:] >= 0)).sum(dim=3) + (tiles[..., 0] >= 0).long()
+    union = distinct.double().mean().item()
+    res = {"config": f"{w.name}, one sparse layer, top-{w.topk} blocks per query position (group max)",
+           "full_ms": round(ms_full, 4), "topk_ms": round(ms_topk, 4), "sparse_ms": round(ms_sparse, 4),
+           "sparse_alg_tflops": round(alg_flops / (ms_sparse / 1e3) / 1e12, 2),
+           "sparse_alg_frac": round(alg_flops / (ms_sparse / 1e3) / 1e12 / peak_tf, 4),
+           "mean_union_blocks_per_tile": round(union, 1)}
+    del o, sc, idx
+    torch.cuda.empty_cache()
     return res
 
 
@@ -797,6 +835,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-token", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-position selection leg")
     ap.add_argument("--token-workload", default="token", help="token-variant workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()

@@ -65,7 +65,7 @@ typedef enum {
 typedef enum { HYS_F32 = 0, HYS_BF16 = 1 } hys_dtype;
 
 /* Granularity of the importance scores the full layer emits. */
-typedef enum { HYS_GRAN_BLOCK = 0, HYS_GRAN_TOKEN = 1 } hys_gran;
+typedef enum { HYS_GRAN_BLOCK = 0, HYS_GRAN_TOKEN = 1, HYS_GRAN_BLOCK_ROW = 2 } hys_gran;
 
 /* Aggregation R over the query heads of a KV group and the rows of a 64-query tile.
  * SUM is the default; MAX is the paper's conservative group-wise maximum. */
@@ -113,6 +113,12 @@ HYS_API hys_status hysparse_get_device_status(hys_stream_t stream, int reset, in
  * gran = HYS_GRAN_TOKEN: scores [B,Hkv,T,N] with
  *   scores[b,g,I,i] = sum_{h in g} sum_{t in tile I, t >= i} P^h_{t,i}   ([HS2], token
  *   selection; red must be HYS_REDUCE_SUM).
+ * gran = HYS_GRAN_BLOCK_ROW: scores [B,Hkv,N,NB] per query position with
+ *   scores[b,g,t,j] = max_{h in g} S^h_{t,j}   for j <= floor(t/64), 0 beyond
+ *   ([HS] 3.4.1 group-wise maximum per (query position, key block) entry; 3.4.2 selection
+ *   per query position).  red must be HYS_REDUCE_MAX; bf16 with D in {64, 128}, an even
+ *   group size and NB <= 2048 (N <= 131072) only (HYS_ERR_UNSUPPORTED otherwise).  The
+ *   workspace is the HYS_GRAN_BLOCK one.
  * lse_opt: NULL or [B,Hq,N] fp32, receives LSE_t = log sum_i exp(tau q_t.k_i).
  * ------------------------------------------------------------------------------------ */
 HYS_API hys_status hysparse_full_attn_select_workspace_size(const hys_shape* shape, hys_dtype dtype,
@@ -131,6 +137,13 @@ HYS_API hys_status hysparse_full_attn_select(const hys_shape* shape, hys_dtype d
  * ------------------------------------------------------------------------------------ */
 HYS_API hys_status hysparse_topk(const hys_shape* shape, const float* scores, int k, int* idx,
                          hys_stream_t stream);
+
+/* Per-position TopK ([HS] 3.4.2, for each query position t and group): the k largest of
+ * scores[b,g,t,0..floor(t/64)] from HYS_GRAN_BLOCK_ROW, ties to the lower block index,
+ * fewer candidates than k selects all; idx [B,Hkv,N,k] int32, ascending, padded with -1.
+ * 1 <= k <= 1024, NB <= 8192.  No workspace. */
+HYS_API hys_status hysparse_topk_rows(const hys_shape* shape, const float* scores, int k, int* idx,
+                              hys_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * TopK token selection with a forced recent window ([HS2]).  Candidates of tile I are
@@ -166,6 +179,17 @@ HYS_API hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype,
                                 int k, const void* k_swa, const void* v_swa, int window,
                                 const float* gate_logits, const float* sinks, void* o,
                                 void* workspace, size_t workspace_bytes, hys_stream_t stream);
+
+/* The sparse layer with per-position selection ([HS] 3.4.2 'computed per query position'):
+ * as hysparse_sparse_attn, but idx is [B,Hkv,N,k] and row t's sparse branch attends
+ * {i <= t : floor(i/64) in idx[b,g,t,:]} (entries past floor(t/64) and -1 are ignored).
+ * bf16 with D in {64, 128}, an even group size, k <= 256 and N <= 32768 only
+ * (HYS_ERR_UNSUPPORTED otherwise).  workspace: hysparse_sparse_attn_workspace_size() bytes. */
+HYS_API hys_status hysparse_sparse_attn_rows(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                     const void* k_shared, const void* v_shared, const int* idx,
+                                     int k, const void* k_swa, const void* v_swa, int window,
+                                     const float* gate_logits, const float* sinks, void* o,
+                                     void* workspace, size_t workspace_bytes, hys_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Token-sparse layer ([HS2]): row t of tile I attends idx[b,g,I,:] (token positions,

@@ -116,6 +116,32 @@ def test_token_decode_entry_points_validate(lib):
                                                 None) == H.HYS_ERR_WORKSPACE
 
 
+def test_per_position_entry_points_validate(lib):
+    """Per-position selection: group max only, tensor-core shapes only, N <= 32768 for the
+    sparse layer; every check fails before a launch."""
+    sh = H.hys_shape(1, 1000, 8, 2, 128, 64)
+    # HYS_GRAN_BLOCK_ROW needs the max aggregation, bf16 and an even group
+    assert H.hysparse_full_attn_select(sh, H.HYS_BF16, 16, 16, 16, 16, 16, H.HYS_GRAN_BLOCK_ROW, H.HYS_REDUCE_SUM,
+                                       None, 16, 1 << 20, None) == H.HYS_ERR_UNSUPPORTED
+    assert H.hysparse_full_attn_select(sh, H.HYS_F32, 16, 16, 16, 16, 16, H.HYS_GRAN_BLOCK_ROW, H.HYS_REDUCE_MAX,
+                                       None, 16, 1 << 20, None) == H.HYS_ERR_UNSUPPORTED
+    assert H.hysparse_full_attn_select_workspace_size(sh, H.HYS_BF16, H.HYS_GRAN_BLOCK_ROW) == \
+        H.hysparse_full_attn_select_workspace_size(sh, H.HYS_BF16, H.HYS_GRAN_BLOCK)
+    assert H.hysparse_topk_rows(sh, 16, 0, 16, None) == H.HYS_ERR_INVALID_ARG
+    assert H.hysparse_topk_rows(sh, 8, 4, 16, None) == H.HYS_ERR_INVALID_ARG
+    rows = H.hysparse_sparse_attn_rows
+    assert rows(sh, H.HYS_F32, 16, 16, 16, 16, 4, 16, 16, 128, 16, None, 16, 16, 1 << 20, None) \
+        == H.HYS_ERR_UNSUPPORTED
+    long_sh = H.hys_shape(1, 40000, 8, 2, 128, 64)
+    assert rows(long_sh, H.HYS_BF16, 16, 16, 16, 16, 4, 16, 16, 128, 16, None, 16, 16, 1 << 20, None) \
+        == H.HYS_ERR_UNSUPPORTED
+    assert rows(sh, H.HYS_BF16, 16, 16, 16, 16, 300, 16, 16, 128, 16, None, 16, 16, 1 << 20, None) \
+        == H.HYS_ERR_UNSUPPORTED
+    assert rows(sh, H.HYS_BF16, 16, 16, 16, 16, 4, 16, 16, 128, 16, None, 16, 16, 0, None) == H.HYS_ERR_WORKSPACE
+    assert rows(sh, H.HYS_BF16, 16, 16, 16, 16, 4, 16, 16, 128, 16, 8, 16, 16, 1 << 20, None) \
+        == H.HYS_ERR_INVALID_ARG
+
+
 def test_fp8_token_decode_entry_points_validate(lib):
     """FP8-cache token decode: the scales are required (4-byte aligned), D must be 128, and the
     workspace is the bf16 call's; every check fails before a launch."""

@@ -202,6 +202,56 @@ def test_decode(case):
     assert np.max(np.abs(to_np(osp) - ref)) <= TOL[dt]
 
 
+ROW_PREFILL_CASES = [
+    # name, B, N, Hq, Hkv, D, k, window, with sinks
+    ("d128_g4_ragged", 2, 1000, 8, 2, 128, 4, 128, False),
+    ("d64_g8", 1, 333, 8, 1, 64, 3, 100, True),
+    ("d128_g2_k_all", 1, 700, 4, 2, 128, 16, 64, False),     # k covers every block: dense branch
+    ("d128_g8_many_units", 1, 2048, 16, 2, 128, 6, 128, False),
+]
+
+
+@pytest.mark.parametrize("case", ROW_PREFILL_CASES, ids=[c[0] for c in ROW_PREFILL_CASES])
+def test_per_position_selection(case):
+    """Per-position selection ([HS] 3.4.1-3.4.2 as printed): group-max scores [B,Hkv,N,NB], the
+    top k of each row's floor(t/64)+1 blocks, and the sparse layer with each row's own blocks,
+    against the oracle (the sparse rows on the GPU's own indices)."""
+    name, B, N, Hq, Hkv, D, k, window, with_sinks = case
+    w = _workload("bf16", B, N, Hq, Hkv, D, k, window, seed=17)
+    a = I.prefill_arrays(w, layers=1)
+    q, kk, vv = (to_dev(a[x], "bf16") for x in ("q", "k", "v"))
+    o, sc = H.full_attn_select(q, kk, vv, gran="block_row", reduce="max")
+    idx = H.topk_rows(sc, k)
+    qs, ks, vs = (to_dev(a[x][0], "bf16") for x in ("q_sparse", "k_swa", "v_swa"))
+    gate = to_dev(a["gate"][0], "f32")
+    sinks = I.sink_logits(w, 0) if with_sinks else None
+    osp = H.sparse_attn_rows(qs, kk, vv, idx, ks, vs, window, gate,
+                             sinks=torch.from_numpy(sinks).cuda() if with_sinks else None)
+    torch.cuda.synchronize()
+    assert H.hysparse_get_device_status() == 0
+    o_ref, _ = O.full_attention(a["q"], a["k"], a["v"])
+    assert np.max(np.abs(to_np(o) - o_ref)) <= TOL["bf16"]
+    sc_ref = O.block_scores_rows(a["q"], a["k"])
+    sc_gpu = to_np(sc)
+    assert sc_gpu.shape == sc_ref.shape
+    assert score_rel_err(sc_ref, sc_gpu) <= 1e-3
+    NB = sc_ref.shape[3]
+    gidx = idx.cpu().numpy().astype(np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(N):
+                assert np.all(sc_gpu[b, g, t, t // 64 + 1:] == 0)
+                check_selection(sc_ref[b, g, t], sc_gpu[b, g, t], gidx[b, g, t], min(NB, t // 64 + 1), k)
+    ref = O.sparse_attention_rows(a["q_sparse"][0], a["k"], a["v"], gidx, a["k_swa"][0], a["v_swa"][0], window,
+                                  a["gate"][0], sinks=sinks)
+    assert np.max(np.abs(to_np(osp) - ref)) <= TOL["bf16"]
+    if name.endswith("k_all"):   # every row keeps all its blocks: the per-tile layer with all blocks
+        tidx = H.topk(H.full_attn_select(q, kk, vv)[1], k)
+        otile = H.sparse_attn(qs, kk, vv, tidx, ks, vs, window, gate)
+        torch.cuda.synchronize()
+        assert np.max(np.abs(to_np(osp) - to_np(otile))) <= TOL["bf16"]
+
+
 SINK_PREFILL_CASES = [
     # name, dtype, B, N, Hq, Hkv, D, k, window  (tensor-core path for bf16 D in {64,128}, even G)
     ("bf16_d128_g4_tc", "bf16", 1, 700, 8, 2, 128, 4, 128),
