@@ -586,17 +586,6 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const
     }
     o[((size_t)b * p.Hq + g * p.G + hh) * 128 + d] = __float2bfloat16_rn(out);
   }
-  if (p.mode == 0 && p.tok_scores != nullptr) {
-    // token scores: sum over the group's heads of exp(s - m) / l under the merged statistics
-    float* trow = p.tok_scores + ((size_t)b * p.Hkv + g) * p.L;
-    const float* lg = p.logits + ((size_t)b * p.Hq + g * p.G) * p.L;
-    for (int i = threadIdx.x; i < p.L; i += blockDim.x) {
-      float a = 0.0f;
-      if (i < Lb)
-        for (int hh = 0; hh < p.G; ++hh) a += exp2f((lg[(size_t)hh * p.L + i] - sM[0][hh]) * sc) * sInv[0][hh];
-      trow[i] = a;
-    }
-  }
   if (p.mode == 0 && scores != nullptr) {
     const int nb = (Lb + 63) / 64;
     for (int j = threadIdx.x; j < p.NB; j += blockDim.x) {
@@ -608,6 +597,58 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const Params p, const
         }
       }
       scores[((size_t)b * p.Hkv + g) * p.NB + j] = a;
+    }
+  }
+}
+
+// Token scores of the full layer (token-variant decode): sum over the group's heads of
+// exp(s - m) / l under the merged statistics, for the positions [1024 x, 1024 x + 1024) of
+// (b, g).  Many CTAs per sequence so the logit stream (G fp32 per cached token) runs at HBM speed.
+constexpr int kTokScoreSpan = 1024;
+__global__ void __launch_bounds__(256) decode_token_scores_kernel(const Params p) {
+  __shared__ float sM[16], sInv[16];
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int Lb = p.seqlens ? max(1, min(p.seqlens[b], p.L)) : p.L;
+  const float sc = p.k_scale ? p.scale_log2 * p.k_scale[g] : p.scale_log2;
+  if (threadIdx.x < p.G) {
+    const size_t ph = ((size_t)b * p.Hq + g * p.G + threadIdx.x) * p.nsplit;
+    float M = -INFINITY;
+    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.pm[ph + s]);
+    float L = 0.0f;
+    for (int s = 0; s < p.nsplit; ++s)
+      if (p.pm[ph + s] != -INFINITY) L += p.pl[ph + s] * exp2f((p.pm[ph + s] - M) * sc);
+    sM[threadIdx.x] = M * sc;
+    sInv[threadIdx.x] = L > 0.0f ? 1.0f / L : 0.0f;
+  }
+  __syncthreads();
+  float* trow = p.tok_scores + ((size_t)b * p.Hkv + g) * p.L;
+  const float* lg = p.logits + ((size_t)b * p.Hq + g * p.G) * p.L;
+  const int i0 = blockIdx.x * kTokScoreSpan, i1 = min(p.L, i0 + kTokScoreSpan);
+  if ((p.L & 3) == 0) {
+    // four positions per thread: 16-byte loads of each head's logits, one 16-byte store
+    for (int i = i0 + 4 * threadIdx.x; i < i1; i += 4 * blockDim.x) {
+      float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (i < Lb) {
+        for (int hh = 0; hh < p.G; ++hh) {
+          const float4 x = *reinterpret_cast<const float4*>(lg + (size_t)hh * p.L + i);
+          const float m = sM[hh], w = sInv[hh];
+          a.x += exp2f(fmaf(x.x, sc, -m)) * w;
+          a.y += exp2f(fmaf(x.y, sc, -m)) * w;
+          a.z += exp2f(fmaf(x.z, sc, -m)) * w;
+          a.w += exp2f(fmaf(x.w, sc, -m)) * w;
+        }
+        if (i + 1 >= Lb) a.y = 0.0f;
+        if (i + 2 >= Lb) a.z = 0.0f;
+        if (i + 3 >= Lb) a.w = 0.0f;
+      }
+      *reinterpret_cast<float4*>(trow + i) = a;
+    }
+  } else {
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+      float a = 0.0f;
+      if (i < Lb)
+        for (int hh = 0; hh < p.G; ++hh) a += exp2f(fmaf(lg[(size_t)hh * p.L + i], sc, -sM[hh])) * sInv[hh];
+      trow[i] = a;
     }
   }
 }
@@ -799,6 +840,9 @@ cudaError_t full_tokens(const DecodeDims& d, const void* q, const void* kc, cons
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_token_scores_kernel<<<dim3((d.L + kTokScoreSpan - 1) / kTokScoreSpan, d.Hkv, d.B), 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

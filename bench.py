@@ -97,7 +97,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -107,6 +107,14 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+
+    def wait_ready(self, timeout_s: float = 3.0):
+        """Block until the sampler has printed its first line, so that it runs for the whole
+        timed region; the samples taken before the region are dropped."""
+        t_end = time.time() + timeout_s
+        while self.proc is not None and not self.lines and time.time() < t_end:
+            time.sleep(0.01)
+        self.lines.clear()
 
     def stop(self):
         if self.proc is None:
@@ -295,6 +303,7 @@ def run_ours(args, torch, dist, rank, world, dev):
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
+    clocks.wait_ready()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)

@@ -312,6 +312,7 @@ TOKEN_DECODE_CASES = [
     ("g8_ragged", 3, 1500, 16, 2, 100, 64, True),
     ("g16_long", 2, 5000, 16, 1, 700, 128, False),
     ("g8_keep_all", 2, 600, 16, 2, 4096, 64, True),    # every candidate kept: dense decode
+    ("g8_odd_L", 2, 1001, 16, 2, 90, 64, True),        # cache length not a multiple of 4
 ]
 
 
