@@ -9,7 +9,9 @@
 // One CTA per candidate row.  Radix select finds the k-th largest key in four 8-bit passes
 // (per-warp histograms in shared memory, then a suffix scan over the 256 bins); one
 // index-ordered sweep then takes every key above it plus the lowest-index ties, and a
-// block-wide scan places them in ascending order.
+// block-wide scan places them in ascending order.  Each thread loads eight keys before it
+// touches the histogram (their latencies overlap), and the sweep gives each thread eight
+// consecutive keys per step, so a step costs two block scans for 8 * NT keys.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -66,9 +68,16 @@ __device__ void radix_topk(KeyFn key, int n, int k, int* out, RadixSmem<NT / 32>
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < NW * 256; i += NT) (&sm.hist[0][0])[i] = 0;
     __syncthreads();
-    for (int c = tid; c < n; c += NT) {
-      const uint32_t kc = key(c);
-      if ((kc & pmask) == prefix) atomicAdd(&sm.hist[warp][(kc >> shift) & 255u], 1);
+    for (int c0 = tid; c0 < n; c0 += 8 * NT) {
+      uint32_t kv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + u * NT;
+        kv[u] = c < n ? key(c) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (c0 + u * NT < n && (kv[u] & pmask) == prefix) atomicAdd(&sm.hist[warp][(kv[u] >> shift) & 255u], 1);
     }
     __syncthreads();
     // bin counts in descending bin order: thread t < 256 owns bin 255 - t
@@ -93,17 +102,33 @@ __device__ void radix_topk(KeyFn key, int n, int k, int* out, RadixSmem<NT / 32>
   // prefix is the k-th largest key: take the greater keys and the `need` lowest-index ties
   const uint32_t kth = prefix;
   int ties_before = 0, written = 0;
-  for (int base = 0; base < n; base += NT) {
-    const int c = base + tid;
-    const uint32_t kc = c < n ? key(c) : 0u;
-    const int is_tie = (c < n && kc == kth) ? 1 : 0;
+  for (int base = 0; base < n; base += 8 * NT) {
+    const int c0 = base + 8 * tid;   // this thread's eight consecutive candidates
+    uint32_t kv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) kv[u] = c0 + u < n ? key(c0 + u) : 0u;
+    int nt = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) nt += (c0 + u < n && kv[u] == kth) ? 1 : 0;
     int tie_total;
-    const int tie_rank = ties_before + block_exclusive_scan<NT>(is_tie, &tie_total, sm.sbuf);
+    int tie_rank = ties_before + block_exclusive_scan<NT>(nt, &tie_total, sm.sbuf);
     ties_before += tie_total;
-    const int sel = (c < n) && (kc > kth || (is_tie && tie_rank < need));
+    uint32_t selm = 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (c0 + u >= n) continue;
+      if (kv[u] > kth) {
+        selm |= 1u << u;
+      } else if (kv[u] == kth) {
+        if (tie_rank < need) selm |= 1u << u;
+        ++tie_rank;
+      }
+    }
     int sel_total;
-    const int pos = written + block_exclusive_scan<NT>(sel, &sel_total, sm.sbuf);
-    if (sel) out[pos] = c;
+    int pos = written + block_exclusive_scan<NT>(__popc(selm), &sel_total, sm.sbuf);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if ((selm >> u) & 1u) out[pos++] = c0 + u;
     written += sel_total;
   }
 }
