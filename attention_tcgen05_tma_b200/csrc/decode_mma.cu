@@ -9,9 +9,9 @@
 // tensor, 32 KB per block) into C stages; consumer warp w owns stage w and takes blocks
 // w, w+C, ... of the split, so every stage's barrier phases are consumed by one warp in
 // order (a parity wait cannot be fooled by a phase two ahead) and the max logit of a
-// block (HySparse's m~) is a warp-local reduction.  A sparse layer's split holds 16 of the
+// block (HySparse's m~) is a warp-local reduction.  A sparse layer's split holds 32 of the
 // selected blocks; its SWA ring is a split of its own.  A token-sparse layer's split holds up
-// to 1024 selected tokens, copied row by row with cp.async into the same stage layout, and the
+// to 2048 selected tokens, copied row by row with cp.async into the same stage layout, and the
 // forced newest tokens are a split of contiguous boxes.
 // The G <= 16 query heads of the group form the 16 rows of mma.sync.m16n8k16 tiles
 // (zero-padded): S = Q K^T (64 mma per block), online softmax in registers, O += P V (64
@@ -52,16 +52,16 @@ struct Stg {
 };
 constexpr int kMaxList = 72;                     // blocks per split (incl. padding)
 #ifndef HYS_DECODE_TOK_SPLIT
-#define HYS_DECODE_TOK_SPLIT 1024
+#define HYS_DECODE_TOK_SPLIT 2048
 #endif
 constexpr int kTokSplit = HYS_DECODE_TOK_SPLIT;  // selected tokens per token-sparse split (stages of 64)
-static_assert(kTokSplit % 32 == 0 && kTokSplit <= 1024, "a split's list is read in one pass of 32-entry chunks");
+static_assert(kTokSplit % 32 == 0 && kTokSplit <= 4096 && kTokSplit / 64 <= 72, "a split's list fits the entry list");
 constexpr int kPartBytes = kConsumers * 16 * (128 + 2) * 4;
 static_assert(kPartBytes <= kStages * kStageBytes, "partials reuse the stage buffers");
 constexpr int kSmemBytes = kStages * kStageBytes + kMaxList * 16 + 256 + kTokSplit * 4 + 1024;
 constexpr int kTargetCtas = 4 * 148;
 #ifndef HYS_DECODE_SPARSE_BPS
-#define HYS_DECODE_SPARSE_BPS 16
+#define HYS_DECODE_SPARSE_BPS 32
 #endif
 constexpr int kSparseBps = HYS_DECODE_SPARSE_BPS;   // selected blocks per sparse-layer split (<= 32)
 static_assert(kSparseBps <= 32 && kSparseBps <= kMaxList, "one warp gathers a split's entries");
@@ -198,19 +198,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int lim = Lb - p.forced;
     const int* sel = p.idx + ((size_t)b * p.Hkv + g) * p.kb;
     const int e_lo = sp * kTokSplit, e_hi = min(p.kb, e_lo + kTokSplit);
-    int jv[kTokSplit / 32];
-#pragma unroll
-    for (int c = 0; c < kTokSplit / 32; ++c) {
-      const int e = e_lo + 32 * c + lane;
-      jv[c] = e < e_hi ? sel[e] : -1;
-    }
+    constexpr int kPass = kTokSplit < 1024 ? kTokSplit : 1024;   // entries loaded per pass (32 per lane)
     int cnt = 0;
+    for (int e_pass = e_lo; e_pass < e_hi; e_pass += kPass) {
+      int jv[kPass / 32];
 #pragma unroll
-    for (int c = 0; c < kTokSplit / 32; ++c) {
-      const bool keep = jv[c] >= 0 && jv[c] < lim;
-      const unsigned m = __ballot_sync(0xffffffffu, keep);
-      if (keep) tok[cnt + __popc(m & ((1u << lane) - 1u))] = jv[c];
-      cnt += __popc(m);
+      for (int c = 0; c < kPass / 32; ++c) {
+        const int e = e_pass + 32 * c + lane;
+        jv[c] = e < e_hi ? sel[e] : -1;
+      }
+#pragma unroll
+      for (int c = 0; c < kPass / 32; ++c) {
+        const bool keep = jv[c] >= 0 && jv[c] < lim;
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (keep) tok[cnt + __popc(m & ((1u << lane) - 1u))] = jv[c];
+        cnt += __popc(m);
+      }
     }
     if (lane == 0) {
       int n = 0;
