@@ -9,9 +9,10 @@
 // One CTA per candidate row.  Radix select finds the k-th largest key in four 8-bit passes
 // (per-warp histograms in shared memory, then a suffix scan over the 256 bins); one
 // index-ordered sweep then takes every key above it plus the lowest-index ties, and a
-// block-wide scan places them in ascending order.  Each thread loads eight keys before it
-// touches the histogram (their latencies overlap), and the sweep gives each thread eight
-// consecutive keys per step, so a step costs two block scans for 8 * NT keys.
+// block-wide scan places them in ascending order.  On long rows (token candidates) each thread
+// loads eight keys before it touches the histogram (their latencies overlap), and the sweep
+// gives each thread eight consecutive keys per step, so a step costs two block scans for
+// 8 * NT keys; short rows keep one key per thread and step.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -68,7 +69,12 @@ __device__ void radix_topk(KeyFn key, int n, int k, int* out, RadixSmem<NT / 32>
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < NW * 256; i += NT) (&sm.hist[0][0])[i] = 0;
     __syncthreads();
-    for (int c0 = tid; c0 < n; c0 += 8 * NT) {
+    if (NT < 1024 || n <= 2 * NT) {   // short rows (block candidates): one key per thread and step
+      for (int c = tid; c < n; c += NT) {
+        const uint32_t kc = key(c);
+        if ((kc & pmask) == prefix) atomicAdd(&sm.hist[warp][(kc >> shift) & 255u], 1);
+      }
+    } else for (int c0 = tid; c0 < n; c0 += 8 * NT) {
       uint32_t kv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -102,6 +108,22 @@ __device__ void radix_topk(KeyFn key, int n, int k, int* out, RadixSmem<NT / 32>
   // prefix is the k-th largest key: take the greater keys and the `need` lowest-index ties
   const uint32_t kth = prefix;
   int ties_before = 0, written = 0;
+  if (NT < 1024 || n <= 2 * NT) {
+    for (int base = 0; base < n; base += NT) {
+      const int c = base + tid;
+      const uint32_t kc = c < n ? key(c) : 0u;
+      const int is_tie = (c < n && kc == kth) ? 1 : 0;
+      int tie_total;
+      const int tie_rank = ties_before + block_exclusive_scan<NT>(is_tie, &tie_total, sm.sbuf);
+      ties_before += tie_total;
+      const int sel = (c < n) && (kc > kth || (is_tie && tie_rank < need));
+      int sel_total;
+      const int pos = written + block_exclusive_scan<NT>(sel, &sel_total, sm.sbuf);
+      if (sel) out[pos] = c;
+      written += sel_total;
+    }
+    return;
+  }
   for (int base = 0; base < n; base += 8 * NT) {
     const int c0 = base + 8 * tid;   // this thread's eight consecutive candidates
     uint32_t kv[8];
