@@ -191,3 +191,49 @@ def test_hybrid_block_backward_sums_the_shared_cache_gradients():
     loss.backward()
     np.testing.assert_allclose(got["dk"], tk.grad.numpy(), rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(got["dv"], tv.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_backward_pins_catch_planted_mistakes(monkeypatch):
+    """Plant plausible mistakes in the gradient oracle (a dropped D_t term, a missing scale, the
+    gate derivative without the 1 - sigmoid factor) and check that a pin above fails."""
+    import pytest
+    orig = BW.attention_rows_backward
+
+    def no_d_term(q_rows, t_rows, k, v, d_o, keys_visible=None, sink=None):
+        q_rows, k, v, d_o = (np.asarray(x, np.float64) for x in (q_rows, k, v, d_o))
+        tau = 1.0 / math.sqrt(q_rows.shape[1])
+        p, _, _ = O.causal_softmax(q_rows, t_rows, k, keys_visible, sink)
+        ds = p * (d_o @ v.T)                    # D_t dropped
+        return tau * (ds @ k), tau * (ds.T @ q_rows), p.T @ d_o, 0.0
+
+    monkeypatch.setattr(BW, "attention_rows_backward", no_d_term)
+    with pytest.raises(AssertionError):
+        test_rows_backward_matches_autograd()
+    with pytest.raises(AssertionError):
+        test_full_backward_matches_sdpa_autograd()
+
+    def no_scale(*a, **kw):
+        dq, dk, dv, ds = orig(*a, **kw)
+        return dq * math.sqrt(np.asarray(a[0]).shape[1]), dk, dv, ds
+
+    monkeypatch.setattr(BW, "attention_rows_backward", no_scale)
+    with pytest.raises(AssertionError):
+        test_rows_backward_matches_autograd()
+    monkeypatch.undo()
+
+    # the gate derivative without the (1 - sigmoid) factor differs from autograd's
+    rng = np.random.default_rng(46)
+    B, Hq, Hkv, N, D, win = 1, 2, 1, 70, 8, 12
+    q_s, do = rng.standard_normal((B, Hq, N, D)), rng.standard_normal((B, Hq, N, D))
+    k, v, ks, vs = (rng.standard_normal((B, Hkv, N, D)) for _ in range(4))
+    gate = rng.standard_normal((B, Hq, N, 2))
+    idx = np.array([[[[0], [1]]]])
+    good = BW.sparse_attention_backward(q_s, k, v, idx, ks, vs, win, gate, do)
+    bad = good["dgate"] / (1.0 - BW.sigmoid(gate))
+    tg = _t(gate)
+    sel_sets = {(0, 0, 0): [0], (0, 0, 1): [1]}
+    o = _torch_sparse_layer(_t(q_s, False), _t(k, False), _t(v, False), sel_sets, _t(ks, False), _t(vs, False), win,
+                            tg, None, [(0, O.tile_rows(0, N)), (1, O.tile_rows(1, N))])
+    (o * torch.from_numpy(do)).sum().backward()
+    np.testing.assert_allclose(good["dgate"], tg.grad.numpy(), rtol=1e-9, atol=1e-11)
+    assert not np.allclose(bad, tg.grad.numpy(), rtol=1e-6, atol=1e-9)
