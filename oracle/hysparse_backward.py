@@ -126,6 +126,31 @@ def sparse_attention_backward(q_s, k, v, idx, k_swa, v_swa, window: int, gate, d
     return out
 
 
+def token_sparse_backward(q_s, k, v, idx, forced: int, d_o, block: int = 64) -> Dict[str, np.ndarray]:
+    """Gradients of one token-sparse layer ([HS2] "Precise retrieval without a separate indexer":
+    row t of tile I attends Sel_I united with [max(0, t-forced+1), t] over the shared K, V, no
+    gate).  idx [B,Hkv,T,k_tokens]; returns dq, dk, dv."""
+    B, Hq, N, D = q_s.shape
+    G = Hq // k.shape[1]
+    T = (N + block - 1) // block
+    out = {"dq": np.zeros((B, Hq, N, D)), "dk": np.zeros(k.shape), "dv": np.zeros(v.shape)}
+    kpos = np.arange(N)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for I in range(T):
+                rows = tile_rows(I, N, block)
+                in_sel = np.zeros(N, dtype=bool)
+                sel = np.asarray([i for i in idx[b, g, I] if i >= 0], dtype=np.int64)
+                in_sel[sel] = True
+                vis = in_sel[None, :] | (kpos[None, :] >= rows[:, None] - forced + 1)
+                dq, dk, dv, _ = attention_rows_backward(q_s[b, h, rows], rows, k[b, g], v[b, g], d_o[b, h, rows], vis)
+                out["dq"][b, h, rows] = dq
+                out["dk"][b, g] += dk
+                out["dv"][b, g] += dv
+    return out
+
+
 def hybrid_block_backward(q, k, v, d_o_full, sparse_layers: Sequence[dict], window: int, block: int = 64):
     """The hybrid block's gradients: the full layer plus the sparse layers, whose gradients of the
     shared K, V are added to the full layer's.  Each sparse layer is a dict with q_s, idx, k_swa,

@@ -193,6 +193,40 @@ def test_hybrid_block_backward_sums_the_shared_cache_gradients():
     np.testing.assert_allclose(got["dv"], tv.grad.numpy(), rtol=1e-9, atol=1e-11)
 
 
+def test_token_sparse_backward_matches_autograd():
+    """Token-sparse layer: the selected tokens united with the forced newest window, each once."""
+    rng = np.random.default_rng(47)
+    B, Hq, Hkv, N, D, W, kt = 1, 4, 2, 150, 8, 16, 10
+    T = (N + 63) // 64
+    q_s, do = rng.standard_normal((B, Hq, N, D)), rng.standard_normal((B, Hq, N, D))
+    k, v = rng.standard_normal((B, Hkv, N, D)), rng.standard_normal((B, Hkv, N, D))
+    idx = np.full((B, Hkv, T, kt), -1)
+    for g in range(Hkv):
+        for I_ in range(T):
+            n = max(0, min(N, 64 * I_ + 64) - W)
+            c = np.sort(rng.permutation(n)[:kt])
+            idx[0, g, I_, :len(c)] = c
+    got = BW.token_sparse_backward(q_s, k, v, idx, W, do)
+    tq, tk, tv = _t(q_s), _t(k), _t(v)
+    kpos = torch.arange(N)
+    outs = []
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        o_h = torch.zeros(N, D, dtype=torch.float64)
+        for I_ in range(T):
+            rows = torch.from_numpy(O.tile_rows(I_, N))
+            in_sel = torch.zeros(N, dtype=torch.bool)
+            for i in idx[0, g, I_]:
+                if i >= 0:
+                    in_sel[i] = True
+            vis = (kpos[None, :] <= rows[:, None]) & (in_sel[None, :] | (kpos[None, :] >= rows[:, None] - W + 1))
+            o_h = o_h.index_put((rows,), _torch_attention(tq[0, h, rows], tk[0, g], tv[0, g], vis))
+        outs.append(o_h)
+    (torch.stack(outs)[None] * torch.from_numpy(do)).sum().backward()
+    for name, ten in (("dq", tq), ("dk", tk), ("dv", tv)):
+        np.testing.assert_allclose(got[name], ten.grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=name)
+
+
 def test_backward_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the gradient oracle (a dropped D_t term, a missing scale, the
     gate derivative without the 1 - sigmoid factor) and check that a pin above fails."""
