@@ -816,8 +816,12 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   return cudaGetLastError();
 }
 
+// the logits follow the split partials at a 256-byte boundary (the token-score kernel reads
+// them with 16-byte loads)
+static size_t logits_offset(const DecodeDims& d) { return (decode_mma_full_workspace(d) + 255) & ~size_t(255); }
+
 size_t decode_mma_full_tokens_workspace(const DecodeDims& d) {
-  return decode_mma_full_workspace(d) + sizeof(float) * (size_t)d.B * d.Hq * d.L;
+  return logits_offset(d) + sizeof(float) * (size_t)d.B * d.Hq * d.L;
 }
 
 namespace {
@@ -837,7 +841,7 @@ cudaError_t full_tokens(const DecodeDims& d, const void* q, const void* kc, cons
   p.bps = bps;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
-  p.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + decode_mma_full_workspace(d));
+  p.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + logits_offset(d));
   p.tok_scores = tok_scores;
   decode_split_kernel<F8><<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
