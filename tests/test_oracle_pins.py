@@ -97,6 +97,36 @@ class TestWorkedExample:
             o = O.token_sparse_rows(self.q[0, 0][rows], rows, self.k[0, 0], self.v[0, 0], sel, 1)[:, 0]
             np.testing.assert_allclose(o, self.g["token_sparse"][rows], atol=1e-13)
 
+    def test_per_position(self):
+        sc = O.block_scores_rows(self.q, self.k, block=2)
+        for t in range(4):
+            np.testing.assert_allclose(sc[0, 0, t], self.g[f"smax_t{t}"], atol=1e-13)
+        idx = O.topk_blocks_rows(sc, 1, block=2)
+        assert idx[0, 0, :, 0].tolist() == self.g["rows_top1"].tolist()
+        rows = np.arange(4)
+        o_sp = np.concatenate([O.sparse_branch_rows(self.q[0, 0][[t]], np.array([t]), self.k[0, 0], self.v[0, 0],
+                                                    idx[0, 0, t], 2) for t in rows])[:, 0]
+        np.testing.assert_allclose(o_sp, self.g["rows_sparse_branch"], atol=1e-13)
+        gate = np.zeros((1, 1, 4, 2))
+        o = O.sparse_attention_rows(self.q, self.k, self.v, idx, self.k, self.v, 1, gate, block=2)
+        np.testing.assert_allclose(o[0, 0, :, 0], self.g["rows_gated"], atol=1e-13)
+
+    def test_token_decode(self):
+        q = np.ones((1, 1, 1))
+        ts = O.decode_token_scores(q, self.k)
+        np.testing.assert_allclose(ts[0, 0], self.g["decode_token_scores"], atol=1e-13)
+        idx = O.topk_decode_tokens(ts, 1, 1)
+        assert idx[0, 0, 0] == self.g["decode_token_top1"][0]
+        o = O.decode_token_sparse(q, self.k, self.v, idx, 1)
+        np.testing.assert_allclose(o[0, 0], self.g["decode_token_sparse"], atol=1e-13)
+
+    def test_gradients(self):
+        dq, dk, dv = O.backward.full_attention_backward(self.q, self.k, self.v, np.ones((1, 1, 4, 1)))
+        np.testing.assert_allclose(dv[0, 0, :, 0], self.g["grad_dv"], atol=1e-13)
+        np.testing.assert_allclose(dk[0, 0, :, 0], self.g["grad_dk"], atol=1e-13)
+        want = self.g["grad_dq_ln2"] * math.log(2.0) + self.g["grad_dq_ln3"] * math.log(3.0)
+        np.testing.assert_allclose(dq[0, 0, :, 0], want, atol=1e-13)
+
     def test_decode(self):
         q = np.ones((1, 1, 1))
         o, sc = O.decode_full(q, self.k, self.v, block=2)
