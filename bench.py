@@ -9,6 +9,14 @@ each with its own Q', K', V' and gate logits.  ``value`` is prefill tokens/s ove
 whole job.  The decode workload (64 sequences x 131072 cached tokens, 1 full + 11
 sparse layers) is timed in the same run and reported as ``decode`` (us/token).
 
+Further legs, each outside the headline's timed region and reported under its own key:
+``rows`` (per-position selection on the prefill inputs, one layer), ``decode_tokens`` (the
+token-variant decode step over the decode cache, bf16 and FP8 E4M3, us/token), ``token`` (the
+token-variant prefill, N=131072), ``e2e`` (the headline through the C ABI with host buffers
+copied in and out every step) and ``cpu_baseline`` (the float64 oracle on a bounded sample).
+Flags ``--no-rows``, ``--no-decode``, ``--no-decode-tokens``, ``--no-token``, ``--no-e2e`` and
+``--no-cpu`` skip them.
+
 Multi-GPU (torchrun): every rank runs its own independent batch (weak scaling, no
 data-path collective); the time is the max over ranks.
 """
