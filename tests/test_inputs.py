@@ -55,3 +55,28 @@ def test_sampled_tiles_include_last():
         w = I.WORKLOADS[name]
         t = I.sampled_tiles(w, 8)
         assert (0, 0, w.T - 1) in t and len(t) == 8
+
+
+def test_fp8_cache_codes():
+    """The FP8 decode cache: per-KV-head scales in the stated range, no NaN codes, and every code
+    within E4M3's rounding of the seeded value / scale (half a unit in the last place: 2^-4
+    relative for normal codes, 2^-10 absolute below the smallest normal 2^-6)."""
+    import oracle as O
+    w = I.scaled(I.WORKLOADS["decode"], B=2, N=300, layers=1)
+    c = I.decode_fp8_cache(w)
+    base = w.scale_std / 32.0
+    for sc in (c["k_scale"], c["v_scale"]):
+        assert sc.dtype == np.float32 and sc.shape == (w.Hkv,)
+        assert np.all(sc >= 0.75 * base * (1 - 1e-6)) and np.all(sc <= 1.25 * base * (1 + 1e-6))
+    for name, sc in (("k8", c["k_scale"]), ("v8", c["v_scale"])):
+        codes = c[name]
+        assert codes.dtype == np.uint8 and codes.shape == (w.B, w.Hkv, w.N, w.D)
+        assert not np.any((codes & 0x7F) == 0x7F)             # no NaN codes
+        vals = O.e4m3_to_float(codes)
+        for b in range(w.B):
+            for g in range(w.Hkv):
+                x = I.normal_slice(w.seed, I.TID_K if name == "k8" else I.TID_V, b, g, (w.N, w.D), w.scale_std,
+                                   False).astype(np.float64) / np.float64(np.float32(sc[g]))
+                err = np.abs(vals[b, g] - x)
+                bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10)
+                assert np.all(err <= bound * (1 + 1e-6))
