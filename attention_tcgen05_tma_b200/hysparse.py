@@ -515,6 +515,8 @@ def sparse_attn_decode_tokens(q, k_cache, v_cache, idx, forced_window: int, *, s
 
 def _fp8_cache_ok(q, k_cache, v_cache, k_scale, v_scale):
     torch = _torch()
+    if q.dtype != torch.bfloat16:
+        raise TypeError("the FP8-cache decode takes a bf16 query")
     for t in (k_cache, v_cache):
         if t.element_size() != 1:
             raise TypeError("the FP8 cache holds one-byte E4M3 codes (torch.uint8 or torch.float8_e4m3fn)")
