@@ -23,6 +23,8 @@
 #include <cuda_fp16.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -741,12 +743,17 @@ void fill_common(Params& p, const DecodeDims& d, const void* q, const int* seqle
   p.nsp = 0;
 }
 
+// The shared-memory opt-in is a per-device attribute: remember it per device (one bit each).
 template <bool F8>
 cudaError_t set_smem() {
-  static bool done = false;
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e == cudaSuccess) done = true;
+  static std::atomic<unsigned long long> done{0ull};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+  if (bit != 0ull && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(decode_split_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_relaxed);
   return e;
 }
 
