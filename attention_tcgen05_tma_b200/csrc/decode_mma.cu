@@ -18,7 +18,10 @@
 // mma per block).  The warps' partial (m, l, O) are merged in shared memory (reusing the stages) and the
 // split's partial goes to the workspace; a combine kernel merges the splits, writes o and
 // (full layer) the block scores exp(m~ - m)/l aggregated over the group's heads, or
-// (sparse layer) the gated sum of the sparse-branch and SWA-ring branches.
+// (sparse layer) the gated sum of the sparse-branch and SWA-ring branches.  In the token
+// variant the full layer also writes every key's logit and a wide kernel turns them into the
+// token scores.  An FP8 (E4M3) cache runs in its own instance: 16 KB blocks, six stages
+// (warp w owns stages w and w + C), codes converted to f16 inside the MMA fragments.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <math.h>
