@@ -3,22 +3,42 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.h"
 
 namespace hys {
 __device__ int g_device_status = 0;
 
+// Device address of g_device_status on the current device, resolved once per device under a
+// lock (host threads may make their first calls concurrently).
 int* device_status_ptr() {
+  static std::mutex mu;
   static int* cached[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!cached[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
     cached[dev] = static_cast<int*>(p);
   }
   return cached[dev];
+}
+
+EncodeTiledFn tma_encode_fn() {
+  // a function-local static is initialised exactly once, even under concurrent first calls
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    return nullptr;
+  }();
+  return fn;
 }
 }  // namespace hys
 

@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.h"
 #include "tc_ptx.cuh"
 
 namespace hys {
@@ -661,24 +662,8 @@ __global__ void __launch_bounds__(256) decode_token_scores_kernel(const Params p
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 bool make_map(CUtensorMap* m, const void* base, int rows, int heads) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = tma_encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)heads};
   cuuint64_t strides[2] = {256, (cuuint64_t)rows * 256};
@@ -691,7 +676,7 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int heads) {
 
 // FP8 codes: [heads][rows][128] bytes, box 128 bytes x 64 rows x 1 head
 bool make_map8(CUtensorMap* m, const void* base, int rows, int heads) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = tma_encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)heads};
   cuuint64_t strides[2] = {128, (cuuint64_t)rows * 128};

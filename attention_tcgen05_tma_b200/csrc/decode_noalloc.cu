@@ -10,7 +10,10 @@
 //
 // The array has a fixed capacity (kNoAllocScratchBytes).  Every GPU that loads the
 // library holds it until the process exits.  Its device address is resolved once per
-// device, on the first call made with that device current.
+// device, on the first call made with that device current; under the driver's lazy module
+// loading that first call is also when the driver loads this file's module and places the
+// array on the device, so the first call may allocate and synchronise and belongs in the
+// caller's set-up (before any stream capture).  Later calls allocate nothing.
 #include <mutex>
 
 #include "common.cuh"

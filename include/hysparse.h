@@ -231,9 +231,12 @@ HYS_API hys_status hysparse_full_attn_select_decode(const hys_decode_shape* shap
  * loads the library until the process exits.
  *   - Shapes whose scratch (the value hysparse_full_attn_select_decode_workspace_size
  *     returns) exceeds 16 MiB return HYS_ERR_WORKSPACE and launch nothing.
- *   - The call allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
- *   - The first call on a device resolves the array's device address with that device
- *     current; make that first call before any stream capture.
+ *   - The call makes no cudaMalloc/cudaFree and no allocating library call.
+ *   - The first call on a device is the set-up: with that device current it resolves the
+ *     array's device address, and under the CUDA driver's lazy module loading (the default)
+ *     that is also when the driver loads the array onto the device, so this first call may
+ *     allocate the array's 16 MiB and synchronise.  Make it during set-up, before any
+ *     stream capture; later calls on that device allocate nothing.
  *   - All calls share the one array: calls whose work overlaps on the GPU (different
  *     streams, or different host threads on the same device) race and must be ordered
  *     by the caller.  Nothing in the array needs clearing between calls.

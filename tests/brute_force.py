@@ -36,12 +36,22 @@ def attend(q, keys, kmat, vmat):
     return out
 
 
-def block_score(qs_group, kmat, tile, j, n, block, reduce="sum"):
+def _row_probs(q_head, t, kmat, memo, h):
+    """Probabilities of row t over keys 0..t; memo (a dict or None) keeps them per (head, row)."""
+    if memo is not None and (h, t) in memo:
+        return memo[(h, t)]
+    probs = dict(softmax_over(q_head[t], list(range(t + 1)), kmat))
+    if memo is not None:
+        memo[(h, t)] = probs
+    return probs
+
+
+def block_score(qs_group, kmat, tile, j, n, block, reduce="sum", memo=None):
     """R_h R_{t in tile} max_{i in block j, i <= t} P_{t,i}."""
     vals = []
-    for q_head in qs_group:
+    for h, q_head in enumerate(qs_group):
         for t in range(tile * block, min(n, (tile + 1) * block)):
-            probs = dict(softmax_over(q_head[t], list(range(t + 1)), kmat))
+            probs = _row_probs(q_head, t, kmat, memo, h)
             in_block = [probs[i] for i in range(j * block, min(n, (j + 1) * block)) if i <= t]
             vals.append(max(in_block) if in_block else 0.0)
     return sum(vals) if reduce == "sum" else max(vals)
@@ -76,11 +86,11 @@ def gated_row(q, t, k, v, sel, ks, vs, window, gate, block):
     return [g0 * x + g1 * y for x, y in zip(a, b)]
 
 
-def token_score(qs_group, kmat, tile, i, n, block):
+def token_score(qs_group, kmat, tile, i, n, block, memo=None):
     s = 0.0
-    for q_head in qs_group:
+    for h, q_head in enumerate(qs_group):
         for t in range(max(i, tile * block), min(n, (tile + 1) * block)):
-            probs = dict(softmax_over(q_head[t], list(range(t + 1)), kmat))
+            probs = _row_probs(q_head, t, kmat, memo, h)
             s += probs[i]
     return s
 

@@ -43,20 +43,39 @@ def to_np(t) -> np.ndarray:
 
 
 def check_selection(oracle_scores: np.ndarray, gpu_scores: np.ndarray, gpu_idx: np.ndarray, n_cand: int, k: int):
-    """Apply rules 1/2 to one tile. Returns 'rule1' or 'rule2'; raises on violation."""
+    """Apply rules 1/2 to one tile (raises on a violation) and return what decided it:
+
+    * ``rule``: 'rule1' (the oracle's k-th and (k+1)-th scores differ by more than the gap, or
+      there are at most k candidates: the GPU set equals the oracle's) or 'rule2' (near tie: the
+      GPU set equals the oracle's selection routine on the GPU's own scores);
+    * ``decided_in`` / ``decided_out``: candidates whose oracle score clears the k-th/(k+1)-th
+      boundary by more than the gap plus twice the GPU's largest score error on this tile, which
+      no correct selection on the GPU's scores can move: each must be selected / left out, on
+      rule-2 tiles too (a planted block far above the boundary is always decided in)."""
     s = oracle_scores[:n_cand]
     order = np.lexsort((np.arange(n_cand), -s))
     want_oracle = O.select_topk(oracle_scores, n_cand, k)
     if n_cand <= k:
         assert np.array_equal(gpu_idx, want_oracle), (gpu_idx, want_oracle)
-        return "rule1"
+        return {"rule": "rule1", "decided_in": list(range(n_cand)), "decided_out": []}
     sk, sk1 = s[order[k - 1]], s[order[k]]
     if sk > 0 and (sk - sk1) / sk > GAP:
         assert np.array_equal(gpu_idx, want_oracle), (gpu_idx, want_oracle)
-        return "rule1"
-    want_gpu = O.select_topk(gpu_scores.astype(np.float64), n_cand, k)
-    assert np.array_equal(gpu_idx, want_gpu), (gpu_idx, want_gpu)
-    return "rule2"
+        rule = "rule1"
+    else:
+        want_gpu = O.select_topk(gpu_scores.astype(np.float64), n_cand, k)
+        assert np.array_equal(gpu_idx, want_gpu), (gpu_idx, want_gpu)
+        rule = "rule2"
+    g = gpu_scores[:n_cand].astype(np.float64)
+    pos = s > 0
+    err = float(np.max(np.abs(g[pos] - s[pos]) / s[pos])) if pos.any() else 0.0
+    margin = GAP + 3.0 * err
+    chosen = set(int(j) for j in gpu_idx if j >= 0)
+    d_in = [int(j) for j in range(n_cand) if s[j] > sk1 * (1.0 + margin)]
+    d_out = [int(j) for j in range(n_cand) if s[j] < sk * (1.0 - margin)]
+    assert all(j in chosen for j in d_in), ("decided-in block not selected", d_in, sorted(chosen))
+    assert not any(j in chosen for j in d_out), ("decided-out block selected", sorted(chosen))
+    return {"rule": rule, "decided_in": d_in, "decided_out": d_out}
 
 
 def score_rel_err(oracle_scores: np.ndarray, gpu_scores: np.ndarray, floor: float = 1e-6) -> float:

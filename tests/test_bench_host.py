@@ -39,4 +39,18 @@ def test_reference_arm_json_contract():
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert "workload" in d["config"]
+    # the same config object as our arm prints, and a step time that is the sample's own
+    from attention_tcgen05_tma_b200 import inputs as I
+    assert d["config"] == bench.workload_config(I.WORKLOADS["tiny"], 1)
+    assert d["ms_per_step"] > 0 and "extrapolated" in d["ms_per_step_kind"]
+
+
+def test_cpu_baseline_is_unbiased_over_tile_position():
+    """The baseline's estimate is mean time per sampled tile x all tiles, with tiles stratified
+    over the tile index: two samples of different sizes give the same order of magnitude."""
+    from attention_tcgen05_tma_b200 import inputs as I
+    w = I.WORKLOADS["tiny"]
+    a = bench.cpu_baseline(w, budget_s=0.0, n_tiles=4, seed=1)
+    b = bench.cpu_baseline(w, budget_s=60.0, n_tiles=16, seed=2)
+    assert a["tiles"] == 1 and b["tiles"] == 16
+    assert 0.2 < a["value"] / b["value"] < 5.0

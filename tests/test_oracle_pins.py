@@ -377,6 +377,45 @@ def test_brute_force(seed, N, D, G):
                                        atol=1e-12)
 
 
+@pytest.mark.parametrize("seed,N,D,G,Hkv", [(10, 65, 128, 8, 2), (11, 256, 64, 4, 2), (12, 200, 128, 4, 1),
+                                             (13, 129, 64, 8, 1)])
+def test_brute_force_gqa(seed, N, D, G, Hkv):
+    """The head dims and group sizes of the workloads (D 64/128, G 4/8), with two KV groups where
+    the head-to-group mapping matters: block scores under both reductions, the top-k, gated
+    sparse rows and token scores against the scalar transcription, group by group."""
+    rng = np.random.default_rng(200 + seed)
+    Hq = G * Hkv
+    q, k, v = _rand(rng, 1, Hq, N, D), _rand(rng, 1, Hkv, N, D), _rand(rng, 1, Hkv, N, D)
+    ks, vs = _rand(rng, 1, Hkv, N, D), _rand(rng, 1, Hkv, N, D)
+    gate = _rand(rng, 1, Hq, N, 2)
+    T = (N + 63) // 64
+    sc = {red: O.block_scores(q, k, red) for red in ("sum", "max")}
+    kb, window = 2, 40
+    idx = O.topk_blocks(sc["sum"], kb)
+    o = O.sparse_attention(q, k, v, idx, ks, vs, window, gate)
+    for g in range(Hkv):
+        kk, vv, kl, vl = k[0, g].tolist(), v[0, g].tolist(), ks[0, g].tolist(), vs[0, g].tolist()
+        heads = list(range(g * G, (g + 1) * G))
+        qg = [q[0, h].tolist() for h in heads]
+        memo = {}
+        for red in ("sum", "max"):
+            for I in range(T):
+                for j in range(I + 1):
+                    want = BF.block_score(qg, kk, I, j, N, 64, red, memo)
+                    assert abs(sc[red][0, g, I, j] - want) <= 1e-12 * max(1.0, abs(want))
+                assert np.all(sc[red][0, g, I, I + 1:] == 0)
+        for I in range(T):
+            assert idx[0, g, I].tolist() == BF.topk(sc["sum"][0, g, I].tolist(), I + 1, kb)
+            for t in O.tile_rows(I, N)[::13]:
+                for h in (heads[0], heads[-1]):
+                    want = BF.gated_row(q[0, h, t].tolist(), t, kk, vv, idx[0, g, I].tolist(), kl, vl, window,
+                                        gate[0, h, t].tolist(), 64)
+                    np.testing.assert_allclose(o[0, h, t], want, atol=1e-12)
+            ts = O.token_scores_tile(q[0, g * G:(g + 1) * G], k[0, g], I)
+            for i in range(0, N, 11):
+                assert abs(ts[i] - BF.token_score(qg, kk, I, i, N, 64, memo)) <= 1e-12
+
+
 def test_brute_force_decode():
     rng = np.random.default_rng(9)
     L, D, G = 190, 8, 2
