@@ -271,6 +271,98 @@ hys_status hysparse_sparse_attn(const hys_shape* shape, hys_dtype dtype, const v
                                            gate_logits, sinks, o, s));
 }
 
+// ----------------------------------------------------------------------------- training
+hys_status hysparse_sparse_attn_train(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                      const void* k_shared, const void* v_shared, const int* idx, int k,
+                                      const void* k_swa, const void* v_swa, int window, const float* gate_logits,
+                                      const float* sinks, void* o, void* o_sparse, float* branch_lse, void* workspace,
+                                      size_t workspace_bytes, hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (!q_sparse || !k_shared || !v_shared || !idx || !k_swa || !v_swa || !gate_logits || !o || !o_sparse ||
+      !branch_lse)
+    return HYS_ERR_INVALID_ARG;
+  if (k < 1 || k > 1024 || window < 1) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q_sparse) || !aligned16(k_shared) || !aligned16(v_shared) || !aligned16(idx) || !aligned16(k_swa) ||
+      !aligned16(v_swa) || !aligned16(gate_logits) || !aligned16(sinks) || !aligned16(o) || !aligned16(o_sparse) ||
+      !aligned16(branch_lse) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (sparse_attn_tc_supported(d, dtype) && k <= 256) {
+    if (workspace == nullptr || workspace_bytes < align256(sparse_attn_tc_workspace(d))) return HYS_ERR_WORKSPACE;
+    return from_cuda(launch_sparse_attn_tc(d, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window, gate_logits,
+                                           sinks, o, workspace, workspace_bytes, s, false, branch_lse, o_sparse));
+  }
+  return from_cuda(launch_sparse_attn_simt(d, dtype, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window,
+                                           gate_logits, sinks, o, s, branch_lse, o_sparse));
+}
+
+hys_status hysparse_full_attn_backward_workspace_size(const hys_shape* shape, hys_dtype dtype, size_t* bytes) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype) || !bytes) return HYS_ERR_INVALID_ARG;
+  *bytes = align256(full_bwd_workspace(d, dtype));
+  return HYS_OK;
+}
+
+hys_status hysparse_full_attn_backward(const hys_shape* shape, hys_dtype dtype, const void* q, const void* k,
+                                       const void* v, const void* o, const void* d_o, const float* lse, void* dq,
+                                       float* dk, float* dv, int accumulate_kv, void* workspace,
+                                       size_t workspace_bytes, hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !d_o || !lse || !dq || !dk || !dv) return HYS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return HYS_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < align256(full_bwd_workspace(d, dtype))) return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_full_bwd(d, dtype, q, k, v, o, d_o, lse, dq, dk, dv, accumulate_kv != 0, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hys_status hysparse_sparse_attn_backward_workspace_size(const hys_shape* shape, hys_dtype dtype, size_t* bytes) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype) || !bytes) return HYS_ERR_INVALID_ARG;
+  *bytes = align256(sparse_bwd_workspace(d));
+  return HYS_OK;
+}
+
+hys_status hysparse_sparse_attn_backward(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                         const void* k_shared, const void* v_shared, const int* idx, int k,
+                                         const void* k_swa, const void* v_swa, int window, const float* gate_logits,
+                                         const float* sinks, const void* o, const void* o_sparse,
+                                         const float* branch_lse, const void* d_o, void* dq, float* dk_shared,
+                                         float* dv_shared, float* dk_swa, float* dv_swa, float* dgate, float* dsinks,
+                                         void* workspace, size_t workspace_bytes, hys_stream_t stream) {
+  PrefillDims d;
+  hys_status st = check_prefill(shape, &d);
+  if (st != HYS_OK) return st;
+  if (!dtype_ok(dtype)) return HYS_ERR_INVALID_ARG;
+  if (!q_sparse || !k_shared || !v_shared || !idx || !k_swa || !v_swa || !gate_logits || !o || !o_sparse ||
+      !branch_lse || !d_o || !dq || !dk_shared || !dv_shared || !dk_swa || !dv_swa || !dgate)
+    return HYS_ERR_INVALID_ARG;
+  if (sinks != nullptr && dsinks == nullptr) return HYS_ERR_INVALID_ARG;
+  if (k < 1 || k > 1024 || window < 1) return HYS_ERR_INVALID_ARG;
+  // gradient outputs are distinct buffers (the window branch's are overwritten, the shared ones added to)
+  if (dk_swa == dk_shared || dv_swa == dv_shared || dk_swa == dv_shared || dv_swa == dk_shared)
+    return HYS_ERR_INVALID_ARG;
+  const void* ptrs[] = {q_sparse, k_shared, v_shared, idx, k_swa, v_swa, gate_logits, sinks, o, o_sparse, branch_lse,
+                        d_o, dq, dk_shared, dv_shared, dk_swa, dv_swa, dgate, dsinks, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return HYS_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < align256(sparse_bwd_workspace(d))) return HYS_ERR_WORKSPACE;
+  return from_cuda(launch_sparse_bwd(d, dtype, q_sparse, k_shared, v_shared, idx, k, k_swa, v_swa, window, gate_logits,
+                                     sinks, o, o_sparse, branch_lse, d_o, dq, dk_shared, dv_shared, dk_swa, dv_swa,
+                                     dgate, dsinks, workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 hys_status hysparse_sparse_attn_rows(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
                                      const void* k_shared, const void* v_shared, const int* idx, int k,
                                      const void* k_swa, const void* v_swa, int window, const float* gate_logits,

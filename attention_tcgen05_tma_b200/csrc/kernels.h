@@ -72,7 +72,7 @@ cudaError_t launch_topk_decode_tokens(const float* scores, int* idx, int B, int 
 cudaError_t launch_sparse_attn_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
                                     const void* v, const int* idx, int kb, const void* ks,
                                     const void* vs, int window, const float* gate, const float* sinks, void* o,
-                                    cudaStream_t s);
+                                    cudaStream_t s, float* blse = nullptr, void* osp = nullptr);
 cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,
                                       const void* v, const int* idx, int kt, int forced, void* o,
                                       cudaStream_t s);
@@ -81,10 +81,45 @@ bool sparse_attn_tc_supported(const PrefillDims& d, hys_dtype dt);
 size_t sparse_attn_tc_workspace(const PrefillDims& d);
 // per_row: idx is [B,Hkv,N,kb], one block list per query position (NB <= 512)
 bool sparse_attn_rows_tc_supported(const PrefillDims& d, hys_dtype dt);
+// blse / osp (training forward, per-tile selection only): [B,Hq,N,2] branch LSEs and [B,Hq,N,D] the
+// gated sparse-branch part sigmoid(g0) o~
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
                                   int kb, const void* ks, const void* vs, int window, const float* gate,
                                   const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s,
-                                  bool per_row = false);
+                                  bool per_row = false, float* blse = nullptr, void* osp = nullptr);
+
+// ---- backward (tcgen05, key-major; bf16, D = 128, even G) ----------------------------------
+bool attn_bwd_tc_supported(const PrefillDims& d, hys_dtype dt);
+size_t full_bwd_tc_workspace(const PrefillDims& d);
+// full layer: dq (bf16) from lse [B,Hq,N] and o; dk, dv fp32, overwritten or (accumulate) added to
+cudaError_t launch_full_bwd_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const void* o,
+                               const void* d_o, const float* lse, void* dq, float* dk, float* dv, int accumulate,
+                               void* ws, cudaStream_t s);
+// one key set of a sparse layer into the fp32 dq accumulator: the window over K', V' (dk, dv
+// overwritten) or the selected blocks over the shared K, V (dk, dv added to; list/list_cnt per
+// (b, g, 128-key tile): query tiles << 2 | block-half mask).  lse2 in log2 units, dsum = D_t,
+// sig = the branch's gate sigma_t per row
+cudaError_t launch_attn_bwd_tc_window(const PrefillDims& d, const void* q, const void* d_o, const void* k,
+                                      const void* v, const float* lse2, const float* dsum, const float* sig,
+                                      float* dq_acc, float* dk, float* dv, int window, int* counter, cudaStream_t s);
+cudaError_t launch_attn_bwd_tc_sparse(const PrefillDims& d, const void* q, const void* d_o, const void* k,
+                                      const void* v, const float* lse2, const float* dsum, const float* sig,
+                                      float* dq_acc, float* dk, float* dv, const int* list, const int* list_cnt,
+                                      int* counter, cudaStream_t s);
+// dq (bf16) = acc / sqrt(128); n a multiple of 8
+cudaError_t launch_bwd_dq_out(const float* acc, void* dq, size_t n, cudaStream_t s);
+
+// ---- backward, any supported dtype / D / G (tcgen05 where it applies, SIMT otherwise) --------
+size_t full_bwd_workspace(const PrefillDims& d, hys_dtype dt);
+cudaError_t launch_full_bwd(const PrefillDims& d, hys_dtype dt, const void* q, const void* k, const void* v,
+                            const void* o, const void* d_o, const float* lse, void* dq, float* dk, float* dv,
+                            int accumulate, void* ws, cudaStream_t s);
+size_t sparse_bwd_workspace(const PrefillDims& d);
+cudaError_t launch_sparse_bwd(const PrefillDims& d, hys_dtype dt, const void* q, const void* k, const void* v,
+                              const int* idx, int kb, const void* ks, const void* vs, int window, const float* gate,
+                              const float* sinks, const void* o, const void* osp, const float* blse, const void* d_o,
+                              void* dq, float* dk, float* dv, float* dks, float* dvs, float* dgate, float* dsinks,
+                              void* ws, cudaStream_t s);
 
 // ---- decode ----------------------------------------------------------------------------------
 size_t decode_full_workspace(const DecodeDims& d);

@@ -70,7 +70,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) sparse_attn_simt_kernel(
     PrefillDims d, const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int* __restrict__ idx, int kb, const T* __restrict__ ks, const T* __restrict__ vs, int window,
-    const float* __restrict__ gate, const float* __restrict__ sinks, T* __restrict__ o) {
+    const float* __restrict__ gate, const float* __restrict__ sinks, T* __restrict__ o, float* __restrict__ blse,
+    T* __restrict__ osp) {
   constexpr int DL = D / 4;
   __shared__ float sk[kKC][D];
   __shared__ float sv[kKC][D];
@@ -136,6 +137,21 @@ __global__ void __launch_bounds__(kThreads) sparse_attn_simt_kernel(
   T* oh = o + ((size_t)b * d.Hq + h) * d.N * D + (size_t)t * D;
 #pragma unroll
   for (int c = 0; c < DL; ++c) Elem<T>::store(oh + c * 4 + lg, a_sp[c] * i_sp + a_sw[c] * i_sw);
+  if (blse != nullptr) {
+    // training forward: each branch's LSE (natural-log units of the scaled logits, sink included;
+    // a branch without keys: the sink alone, or -inf) and the gated sparse part sigmoid(g0) o~
+    if (lg == 0) {
+      const float sk0 = sinks ? sinks[2 * h] * kLog2e : -INFINITY, sk1 = sinks ? sinks[2 * h + 1] * kLog2e : -INFINITY;
+      const float a = st_sp.m == -INFINITY ? sk0 : st_sp.m + log2f(l_sp);
+      const float c = st_sw.m == -INFINITY ? sk1 : st_sw.m + log2f(l_sw);
+      float* lrow = blse + (((size_t)b * d.Hq + h) * d.N + t) * 2;
+      lrow[0] = a * 0.6931471805599453f;
+      lrow[1] = c * 0.6931471805599453f;
+    }
+    T* sph = osp + ((size_t)b * d.Hq + h) * d.N * D + (size_t)t * D;
+#pragma unroll
+    for (int c = 0; c < DL; ++c) Elem<T>::store(sph + c * 4 + lg, a_sp[c] * i_sp);
+  }
 }
 
 template <typename T, int D>
@@ -201,10 +217,11 @@ __global__ void __launch_bounds__(kThreads) sparse_tokens_simt_kernel(PrefillDim
 template <typename T, int D>
 cudaError_t launch_sparse_typed(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
                                 int kb, const void* ks, const void* vs, int window, const float* gate,
-                                const float* sinks, void* o, cudaStream_t s) {
+                                const float* sinks, void* o, cudaStream_t s, float* blse, void* osp) {
   dim3 grid(d.T, d.Hq, d.B);
   sparse_attn_simt_kernel<T, D><<<grid, kThreads, 0, s>>>(d, (const T*)q, (const T*)k, (const T*)v, idx, kb,
-                                                          (const T*)ks, (const T*)vs, window, gate, sinks, (T*)o);
+                                                          (const T*)ks, (const T*)vs, window, gate, sinks, (T*)o,
+                                                          blse, (T*)osp);
   return cudaGetLastError();
 }
 
@@ -221,12 +238,16 @@ cudaError_t launch_tokens_typed(const PrefillDims& d, const void* q, const void*
 
 cudaError_t launch_sparse_attn_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k, const void* v,
                                     const int* idx, int kb, const void* ks, const void* vs, int window,
-                                    const float* gate, const float* sinks, void* o, cudaStream_t s) {
+                                    const float* gate, const float* sinks, void* o, cudaStream_t s, float* blse,
+                                    void* osp) {
   if (dt == HYS_F32)
-    return d.D == 64 ? launch_sparse_typed<float, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s)
-                     : launch_sparse_typed<float, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s);
-  return d.D == 64 ? launch_sparse_typed<__nv_bfloat16, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s)
-                   : launch_sparse_typed<__nv_bfloat16, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s);
+    return d.D == 64
+               ? launch_sparse_typed<float, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s, blse, osp)
+               : launch_sparse_typed<float, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s, blse, osp);
+  return d.D == 64 ? launch_sparse_typed<__nv_bfloat16, 64>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s,
+                                                            blse, osp)
+                   : launch_sparse_typed<__nv_bfloat16, 128>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, s,
+                                                             blse, osp);
 }
 
 cudaError_t launch_sparse_tokens_simt(const PrefillDims& d, hys_dtype dt, const void* q, const void* k,

@@ -64,6 +64,8 @@ struct Params {
   const float* sinks;  // [Hq,2] sink logits of the two branches, or null
   __nv_bfloat16* o;
   int o_v8;            // o is 32-byte aligned (256-bit stores)
+  float* blse;         // training forward: [B,Hq,N,2] LSE of the sparse and window branches
+  __nv_bfloat16* osp;  // training forward: [B,Hq,N,D] the gated sparse-branch part sigmoid(g0) o~
   int* counter;        // work-unit counter (zeroed before the launch)
   int* status;
   float scale_log2;
@@ -203,7 +205,8 @@ __device__ __forceinline__ void fail(volatile int* abort, int* status) {
   report_status(status, HYS_ERR_TIMEOUT);
 }
 
-template <int D, bool PR>   // PR: per-position selection (idx [B,Hkv,N,kb])
+template <int D, bool PR, bool TR>   // PR: per-position selection (idx [B,Hkv,N,kb]); TR: training
+                                     // forward (also writes the branch LSEs and sigmoid(g0) o~)
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKs,
@@ -543,6 +546,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) tc::tmem_st32(tOrow + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(ov + 32 * c));
+            if (TR && valid) {
+              uint4* dst = reinterpret_cast<uint4*>(p.osp + (((size_t)x.b * p.Hq + h) * p.N + t) * D);
+#pragma unroll
+              for (int i = 0; i < D / 8; ++i)
+                dst[i] = make_uint4(tc::pack_bf16x2(__uint_as_float(ov[8 * i]), __uint_as_float(ov[8 * i + 1])),
+                                    tc::pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3])),
+                                    tc::pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5])),
+                                    tc::pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7])));
+            }
           }
           // visible columns of the two 64-key halves of this tile (empty by default)
           const int wi = kind == kWinStats ? tau - x.n_sp : tau - x.n_sp - x.n_sw;
@@ -687,6 +699,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mbar_arrive(&bars->p_full[s]);
         }
         if (!ok) break;
+        if (TR && valid) {
+          // LSE of each branch in natural-log units of the scaled logits, the sink term included
+          // (a branch without keys: the sink alone, or -inf)
+          const float a = m_used == -INFINITY ? sk.x : m_used * sc + __log2f(l + exp2f(sk.x - m_used * sc));
+          const float c = mw == -INFINITY ? sk.y : mw * sc + __log2f(lw + exp2f(sk.y - mw * sc));
+          *reinterpret_cast<float2*>(p.blse + (((size_t)x.b * p.Hq + h) * p.N + t) * 2) =
+              make_float2(a * 0.6931471805599453f, c * 0.6931471805599453f);
+          if (x.n_sp == 0) {   // no sparse tile: the gated sparse part is zero
+            uint4* dst = reinterpret_cast<uint4*>(p.osp + (((size_t)x.b * p.Hq + h) * p.N + t) * D);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
         // ---- epilogue: O already holds sigmoid(g0) o~ + sigmoid(g1) o'
         if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_full[s], o_cnt & 1u, abort)))) break;
         ++o_cnt;
@@ -742,10 +767,10 @@ bool make_map(CUtensorMap* m, const void* base, int D, int rows, int heads) {
 int num_units(const PrefillDims& d) { return d.B * d.Hkv * d.T; }
 int grid_size(const PrefillDims& d) { return num_units(d) < kMaxGrid ? num_units(d) : kMaxGrid; }
 
-template <int D, bool PR>
+template <int D, bool PR, bool TR>
 cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx, int kb,
                          const void* ks, const void* vs, int window, const float* gate, const float* sinks,
-                         void* o, void* ws, cudaStream_t s) {
+                         void* o, void* ws, cudaStream_t s, float* blse, void* osp) {
   CUtensorMap mq, mk, mv, mks, mvs;
   if (!make_map(&mq, q, D, d.N, d.B * d.Hq) || !make_map(&mk, k, D, d.N, d.B * d.Hkv) ||
       !make_map(&mv, v, D, d.N, d.B * d.Hkv) || !make_map(&mks, ks, D, d.N, d.B * d.Hkv) ||
@@ -766,6 +791,8 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.sinks = sinks;
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
+  p.blse = blse;
+  p.osp = reinterpret_cast<__nv_bfloat16*>(osp);
   p.counter = reinterpret_cast<int*>(ws);
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
@@ -773,16 +800,16 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   static int regs = -1;   // the register split assumes exactly kLaunchRegs per thread at launch
   if (regs < 0) {
     cudaFuncAttributes fa;
-    cudaError_t e0 = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<D, PR>);
+    cudaError_t e0 = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<D, PR, TR>);
     if (e0 != cudaSuccess) return e0;
     regs = fa.numRegs;
   }
   if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D, PR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D, PR, TR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
-  sparse_attn_tc_kernel<D, PR><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, mks, mvs, p);
+  sparse_attn_tc_kernel<D, PR, TR><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, mks, mvs, p);
   return cudaGetLastError();
 }
 
@@ -801,14 +828,24 @@ bool sparse_attn_rows_tc_supported(const PrefillDims& d, hys_dtype dt) {
 cudaError_t launch_sparse_attn_tc(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx,
                                   int kb, const void* ks, const void* vs, int window, const float* gate,
                                   const float* sinks, void* o, void* ws, size_t ws_bytes, cudaStream_t s,
-                                  bool per_row) {
+                                  bool per_row, float* blse, void* osp) {
   if (ws_bytes < sparse_attn_tc_workspace(d)) return cudaErrorInvalidValue;
   if (per_row && d.NB > 32 * kRowWords) return cudaErrorInvalidValue;
+  if (per_row && blse != nullptr) return cudaErrorInvalidValue;   // training outputs: per-tile selection only
   if (per_row)
-    return d.D == 64 ? launch_typed<64, true>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s)
-                     : launch_typed<128, true>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s);
-  return d.D == 64 ? launch_typed<64, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s)
-                   : launch_typed<128, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s);
+    return d.D == 64 ? launch_typed<64, true, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s,
+                                                     nullptr, nullptr)
+                     : launch_typed<128, true, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s,
+                                                      nullptr, nullptr);
+  if (blse != nullptr)
+    return d.D == 64 ? launch_typed<64, false, true>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s, blse,
+                                                     osp)
+                     : launch_typed<128, false, true>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s,
+                                                      blse, osp);
+  return d.D == 64 ? launch_typed<64, false, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s,
+                                                    nullptr, nullptr)
+                   : launch_typed<128, false, false>(d, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, ws, s,
+                                                     nullptr, nullptr);
 }
 
 }  // namespace hys

@@ -35,6 +35,8 @@ EXPORTED = (
     "hysparse_sparse_attn_decode_tokens",
     "hysparse_full_attn_select_decode_tokens_fp8", "hysparse_sparse_attn_decode_tokens_fp8",
     "hysparse_topk_rows", "hysparse_sparse_attn_rows",
+    "hysparse_sparse_attn_train", "hysparse_full_attn_backward_workspace_size", "hysparse_full_attn_backward",
+    "hysparse_sparse_attn_backward_workspace_size", "hysparse_sparse_attn_backward",
 )
 
 
@@ -89,6 +91,12 @@ _SIGS = {
     "hysparse_sparse_attn_decode_tokens": ([_DSH, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P], _I),
     "hysparse_full_attn_select_decode_tokens_fp8": ([_DSH, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "hysparse_sparse_attn_decode_tokens_fp8": ([_DSH, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _SZ, _P], _I),
+    "hysparse_sparse_attn_train": ([_SH, _I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "hysparse_full_attn_backward_workspace_size": ([_SH, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_full_attn_backward": ([_SH, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _SZ, _P], _I),
+    "hysparse_sparse_attn_backward_workspace_size": ([_SH, _I, ctypes.POINTER(_SZ)], _I),
+    "hysparse_sparse_attn_backward": ([_SH, _I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                       _P, _P, _P, _P, _P, _SZ, _P], _I),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -270,6 +278,39 @@ def hysparse_sparse_attn_decode_tokens_fp8(shape, q, kc, vc, k_scale, v_scale, s
                                            ws_bytes, stream) -> int:
     return load().hysparse_sparse_attn_decode_tokens_fp8(ctypes.byref(shape), q, kc, vc, k_scale, v_scale, seqlens,
                                                          idx, k_tokens, forced, o, ws, ws_bytes, stream)
+
+
+def hysparse_sparse_attn_train(shape, dtype, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, o_sparse, blse, ws,
+                               ws_bytes, stream) -> int:
+    return load().hysparse_sparse_attn_train(ctypes.byref(shape), dtype, q, k, v, idx, kb, ks, vs, window, gate,
+                                             sinks, o, o_sparse, blse, ws, ws_bytes, stream)
+
+
+def hysparse_full_attn_backward_workspace_size(shape: hys_shape, dtype: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_full_attn_backward_workspace_size(ctypes.byref(shape), dtype, ctypes.byref(n)),
+           "hysparse_full_attn_backward_workspace_size")
+    return n.value
+
+
+def hysparse_full_attn_backward(shape, dtype, q, k, v, o, d_o, lse, dq, dk, dv, accumulate, ws, ws_bytes,
+                                stream) -> int:
+    return load().hysparse_full_attn_backward(ctypes.byref(shape), dtype, q, k, v, o, d_o, lse, dq, dk, dv,
+                                              accumulate, ws, ws_bytes, stream)
+
+
+def hysparse_sparse_attn_backward_workspace_size(shape: hys_shape, dtype: int) -> int:
+    n = _SZ(0)
+    _check(load().hysparse_sparse_attn_backward_workspace_size(ctypes.byref(shape), dtype, ctypes.byref(n)),
+           "hysparse_sparse_attn_backward_workspace_size")
+    return n.value
+
+
+def hysparse_sparse_attn_backward(shape, dtype, q, k, v, idx, kb, ks, vs, window, gate, sinks, o, o_sparse, blse,
+                                  d_o, dq, dk, dv, dks, dvs, dgate, dsinks, ws, ws_bytes, stream) -> int:
+    return load().hysparse_sparse_attn_backward(ctypes.byref(shape), dtype, q, k, v, idx, kb, ks, vs, window, gate,
+                                                sinks, o, o_sparse, blse, d_o, dq, dk, dv, dks, dvs, dgate, dsinks,
+                                                ws, ws_bytes, stream)
 
 
 # ----------------------------------------------------------------------------- torch helpers
@@ -563,3 +604,73 @@ def sparse_attn_decode_tokens_fp8(q, k_cache, v_cache, k_scale, v_scale, idx, fo
                                                   _stream(stream)),
            "hysparse_sparse_attn_decode_tokens_fp8")
     return o
+
+
+# ----------------------------------------------------------------------------- training
+def sparse_attn_train(q_sparse, k_shared, v_shared, idx, k_swa, v_swa, window: int, gate_logits, *, sinks=None,
+                      o=None, o_sparse=None, branch_lse=None, workspace=None, stream=None):
+    """Sparse layer forward of a training step. Returns (o, o_sparse, branch_lse): the layer
+    output, its gated sparse-branch part sigmoid(g0) o~ and the two branches' LSE [B,Hq,N,2]."""
+    torch = _torch()
+    sh = prefill_shape(q_sparse, k_shared)
+    o = torch.empty_like(q_sparse) if o is None else o
+    o_sparse = torch.empty_like(q_sparse) if o_sparse is None else o_sparse
+    if branch_lse is None:
+        branch_lse = torch.empty((sh.B, sh.Hq, sh.N, 2), dtype=torch.float32, device=q_sparse.device)
+    if workspace is None:
+        workspace = workspace_for(hysparse_sparse_attn_workspace_size(sh, _dt(q_sparse)), q_sparse.device)
+    _check(hysparse_sparse_attn_train(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k_shared), _ptr(v_shared), _ptr(idx),
+                                      idx.shape[-1], _ptr(k_swa), _ptr(v_swa), window, _ptr(gate_logits), _ptr(sinks),
+                                      _ptr(o), _ptr(o_sparse), _ptr(branch_lse), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)),
+           "hysparse_sparse_attn_train")
+    return o, o_sparse, branch_lse
+
+
+def full_attn_backward(q, k, v, o, d_o, lse, *, dq=None, dk=None, dv=None, accumulate: bool = False,
+                       workspace=None, stream=None):
+    """Gradients of the full layer. Returns (dq [input type], dk fp32, dv fp32); with
+    accumulate, dk and dv (given) receive the gradient added to their contents."""
+    torch = _torch()
+    sh = prefill_shape(q, k)
+    dq = torch.empty_like(q) if dq is None else dq
+    if dk is None:
+        dk = torch.empty(k.shape, dtype=torch.float32, device=k.device)
+    if dv is None:
+        dv = torch.empty(v.shape, dtype=torch.float32, device=v.device)
+    if workspace is None:
+        workspace = workspace_for(hysparse_full_attn_backward_workspace_size(sh, _dt(q)), q.device)
+    _check(hysparse_full_attn_backward(sh, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq),
+                                       _ptr(dk), _ptr(dv), int(accumulate), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)),
+           "hysparse_full_attn_backward")
+    return dq, dk, dv
+
+
+def sparse_attn_backward(q_sparse, k_shared, v_shared, idx, k_swa, v_swa, window: int, gate_logits, o, o_sparse,
+                         branch_lse, d_o, dk_shared, dv_shared, *, sinks=None, dq=None, dk_swa=None, dv_swa=None,
+                         dgate=None, dsinks=None, workspace=None, stream=None):
+    """Gradients of one sparse layer. dk_shared / dv_shared (fp32, given) receive the sparse
+    branch's gradient of the shared cache ADDED to their contents. Returns
+    (dq, dk_swa, dv_swa, dgate, dsinks)."""
+    torch = _torch()
+    sh = prefill_shape(q_sparse, k_shared)
+    dev = q_sparse.device
+    dq = torch.empty_like(q_sparse) if dq is None else dq
+    if dk_swa is None:
+        dk_swa = torch.empty(k_swa.shape, dtype=torch.float32, device=dev)
+    if dv_swa is None:
+        dv_swa = torch.empty(v_swa.shape, dtype=torch.float32, device=dev)
+    if dgate is None:
+        dgate = torch.empty((sh.B, sh.Hq, sh.N, 2), dtype=torch.float32, device=dev)
+    if sinks is not None and dsinks is None:
+        dsinks = torch.empty((sh.Hq, 2), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = workspace_for(hysparse_sparse_attn_backward_workspace_size(sh, _dt(q_sparse)), dev)
+    _check(hysparse_sparse_attn_backward(sh, _dt(q_sparse), _ptr(q_sparse), _ptr(k_shared), _ptr(v_shared), _ptr(idx),
+                                         idx.shape[-1], _ptr(k_swa), _ptr(v_swa), window, _ptr(gate_logits),
+                                         _ptr(sinks), _ptr(o), _ptr(o_sparse), _ptr(branch_lse), _ptr(d_o), _ptr(dq),
+                                         _ptr(dk_shared), _ptr(dv_shared), _ptr(dk_swa), _ptr(dv_swa), _ptr(dgate),
+                                         _ptr(dsinks), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hysparse_sparse_attn_backward")
+    return dq, dk_swa, dv_swa, dgate, dsinks

@@ -39,10 +39,11 @@ import numpy as np
 # tensor ids (stream keys).  Per sparse layer l the ids are 16 + 8*l + {0..3}.
 # ----------------------------------------------------------------------------
 TID_Q, TID_K, TID_V = 0, 1, 2
+TID_DO = 12          # output gradient of the full layer (training workloads)
 TID_FP8_SCALE = 14
 TID_PLANT = 15
 _TID_LAYER0 = 16
-SPARSE_Q, SPARSE_KSWA, SPARSE_VSWA, SPARSE_GATE, SPARSE_SINK = 0, 1, 2, 3, 4
+SPARSE_Q, SPARSE_KSWA, SPARSE_VSWA, SPARSE_GATE, SPARSE_SINK, SPARSE_DO = 0, 1, 2, 3, 4, 5
 
 
 def layer_tid(layer: int, which: int) -> int:
@@ -247,6 +248,16 @@ def gate_slice(w: Workload, layer: int, b: int, h: int) -> np.ndarray:
     return normal_slice(w.seed, layer_tid(layer, SPARSE_GATE), b, h, shape, 1.0, False)
 
 
+def d_o_slice(w: Workload, b: int, h: int) -> np.ndarray:
+    """Output gradient of the full layer (training): N(0, std^2) draws like Q, [N, D]."""
+    return normal_slice(w.seed, TID_DO, b, h, (w.N, w.D), w.scale_std, _bf16(w))
+
+
+def sparse_d_o_slice(w: Workload, layer: int, b: int, h: int) -> np.ndarray:
+    """Output gradient of a sparse layer (training), [N, D]."""
+    return normal_slice(w.seed, layer_tid(layer, SPARSE_DO), b, h, (w.N, w.D), w.scale_std, _bf16(w))
+
+
 def sink_logits(w: Workload, layer: int, std: float = 2.0) -> np.ndarray:
     """Per-head sink logits of a sparse layer, [Hq, 2] fp32 (index 0: sparse branch, 1: SWA
     branch); standard deviation 2 so that sinks range from negligible to dominant."""
@@ -315,11 +326,13 @@ def _fill(shape, fn, keys, threads: int = 8) -> np.ndarray:
     return out
 
 
-def prefill_arrays(w: Workload, layers: Optional[int] = None, threads: int = 8) -> Dict[str, object]:
+def prefill_arrays(w: Workload, layers: Optional[int] = None, threads: int = 8,
+                   grads: bool = False) -> Dict[str, object]:
     """All prefill tensors of a workload as float32 numpy arrays ([B, H, N, D] layout).
 
     Keys: q, k, v, and per sparse layer l: q_sparse[l], k_swa[l], v_swa[l], gate[l]
-    (gate is [B, Hq, N, 2]).
+    (gate is [B, Hq, N, 2]); with grads, also the output gradients d_o (full layer) and
+    d_o_sparse[l].
     """
     L = w.layers if layers is None else layers
     bq = [(b, h) for b in range(w.B) for h in range(w.Hq)]
@@ -336,6 +349,10 @@ def prefill_arrays(w: Workload, layers: Optional[int] = None, threads: int = 8) 
         out["k_swa"].append(_fill((w.B, w.Hkv, w.N, w.D), lambda b, g: swa_k_slice(w, l, b, g), bk, threads))
         out["v_swa"].append(_fill((w.B, w.Hkv, w.N, w.D), lambda b, g: swa_v_slice(w, l, b, g), bk, threads))
         out["gate"].append(_fill((w.B, w.Hq, w.N, 2), lambda b, h: gate_slice(w, l, b, h), bq, threads))
+    if grads:
+        out["d_o"] = _fill((w.B, w.Hq, w.N, w.D), lambda b, h: d_o_slice(w, b, h), bq, threads)
+        out["d_o_sparse"] = [_fill((w.B, w.Hq, w.N, w.D), lambda b, h: sparse_d_o_slice(w, l, b, h), bq, threads)
+                             for l in range(L)]
     return out
 
 

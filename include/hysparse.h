@@ -192,6 +192,70 @@ HYS_API hys_status hysparse_sparse_attn_rows(const hys_shape* shape, hys_dtype d
                                      void* workspace, size_t workspace_bytes, hys_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * Training: the sparse layer's forward with saved statistics, and the backward of the full
+ * and sparse layers ([HS] 3.4.6, training pipeline: no auxiliary loss for the selection, the
+ * selected indices are constants of the step; the sparse layers' gradients reach the full
+ * layer's K and V through the shared cache of 3.4.4).  Gradients of attention over a key set
+ * with p = softmax(tau q.k) and o = sum_i p_i v_i: dV_i = sum_t p_ti dO_t, dK_i = tau sum_t
+ * dS_ti q_t, dQ_t = tau sum_i dS_ti k_i, dS_ti = p_ti (dO_t.v_i - dO_t.o_t); for the gated layer
+ * ([HS] 3.4.3) each branch b sees dO scaled by sigmoid(g_b), and d g_b = sigmoid(g_b)
+ * (1 - sigmoid(g_b)) dO.o_b; a sink logit's gradient is -sum_t p_sink,t sigmoid(g_b) dO_t.o_b,t.
+ * Key and value gradients are fp32 (they are sums over layers and heads); dq takes the input
+ * type.  bf16 with D = 128 and an even group size runs on the tensor cores (key-major tcgen05
+ * kernel, dQ accumulated in fp32 with vector reductions); other shapes and fp32 run SIMT
+ * fp32-accumulate kernels.
+ * ------------------------------------------------------------------------------------ */
+
+/* The sparse layer of a training step: hysparse_sparse_attn (same arguments, limits and
+ * workspace) that also saves
+ *   o_sparse    [B,Hq,N,D] input type: the gated sparse-branch part sigmoid(g0) o~ of o;
+ *   branch_lse  [B,Hq,N,2] fp32: log of each branch's softmax normaliser in units of the
+ *               scaled logits, LSE = log(sum_i exp(tau q.k_i) + exp(sink)), index 0 the sparse
+ *               branch and 1 the window branch (a branch without keys: the sink, or -inf). */
+HYS_API hys_status hysparse_sparse_attn_train(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                              const void* k_shared, const void* v_shared, const int* idx, int k,
+                                              const void* k_swa, const void* v_swa, int window,
+                                              const float* gate_logits, const float* sinks, void* o, void* o_sparse,
+                                              float* branch_lse, void* workspace, size_t workspace_bytes,
+                                              hys_stream_t stream);
+
+/* Backward of the full layer (causal GQA attention, [HS] 3.4.1).  Inputs q, k, v, o and the
+ * output gradient d_o as for hysparse_full_attn_select, lse [B,Hq,N] fp32 the forward's lse_opt.
+ * Outputs: dq [B,Hq,N,D] (input type); dk, dv [B,Hkv,N,D] fp32, summed over the group's heads,
+ * overwritten (accumulate_kv == 0) or added to (accumulate_kv != 0).  workspace: at least
+ * hysparse_full_attn_backward_workspace_size() bytes. */
+HYS_API hys_status hysparse_full_attn_backward_workspace_size(const hys_shape* shape, hys_dtype dtype,
+                                                              size_t* bytes);
+HYS_API hys_status hysparse_full_attn_backward(const hys_shape* shape, hys_dtype dtype, const void* q, const void* k,
+                                               const void* v, const void* o, const void* d_o, const float* lse,
+                                               void* dq, float* dk, float* dv, int accumulate_kv, void* workspace,
+                                               size_t workspace_bytes, hys_stream_t stream);
+
+/* Backward of one sparse layer (per-tile selection, [HS] 3.4.3).  Inputs as for
+ * hysparse_sparse_attn_train, plus its outputs o, o_sparse and branch_lse, and d_o [B,Hq,N,D].
+ * Outputs:
+ *   dq                 [B,Hq,N,D] input type, both branches;
+ *   dk_shared,
+ *   dv_shared          [B,Hkv,N,D] fp32, the sparse branch's gradient of the shared cache, ADDED
+ *                      to the buffers (pass the full layer's gradient, or zeros, and call the
+ *                      block's sparse layers one after another to sum the block);
+ *   dk_swa, dv_swa     [B,Hkv,N,D] fp32, the window branch's gradient of K', V', overwritten;
+ *   dgate              [B,Hq,N,2] fp32, overwritten;
+ *   dsinks             [Hq,2] fp32 (required when sinks is given, else ignored), overwritten.
+ * The gradient buffers must not alias one another (inputs may: K'/V' may be K/V).  workspace:
+ * at least hysparse_sparse_attn_backward_workspace_size() bytes. */
+HYS_API hys_status hysparse_sparse_attn_backward_workspace_size(const hys_shape* shape, hys_dtype dtype,
+                                                                size_t* bytes);
+HYS_API hys_status hysparse_sparse_attn_backward(const hys_shape* shape, hys_dtype dtype, const void* q_sparse,
+                                                 const void* k_shared, const void* v_shared, const int* idx, int k,
+                                                 const void* k_swa, const void* v_swa, int window,
+                                                 const float* gate_logits, const float* sinks, const void* o,
+                                                 const void* o_sparse, const float* branch_lse, const void* d_o,
+                                                 void* dq, float* dk_shared, float* dv_shared, float* dk_swa,
+                                                 float* dv_swa, float* dgate, float* dsinks, void* workspace,
+                                                 size_t workspace_bytes, hys_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * Token-sparse layer ([HS2]): row t of tile I attends idx[b,g,I,:] (token positions,
  * ascending, -1 padded, all <= t) united with [max(0, t-forced_window+1), t], each
  * token once, over the shared K, V; no gate.  sinks must be NULL.  workspace: at least

@@ -83,3 +83,16 @@ def score_rel_err(oracle_scores: np.ndarray, gpu_scores: np.ndarray, floor: floa
     if not mask.any():
         return 0.0
     return float(np.max(np.abs(gpu_scores[mask] - oracle_scores[mask]) / np.abs(oracle_scores[mask])))
+
+
+# Gradients: the largest error relative to the gradient's largest element.  bf16 inputs: 2e-2 (the
+# bound set for bf16 attention outputs; P and dS are rounded to bf16 before the contractions and dq is
+# stored in bf16, each a relative 2^-9 per term); fp32 inputs (fp32 kernels throughout): 1e-4.
+GRAD_TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def grad_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+    scale = float(np.max(np.abs(ref)))
+    if scale == 0.0:
+        return float(np.max(np.abs(gpu)))
+    return float(np.max(np.abs(np.asarray(gpu, np.float64) - ref))) / scale

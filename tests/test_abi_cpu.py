@@ -161,3 +161,33 @@ def test_fp8_token_decode_entry_points_validate(lib):
     assert sparse(dsh, 16, 16, 16, 16, None, None, 16, 64, 64, 16, 16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
     assert sparse(dsh, 16, 16, 16, 16, 16, None, 16, 64, 5000, 16, 16, 1 << 20, None) == H.HYS_ERR_INVALID_ARG
     assert sparse(dsh, 16, 16, 16, 16, 16, None, 16, 64, 64, 16, 16, 64, None) == H.HYS_ERR_WORKSPACE
+
+
+def test_training_entry_points_reject_bad_arguments_without_launching(lib):
+    sh = H.hys_shape(1, 256, 4, 2, 128, 64)
+    assert H.hysparse_full_attn_backward_workspace_size(sh, H.HYS_BF16) > 0
+    assert H.hysparse_sparse_attn_backward_workspace_size(sh, H.HYS_BF16) > 0
+    P = 256   # an aligned stand-in pointer: every call below fails validation before any launch
+    # missing inputs / outputs
+    assert H.hysparse_full_attn_backward(sh, H.HYS_BF16, P, P, P, P, P, None, P, P, P, 0, P, 1 << 30, None) \
+        == H.HYS_ERR_INVALID_ARG
+    # misaligned gradient output
+    assert H.hysparse_full_attn_backward(sh, H.HYS_BF16, P, P, P, P, P, P, P + 4, P, P, 0, P, 1 << 30, None) \
+        == H.HYS_ERR_INVALID_ARG
+    # workspace too small
+    assert H.hysparse_full_attn_backward(sh, H.HYS_BF16, P, P, P, P, P, P, P, P, P, 0, P, 16, None) \
+        == H.HYS_ERR_WORKSPACE
+    args = [P] * 4 + [2, P, P, 128, P, None, P, P, P, P]   # q, k, v, idx, k, ks, vs, window, gate, sinks, o, osp, lse, do
+    outs = [512, 768, 1024, 1280, 1536, 1792, None]         # dq, dk, dv, dk_swa, dv_swa, dgate, dsinks
+    ok = H.hysparse_sparse_attn_backward(sh, H.HYS_BF16, *args, *outs, P, 16, None)
+    assert ok == H.HYS_ERR_WORKSPACE                        # valid arguments, workspace too small
+    alias = list(outs)
+    alias[3] = alias[1]                                     # dk_swa aliases dk_shared
+    assert H.hysparse_sparse_attn_backward(sh, H.HYS_BF16, *args, *alias, P, 1 << 30, None) == H.HYS_ERR_INVALID_ARG
+    with_sinks = list(args)
+    with_sinks[9] = P                                       # sinks given without a dsinks output
+    assert H.hysparse_sparse_attn_backward(sh, H.HYS_BF16, *with_sinks, *outs, P, 1 << 30, None) \
+        == H.HYS_ERR_INVALID_ARG
+    # the training forward needs both saved outputs
+    assert H.hysparse_sparse_attn_train(sh, H.HYS_BF16, P, P, P, P, 2, P, P, 128, P, None, P, None, P, P, 1 << 20,
+                                        None) == H.HYS_ERR_INVALID_ARG
