@@ -36,7 +36,11 @@ constexpr int kThreads = 384;
 // kLaunchRegs; the producer/MMA warpgroup drops to kLowRegs and each softmax warpgroup rises to
 // kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
 // the host checks the compiled register count before every launch.
-constexpr int kLaunchRegs = 168, kLowRegs = 88, kHighRegs = 208;
+#ifndef HYS_SPARSE_LOW_REGS
+#define HYS_SPARSE_LOW_REGS 88
+#endif
+constexpr int kLaunchRegs = 168, kLowRegs = HYS_SPARSE_LOW_REGS, kHighRegs = (3 * kLaunchRegs - kLowRegs) / 2;
+static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 static_assert(kLowRegs + 2 * kHighRegs == 3 * kLaunchRegs, "register split must match the launch allocation");
 constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;

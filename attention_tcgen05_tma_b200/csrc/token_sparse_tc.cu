@@ -39,7 +39,11 @@ constexpr int kPolyPairs = HYS_TOKEN_POLY_PAIRS;
 // kLaunchRegs; the producer/MMA warpgroup drops to kLowRegs and each softmax warpgroup rises to
 // kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
 // the host checks the compiled register count before every launch.
-constexpr int kLaunchRegs = 168, kLowRegs = 88, kHighRegs = 208;
+#ifndef HYS_TOKEN_LOW_REGS
+#define HYS_TOKEN_LOW_REGS 88
+#endif
+constexpr int kLaunchRegs = 168, kLowRegs = HYS_TOKEN_LOW_REGS, kHighRegs = (3 * kLaunchRegs - kLowRegs) / 2;
+static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 static_assert(kLowRegs + 2 * kHighRegs == 3 * kLaunchRegs, "register split must match the launch allocation");
 
 __device__ __forceinline__ float2 exp2_pair(float2 x, int i) {

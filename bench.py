@@ -11,11 +11,12 @@ sparse layers) is timed in the same run and reported as ``decode`` (us/token).
 
 Further legs, each outside the headline's timed region and reported under its own key:
 ``rows`` (per-position selection on the prefill inputs, one layer), ``dense7b`` (the 7B-dense-shaped
-1:3 block: B1 N8192, 32/8 heads, top-16 blocks, 3 sparse layers), ``decode_tokens`` (the
+1:3 block: B1 N8192, 32/8 heads, top-16 blocks, 3 sparse layers), ``backward`` (the training
+backward of the full layer and of one sparse layer on the headline inputs), ``decode_tokens`` (the
 token-variant decode step over the decode cache, bf16 and FP8 E4M3, us/token), ``token`` (the
 token-variant prefill, N=131072), ``e2e`` (the headline through the C ABI with host buffers
 copied in and out every step) and ``cpu_baseline`` (the float64 oracle on a bounded sample).
-Flags ``--no-rows``, ``--no-dense7b``, ``--no-decode``, ``--no-decode-tokens``, ``--no-token``,
+Flags ``--no-rows``, ``--no-dense7b``, ``--no-backward``, ``--no-decode``, ``--no-decode-tokens``, ``--no-token``,
 ``--no-e2e`` and ``--no-cpu`` skip them.
 
 Multi-GPU (torchrun): every rank runs its own independent batch (weak scaling, no
@@ -376,6 +377,7 @@ def run_ours(args, torch, dist, rank, world, dev):
     kernels["sparse_attn_same_layer_no_sinks_ms"] = round(ms_plain, 4)   # same repeated-call timing
     kernels["sparse_attn_sinks_tflops"] = round(sp_flops / (ms_sinks / 1e3) / 1e12, 2)
     rows = None if args.no_rows else run_rows(torch, H, w, x, step, peak_tf)
+    backward = None if args.no_backward else run_backward(torch, H, w, x, step, peak_tf)
 
     res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -384,6 +386,8 @@ def run_ours(args, torch, dist, rank, world, dev):
            "kernels": kernels, "roofline": roof, "clocks": clk, "gpu_launches": launches}
     if rows is not None:
         res["rows"] = rows
+    if backward is not None:
+        res["backward"] = backward
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, torch, dist, world, w, x, step, dev)
     del x, step
@@ -433,6 +437,51 @@ def run_rows(torch, H, w, x, step, peak_tf):
            "sparse_alg_frac": round(alg_flops / (ms_sparse / 1e3) / 1e12 / peak_tf, 4),
            "mean_union_blocks_per_tile": round(union, 1)}
     del o, sc, idx
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_backward(torch, H, w, x, step, peak_tf):
+    """Training backward on the headline inputs, each call timed on its own: the full layer's
+    gradients (dq, and fp32 dk, dv of the shared cache) and one sparse layer's (dq, its share of the
+    shared dk, dv, dk', dv', gate gradients) after its training forward.  Algorithmic work: five
+    contractions of 2*D flops per attended (row, head, key) = 10*D, i.e. 2.5x the forward's."""
+    gen = torch.Generator(device=x["q"].device)
+    gen.manual_seed(1234)
+    d_o = (torch.randn(x["q"].shape, generator=gen, device=x["q"].device) / math.sqrt(w.D)).to(torch.bfloat16)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=x["q"].device)
+    o = torch.empty_like(x["q"])
+    H.full_attn_select(x["q"], x["k"], x["v"], o=o, scores=step.scores, lse=lse, workspace=step.ws)
+    H.topk(step.scores, w.topk, idx=step.idx)
+    dq = torch.empty_like(x["q"])
+    dk = torch.empty(x["k"].shape, dtype=torch.float32, device=x["q"].device)
+    dv = torch.empty_like(dk)
+    ws_f = H.workspace_for(H.hysparse_full_attn_backward_workspace_size(H.prefill_shape(x["q"], x["k"]), H.HYS_BF16),
+                           x["q"].device)
+    full = lambda: H.full_attn_backward(x["q"], x["k"], x["v"], o, d_o, lse, dq=dq, dk=dk, dv=dv, workspace=ws_f)
+    ms_full = time_call(torch, full, n=3, warm=1)
+    del ws_f
+    lx = [x[key][0] for key in ("q_sparse", "k_swa", "v_swa", "gate")]
+    o_l, osp, blse = H.sparse_attn_train(lx[0], x["k"], x["v"], step.idx, lx[1], lx[2], w.window, lx[3],
+                                         workspace=step.ws_sp)
+    dks = torch.empty(x["k"].shape, dtype=torch.float32, device=x["q"].device)
+    dvs = torch.empty_like(dks)
+    dgate = torch.empty((w.B, w.Hq, w.N, 2), dtype=torch.float32, device=x["q"].device)
+    ws_s = H.workspace_for(H.hysparse_sparse_attn_backward_workspace_size(H.prefill_shape(x["q"], x["k"]),
+                                                                         H.HYS_BF16), x["q"].device)
+    sparse = lambda: H.sparse_attn_backward(lx[0], x["k"], x["v"], step.idx, lx[1], lx[2], w.window, lx[3], o_l, osp,
+                                            blse, d_o, dk, dv, dq=dq, dk_swa=dks, dv_swa=dvs, dgate=dgate,
+                                            workspace=ws_s)
+    ms_sparse = time_call(torch, sparse, n=3, warm=1)
+    full_flops = 2.5 * 4.0 * w.D * w.Hq * w.B * w.N * (w.N + 1) / 2
+    sp_flops = 2.5 * sparse_flops(step.idx.cpu().numpy(), w.N, w.G, w.D, w.window)
+    res = {"config": f"{w.name}: full layer and one sparse layer, bf16 inputs, fp32 K/V gradients",
+           "full_bwd_ms": round(ms_full, 3), "full_bwd_tflops": round(full_flops / ms_full / 1e9, 1),
+           "full_bwd_frac": round(full_flops / ms_full / 1e9 / peak_tf, 4),
+           "sparse_bwd_ms": round(ms_sparse, 3), "sparse_bwd_tflops": round(sp_flops / ms_sparse / 1e9, 1),
+           "sparse_bwd_frac": round(sp_flops / ms_sparse / 1e9 / peak_tf, 4),
+           "full_bwd_flops": full_flops, "sparse_bwd_flops": sp_flops}
+    del d_o, lse, o, dq, dk, dv, dks, dvs, dgate, ws_s, o_l, osp, blse
     torch.cuda.empty_cache()
     return res
 
@@ -945,6 +994,7 @@ def main():
     ap.add_argument("--no-token", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-position selection leg")
     ap.add_argument("--no-dense7b", action="store_true", help="skip the 7B-dense-shaped block leg")
+    ap.add_argument("--no-backward", action="store_true", help="skip the training backward leg")
     ap.add_argument("--token-workload", default="token", help="token-variant workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
