@@ -3,15 +3,20 @@
 //
 //   score[b,g,I,i] = sum_{h in g} sum_{t in tile I, t >= i} exp(tau q_t.k_i - LSE_t)
 //
-// LSE_t comes from the first pass (the full-attention kernel), so every probability is
-// exact without an online softmax.  Per 128-key tile and 128-row M-tile (two heads x the
-// 64 positions of tile I, as in the full layer): S = Q K^T (tcgen05, TMEM); the softmax
-// warpgroup writes P * 2^12 as fp16 into shared memory (the scale keeps probabilities down
-// to 1.5e-8 in the normal fp16 range; the sum is scaled back at the end); the column sums
-// over the 128 rows are one more MMA, D = ONES(128 x 128) * P, accumulated over both
-// M-tiles of a round in TMEM.  Warps 2-3 drain D (double-buffered) into the score row;
-// later rounds of a unit add to what the first wrote, in a fixed order (deterministic).
+// LSE_t comes from the first pass (the full-attention kernel), so every probability is exact
+// without an online softmax.  The scores are column sums of P, so the kernel computes the
+// transposed logits S^T = K Q^T (tcgen05, TMEM): a TMEM lane is then a key and its 128 columns
+// are the query rows of an M-tile (two heads x the 64 positions of tile I), and each key's sum
+// over the rows is a sum inside one thread -- no cross-thread reduction, no P in shared memory.
+//
+// A work unit is (b, g, I); up to four M-tiles (head pairs) stay in shared memory while the
+// key tiles 0..I/2 stream through a two-stage ring.  Every (key tile, M-tile) item is one MMA
+// into one of four 128-column TMEM buffers (a ring over the items).  Two softmax warpgroups
+// take the items of even and odd M-tiles; per key tile the odd group's per-key partial goes to
+// the even group through shared memory, which adds its own and writes score[b,g,I,key] once
+// (fixed order: deterministic).  Part of the exponentials run as a polynomial on the FMA pipe.
 #include <cuda.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -22,10 +27,16 @@ namespace hys {
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 384;     // warp 0 TMA, warp 1 MMA, warps 4-7 / 8-11 softmax groups 0 / 1
 constexpr int kStages = 2;        // K ring
+constexpr int kMaxMT = 4;         // M-tiles resident per round
+constexpr int kBufs = 4;          // TMEM buffers of 128 columns
 constexpr int kMaxGrid = 148;
-constexpr float kPScaleLog2 = 12.0f;
+#ifndef HYS_TSCORE_POLY_PAIRS
+#define HYS_TSCORE_POLY_PAIRS 16
+#endif
+// column pairs (of the 64 in a 128-row item) whose exp2 runs on the FMA pipe instead of MUFU
+constexpr int kPolyPairs = HYS_TSCORE_POLY_PAIRS;
 
 struct Params {
   int B, N, Hq, Hkv, G, T;
@@ -35,33 +46,36 @@ struct Params {
   int* counter;
   int* status;
   float scale_log2;
+  uint64_t wait_ns;   // limit of every bounded wait
+  int probe;          // watchdog probe: the producer never issues the first unit's Q copies
 };
 
 struct Bars {
   uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], p_empty[2], d_full[2], d_empty[2];
+  uint64_t q_full, q_empty, s_full[kBufs], s_free[kBufs];
+  uint64_t rows_ready[2], comb_full[2], comb_empty[2];
   uint64_t mma_drain, spare;
-  tc::UnitQueue queue;
 };
 
 template <int D>
 struct Cfg {
   static constexpr int kChunks = D / 64;
-  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kQBytes = 128 * D * 2;   // one M-tile
   static constexpr int kKBytes = 128 * D * 2;
-  static constexpr int kPBytes = 128 * 128 * 2;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = 2 * kQBytes;
-  static constexpr int kOffP = kOffK + kStages * kKBytes;
-  static constexpr int kOffOnes = kOffP + 2 * kPBytes;
-  static constexpr int kOffBar = kOffOnes + 16384;
+  static constexpr int kOffK = kMaxMT * kQBytes;
+  static constexpr int kOffLse = kOffK + kStages * kKBytes;      // [2 rounds][kMaxMT][128] lse2
+  static constexpr int kOffRed = kOffLse + 2 * kMaxMT * 128 * 4; // [2][128] odd-group partials
+  static constexpr int kOffBar = kOffRed + 2 * 128 * 4;
   static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 };
+static_assert(Cfg<128>::kSmemBytes <= 232448, "shared memory of one CTA");
 
+// unit u -> (b, g, I), the longest (largest I) first over all (b, g)
 __device__ __forceinline__ void unit_coords(const Params& p, int u, int& b, int& g, int& I) {
-  const int bg = u / p.T;
-  I = p.T - 1 - u % p.T;
+  const int bg = u % (p.B * p.Hkv);
+  I = p.T - 1 - u / (p.B * p.Hkv);
   b = bg / p.Hkv;
   g = bg % p.Hkv;
 }
@@ -69,16 +83,6 @@ __device__ __forceinline__ void unit_coords(const Params& p, int u, int& b, int&
 __device__ __forceinline__ void fail(volatile int* abort, int* status) {
   *abort = 1;
   report_status(status, HYS_ERR_TIMEOUT);
-}
-
-// instruction descriptor: fp16 A and B (kind::f16 format 0), fp32 accumulate
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
-  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
 }
 
 template <int D>
@@ -91,36 +95,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 16);
+  int* s_unit = reinterpret_cast<int*>(smem + C::kOffMisc + 32);
+  float* s_lse = reinterpret_cast<float*>(smem + C::kOffLse);
+  float* s_red = reinterpret_cast<float*>(smem + C::kOffRed);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MT = p.G / 2;
-  const int rounds = (MT + 1) / 2;
+  const int rounds = (MT + kMaxMT - 1) / kMaxMT;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bars->k_full[i], 1);
       tc::mbar_init(&bars->k_empty[i], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->q_full[s], 1);
-      tc::mbar_init(&bars->q_empty[s], 1);
-      tc::mbar_init(&bars->s_full[s], 1);
-      tc::mbar_init(&bars->p_full[s], 128);
-      tc::mbar_init(&bars->p_empty[s], 1);
-      tc::mbar_init(&bars->d_full[s], 1);
-      tc::mbar_init(&bars->d_empty[s], 64);
+    tc::mbar_init(&bars->q_full, 1);
+    tc::mbar_init(&bars->q_empty, 1);
+    for (int i = 0; i < kBufs; ++i) {
+      tc::mbar_init(&bars->s_full[i], 1);
+      tc::mbar_init(&bars->s_free[i], 128);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bars->rows_ready[i], 128);
+      tc::mbar_init(&bars->comb_full[i], 128);
+      tc::mbar_init(&bars->comb_empty[i], 128);
     }
     tc::mbar_init(&bars->mma_drain, 1);
-    tc::queue_init(&bars->queue, 1 + 256 + 64);  // MMA thread, softmax warpgroups, drain warps
     *abort = 0;
     tc::fence_barrier_init();
-  }
-  // the all-ones A operand: 128 rows x 64 fp16 (one 128-byte swizzled chunk, reused for both k halves)
-  {
-    uint4* ones = reinterpret_cast<uint4*>(smem + C::kOffOnes);
-    const uint32_t one2 = 0x3C003C00u;
-    for (int i = threadIdx.x; i < 16384 / 16; i += kThreads) ones[i] = make_uint4(one2, one2, one2, one2);
-    tc::fence_proxy_async_shared();
   }
   if (warp == 0 && lane == 0) {
     tc::prefetch_tensormap(&tmQ);
@@ -135,253 +136,172 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ============================================================== TMA producer
-    if (lane == 0) {
-      uint32_t k_it = 0, q_cnt[2] = {0, 0};
-      bool ok = true;
-      for (uint32_t n = 0; ok; ++n) {
-        const int c = atomicAdd(p.counter, 1);
-        const int u = c < p.num_units ? c : -1;
-        if (!(ok = tc::queue_push(&bars->queue, n, u, abort))) break;
-        if (u < 0) break;
-        int b, g, I;
-        unit_coords(p, u, b, g, I);
-        const int nkt = I / 2 + 1;
-        for (int r = 0; r < rounds && ok; ++r) {
-          for (int s = 0; s < 2 && ok; ++s) {
-            const int mt = 2 * r + s;
-            if (mt >= MT) continue;
-            if (!(ok = tc::mbar_wait(&bars->q_empty[s], (q_cnt[s] & 1u) ^ 1u, abort))) break;
-            ++q_cnt[s];
-            tc::mbar_arrive_expect_tx(&bars->q_full[s], C::kQBytes);
-            uint8_t* qdst = smem + C::kOffQ + s * C::kQBytes;
-            const int h0 = g * p.G + 2 * mt;
-            for (int hh = 0; hh < 2; ++hh)
-              for (int ch = 0; ch < C::kChunks; ++ch)
-                tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + ch * 16384 + hh * 8192, ch * 64, 64 * I,
-                                b * p.Hq + h0 + hh);
+  // every role walks the same unit sequence (one thread claims, all read it back); counters of
+  // rounds (rc), key-tile items (ni), K tiles (kc) and combines (cc) advance identically in all roles
+  uint32_t rc = 0, ni = 0, kc = 0, cc = 0;
+  for (;;) {
+    if (threadIdx.x == 0) *s_unit = atomicAdd(p.counter, 1);
+    __syncthreads();
+    const int u = *s_unit;
+    const bool stop = u >= p.num_units || *abort;
+    __syncthreads();
+    if (stop) break;
+    int b, g, I;
+    unit_coords(p, u, b, g, I);
+    const int nkt = I / 2 + 1;
+    float* srow = p.scores + (((size_t)b * p.Hkv + g) * p.T + I) * (size_t)p.N;
+
+    for (int r = 0; r < rounds; ++r) {
+      const int mt0 = kMaxMT * r;
+      const int nm = min(kMaxMT, MT - mt0);
+      if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+          bool ok = tc::mbar_wait(&bars->q_empty, (rc & 1u) ^ 1u, abort, p.wait_ns);
+          // watchdog probe (tests only): the first unit's Q copies are never issued, so the MMA
+          // warp's wait on them runs out and the kernel must end with HYS_ERR_TIMEOUT
+          if (ok && !(p.probe && rc == 0)) {
+            tc::mbar_arrive_expect_tx(&bars->q_full, nm * C::kQBytes);
+            for (int m = 0; m < nm; ++m)
+              for (int hh = 0; hh < 2; ++hh)
+                for (int ch = 0; ch < C::kChunks; ++ch)
+                  tc::tma_load_3d(&tmQ, &bars->q_full, smem + C::kOffQ + m * C::kQBytes + ch * 16384 + hh * 8192,
+                                  ch * 64, 64 * I, b * p.Hq + g * p.G + 2 * (mt0 + m) + hh);
           }
-          for (int tau = 0; tau < nkt && ok; ++tau) {
-            const uint32_t st = k_it % kStages;
-            if (!(ok = tc::mbar_wait(&bars->k_empty[st], ((k_it / kStages) & 1u) ^ 1u, abort))) break;
+          for (int j = 0; j < nkt && ok; ++j) {
+            const uint32_t k = kc + j, st = k % kStages;
+            if (!(ok = tc::mbar_wait(&bars->k_empty[st], ((k / kStages) & 1u) ^ 1u, abort, p.wait_ns))) break;
             tc::mbar_arrive_expect_tx(&bars->k_full[st], C::kKBytes);
-            uint8_t* dst = smem + C::kOffK + st * C::kKBytes;
             for (int ch = 0; ch < C::kChunks; ++ch)
-              tc::tma_load_3d(&tmK, &bars->k_full[st], dst + ch * 16384, ch * 64, 128 * tau, b * p.Hkv + g);
-            ++k_it;
+              tc::tma_load_3d(&tmK, &bars->k_full[st], smem + C::kOffK + st * C::kKBytes + ch * 16384, ch * 64,
+                              128 * j, b * p.Hkv + g);
           }
+          if (!ok) fail(abort, p.status);
         }
-      }
-      if (!ok) fail(abort, p.status);
-      for (uint32_t i = (k_it > kStages ? k_it - kStages : 0); i < k_it; ++i)
-        tc::mbar_wait(&bars->k_full[i % kStages], (i / kStages) & 1u, abort, 100000000ull);
-      for (int s = 0; s < 2; ++s)
-        if (q_cnt[s] > 0) tc::mbar_wait(&bars->q_full[s], (q_cnt[s] - 1) & 1u, abort, 100000000ull);
-    }
-  } else if (warp == 1) {
-    // ============================================================== MMA issuer
-    if (lane == 0) {
-      const uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
-      const uint32_t idC = idesc_f16_f32(128, 128, true);
-      const uint32_t tS[2] = {tmem_base, tmem_base + 128};
-      const uint32_t tD[2] = {tmem_base + 256, tmem_base + 384};
-      const uint32_t qaddr = tc::smem_u32(smem + C::kOffQ);
-      const uint32_t kaddr = tc::smem_u32(smem + C::kOffK);
-      const uint32_t paddr = tc::smem_u32(smem + C::kOffP);
-      const uint32_t oaddr = tc::smem_u32(smem + C::kOffOnes);
-      uint32_t k_it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0}, d_cnt = 0;
-      bool ok = true;
-      auto issue_S = [&](int s, uint32_t st) {
-        const uint32_t qb = qaddr + s * C::kQBytes, kb = kaddr + st * C::kKBytes;
+      } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer: S^T = K Q^T
+        if (lane == 0) {
+          const uint32_t idS = tc::idesc_bf16_f32(128, 128, false);
+          bool ok = tc::mbar_wait(&bars->q_full, rc & 1u, abort, p.wait_ns);
+          for (int j = 0; j < nkt && ok; ++j) {
+            const uint32_t k = kc + j, st = k % kStages;
+            if (!(ok = tc::mbar_wait(&bars->k_full[st], (k / kStages) & 1u, abort, p.wait_ns))) break;
+            const uint32_t kb = tc::smem_u32(smem + C::kOffK + st * C::kKBytes);
+            for (int m = 0; m < nm && ok; ++m) {
+              const uint32_t n = ni + j * nm + m, bf = n % kBufs, use = n / kBufs;
+              if (use > 0 && !(ok = tc::mbar_wait(&bars->s_free[bf], (use - 1) & 1u, abort, p.wait_ns))) break;
+              tc::fence_after_sync();
+              const uint32_t qb = tc::smem_u32(smem + C::kOffQ + m * C::kQBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc::mma_ss(tS[s], tc::sdesc_sw128(qb + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024), idS,
-                     kk > 0 ? 1u : 0u);
-        }
-      };
-      // D[buf] (+)= ONES * P_s : K = the 128 query rows of the M-tile, N = the 128 keys
-      auto issue_C = [&](int s, uint32_t buf, bool acc) {
-        const uint32_t pb = paddr + s * C::kPBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc::mma_ss(tD[buf], tc::sdesc_sw128(oaddr + (kk & 3) * 32, 16, 1024),
-                     tc::sdesc_sw128(pb + kk * 2048, 16384, 1024), idC, (acc || kk > 0) ? 1u : 0u);
-      };
-      for (uint32_t n = 0; ok; ++n) {
-        const int u = tc::queue_pop(&bars->queue, n, abort, ok);
-        if (u < 0) break;
-        int b, g, I;
-        unit_coords(p, u, b, g, I);
-        const int nkt = I / 2 + 1;
-        for (int r = 0; r < rounds && ok; ++r) {
-          bool act[2];
-          for (int s = 0; s < 2; ++s) {
-            act[s] = (2 * r + s) < MT;
-            if (act[s] && ok) {
-              ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort);
-              ++q_cnt[s];
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                tc::mma_ss(tmem_base + 128 * bf, tc::sdesc_sw128(kb + off, 16, 1024),
+                           tc::sdesc_sw128(qb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+              }
+              tc::mma_commit(&bars->s_full[bf]);
             }
+            tc::mma_commit(&bars->k_empty[st]);
+          }
+          if (ok) tc::mma_commit(&bars->q_empty);
+          else fail(abort, p.status);
+        }
+      } else if (warp >= 4) {
+        // ---------------------------------------------------------- softmax groups
+        const int grp = (warp - 4) >> 2;                 // 0: even M-tiles, 1: odd M-tiles
+        const int key = 32 * (warp & 3) + lane;          // TMEM lane = key of the tile
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        const float sc = p.scale_log2;
+        float* lse_r = s_lse + (rc & 1u) * kMaxMT * 128;
+        bool ok = true;
+        // this group's M-tiles' row LSEs (log2 units; rows past N never count)
+        for (int m = grp; m < nm; m += 2) {
+          const int h = g * p.G + 2 * (mt0 + m) + (key >> 6);
+          const int t = 64 * I + (key & 63);
+          lse_r[m * 128 + key] = t < p.N ? p.lse[((size_t)b * p.Hq + h) * p.N + t] * kLog2e : INFINITY;
+        }
+        if (grp == 0 && r == 0)
+          for (int i = 128 * nkt + key; i < p.N; i += 128) srow[i] = 0.0f;   // keys past the last tile
+        tc::mbar_arrive(&bars->rows_ready[grp]);
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->rows_ready[grp], rc & 1u, abort, p.wait_ns));
+        const bool two = nm >= 2;
+        for (int j = 0; j < nkt && ok; ++j) {
+          float acc = 0.0f;
+          const int kp = 128 * j + key;
+          for (int m = grp; m < nm; m += 2) {
+            const uint32_t n = ni + j * nm + m, bf = n % kBufs, use = n / kBufs;
+            if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[bf], use & 1u, abort, p.wait_ns)))) break;
+            tc::fence_after_sync();
+            const float* lr = lse_r + m * 128;
+            // causal: key kp counts for query column q when kp <= 64 I + (q & 63)
+            const int lim = kp - 64 * I;   // columns with (q & 63) >= lim are visible
+            float2 a2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll 2
+            for (int c = 0; c < 4; ++c) {
+              uint32_t v[32];
+              tc::tmem_ld32(tmem_base + 128 * bf + 32 * c + lane_off, v);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int q = 32 * c + 2 * e;
+                const float2 x = tc::ffma2(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])),
+                                           make_float2(sc, sc), make_float2(-lr[q], -lr[q + 1]));
+                float2 pv = (16 * c + e) % 4 < kPolyPairs / 16 ? tc::exp2_poly3_x2(x)
+                                                                : make_float2(exp2f(x.x), exp2f(x.y));
+                if (lim > 0) {
+                  pv.x = (q & 63) >= lim ? pv.x : 0.0f;
+                  pv.y = ((q + 1) & 63) >= lim ? pv.y : 0.0f;
+                }
+                a2[e & 1] = tc::fadd2(a2[e & 1], pv);
+              }
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&bars->s_free[bf]);
+            const float2 a = tc::fadd2(a2[0], a2[1]);
+            acc += a.x + a.y;
           }
           if (!ok) break;
-          uint32_t kst = k_it % kStages;
-          if (!(ok = tc::mbar_wait(&bars->k_full[kst], (k_it / kStages) & 1u, abort))) break;
-          ++k_it;
-          tc::fence_after_sync();
-          for (int s = 0; s < 2; ++s)
-            if (act[s]) {
-              issue_S(s, kst);
-              tc::mma_commit(&bars->s_full[s]);
-            }
-          tc::mma_commit(&bars->k_empty[kst]);
-          for (int tau = 1; tau <= nkt && ok; ++tau) {
-            // column sums of tile tau-1 into D[d_cnt & 1], then S of tile tau
-            const uint32_t buf = d_cnt & 1u;
-            if (!(ok = tc::mbar_wait(&bars->d_empty[buf], ((d_cnt >> 1) & 1u) ^ 1u, abort))) break;
-            bool have_k = false, first = true;
-            for (int s = 0; s < 2 && ok; ++s) {
-              if (!act[s]) continue;
-              if (!(ok = tc::mbar_wait(&bars->p_full[s], p_cnt[s] & 1u, abort))) break;
-              ++p_cnt[s];
-              tc::fence_after_sync();
-              issue_C(s, buf, !first);
-              first = false;
-              tc::mma_commit(&bars->p_empty[s]);
-              if (tau < nkt) {
-                if (!have_k) {
-                  kst = k_it % kStages;
-                  if (!(ok = tc::mbar_wait(&bars->k_full[kst], (k_it / kStages) & 1u, abort))) break;
-                  ++k_it;
-                  have_k = true;
-                  tc::fence_after_sync();
-                }
-                issue_S(s, kst);
-                tc::mma_commit(&bars->s_full[s]);
-              }
-            }
-            tc::mma_commit(&bars->d_full[buf]);
-            ++d_cnt;
-            if (have_k) tc::mma_commit(&bars->k_empty[kst]);
-          }
-          for (int s = 0; s < 2; ++s)
-            if (act[s]) tc::mma_commit(&bars->q_empty[s]);
-        }
-      }
-      if (!ok) fail(abort, p.status);
-      tc::mma_commit(&bars->mma_drain);
-      tc::mbar_wait(&bars->mma_drain, 0, abort, 100000000ull);
-    }
-  } else if (warp == 2 || warp == 3) {
-    // ============================================================== column-sum drain
-    // All rows of D are equal; warp w reads its own TMEM lane quarter and lane l keeps column l.
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const int half = warp - 2;  // columns [64*half, 64*half + 64)
-    const float inv = exp2f(-kPScaleLog2);
-    uint32_t d_cnt = 0;
-    bool ok = true;
-    for (uint32_t n = 0; ok; ++n) {
-      const int u = tc::queue_pop(&bars->queue, n, abort, ok);
-      ok = __all_sync(0xffffffffu, ok);   // warp-uniform: TMEM accesses are warp-collective
-      if (__any_sync(0xffffffffu, u < 0)) break;
-      int b, g, I;
-      unit_coords(p, u, b, g, I);
-      const int nkt = I / 2 + 1;
-      float* srow = p.scores + (((size_t)b * p.Hkv + g) * p.T + I) * (size_t)p.N;
-      // keys past the last key tile receive no probability
-      for (int i = 128 * nkt + 64 * half + lane; i < p.N; i += 64) srow[i] = 0.0f;
-      for (int r = 0; r < rounds && ok; ++r) {
-        for (int tau = 0; tau < nkt; ++tau) {
-          const uint32_t buf = d_cnt & 1u;
-          if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->d_full[buf], (d_cnt >> 1) & 1u, abort)))) break;
-          ++d_cnt;
-          tc::fence_after_sync();
-          uint32_t v0[32], v1[32];
-          tc::tmem_ld32(tmem_base + 256 + 128 * buf + 64 * half + lane_off, v0);
-          tc::tmem_ld32(tmem_base + 256 + 128 * buf + 64 * half + 32 + lane_off, v1);
-          tc::tmem_wait_ld();
-          float a = 0.0f, c = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            a = (i == lane) ? __uint_as_float(v0[i]) : a;
-            c = (i == lane) ? __uint_as_float(v1[i]) : c;
-          }
-          tc::fence_before_sync();
-          tc::mbar_arrive(&bars->d_empty[buf]);
-          const int i0 = 128 * tau + 64 * half + lane, i1 = i0 + 32;
-          if (i0 < p.N) srow[i0] = (r == 0 ? 0.0f : srow[i0]) + a * inv;
-          if (i1 < p.N) srow[i1] = (r == 0 ? 0.0f : srow[i1]) + c * inv;
-        }
-      }
-    }
-    if (!ok) fail(abort, p.status);
-  } else if (warp >= 4) {
-    // ============================================================== probabilities -> fp16 P in smem
-    const int s = (warp - 4) >> 2;
-    const int row = 32 * (warp & 3) + lane;
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tSrow = tmem_base + 128 * s + lane_off;
-    uint8_t* pbuf = smem + C::kOffP + s * C::kPBytes;
-    const float sc = p.scale_log2;
-    uint32_t s_cnt = 0, pe_cnt = 0;
-    bool ok = true;
-    for (uint32_t n = 0; ok; ++n) {
-      const int u = tc::queue_pop(&bars->queue, n, abort, ok);
-      ok = __all_sync(0xffffffffu, ok);   // warp-uniform: TMEM accesses are warp-collective
-      if (__any_sync(0xffffffffu, u < 0)) break;
-      int b, g, I;
-      unit_coords(p, u, b, g, I);
-      const int nkt = I / 2 + 1;
-      for (int r = 0; r < rounds && ok; ++r) {
-        const int mt = 2 * r + s;
-        if (mt >= MT) continue;
-        const int h = g * p.G + 2 * mt + (row >> 6);
-        const int t = 64 * I + (row & 63);
-        const bool valid = t < p.N;
-        // p * 2^12 = exp2(s * sc - LSE_t * log2(e) + 12); invalid rows contribute nothing
-        const float bias = valid ? kPScaleLog2 - p.lse[((size_t)b * p.Hq + h) * p.N + t] * kLog2e : -INFINITY;
-        for (int tau = 0; tau < nkt; ++tau) {
-          if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[s], s_cnt & 1u, abort)))) break;
-          ++s_cnt;
-          tc::fence_after_sync();
-          uint32_t r0[32], r1[32], r2[32], r3[32];
-          tc::tmem_ld32(tSrow + 0, r0);
-          tc::tmem_ld32(tSrow + 32, r1);
-          tc::tmem_ld32(tSrow + 64, r2);
-          tc::tmem_ld32(tSrow + 96, r3);
-          tc::tmem_wait_ld();
-          // P buffer of this slot is free once the previous column-sum MMA has read it
-          if (!(ok = tc::mbar_wait(&bars->p_empty[s], (pe_cnt & 1u) ^ 1u, abort))) break;
-          ++pe_cnt;
-          const int cmax = (tau == nkt - 1) ? t - 128 * tau : 127;  // causal: keys <= t
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {        // 64-key chunk
-#pragma unroll
-            for (int un = 0; un < 8; ++un) {      // 16-byte unit = 8 keys
-              uint32_t w[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int col = 64 * ch + 8 * un + 2 * e;
-                const uint32_t* src = ch == 0 ? (col < 32 ? r0 : r1) : (col < 96 ? r2 : r3);
-                const int ci = col & 31;
-                const float x0 = col <= cmax ? exp2f(fmaf(__uint_as_float(src[ci]), sc, bias)) : 0.0f;
-                const float x1 = col + 1 <= cmax ? exp2f(fmaf(__uint_as_float(src[ci + 1]), sc, bias)) : 0.0f;
-                w[e] = pack_f16x2(x0, x1);
-              }
-              // MN-major 128-byte swizzle: row `row`, 16-byte unit `un` of chunk `ch`
-              *reinterpret_cast<uint4*>(pbuf + ch * 16384 + row * 128 + ((un ^ (row & 7)) << 4)) =
-                  make_uint4(w[0], w[1], w[2], w[3]);
+          // combine the two groups' partials of key kp and write the score once
+          if (two) {
+            const uint32_t slot = (cc + j) & 1u, use = (cc + j) >> 1;
+            if (grp == 1) {
+              if (use > 0 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->comb_empty[slot], (use - 1) & 1u, abort, p.wait_ns))))
+                break;
+              s_red[slot * 128 + key] = acc;
+              tc::mbar_arrive(&bars->comb_full[slot]);
+            } else {
+              if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->comb_full[slot], use & 1u, abort, p.wait_ns)))) break;
+              acc += s_red[slot * 128 + key];
+              tc::mbar_arrive(&bars->comb_empty[slot]);
             }
           }
-          tc::fence_proxy_async_shared();  // generic-proxy writes -> visible to the tensor core
-          tc::fence_before_sync();
-          tc::mbar_arrive(&bars->p_full[s]);
+          if (grp == 0 && kp < p.N) srow[kp] = (r == 0 ? 0.0f : srow[kp]) + acc;
         }
+        if (!ok) fail(abort, p.status);
       }
+      ni += (uint32_t)(nkt * nm);
+      kc += (uint32_t)nkt;
+      cc += nm >= 2 ? (uint32_t)nkt : 0u;
+      ++rc;
     }
-    if (!ok) fail(abort, p.status);
+    __syncthreads();   // every role finished the unit (a failed wait set abort)
   }
 
+  // the MMAs and copies issued have completed before TMEM is released
+  if (warp == 1 && lane == 0) {
+    tc::mma_commit(&bars->mma_drain);
+    const uint64_t t0 = tc::globaltimer();
+    while (!tc::mbar_try_wait(&bars->mma_drain, 0) && tc::globaltimer() - t0 < 100000000ull) {
+    }
+  }
+  if (warp == 0 && lane == 0 && rc > 0) {
+    const uint32_t k = kc - 1;
+    const uint64_t t0 = tc::globaltimer();
+    while (!tc::mbar_try_wait(&bars->q_full, (rc - 1) & 1u) && tc::globaltimer() - t0 < 100000000ull) {
+    }
+    while (kc > 0 && !tc::mbar_try_wait(&bars->k_full[k % kStages], (k / kStages) & 1u) &&
+           tc::globaltimer() - t0 < 100000000ull) {
+    }
+  }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {
@@ -424,6 +344,13 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.counter = reinterpret_cast<int*>(ws);
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
+  // HYS_WATCHDOG_PROBE=1 (tests only) arms the probe above with a 0.2 s wait limit
+  static const bool probe = [] {
+    const char* e = getenv("HYS_WATCHDOG_PROBE");
+    return e != nullptr && e[0] == '1';
+  }();
+  p.probe = probe ? 1 : 0;
+  p.wait_ns = probe ? 200000000ull : 4000000000ull;
   const int smem = Cfg<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(token_scores_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
