@@ -85,13 +85,6 @@ __device__ __forceinline__ void fail(volatile int* abort, int* status) {
   report_status(status, HYS_ERR_TIMEOUT);
 }
 
-// Wait for a phase with a time limit only (no abort check): used after a failure, to let the
-// copies and MMAs already issued complete before the kernel leaves.
-__device__ __forceinline__ void wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  const uint64_t t0 = tc::globaltimer();
-  while (!tc::mbar_try_wait(bar, parity))
-    if (tc::globaltimer() - t0 > limit_ns) return;
-}
 
 // unit u -> (b, g, j), key tiles in increasing j across all (b, g) first: small j has the most
 // query tiles in the full and sparse modes, so the longest units start first
@@ -226,10 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) {
           fail(abort, p.status);
           // the copies already issued land before the kernel leaves
-          if (kv_issued) wait_bounded(&bars->kv_full, par, 100000000ull);
+          if (kv_issued) tc::mbar_wait_drain(&bars->kv_full, par);
           if (q_issued > 0) {
             const uint32_t n = q_issued - 1;
-            wait_bounded(&bars->q_full[n & 1u], (n >> 1) & 1u, 100000000ull);
+            tc::mbar_wait_drain(&bars->q_full[n & 1u], (n >> 1) & 1u);
           }
         }
       }
@@ -307,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // every MMA of the unit has completed before the next unit (or the TMEM release)
         tc::mma_commit(&bars->mma_drain);
-        wait_bounded(&bars->mma_drain, nu & 1u, 100000000ull);
+        tc::mbar_wait_drain(&bars->mma_drain, nu & 1u);
       }
     } else if (warp >= 4) {
       // ------------------------------------------------------------ softmax / drains

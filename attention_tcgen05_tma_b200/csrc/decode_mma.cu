@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         report_status(p.status, HYS_ERR_TIMEOUT);
       }
       for (int i = max(0, nlist - NS); i < nlist; ++i)
-        tc::mbar_wait(&full[i % NS], (i / NS) & 1, abort, 100000000ull);
+        tc::mbar_wait_drain(&full[i % NS], (i / NS) & 1);
     }
     cp_async_wait_all();
     __syncwarp();

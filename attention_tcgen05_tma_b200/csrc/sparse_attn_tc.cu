@@ -377,9 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       if (!ok) fail(abort, p.status);
       for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i)
-        tc::mbar_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u, abort, 100000000ull);
+        tc::mbar_wait_drain(&bars->kv_full[i % kStages], (i / kStages) & 1u);
       for (int s = 0; s < 2; ++s)
-        if (q_cnt[s] > 0) tc::mbar_wait(&bars->q_full[s], (q_cnt[s] - 1) & 1u, abort, 100000000ull);
+        if (q_cnt[s] > 0) tc::mbar_wait_drain(&bars->q_full[s], (q_cnt[s] - 1) & 1u);
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) fail(abort, p.status);
       tc::mma_commit(&bars->mma_drain);
-      tc::mbar_wait(&bars->mma_drain, 0, abort, 100000000ull);
+      tc::mbar_wait_drain(&bars->mma_drain, 0);
     }
   } else if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));

@@ -73,6 +73,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait for a phase with a time limit only, whatever the abort flag says: used once a role has
+// left its loop (possibly on an abort), so that the copies and MMAs it issued complete before
+// the kernel releases TMEM or leaves.  Returns false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 100000000ull) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > limit_ns) return false;
+  return true;
+}
+
 // ------------------------------------------------------------------ TMA
 // 3-D tiled load of one box into shared memory, completing on an mbarrier (tx bytes).
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1,

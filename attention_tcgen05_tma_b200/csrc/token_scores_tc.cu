@@ -289,18 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the MMAs and copies issued have completed before TMEM is released
   if (warp == 1 && lane == 0) {
     tc::mma_commit(&bars->mma_drain);
-    const uint64_t t0 = tc::globaltimer();
-    while (!tc::mbar_try_wait(&bars->mma_drain, 0) && tc::globaltimer() - t0 < 100000000ull) {
-    }
+    tc::mbar_wait_drain(&bars->mma_drain, 0);
   }
   if (warp == 0 && lane == 0 && rc > 0) {
-    const uint32_t k = kc - 1;
-    const uint64_t t0 = tc::globaltimer();
-    while (!tc::mbar_try_wait(&bars->q_full, (rc - 1) & 1u) && tc::globaltimer() - t0 < 100000000ull) {
-    }
-    while (kc > 0 && !tc::mbar_try_wait(&bars->k_full[k % kStages], (k / kStages) & 1u) &&
-           tc::globaltimer() - t0 < 100000000ull) {
-    }
+    tc::mbar_wait_drain(&bars->q_full, (rc - 1) & 1u);
+    if (kc > 0) tc::mbar_wait_drain(&bars->k_full[(kc - 1) % kStages], ((kc - 1) / kStages) & 1u);
   }
   tc::fence_before_sync();
   __syncthreads();
