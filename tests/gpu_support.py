@@ -88,7 +88,12 @@ def score_rel_err(oracle_scores: np.ndarray, gpu_scores: np.ndarray, floor: floa
 # Gradients: the largest error relative to the gradient's largest element.  bf16 inputs: 2e-2 (the
 # bound set for bf16 attention outputs; P and dS are rounded to bf16 before the contractions and dq is
 # stored in bf16, each a relative 2^-9 per term); fp32 inputs (fp32 kernels throughout): 1e-4.
+# dq of bf16 inputs: 5e-2.  The backward forms D_t = dO_t . o_t from the forward's stored bf16 output
+# o; its rounding (2^-9 relative per element) shifts D_t by dD_t and dq_t by tau dD_t sum_i P_ti k_i,
+# which the planted keys (norm 3 sqrt(D), far above the others) carry to 2.5% of max|dq| with every
+# other step exact (a float64 emulation of just that step on the 2 x 300 ragged case).
 GRAD_TOL = {"f32": 1e-4, "bf16": 2e-2}
+DQ_TOL = {"f32": 1e-4, "bf16": 5e-2}
 
 
 def grad_err(gpu: np.ndarray, ref: np.ndarray) -> float:

@@ -11,7 +11,7 @@ import oracle as O
 from oracle import hysparse_backward as OB
 from attention_tcgen05_tma_b200 import hysparse as H
 from attention_tcgen05_tma_b200 import inputs as I
-from tests.gpu_support import GRAD_TOL, TOL, grad_err, to_dev, to_np
+from tests.gpu_support import DQ_TOL, GRAD_TOL, TOL, grad_err, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -49,11 +49,14 @@ def test_full_layer_backward(case):
     assert H.hysparse_get_device_status() == 0
     ref_q, ref_k, ref_v = OB.full_attention_backward(a["q"], a["k"], a["v"], a["d_o"])
     tol = GRAD_TOL[dt]
-    assert grad_err(to_np(dq), ref_q) <= tol, grad_err(to_np(dq), ref_q)
+    assert grad_err(to_np(dq), ref_q) <= DQ_TOL[dt], grad_err(to_np(dq), ref_q)
     assert grad_err(to_np(dk), ref_k) <= tol, grad_err(to_np(dk), ref_k)
     assert grad_err(to_np(dv), ref_v) <= tol, grad_err(to_np(dv), ref_v)
-    assert torch.allclose(dk2 - base_k, dk, atol=1e-5 * float(dk.abs().max())) and \
-        torch.allclose(dv2 - base_v, dv, atol=1e-5 * float(dv.abs().max()))
+    # the kernels are deterministic: the accumulated result is the buffer plus the same gradient, up
+    # to the rounding of that one fp32 addition (a fused multiply-add may skip the product's rounding)
+    ulp = 1.2e-7
+    assert torch.allclose(dk2, base_k + dk, rtol=0, atol=4 * ulp * float(base_k.abs().max()))
+    assert torch.allclose(dv2, base_v + dv, rtol=0, atol=4 * ulp * float(base_v.abs().max()))
 
 
 def _branch_lse(q_s, k, v, idx, k_swa, window, sinks, G, block=64):
@@ -132,7 +135,7 @@ def test_sparse_layer_train_and_backward(case, with_sinks):
         checks["dsinks"] = to_np(dsinks)
     for key, val in checks.items():
         e = grad_err(val, ref[key])
-        assert e <= tol, (key, e)
+        assert e <= (DQ_TOL[dt] if key == "dq" else tol), (key, e)
 
 
 def test_hybrid_block_backward():
@@ -160,9 +163,9 @@ def test_hybrid_block_backward():
                                          gate=a["gate"][l], d_o=a["d_o_sparse"][l]) for l in range(w.layers)],
                                    w.window)
     tol = GRAD_TOL[dt]
-    assert grad_err(to_np(dq), ref["dq"]) <= tol
+    assert grad_err(to_np(dq), ref["dq"]) <= DQ_TOL[dt]
     assert grad_err(to_np(dk), ref["dk"]) <= tol
     assert grad_err(to_np(dv), ref["dv"]) <= tol
     for l in range(w.layers):
-        assert grad_err(to_np(layers[l][0]), ref["layers"][l]["dq"]) <= tol
+        assert grad_err(to_np(layers[l][0]), ref["layers"][l]["dq"]) <= DQ_TOL[dt]
         assert grad_err(to_np(layers[l][3]), ref["layers"][l]["dgate"]) <= tol
