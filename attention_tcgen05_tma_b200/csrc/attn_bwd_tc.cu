@@ -22,9 +22,10 @@
 // from TMEM to an fp32 accumulator in global memory with vector reductions (red.add), scaled by
 // tau and rounded to the output type afterwards.
 //
-// Warp roles (256 threads): warp 0 TMA producer (K_j, V_j once per unit; Q and dO of every
-// M-tile, two stages), warp 1 MMA issuer (and TMEM owner), warps 4-7 softmax and drains (thread
-// = key row r of the tile = TMEM lane).  TMEM: tS (S^T, then sigma P^T as bf16), tP (dP^T, then
+// Warp roles (384 threads): warp 0 TMA producer (K_j, V_j once per unit; Q and dO of every
+// M-tile, two stages), warp 1 MMA issuer (and TMEM owner), warps 4-7 and 8-11 two softmax and
+// drain groups (thread = key row r of the tile = TMEM lane; each group takes half of the row's
+// query columns, and half of the head-dim columns in the drains).  TMEM: tS (S^T, then sigma P^T as bf16), tP (dP^T, then
 // dS^T as bf16, then the M-tile's dQ part), tdV, tdK: 4 x 128 columns.  The MMA order per M-tile
 // is dV, dK, dQ (into tP), then S^T of the next M-tile into tS, which overlaps the drain of dQ.
 // Every mbarrier wait is bounded; a timeout records HYS_ERR_TIMEOUT, waits (bounded) for the
@@ -39,7 +40,7 @@
 namespace hys {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4-7 / 8-11 softmax groups
 constexpr int kD = 128;
 constexpr int kMaxGrid = 148;
 constexpr int kTile = 128 * kD * 2;  // 128 rows x 128 bf16: two 64-column swizzled chunks of 16 KB
@@ -70,7 +71,7 @@ struct Params {
 
 struct Bars {
   uint64_t kv_full, kv_empty, q_full[2], q_empty[2], s_full, p_full, dq_full, s_free, ds_free, acc_full, acc_free;
-  uint64_t mma_drain, rows_ready;
+  uint64_t mma_drain, rows_ready[2];
 };
 
 constexpr int kOffK = 0, kOffV = kTile, kOffQ = 2 * kTile, kOffDO = 4 * kTile, kOffDS = 6 * kTile;
@@ -145,14 +146,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->q_empty[s], 1);
     }
     tc::mbar_init(&bars->s_full, 1);
-    tc::mbar_init(&bars->p_full, 128);
+    tc::mbar_init(&bars->p_full, 256);
     tc::mbar_init(&bars->dq_full, 1);
-    tc::mbar_init(&bars->s_free, 128);
+    tc::mbar_init(&bars->s_free, 256);
     tc::mbar_init(&bars->ds_free, 1);
     tc::mbar_init(&bars->acc_full, 1);
-    tc::mbar_init(&bars->acc_free, 128);
+    tc::mbar_init(&bars->acc_free, 256);
     tc::mbar_init(&bars->mma_drain, 1);
-    tc::mbar_init(&bars->rows_ready, 128);
+    tc::mbar_init(&bars->rows_ready[0], 128);
+    tc::mbar_init(&bars->rows_ready[1], 128);
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -304,6 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp >= 4) {
       // ------------------------------------------------------------ softmax / drains
+      // Two groups share every M-tile: group wg takes the query columns (and, in the drains, the
+      // head-dim columns) [64 wg, 64 wg + 64) of the thread's TMEM lane.
+      const int wg = (warp - 4) >> 2;
       const int r = 32 * (warp & 3) + lane;              // TMEM lane: key row, later query row
       const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
       const int kp = 128 * j + r;                        // this thread's key position
@@ -312,20 +317,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t n = mc + m;
         int i, hp, mask;
         mtile<MODE>(p, j, lu, m, i, hp, mask);
-        // the M-tile's row statistics (row r: head 2hp + r/64, position 64i + r%64)
-        {
-          const int head = b * p.Hq + g * p.G + 2 * hp + (r >> 6);
-          const int pos = 64 * i + (r & 63);
+        // the statistics of this group's 64 query rows (head 2hp + wg, positions 64i ..)
+        if (r < 64) {
+          const int q = 64 * wg + r;
+          const int head = b * p.Hq + g * p.G + 2 * hp + wg;
+          const int pos = 64 * i + r;
           const size_t rix = (size_t)head * p.N + pos;
-          s_lse[r] = pos < p.N ? p.lse2[rix] : INFINITY;
-          s_dsum[r] = pos < p.N ? p.dsum[rix] : 0.0f;
-          s_sig[r] = (pos < p.N && p.sig != nullptr) ? p.sig[rix] : 1.0f;
+          s_lse[q] = pos < p.N ? p.lse2[rix] : INFINITY;
+          s_dsum[q] = pos < p.N ? p.dsum[rix] : 0.0f;
+          s_sig[q] = (pos < p.N && p.sig != nullptr) ? p.sig[rix] : 1.0f;
         }
-        // all 128 rows written (a bounded wait: a warp that left on a failed wait cannot block the
-        // others); the previous M-tile's values were read by every thread before its p_full arrival,
-        // which the dq_full wait above covered
-        tc::mbar_arrive(&bars->rows_ready);
-        if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->rows_ready, n & 1u, abort)))) break;
+        // the group's rows written (a bounded wait: a warp that left on a failed wait cannot block
+        // the others); the previous M-tile's values were read by every thread before its p_full
+        // arrival, which the previous dq_full wait covered
+        tc::mbar_arrive(&bars->rows_ready[wg]);
+        if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->rows_ready[wg], n & 1u, abort)))) break;
         if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full, n & 1u, abort)))) break;
         if (n > 0 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->ds_free, (n - 1) & 1u, abort)))) break;
         tc::fence_after_sync();
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the causal line (and the window's lower edge)
         const bool row_on = kp < p.N && (MODE != kModeSparse || ((mask >> (r >> 6)) & 1));
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {                      // 32 query columns per chunk
+        for (int c = 2 * wg; c < 2 * wg + 2; ++c) {        // 32 query columns per chunk
           uint32_t sr[32], dr[32];
           tc::tmem_ld32(tS + 32 * c + lane_off, sr);
           tc::tmem_ld32(tP + 32 * c + lane_off, dr);
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int pos = 64 * i + (r & 63);
           float* dqrow = p.dq + ((size_t)head * p.N + pos) * kD;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 2 * wg; c < 2 * wg + 2; ++c) {      // this group's 64 head-dim columns
             uint32_t v[32];
             tc::tmem_ld32(tP + 32 * c + lane_off, v);
             tc::tmem_wait_ld();
@@ -404,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* dst = (t2 ? p.dv : p.dk) + (((size_t)b * p.Hkv + g) * p.N + kp) * kD;
           const float f = t2 ? 1.0f : p.tau;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 2 * wg; c < 2 * wg + 2; ++c) {
             uint32_t v[32];
             tc::tmem_ld32(tsrc + 32 * c + lane_off, v);
             tc::tmem_wait_ld();

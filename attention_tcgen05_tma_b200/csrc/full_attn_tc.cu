@@ -53,7 +53,7 @@ constexpr int kPolyPairs = HYS_FULL_POLY_PAIRS;
 // kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
 // the host checks the compiled register count before every launch.
 #ifndef HYS_FULL_LOW_REGS
-#define HYS_FULL_LOW_REGS 88
+#define HYS_FULL_LOW_REGS 104
 #endif
 constexpr int kLaunchRegs = 168, kLowRegs = HYS_FULL_LOW_REGS, kHighRegs = (3 * kLaunchRegs - kLowRegs) / 2;
 static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multiples of 8");

@@ -33,7 +33,7 @@ constexpr int kMaxMT = 4;         // M-tiles resident per round
 constexpr int kBufs = 4;          // TMEM buffers of 128 columns
 constexpr int kMaxGrid = 148;
 #ifndef HYS_TSCORE_POLY_PAIRS
-#define HYS_TSCORE_POLY_PAIRS 16
+#define HYS_TSCORE_POLY_PAIRS 24
 #endif
 // column pairs (of the 64 in a 128-row item) whose exp2 runs on the FMA pipe instead of MUFU
 constexpr int kPolyPairs = HYS_TSCORE_POLY_PAIRS;

@@ -40,7 +40,7 @@ constexpr int kPolyPairs = HYS_TOKEN_POLY_PAIRS;
 // kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
 // the host checks the compiled register count before every launch.
 #ifndef HYS_TOKEN_LOW_REGS
-#define HYS_TOKEN_LOW_REGS 88
+#define HYS_TOKEN_LOW_REGS 104
 #endif
 constexpr int kLaunchRegs = 168, kLowRegs = HYS_TOKEN_LOW_REGS, kHighRegs = (3 * kLaunchRegs - kLowRegs) / 2;
 static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multiples of 8");
