@@ -107,10 +107,13 @@ __device__ __forceinline__ int num_qtiles(const Params& p, int j, int lu) {
   return p.list_cnt[lu];
 }
 
-// query tile and key-half mask of the unit's M-tile m
+// query tile and key-half mask of the unit's M-tile m.  The query tiles run from the last one
+// down: the units running at the same time then reach the same query tiles (and the same dQ
+// accumulator rows) together, so the accumulator's vector reductions mostly hit L2.
 template <int MODE>
-__device__ __forceinline__ void mtile(const Params& p, int j, int lu, int m, int& i, int& hp, int& mask) {
-  const int n = m / p.MT;
+__device__ __forceinline__ void mtile(const Params& p, int j, int lu, int m, int nmt, int& i, int& hp,
+                                      int& mask) {
+  const int n = (nmt - 1 - m) / p.MT;
   hp = m % p.MT;
   if (MODE == kModeSparse) {
     const int e = p.list[(size_t)lu * p.T + n];
@@ -206,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int m = 0; m < nmt && ok; ++m) {
           const uint32_t n = mc + m, st = n & 1u;
           int i, hp, mask;
-          mtile<MODE>(p, j, lu, m, i, hp, mask);
+          mtile<MODE>(p, j, lu, m, nmt, i, hp, mask);
           if (!(ok = tc::mbar_wait(&bars->q_empty[st], ((n >> 1) & 1u) ^ 1u, abort))) break;
           tc::mbar_arrive_expect_tx(&bars->q_full[st], 2 * kTile);
           for (int hh = 0; hh < 2; ++hh)
@@ -270,12 +273,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::fence_after_sync();
           const uint32_t qb = tc::smem_u32(smem + kOffQ + st * kTile);
           const uint32_t dob = tc::smem_u32(smem + kOffDO + st * kTile);
+          // A operands in TMEM: query rows 0-63 packed at columns 0-31, rows 64-127 at 64-95
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)   // dV += (sigma P)^T dO : K = 128 query rows, 16 per step
-            tc::mma_ts(tdV, tS + kk * 8, tc::sdesc_sw128(dob + kk * 2048, 16384, 1024), idAcc, (m > 0 || kk > 0));
+            tc::mma_ts(tdV, tS + kk * 8 + (kk >= 4 ? 32 : 0), tc::sdesc_sw128(dob + kk * 2048, 16384, 1024), idAcc,
+                       (m > 0 || kk > 0));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)   // dK += dS^T Q
-            tc::mma_ts(tdK, tP + kk * 8, tc::sdesc_sw128(qb + kk * 2048, 16384, 1024), idAcc, (m > 0 || kk > 0));
+            tc::mma_ts(tdK, tP + kk * 8 + (kk >= 4 ? 32 : 0), tc::sdesc_sw128(qb + kk * 2048, 16384, 1024), idAcc,
+                       (m > 0 || kk > 0));
           tc::mma_commit(&bars->q_empty[st]);   // Q_m, dO_m free once these complete
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)   // dQ part = dS K_j : K = 128 keys, 16 per step, into tP
@@ -313,19 +319,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
       const int kp = 128 * j + r;                        // this thread's key position
       bool ok = true;
+      // the statistics of this group's 64 query rows of an M-tile (head 2hp + wg, positions 64i ..),
+      // loaded one M-tile ahead so that their latency overlaps the previous M-tile
+      float nl = INFINITY, nd = 0.0f, ns = 1.0f;
+      auto load_rows = [&](int m) {
+        int i, hp, mask;
+        mtile<MODE>(p, j, lu, m, nmt, i, hp, mask);
+        const int head = b * p.Hq + g * p.G + 2 * hp + wg;
+        const int pos = 64 * i + (r & 63);
+        const size_t rix = (size_t)head * p.N + pos;
+        nl = pos < p.N ? p.lse2[rix] : INFINITY;
+        nd = pos < p.N ? p.dsum[rix] : 0.0f;
+        ns = (pos < p.N && p.sig != nullptr) ? p.sig[rix] : 1.0f;
+      };
+      if (r < 64) load_rows(0);
       for (int m = 0; m < nmt && ok; ++m) {
         const uint32_t n = mc + m;
         int i, hp, mask;
-        mtile<MODE>(p, j, lu, m, i, hp, mask);
-        // the statistics of this group's 64 query rows (head 2hp + wg, positions 64i ..)
+        mtile<MODE>(p, j, lu, m, nmt, i, hp, mask);
         if (r < 64) {
           const int q = 64 * wg + r;
-          const int head = b * p.Hq + g * p.G + 2 * hp + wg;
-          const int pos = 64 * i + r;
-          const size_t rix = (size_t)head * p.N + pos;
-          s_lse[q] = pos < p.N ? p.lse2[rix] : INFINITY;
-          s_dsum[q] = pos < p.N ? p.dsum[rix] : 0.0f;
-          s_sig[q] = (pos < p.N && p.sig != nullptr) ? p.sig[rix] : 1.0f;
+          s_lse[q] = nl;
+          s_dsum[q] = nd;
+          s_sig[q] = ns;
+          if (m + 1 < nmt) load_rows(m + 1);
         }
         // the group's rows written (a bounded wait: a warp that left on a failed wait cannot block
         // the others); the previous M-tile's values were read by every thread before its p_full
@@ -361,8 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[e] = tc::pack_bf16x2(pv[0], pv[1]);
             dk2[e] = tc::pack_bf16x2(dv[0], dv[1]);
           }
-          tc::tmem_st16(tS + 16 * c + lane_off, pk);
-          tc::tmem_st16(tP + 16 * c + lane_off, dk2);
+          // packed bf16 pairs over this group's own fp32 columns, behind its reads (the other group
+          // is still reading its half): group wg's 32 packed columns start at column 64 wg
+          tc::tmem_st16(tS + 64 * wg + 16 * (c - 2 * wg) + lane_off, pk);
+          tc::tmem_st16(tP + 64 * wg + 16 * (c - 2 * wg) + lane_off, dk2);
           // dS^T into shared memory (the dQ MMA's MN-major A): 16-byte units of 8 query columns,
           // 128-byte swizzle by key row
 #pragma unroll
