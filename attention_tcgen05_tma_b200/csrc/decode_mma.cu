@@ -69,6 +69,13 @@ constexpr int kTargetCtas = 4 * 148;
 #ifndef HYS_DECODE_SPARSE_BPS
 #define HYS_DECODE_SPARSE_BPS 32
 #endif
+#ifndef HYS_DECODE_SPLIT_MAJOR
+#define HYS_DECODE_SPLIT_MAJOR 0
+#endif
+// grid of the split kernel: (splits, Hkv, B), or (Hkv, B, splits) with HYS_DECODE_SPLIT_MAJOR
+__host__ __forceinline__ dim3 split_grid(int nsplit, int Hkv, int B) {
+  return HYS_DECODE_SPLIT_MAJOR ? dim3(Hkv, B, nsplit) : dim3(nsplit, Hkv, B);
+}
 constexpr int kSparseBps = HYS_DECODE_SPARSE_BPS;   // selected blocks per sparse-layer split (<= 32)
 static_assert(kSparseBps <= 32 && kSparseBps <= kMaxList, "one warp gathers a split's entries");
 
@@ -179,7 +186,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   volatile int* abort = s_nlist + 1;
   int* tok = reinterpret_cast<int*>(smem + kStages * kStageBytes + kMaxList * 16 + 256);   // mode 2 token rows
 
+#if HYS_DECODE_SPLIT_MAJOR
+  const int sp = blockIdx.z, g = blockIdx.x, b = blockIdx.y;   // every (b, g)'s first split launches first
+#else
   const int sp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+#endif
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Lb = p.seqlens ? max(1, min(p.seqlens[b], p.L)) : p.L;
 
@@ -775,7 +786,7 @@ cudaError_t launch_decode_full_mma(const DecodeDims& d, const void* q, const voi
   fill_common(p, d, q, seqlens, ws, nsplit);
   p.mode = 0;
   p.bps = bps;
-  decode_split_kernel<false><<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  decode_split_kernel<false><<<split_grid(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), scores,
@@ -804,7 +815,7 @@ cudaError_t launch_decode_sparse_mma(const DecodeDims& d, const void* q, const v
   p.W = W;
   p.swa_len = swa_len;
   p.sinks = sinks;
-  decode_split_kernel<false><<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
+  decode_split_kernel<false><<<split_grid(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mkr, mvr, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, gate, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
@@ -838,7 +849,7 @@ cudaError_t full_tokens(const DecodeDims& d, const void* q, const void* kc, cons
   p.v_scale = v_scale;
   p.logits = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + logits_offset(d));
   p.tok_scores = tok_scores;
-  decode_split_kernel<F8><<<dim3(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  decode_split_kernel<F8><<<split_grid(nsplit, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
@@ -891,7 +902,7 @@ cudaError_t sparse_tokens(const DecodeDims& d, const void* q, const void* kc, co
   p.vc = reinterpret_cast<const uint8_t*>(vc);
   p.k_scale = k_scale;
   p.v_scale = v_scale;
-  decode_split_kernel<F8><<<dim3(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
+  decode_split_kernel<F8><<<split_grid(nsp + 1, d.Hkv, d.B), kThreads, kSmemBytes, s>>>(mk, mv, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<<<dim3(d.Hkv, d.B), 256, 0, s>>>(p, nullptr, reinterpret_cast<__nv_bfloat16*>(o), nullptr, 0);
