@@ -70,7 +70,7 @@ constexpr int kTargetCtas = 4 * 148;
 #define HYS_DECODE_SPARSE_BPS 32
 #endif
 #ifndef HYS_DECODE_SPLIT_MAJOR
-#define HYS_DECODE_SPLIT_MAJOR 0
+#define HYS_DECODE_SPLIT_MAJOR 1
 #endif
 // grid of the split kernel: (splits, Hkv, B), or (Hkv, B, splits) with HYS_DECODE_SPLIT_MAJOR
 __host__ __forceinline__ dim3 split_grid(int nsplit, int Hkv, int B) {
