@@ -44,7 +44,7 @@ constexpr int kMaxNB = 2048;       // score accumulator capacity per slot (N <= 
 constexpr int kMaxGrid = 148;      // B200 SM count; the workspace is sized for this grid
 constexpr float kRescaleLog2 = 8.0f;
 #ifndef HYS_FULL_POLY_PAIRS
-#define HYS_FULL_POLY_PAIRS 8
+#define HYS_FULL_POLY_PAIRS 4
 #endif
 // column pairs (of the 64 in a 128-key row) whose exp2 runs on the FMA pipe instead of MUFU
 constexpr int kPolyPairs = HYS_FULL_POLY_PAIRS;

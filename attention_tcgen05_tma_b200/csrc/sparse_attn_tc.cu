@@ -47,7 +47,7 @@ constexpr int kMaxGrid = 148;
 constexpr int kMaxKb = 1024;
 constexpr float kRescaleLog2 = 8.0f;
 #ifndef HYS_SPARSE_POLY_PAIRS
-#define HYS_SPARSE_POLY_PAIRS 8
+#define HYS_SPARSE_POLY_PAIRS 4
 #endif
 // column pairs (of the 64 in a 128-key row) whose exp2 runs on the FMA pipe instead of MUFU
 constexpr int kPolyPairs = HYS_SPARSE_POLY_PAIRS;
