@@ -19,8 +19,9 @@
 // so that dV = sum_t sigma_t P_ti dO_t, dK = tau sum_t dS_ti q_t and dQ = tau sum_i dS_ti k_i are
 // the gradients of o = sigma * softmax(tau q k^T) v with D_t = sigma_t dO_t . o_t.  dK_j and dV_j
 // stay in TMEM for the whole unit and are written (or added) once; every M-tile's dQ part goes
-// from TMEM to an fp32 accumulator in global memory with vector reductions (red.add), scaled by
-// tau and rounded to the output type afterwards.
+// from TMEM through shared memory (the dS^T buffer, free once the dQ MMA has read it) to an fp32
+// accumulator in global memory with TMA reduce-adds, scaled by tau and rounded to the output type
+// afterwards.
 //
 // Warp roles (384 threads): warp 0 TMA producer (K_j, V_j once per unit; Q and dO of every
 // M-tile, two stages), warp 1 MMA issuer (and TMEM owner), warps 4-7 and 8-11 two softmax and
@@ -72,6 +73,7 @@ struct Params {
 struct Bars {
   uint64_t kv_full, kv_empty, q_full[2], q_empty[2], s_full, p_full, dq_full, s_free, ds_free, acc_full, acc_free;
   uint64_t mma_drain, rows_ready[2];
+  uint64_t stage_ready[2], stage_free[2];   // per group: its dQ stage written / read by the TMA reduce
 };
 
 constexpr int kOffK = 0, kOffV = kTile, kOffQ = 2 * kTile, kOffDO = 4 * kTile, kOffDS = 6 * kTile;
@@ -129,7 +131,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                       const Params p) {
+                       const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
@@ -158,6 +160,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bars->mma_drain, 1);
     tc::mbar_init(&bars->rows_ready[0], 128);
     tc::mbar_init(&bars->rows_ready[1], 128);
+    for (int w = 0; w < 2; ++w) {
+      tc::mbar_init(&bars->stage_ready[w], 128);
+      tc::mbar_init(&bars->stage_free[w], 1);
+    }
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -166,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::prefetch_tensormap(&tmDO);
     tc::prefetch_tensormap(&tmK);
     tc::prefetch_tensormap(&tmV);
+    tc::prefetch_tensormap(&tmDQ);
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, 512);
@@ -396,27 +403,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_proxy_async_shared();   // dS^T shared-memory writes -> the MMA (async proxy)
         tc::fence_before_sync();
         tc::mbar_arrive(&bars->p_full);
-        // dQ part of query row r (TMEM lane r of tP): 128 fp32 columns -> vector reductions
+        // dQ part (TMEM lane r of tP = query row r, 128 fp32 columns): the group's two 32-column
+        // chunks go through its half of the dS^T buffer (free: the dQ MMA has read it) into the
+        // fp32 accumulator with TMA reduce-adds, one 64-row box per head
         if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->dq_full, n & 1u, abort)))) break;
         tc::fence_after_sync();
         {
-          const int head = b * p.Hq + g * p.G + 2 * hp + (r >> 6);
-          const int pos = 64 * i + (r & 63);
-          float* dqrow = p.dq + ((size_t)head * p.N + pos) * kD;
+          uint8_t* stg = smem + kOffDS + wg * 16384;
+          const bool elected = (warp & 3) == 0 && lane == 0;
+          const int head0 = b * p.Hq + g * p.G + 2 * hp;
 #pragma unroll 1
-          for (int c = 2 * wg; c < 2 * wg + 2; ++c) {      // this group's 64 head-dim columns
+          for (int cc = 0; cc < 2 && ok; ++cc) {
+            const int c = 2 * wg + cc;
             uint32_t v[32];
             tc::tmem_ld32(tP + 32 * c + lane_off, v);
             tc::tmem_wait_ld();
-            if (pos < p.N) {
+            // the previous round's box has been read out of the stage
+            if (cc > 0 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->stage_free[wg], 0u, abort)))) break;
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dqrow + 32 * c + 4 * e),
-                             "f"(__uint_as_float(v[4 * e])), "f"(__uint_as_float(v[4 * e + 1])),
-                             "f"(__uint_as_float(v[4 * e + 2])), "f"(__uint_as_float(v[4 * e + 3]))
-                             : "memory");
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) =
+                  make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+            tc::fence_proxy_async_shared();   // generic shared-memory writes -> the TMA (async proxy)
+            tc::mbar_arrive(&bars->stage_ready[wg]);
+            if (elected) {
+              if (tc::mbar_wait(&bars->stage_ready[wg], (uint32_t)cc, abort)) {
+                tc::tma_reduce_add_3d(&tmDQ, stg, 32 * c, 64 * i, head0);
+                tc::tma_reduce_add_3d(&tmDQ, stg + 8192, 32 * c, 64 * i, head0 + 1);
+                tc::bulk_commit_group();
+                tc::bulk_wait_group_read0();
+              }
+              tc::mbar_arrive(&bars->stage_free[wg]);
             }
           }
+          // the stage is free again before this group writes the next M-tile's dS^T into it
+          if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->stage_free[wg], 1u, abort));
+          if (!ok) break;
         }
         tc::fence_before_sync();
         tc::mbar_arrive(&bars->s_free);
@@ -461,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();   // every role finished the unit (a failed wait set abort)
   }
 
+  if (warp >= 4 && (warp & 3) == 0 && lane == 0) tc::bulk_wait_group0();   // the dQ reductions have landed
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {
@@ -517,14 +540,29 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int heads, int box_row
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [heads][rows][128] fp32 (the dQ accumulator), box = 32 columns x 64 rows x 1 head, 128-byte
+// swizzle: the target of the TMA reduce-adds
+bool make_map_f32(CUtensorMap* m, const void* base, int rows, int heads) {
+  EncodeTiledFn fn = tma_encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {512, (cuuint64_t)rows * 512};
+  cuuint32_t box[3] = {32, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int MODE>
 cudaError_t launch_mode(const PrefillDims& d, const void* q, const void* d_o, const void* k, const void* v,
                         const float* lse2, const float* dsum, const float* sig, float* dq_acc, float* dk, float* dv,
                         int accumulate, int window, const int* list, const int* list_cnt, int* counter,
                         cudaStream_t s) {
-  CUtensorMap mq, mdo, mk, mv;
+  CUtensorMap mq, mdo, mk, mv, mdq;
   if (!make_map(&mq, q, d.N, d.B * d.Hq, 64) || !make_map(&mdo, d_o, d.N, d.B * d.Hq, 64) ||
-      !make_map(&mk, k, d.N, d.B * d.Hkv, 128) || !make_map(&mv, v, d.N, d.B * d.Hkv, 128))
+      !make_map(&mk, k, d.N, d.B * d.Hkv, 128) || !make_map(&mv, v, d.N, d.B * d.Hkv, 128) ||
+      !make_map_f32(&mdq, dq_acc, d.N, d.B * d.Hq))
     return cudaErrorInvalidValue;
   Params p;
   p.B = d.B;
@@ -555,7 +593,7 @@ cudaError_t launch_mode(const PrefillDims& d, const void* q, const void* d_o, co
   e = cudaFuncSetAttribute(attn_bwd_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.num_units < kMaxGrid ? p.num_units : kMaxGrid;
-  attn_bwd_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(mq, mdo, mk, mv, p);
+  attn_bwd_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(mq, mdo, mk, mv, mdq, p);
   return cudaGetLastError();
 }
 
