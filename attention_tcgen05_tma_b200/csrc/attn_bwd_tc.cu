@@ -111,7 +111,7 @@ __device__ __forceinline__ int num_qtiles(const Params& p, int j, int lu) {
 
 // query tile and key-half mask of the unit's M-tile m.  The query tiles run from the last one
 // down: the units running at the same time then reach the same query tiles (and the same dQ
-// accumulator rows) together, so the accumulator's vector reductions mostly hit L2.
+// accumulator rows) together, so the accumulator's reduce-adds mostly hit L2.
 template <int MODE>
 __device__ __forceinline__ void mtile(const Params& p, int j, int lu, int m, int nmt, int& i, int& hp,
                                       int& mask) {

@@ -202,7 +202,7 @@ HYS_API hys_status hysparse_sparse_attn_rows(const hys_shape* shape, hys_dtype d
  * (1 - sigmoid(g_b)) dO.o_b; a sink logit's gradient is -sum_t p_sink,t sigmoid(g_b) dO_t.o_b,t.
  * Key and value gradients are fp32 (they are sums over layers and heads); dq takes the input
  * type.  bf16 with D = 128 and an even group size runs on the tensor cores (key-major tcgen05
- * kernel, dQ accumulated in fp32 with vector reductions); other shapes and fp32 run SIMT
+ * kernel, dQ accumulated in fp32 by TMA reduce-adds); other shapes and fp32 run SIMT
  * fp32-accumulate kernels.
  * ------------------------------------------------------------------------------------ */
 
