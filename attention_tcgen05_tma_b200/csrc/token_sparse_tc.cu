@@ -13,8 +13,21 @@
 //     part B travel as a bitmask published with the unit.
 // The rest follows the full-layer kernel: 128-row M-tiles of two heads x 64 positions, two
 // in flight, S and O in TMEM, P written back over S, one online softmax, O / l at the end.
+//
+// Gathers bound the layer (one TMA instruction per four 128-byte rows).  With four or more
+// M-tiles per unit a single CTA needs two rounds over the unit's keys and gathers every tile
+// twice, so such units run on a CTA pair (a cluster of two): both CTAs walk the same key
+// tiles, each gathers half of every tile's rows (part B: half-tile boxes) and sends that half
+// into the partner's stage with a shared-to-shared bulk copy, and each CTA computes two of the
+// unit's M-tiles.  A stage is free again once both CTAs' MMAs have read it (the MMA warp's
+// commit arrives on the stage barrier of both CTAs).  Every key row then crosses the TMA unit
+// once per unit instead of once per round.
 #include <cuda.h>
 
+#include <algorithm>
+#include <atomic>
+
+#include "cluster_ptx.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "tma_host.h"
@@ -30,6 +43,9 @@ constexpr int kMaxGrid = 148;
 constexpr int kMaskWords = 16;     // extended window <= 512 keys  ->  W <= 449
 constexpr int kMaxList = 4096;     // selected positions kept in shared memory (larger k: read from L2)
 constexpr float kRescaleLog2 = 8.0f;
+#ifndef HYS_TOKEN_PAIR
+#define HYS_TOKEN_PAIR 1
+#endif
 #ifndef HYS_TOKEN_POLY_PAIRS
 #define HYS_TOKEN_POLY_PAIRS 8
 #endif
@@ -64,6 +80,7 @@ struct Params {
 
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t kv_half[kStages];   // CTA pair: this CTA's half of the stage has landed
   uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_drain, spare;
   tc::UnitQueue queue;
@@ -75,6 +92,7 @@ struct Cfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVBytes = 128 * D * 2;
+  static constexpr int kHalfBytes = kKVBytes / 2;   // 64 key rows
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kQBytes;
   static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
@@ -109,10 +127,13 @@ __device__ __forceinline__ void fail(volatile int* abort, int* status) {
   report_status(status, HYS_ERR_TIMEOUT);
 }
 
-template <int D>
+// PAIR: the kernel runs as clusters of two CTAs, one unit per cluster at a time (see the top of
+// the file); tmKb / tmVb are K and V with 64-row boxes (part B's half tiles).
+template <int D, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     token_sparse_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                           const __grid_constant__ CUtensorMap tmV, const Params p) {
+                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
+                           const __grid_constant__ CUtensorMap tmVb, const Params p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -122,12 +143,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MT = p.G / 2;
-  const int rounds = (MT + 1) / 2;
+  // M-tile mt = kRoundStride * r + mt0 + s (s = TMEM slot): two per CTA and round, four per pair
+  constexpr int kRoundStride = PAIR ? 4 : 2;
+  const int rounds = (MT + kRoundStride - 1) / kRoundStride;
+  const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;
+  const int mt0 = 2 * (int)rank;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&bars->kv_full[i], 1);
-      tc::mbar_init(&bars->kv_empty[i], 1);
+      tc::mbar_init(&bars->kv_empty[i], PAIR ? 2 : 1);   // pair: both CTAs' MMAs release a stage
+      tc::mbar_init(&bars->kv_half[i], 1);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->q_full[s], 1);
@@ -138,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->o_empty[s], 128);
     }
     tc::mbar_init(&bars->mma_drain, 1);
-    tc::queue_init(&bars->queue, 1 + 256);
+    tc::queue_init(&bars->queue, 1 + 256 + (PAIR ? 1 : 0));   // MMA, softmax, pair: copier
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -146,6 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::prefetch_tensormap(&tmQ);
     tc::prefetch_tensormap(&tmK);
     tc::prefetch_tensormap(&tmV);
+    if (PAIR) {
+      tc::prefetch_tensormap(&tmKb);
+      tc::prefetch_tensormap(&tmVb);
+    }
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_slot, 512);
@@ -154,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  if (PAIR) tc::cluster_sync();   // the partner's barriers are initialised before any copy or commit reaches them
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
@@ -163,11 +194,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t kv_it = 0, q_cnt[2] = {0, 0};
     bool ok = true;
     // the next unit is claimed one unit ahead, so the counter's round trip overlaps a unit's work
+    // (a CTA pair takes units in a fixed order instead: both CTAs must see the same sequence)
     int claim = 0;
-    if (lane == 0) claim = atomicAdd(p.counter, 1);
+    if (!PAIR && lane == 0) claim = atomicAdd(p.counter, 1);
     for (uint32_t n = 0; ok; ++n) {
       int u = 0;
-      if (lane == 0) {
+      if (PAIR) {
+        const int c = (int)(blockIdx.x >> 1) + (int)n * (int)(gridDim.x >> 1);
+        u = c < p.num_units ? c : -1;
+      } else if (lane == 0) {
         u = claim < p.num_units ? claim : -1;
         if (u >= 0) claim = atomicAdd(p.counter, 1);
       }
@@ -226,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < rounds && ok; ++r) {
         if (lane == 0) {
           for (int s = 0; s < 2 && ok; ++s) {
-            const int mt = 2 * r + s;
+            const int mt = kRoundStride * r + mt0 + s;
             if (mt >= MT) continue;
             if (!(ok = tc::mbar_wait(&bars->q_empty[s], (q_cnt[s] & 1u) ^ 1u, abort))) break;
             ++q_cnt[s];
@@ -240,7 +275,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        for (int tau = 0; tau < ntiles && ok; ++tau) {
+        for (int tau = 0; tau < ntiles && ok && PAIR; ++tau) {
+          // this CTA's half of the tile: rows 64 rank .. 64 rank + 63.  Part A: lane = (column
+          // chunk, quad of rows) gathers four rows; part B: one 64-row box per column chunk.
+          const bool part_a = tau < x.n_sp;
+          const int ch = lane >> 4, quad = lane & 15;
+          int rows[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = 128 * tau + 64 * (int)rank + 4 * quad + k;
+            const int pos = (part_a && e < x.nA) ? (e < kMaxList ? plist[e] : sel[e]) : 0;  // padding: row 0 (masked)
+            rows[k] = head_row0 + pos;
+          }
+          const int brow = head_row0 + x.w0 + 128 * (tau - x.n_sp) + 64 * (int)rank;  // past e_I: masked
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t st = kv_it % kStages;
+            if (lane == 0) {
+              ok = tc::mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1u) ^ 1u, abort);
+              if (ok) tc::mbar_arrive_expect_tx(&bars->kv_half[st], C::kHalfBytes);
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            uint8_t* dst = smem + C::kOffKV + st * C::kKVBytes + 64 * (int)rank * 128;
+            if (part_a) {
+              if (ch < C::kChunks)
+                tc::tma_gather4(kv ? &tmV : &tmK, &bars->kv_half[st], dst + ch * 16384 + 4 * quad * 128, ch * 64,
+                                rows[0], rows[1], rows[2], rows[3]);
+            } else if (lane == 0) {
+              for (int c = 0; c < C::kChunks; ++c)
+                tc::tma_load_2d(kv ? &tmVb : &tmKb, &bars->kv_half[st], dst + c * 16384, c * 64, brow);
+            }
+            ++kv_it;
+          }
+        }
+        for (int tau = 0; tau < ntiles && ok && !PAIR; ++tau) {
           // key rows of this lane's quad (rows 4*lane .. 4*lane+3 of the tile)
           int rows[4];
 #pragma unroll
@@ -279,6 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_wait_drain(&bars->kv_full[i % kStages], (i / kStages) & 1u);
       for (int s = 0; s < 2; ++s)
         if (q_cnt[s] > 0) tc::mbar_wait_drain(&bars->q_full[s], (q_cnt[s] - 1) & 1u);
+      // pair: this CTA's own gathers of the last uses, and each stage's last use released by
+      // both MMAs, so every half this CTA sent has been read by the partner before either leaves
+      if (PAIR)
+        for (uint32_t i = (kv_it > kStages ? kv_it - kStages : 0); i < kv_it; ++i) {
+          tc::mbar_wait_drain(&bars->kv_half[i % kStages], (i / kStages) & 1u);
+          tc::mbar_wait_drain(&bars->kv_empty[i % kStages], (i / kStages) & 1u);
+        }
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
@@ -301,6 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                      kk > 0 ? 1u : 0u);
         }
       };
+      // a stage is released to both CTAs of a pair (each gathered half of it)
+      auto release_kv = [&](uint32_t st) {
+        if (PAIR)
+          tc::mma_commit_cluster(&bars->kv_empty[st], 0x3);
+        else
+          tc::mma_commit(&bars->kv_empty[st]);
+      };
       auto issue_PV = [&](int s, uint32_t st, bool acc) {
         const uint32_t vb = kvaddr + st * C::kKVBytes;
 #pragma unroll
@@ -317,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < rounds && ok; ++r) {
           bool act[2];
           for (int s = 0; s < 2; ++s) {
-            act[s] = (2 * r + s) < MT;
+            act[s] = (kRoundStride * r + mt0 + s) < MT;
             if (act[s] && ok) {
               ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort);
               ++q_cnt[s];
@@ -333,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               issue_S(s, kst);
               tc::mma_commit(&bars->s_full[s]);
             }
-          tc::mma_commit(&bars->kv_empty[kst]);
+          release_kv(kst);
           for (int tau = 1; tau <= ntiles && ok; ++tau) {
             const uint32_t vst = kv_it % kStages;
             if (!(ok = tc::mbar_wait(&bars->kv_full[vst], (kv_it / kStages) & 1u, abort))) break;
@@ -363,8 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++o_cnt[s];
               }
             }
-            tc::mma_commit(&bars->kv_empty[vst]);
-            if (have_k) tc::mma_commit(&bars->kv_empty[kst]);
+            release_kv(vst);
+            if (have_k) release_kv(kst);
           }
           for (int s = 0; s < 2; ++s)
             if (act[s]) tc::mma_commit(&bars->q_empty[s]);
@@ -377,6 +459,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+    if (PAIR && warp == 2 && lane == 0) {
+      // ============================================================== copier (CTA pair)
+      // once this CTA's half of a stage has landed, send it into the partner's stage (its bytes
+      // complete the partner's kv_full) and expect the partner's half on our own kv_full
+      const uint32_t peer = rank ^ 1u;
+      uint32_t kv_it = 0;
+      bool ok = true;
+      for (uint32_t n = 0; ok; ++n) {
+        int nA = 0, unused = 0;
+        const int u = tc::queue_peek(&bars->queue, n, abort, ok, &nA, &unused);
+        if (u < 0) break;
+        const Unit x = make_unit(p, u, nA);
+        const int nkv = 2 * rounds * (x.n_sp + x.n_w);
+        for (int i = 0; i < nkv && ok; ++i) {
+          const uint32_t st = kv_it % kStages;
+          if (!(ok = tc::mbar_wait(&bars->kv_half[st], (kv_it / kStages) & 1u, abort))) break;
+          ++kv_it;
+          tc::mbar_arrive_expect_tx(&bars->kv_full[st], C::kHalfBytes);
+          const uint32_t bar_peer = tc::peer_addr(&bars->kv_full[st], peer);
+          for (int c = 0; c < C::kChunks; ++c) {
+            const uint8_t* src = smem + C::kOffKV + st * C::kKVBytes + c * 16384 + 64 * (int)rank * 128;
+            tc::bulk_copy_to_peer(tc::peer_addr(src, peer), src, C::kHalfBytes / C::kChunks, bar_peer);
+          }
+        }
+        tc::queue_release(&bars->queue, n);
+      }
+      if (!ok) fail(abort, p.status);
+    }
   } else {
     // ============================================================== softmax / epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
@@ -397,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t* mask = bars->selmask[n % tc::kQueueSlots];
       const int ntiles = x.n_sp + x.n_w;
       for (int r = 0; r < rounds && ok; ++r) {
-        const int mt = 2 * r + s;
+        const int mt = kRoundStride * r + mt0 + s;
         if (mt >= MT) continue;
         const int h = x.g * p.G + 2 * mt + (row >> 6);
         const int t = 64 * x.I + (row & 63);
@@ -548,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem_base, 512);
   }
+  if (PAIR) tc::cluster_sync();   // neither CTA's shared memory goes away while the partner may use it
 }
 
 // Q: [heads][rows][D], box 64 columns x 64 rows x 1 head
@@ -563,13 +674,14 @@ bool make_q_map(CUtensorMap* m, const void* base, int D, int rows, int heads) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// K or V as a 2-D [B*Hkv*N][D] tensor with a one-row box (64 columns) for tile::gather4
-bool make_gather_map(CUtensorMap* m, const void* base, int D, long long rows) {
+// K or V as a 2-D [B*Hkv*N][D] tensor with a box of 64 columns x box_rows rows (one row for
+// tile::gather4, 64 for part B's half tiles)
+bool make_kv_map(CUtensorMap* m, const void* base, int D, long long rows, int box_rows) {
   EncodeTiledFn fn = tma_encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 1};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -579,13 +691,56 @@ bool make_gather_map(CUtensorMap* m, const void* base, int D, long long rows) {
 int num_units(const PrefillDims& d) { return d.B * d.Hkv * d.T; }
 int grid_size(const PrefillDims& d) { return num_units(d) < kMaxGrid ? num_units(d) : kMaxGrid; }
 
+// The register split assumes exactly kLaunchRegs per thread at launch.
+template <int D, bool PAIR>
+cudaError_t check_regs() {
+  static std::atomic<int> regs{-1};
+  int r = regs.load(std::memory_order_relaxed);
+  if (r < 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, token_sparse_tc_kernel<D, PAIR>);
+    if (e != cudaSuccess) return e;
+    r = fa.numRegs;
+    regs.store(r, std::memory_order_relaxed);
+  }
+  return r == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+// Clusters of two that fit on the device at once (per device; 0 = not known yet).
+template <int D>
+int pair_clusters(cudaStream_t s) {
+  static std::atomic<int> known[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int n = known[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * kMaxGrid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg<D>::kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&n, token_sparse_tc_kernel<D, true>, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  known[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 template <int D>
 cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, const void* v, const int* idx, int kt,
                          int W, void* o, void* ws, cudaStream_t s) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mkb, mvb;
   const long long rows = (long long)d.B * d.Hkv * d.N;
-  if (!make_q_map(&mq, q, D, d.N, d.B * d.Hq) || !make_gather_map(&mk, k, D, rows) ||
-      !make_gather_map(&mv, v, D, rows))
+  if (!make_q_map(&mq, q, D, d.N, d.B * d.Hq) || !make_kv_map(&mk, k, D, rows, 1) ||
+      !make_kv_map(&mv, v, D, rows, 1) || !make_kv_map(&mkb, k, D, rows, 64) || !make_kv_map(&mvb, v, D, rows, 64))
     return cudaErrorInvalidValue;
   Params p;
   p.B = d.B;
@@ -604,19 +759,41 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
-  static int regs = -1;   // the register split assumes exactly kLaunchRegs per thread at launch
-  if (regs < 0) {
-    cudaFuncAttributes fa;
-    cudaError_t e0 = cudaFuncGetAttributes(&fa, token_sparse_tc_kernel<D>);
-    if (e0 != cudaSuccess) return e0;
-    regs = fa.numRegs;
-  }
-  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(token_sparse_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // four or more M-tiles per unit: a single CTA would gather every key tile once per round
+  const bool pair = HYS_TOKEN_PAIR && p.G / 2 >= 3;
+  cudaError_t e = pair ? check_regs<D, true>() : check_regs<D, false>();
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(pair ? token_sparse_tc_kernel<D, true> : token_sparse_tc_kernel<D, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int ncl = 0;
+  if (pair) ncl = std::min(pair_clusters<D>(s), p.num_units);
+  if (ncl > 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * ncl);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, token_sparse_tc_kernel<D, true>, mq, mk, mv, mkb, mvb, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  if (pair) {   // no cluster fits: the single-CTA kernel
+    e = check_regs<D, false>();
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(token_sparse_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
   e = cudaMemsetAsync(p.counter, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
-  token_sparse_tc_kernel<D><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, p);
+  token_sparse_tc_kernel<D, false><<<grid_size(d), kThreads, smem, s>>>(mq, mk, mv, mkb, mvb, p);
   return cudaGetLastError();
 }
 

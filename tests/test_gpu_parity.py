@@ -125,6 +125,11 @@ TOKEN_CASES = [
     ("bf16_d64_small_forced", "bf16", 1, 300, 4, 1, 64, 40, 16),
     ("f32_d64", "f32", 1, 400, 4, 1, 64, 64, 128),
     ("bf16_d128_g8_rounds", "bf16", 1, 1500, 16, 2, 128, 300, 128),
+    # four or more M-tiles per unit run on CTA pairs: D 64, three M-tiles (one idle slot), two
+    # rounds of four, fewer units than the device holds clusters
+    ("bf16_d64_g8_pair", "bf16", 1, 900, 8, 1, 64, 120, 128),
+    ("bf16_d128_g6_pair_b2", "bf16", 2, 1000, 12, 2, 128, 200, 64),
+    ("bf16_d128_g16_pair_2rounds", "bf16", 1, 700, 16, 1, 128, 150, 128),
 ]
 
 
