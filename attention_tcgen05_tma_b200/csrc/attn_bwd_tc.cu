@@ -18,7 +18,8 @@
 //   dQ_m += dS K_j                                                (A = dS^T in shared memory)
 // so that dV = sum_t sigma_t P_ti dO_t, dK = tau sum_t dS_ti q_t and dQ = tau sum_i dS_ti k_i are
 // the gradients of o = sigma * softmax(tau q k^T) v with D_t = sigma_t dO_t . o_t.  dK_j and dV_j
-// stay in TMEM for the whole unit and are written (or added) once; every M-tile's dQ part goes
+// stay in TMEM for the whole unit and are written (or added) once (kModeSparse: a key tile's
+// query tiles come in units of at most 16, whose parts are added atomically); every M-tile's dQ part goes
 // from TMEM through shared memory (the dS^T buffer, free once the dQ MMA has read it) to an fp32
 // accumulator in global memory with TMA reduce-adds, scaled by tau and rounded to the output type
 // afterwards.
@@ -44,6 +45,10 @@ namespace {
 constexpr int kThreads = 384;   // warp 0 TMA, warp 1 MMA, warps 4-7 / 8-11 softmax groups
 constexpr int kD = 128;
 constexpr int kMaxGrid = 148;
+#ifndef HYS_BWD_SPARSE_CHUNK
+#define HYS_BWD_SPARSE_CHUNK 16
+#endif
+constexpr int kSparseChunk = HYS_BWD_SPARSE_CHUNK;   // query tiles per selected-block unit
 constexpr int kTile = 128 * kD * 2;  // 128 rows x 128 bf16: two 64-column swizzled chunks of 16 KB
 constexpr int kModeFull = 0, kModeWindow = 1, kModeSparse = 2;
 
@@ -55,6 +60,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 
 struct Params {
   int B, N, Hq, Hkv, G, MT, NK, T, num_units, window;
+  int chunk;           // kModeSparse: query tiles per unit (a key tile's list is cut into pieces)
   const float* lse2;   // [B,Hq,N] row LSE in log2 units (includes any sink term)
   const float* dsum;   // [B,Hq,N] D_t of this key set
   const float* sig;    // [B,Hq,N] per-row factor sigma_t, or null (1)
@@ -89,36 +95,50 @@ __device__ __forceinline__ void fail(volatile int* abort, int* status) {
 }
 
 
+// four fp32 atomic adds in one vector reduction (relaxed, device scope)
+__device__ __forceinline__ void red_add_v4(float4* dst, float4 x) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(x.x), "f"(x.y), "f"(x.z),
+               "f"(x.w)
+               : "memory");
+}
+
 // unit u -> (b, g, j), key tiles in increasing j across all (b, g) first: small j has the most
-// query tiles in the full and sparse modes, so the longest units start first
-__device__ __forceinline__ void unit_coords(const Params& p, int u, int& b, int& g, int& j, int& lu) {
-  const int bg = u % (p.B * p.Hkv);
-  j = u / (p.B * p.Hkv);
+// query tiles in the full mode, so the longest units start first.  In the selected-block mode a
+// key tile's query tiles come in pieces of at most p.chunk (piece `sub`, pieces outermost):
+// how often a block is selected varies a lot, and one popular key tile as a single unit would
+// outlast the rest of the launch.
+template <int MODE>
+__device__ __forceinline__ void unit_coords(const Params& p, int u, int& b, int& g, int& j, int& lu, int& sub) {
+  const int per = p.B * p.Hkv * p.NK;
+  sub = MODE == kModeSparse ? u / per : 0;
+  const int v = MODE == kModeSparse ? u % per : u;
+  const int bg = v % (p.B * p.Hkv);
+  j = v / (p.B * p.Hkv);
   b = bg / p.Hkv;
   g = bg % p.Hkv;
   lu = bg * p.NK + j;
 }
 
 template <int MODE>
-__device__ __forceinline__ int num_qtiles(const Params& p, int j, int lu) {
+__device__ __forceinline__ int num_qtiles(const Params& p, int j, int lu, int sub) {
   if (MODE == kModeFull) return p.T - 2 * j;
   if (MODE == kModeWindow) {
     const int hi = min(p.T - 1, (128 * j + 127 + p.window - 1) / 64);
     return hi - 2 * j + 1;
   }
-  return p.list_cnt[lu];
+  return min(p.chunk, p.list_cnt[lu] - sub * p.chunk);
 }
 
 // query tile and key-half mask of the unit's M-tile m.  The query tiles run from the last one
 // down: the units running at the same time then reach the same query tiles (and the same dQ
 // accumulator rows) together, so the accumulator's reduce-adds mostly hit L2.
 template <int MODE>
-__device__ __forceinline__ void mtile(const Params& p, int j, int lu, int m, int nmt, int& i, int& hp,
+__device__ __forceinline__ void mtile(const Params& p, int j, int lu, int sub, int m, int nmt, int& i, int& hp,
                                       int& mask) {
   const int n = (nmt - 1 - m) / p.MT;
   hp = m % p.MT;
   if (MODE == kModeSparse) {
-    const int e = p.list[(size_t)lu * p.T + n];
+    const int e = p.list[(size_t)lu * p.T + sub * p.chunk + n];
     i = e >> 2;
     mask = e & 3;
   } else {
@@ -195,9 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool stop = u >= p.num_units || *abort;
     __syncthreads();
     if (stop) break;
-    int b, g, j, lu;
-    unit_coords(p, u, b, g, j, lu);
-    const int nmt = num_qtiles<MODE>(p, j, lu) * p.MT;
+    int b, g, j, lu, sub;
+    unit_coords<MODE>(p, u, b, g, j, lu, sub);
+    const int nmt = num_qtiles<MODE>(p, j, lu, sub) * p.MT;
     if (nmt <= 0) continue;
     const uint32_t par = nu & 1u;
 
@@ -216,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int m = 0; m < nmt && ok; ++m) {
           const uint32_t n = mc + m, st = n & 1u;
           int i, hp, mask;
-          mtile<MODE>(p, j, lu, m, nmt, i, hp, mask);
+          mtile<MODE>(p, j, lu, sub, m, nmt, i, hp, mask);
           if (!(ok = tc::mbar_wait(&bars->q_empty[st], ((n >> 1) & 1u) ^ 1u, abort))) break;
           tc::mbar_arrive_expect_tx(&bars->q_full[st], 2 * kTile);
           for (int hh = 0; hh < 2; ++hh)
@@ -331,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float nl = INFINITY, nd = 0.0f, ns = 1.0f;
       auto load_rows = [&](int m) {
         int i, hp, mask;
-        mtile<MODE>(p, j, lu, m, nmt, i, hp, mask);
+        mtile<MODE>(p, j, lu, sub, m, nmt, i, hp, mask);
         const int head = b * p.Hq + g * p.G + 2 * hp + wg;
         const int pos = 64 * i + (r & 63);
         const size_t rix = (size_t)head * p.N + pos;
@@ -343,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int m = 0; m < nmt && ok; ++m) {
         const uint32_t n = mc + m;
         int i, hp, mask;
-        mtile<MODE>(p, j, lu, m, nmt, i, hp, mask);
+        mtile<MODE>(p, j, lu, sub, m, nmt, i, hp, mask);
         if (r < 64) {
           const int q = 64 * wg + r;
           s_lse[q] = nl;
@@ -461,6 +481,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int e = 0; e < 8; ++e) {
                 float4 x = make_float4(__uint_as_float(v[4 * e]) * f, __uint_as_float(v[4 * e + 1]) * f,
                                        __uint_as_float(v[4 * e + 2]) * f, __uint_as_float(v[4 * e + 3]) * f);
+                if (MODE == kModeSparse) {   // pieces of one key tile may run at the same time
+                  red_add_v4(d4 + e, x);
+                  continue;
+                }
                 if (p.accumulate) {
                   const float4 y = d4[e];
                   x.x += y.x;
@@ -573,7 +597,8 @@ cudaError_t launch_mode(const PrefillDims& d, const void* q, const void* d_o, co
   p.MT = p.G / 2;
   p.NK = (d.N + 127) / 128;
   p.T = d.T;
-  p.num_units = d.B * d.Hkv * p.NK;
+  p.chunk = kSparseChunk;
+  p.num_units = d.B * d.Hkv * p.NK * (MODE == kModeSparse ? (d.T + kSparseChunk - 1) / kSparseChunk : 1);
   p.window = window;
   p.lse2 = lse2;
   p.dsum = dsum;
