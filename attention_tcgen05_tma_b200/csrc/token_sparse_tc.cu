@@ -38,10 +38,12 @@ namespace hys {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kStages = 4;
+#ifndef HYS_TOKEN_STAGES
+#define HYS_TOKEN_STAGES 5
+#endif
+constexpr int kStages = HYS_TOKEN_STAGES;   // K / V stages of 128 keys (shared memory holds five)
 constexpr int kMaxGrid = 148;
 constexpr int kMaskWords = 16;     // extended window <= 512 keys  ->  W <= 449
-constexpr int kMaxList = 4096;     // selected positions kept in shared memory (larger k: read from L2)
 constexpr float kRescaleLog2 = 8.0f;
 #ifndef HYS_TOKEN_PAIR
 #define HYS_TOKEN_PAIR 1
@@ -97,8 +99,8 @@ struct Cfg {
   static constexpr int kOffKV = 2 * kQBytes;
   static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
   static constexpr int kOffMisc = kOffBar + (int)((sizeof(Bars) + 15) / 16 * 16);
-  static constexpr int kOffList = kOffMisc + 64;   // the producer's copy of a unit's positions
-  static constexpr int kSmemBytes = kOffList + kMaxList * 4 + 1024;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct Unit {
@@ -190,7 +192,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ============================================================== producer warp (gathers)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
-    int* plist = reinterpret_cast<int*>(smem + C::kOffList);
     uint32_t kv_it = 0, q_cnt[2] = {0, 0};
     bool ok = true;
     // the next unit is claimed one unit ahead, so the counter's round trip overlaps a unit's work
@@ -240,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool live = lane < first_stop;
             nA += __popc(__ballot_sync(0xffffffffu, live && j < x0.w0));
             if (live && j >= x0.w0 && j <= x0.eI) atomicOr(&mask[(j - x0.w0) >> 5], 1u << ((j - x0.w0) & 31));
-            if (live && e < kMaxList) plist[e] = j;
             if (stop) stopped = true;
           }
         }
@@ -275,6 +275,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        // part A positions of this lane's quad, read from the (L2-resident) index list one tile
+        // ahead of their gathers
+        auto positions = [&](int tau, int (&pos)[4]) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = PAIR ? 128 * tau + 64 * (int)rank + 4 * (lane & 15) + k : 128 * tau + 4 * lane + k;
+            pos[k] = (tau < x.n_sp && e < x.nA) ? __ldg(sel + e) : 0;   // padding: row 0 (masked)
+          }
+        };
+        int nxt[4];
+        positions(0, nxt);
         for (int tau = 0; tau < ntiles && ok && PAIR; ++tau) {
           // this CTA's half of the tile: rows 64 rank .. 64 rank + 63.  Part A: lane = (column
           // chunk, quad of rows) gathers four rows; part B: one 64-row box per column chunk.
@@ -282,11 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ch = lane >> 4, quad = lane & 15;
           int rows[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int e = 128 * tau + 64 * (int)rank + 4 * quad + k;
-            const int pos = (part_a && e < x.nA) ? (e < kMaxList ? plist[e] : sel[e]) : 0;  // padding: row 0 (masked)
-            rows[k] = head_row0 + pos;
-          }
+          for (int k = 0; k < 4; ++k) rows[k] = head_row0 + nxt[k];
+          positions(tau + 1, nxt);
           const int brow = head_row0 + x.w0 + 128 * (tau - x.n_sp) + 64 * (int)rank;  // past e_I: masked
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t st = kv_it % kStages;
@@ -314,16 +322,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int rr = 4 * lane + k;
-            int pos;
-            if (tau < x.n_sp) {
-              const int e = 128 * tau + rr;
-              pos = e < x.nA ? (e < kMaxList ? plist[e] : sel[e]) : 0;  // padding rows read row 0 (masked)
-            } else {
+            int pos = nxt[k];
+            if (tau >= x.n_sp) {
               const int i = x.w0 + 128 * (tau - x.n_sp) + rr;
               pos = i <= x.eI ? i : 0;
             }
             rows[k] = head_row0 + pos;
           }
+          positions(tau + 1, nxt);
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t st = kv_it % kStages;
             if (lane == 0) {
