@@ -49,7 +49,7 @@ constexpr float kRescaleLog2 = 8.0f;
 #define HYS_TOKEN_PAIR 1
 #endif
 #ifndef HYS_TOKEN_POLY_PAIRS
-#define HYS_TOKEN_POLY_PAIRS 8
+#define HYS_TOKEN_POLY_PAIRS 0
 #endif
 // column pairs (of the 64 in a 128-key row) whose exp2 runs on the FMA pipe instead of MUFU
 constexpr int kPolyPairs = HYS_TOKEN_POLY_PAIRS;
@@ -58,7 +58,7 @@ constexpr int kPolyPairs = HYS_TOKEN_POLY_PAIRS;
 // kHighRegs.  The sum must equal three launch shares, or setmaxnreg.inc would wait forever;
 // the host checks the compiled register count before every launch.
 #ifndef HYS_TOKEN_LOW_REGS
-#define HYS_TOKEN_LOW_REGS 104
+#define HYS_TOKEN_LOW_REGS 88
 #endif
 constexpr int kLaunchRegs = 168, kLowRegs = HYS_TOKEN_LOW_REGS, kHighRegs = (3 * kLaunchRegs - kLowRegs) / 2;
 static_assert(kLowRegs % 8 == 0 && kHighRegs % 8 == 0, "setmaxnreg takes multiples of 8");
