@@ -20,16 +20,18 @@
 // the gradients of o = sigma * softmax(tau q k^T) v with D_t = sigma_t dO_t . o_t.  dK_j and dV_j
 // stay in TMEM for the whole unit and are written (or added) once (kModeSparse: a key tile's
 // query tiles come in units of at most 16, whose parts are added atomically); every M-tile's dQ part goes
-// from TMEM through shared memory (the dS^T buffer, free once the dQ MMA has read it) to an fp32
-// accumulator in global memory with TMA reduce-adds, scaled by tau and rounded to the output type
-// afterwards.
+// from TMEM into shared memory over the M-tile's own Q and dO stage (free once its MMAs have read
+// them), and a reduce warp sends it to an fp32 accumulator in global memory with TMA reduce-adds
+// while the next M-tile runs; the stage goes back to the producer once the reduce has read it.
+// dQ is scaled by tau and rounded to the output type afterwards.
 //
 // Warp roles (384 threads): warp 0 TMA producer (K_j, V_j once per unit; Q and dO of every
-// M-tile, two stages), warp 1 MMA issuer (and TMEM owner), warps 4-7 and 8-11 two softmax and
+// M-tile, two stages), warp 1 MMA issuer (and TMEM owner), warp 2 dQ reducer, warps 4-7 and 8-11 two softmax and
 // drain groups (thread = key row r of the tile = TMEM lane; each group takes half of the row's
 // query columns, and half of the head-dim columns in the drains).  TMEM: tS (S^T, then sigma P^T as bf16), tP (dP^T, then
 // dS^T as bf16, then the M-tile's dQ part), tdV, tdK: 4 x 128 columns.  The MMA order per M-tile
-// is dV, dK, dQ (into tP), then S^T of the next M-tile into tS, which overlaps the drain of dQ.
+// is dV, dK, dQ (into tP), then S^T of the next M-tile into tS, then its dP^T once the dQ part
+// has been read out of tP.
 // Every mbarrier wait is bounded; a timeout records HYS_ERR_TIMEOUT, waits (bounded) for the
 // copies and MMAs already issued and frees TMEM.
 #include <cuda.h>
@@ -77,9 +79,9 @@ struct Params {
 };
 
 struct Bars {
-  uint64_t kv_full, kv_empty, q_full[2], q_empty[2], s_full, p_full, dq_full, s_free, ds_free, acc_full, acc_free;
+  uint64_t kv_full, kv_empty, q_full[2], q_red[2], s_full, p_full, dq_full, s_free, ds_free, acc_full, acc_free;
   uint64_t mma_drain, rows_ready[2];
-  uint64_t stage_ready[2], stage_free[2];   // per group: its dQ stage written / read by the TMA reduce
+  uint64_t dq_staged;   // an M-tile's dQ part is in its Q / dO stage (both groups)
 };
 
 constexpr int kOffK = 0, kOffV = kTile, kOffQ = 2 * kTile, kOffDO = 4 * kTile, kOffDS = 6 * kTile;
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bars->kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->q_full[s], 1);
-      tc::mbar_init(&bars->q_empty[s], 1);
+      tc::mbar_init(&bars->q_red[s], 1);   // the stage's dQ part has been read by the TMA reduce
     }
     tc::mbar_init(&bars->s_full, 1);
     tc::mbar_init(&bars->p_full, 256);
@@ -180,10 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bars->mma_drain, 1);
     tc::mbar_init(&bars->rows_ready[0], 128);
     tc::mbar_init(&bars->rows_ready[1], 128);
-    for (int w = 0; w < 2; ++w) {
-      tc::mbar_init(&bars->stage_ready[w], 128);
-      tc::mbar_init(&bars->stage_free[w], 1);
-    }
+    tc::mbar_init(&bars->dq_staged, 256);
     *abort = 0;
     tc::fence_barrier_init();
   }
@@ -237,7 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t n = mc + m, st = n & 1u;
           int i, hp, mask;
           mtile<MODE>(p, j, lu, sub, m, nmt, i, hp, mask);
-          if (!(ok = tc::mbar_wait(&bars->q_empty[st], ((n >> 1) & 1u) ^ 1u, abort))) break;
+          // the stage is free once M-tile n - 2's MMAs and the TMA reduce of its dQ part (staged over
+          // its Q and dO) have read it
+          if (!(ok = tc::mbar_wait(&bars->q_red[st], ((n >> 1) & 1u) ^ 1u, abort))) break;
           tc::mbar_arrive_expect_tx(&bars->q_full[st], 2 * kTile);
           for (int hh = 0; hh < 2; ++hh)
             for (int ch = 0; ch < 2; ++ch) {
@@ -309,7 +310,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < 8; ++kk)   // dK += dS^T Q
             tc::mma_ts(tdK, tP + kk * 8 + (kk >= 4 ? 32 : 0), tc::sdesc_sw128(qb + kk * 2048, 16384, 1024), idAcc,
                        (m > 0 || kk > 0));
-          tc::mma_commit(&bars->q_empty[st]);   // Q_m, dO_m free once these complete
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)   // dQ part = dS K_j : K = 128 keys, 16 per step, into tP
             tc::mma_ss(tP, tc::sdesc_sw128(dsb + kk * 2048, 16384, 1024), tc::sdesc_sw128(kb + kk * 2048, 16384, 1024),
@@ -336,6 +336,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // every MMA of the unit has completed before the next unit (or the TMEM release)
         tc::mma_commit(&bars->mma_drain);
         tc::mbar_wait_drain(&bars->mma_drain, nu & 1u);
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------ dQ reducer
+      // every M-tile's staged dQ part (two 64-row boxes per 32-column chunk) into the fp32
+      // accumulator with TMA reduce-adds; the stage goes back to the producer once read
+      if (lane == 0) {
+        bool ok = true;
+        for (int m = 0; m < nmt && ok; ++m) {
+          const uint32_t n = mc + m, st = n & 1u;
+          int i, hp, mask;
+          mtile<MODE>(p, j, lu, sub, m, nmt, i, hp, mask);
+          if (!(ok = tc::mbar_wait(&bars->dq_staged, n & 1u, abort))) break;
+          const int head0 = b * p.Hq + g * p.G + 2 * hp;
+          for (int c = 0; c < 4; ++c) {
+            const uint8_t* stg = smem + (c < 2 ? kOffQ : kOffDO) + st * kTile + (c & 1) * 16384;
+            tc::tma_reduce_add_3d(&tmDQ, stg, 32 * c, 64 * i, head0);
+            tc::tma_reduce_add_3d(&tmDQ, stg + 8192, 32 * c, 64 * i, head0 + 1);
+          }
+          tc::bulk_commit_group();
+          tc::bulk_wait_group_read0();
+          tc::mbar_arrive(&bars->q_red[st]);
+        }
+        if (!ok) fail(abort, p.status);
       }
     } else if (warp >= 4) {
       // ------------------------------------------------------------ softmax / drains
@@ -424,44 +447,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         tc::mbar_arrive(&bars->p_full);
         // dQ part (TMEM lane r of tP = query row r, 128 fp32 columns): the group's two 32-column
-        // chunks go through its half of the dS^T buffer (free: the dQ MMA has read it) into the
-        // fp32 accumulator with TMA reduce-adds, one 64-row box per head
+        // chunks are read out of TMEM (tP is free for the next dP^T from there on) and staged
+        // over this M-tile's Q stage (group 0) or dO stage (group 1), which its MMAs have finished
+        // reading; the reduce warp sends them to the fp32 accumulator while the next M-tile runs
         if (!(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->dq_full, n & 1u, abort)))) break;
         tc::fence_after_sync();
         {
-          uint8_t* stg = smem + kOffDS + wg * 16384;
-          const bool elected = (warp & 3) == 0 && lane == 0;
-          const int head0 = b * p.Hq + g * p.G + 2 * hp;
-#pragma unroll 1
-          for (int cc = 0; cc < 2 && ok; ++cc) {
-            const int c = 2 * wg + cc;
-            uint32_t v[32];
-            tc::tmem_ld32(tP + 32 * c + lane_off, v);
-            tc::tmem_wait_ld();
-            // the previous round's box has been read out of the stage
-            if (cc > 0 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->stage_free[wg], 0u, abort)))) break;
+          uint32_t v0[32], v1[32];
+          tc::tmem_ld32(tP + 64 * wg + lane_off, v0);
+          tc::tmem_ld32(tP + 64 * wg + 32 + lane_off, v1);
+          tc::tmem_wait_ld();
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bars->s_free);
+          uint8_t* stg = smem + (wg == 0 ? kOffQ : kOffDO) + (n & 1u) * kTile;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<uint4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) =
-                  make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-            tc::fence_proxy_async_shared();   // generic shared-memory writes -> the TMA (async proxy)
-            tc::mbar_arrive(&bars->stage_ready[wg]);
-            if (elected) {
-              if (tc::mbar_wait(&bars->stage_ready[wg], (uint32_t)cc, abort)) {
-                tc::tma_reduce_add_3d(&tmDQ, stg, 32 * c, 64 * i, head0);
-                tc::tma_reduce_add_3d(&tmDQ, stg + 8192, 32 * c, 64 * i, head0 + 1);
-                tc::bulk_commit_group();
-                tc::bulk_wait_group_read0();
-              }
-              tc::mbar_arrive(&bars->stage_free[wg]);
-            }
+          for (int u = 0; u < 8; ++u) {
+            const int o = r * 128 + ((u ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(stg + o) = make_uint4(v0[4 * u], v0[4 * u + 1], v0[4 * u + 2], v0[4 * u + 3]);
+            *reinterpret_cast<uint4*>(stg + 16384 + o) =
+                make_uint4(v1[4 * u], v1[4 * u + 1], v1[4 * u + 2], v1[4 * u + 3]);
           }
-          // the stage is free again before this group writes the next M-tile's dS^T into it
-          if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->stage_free[wg], 1u, abort));
-          if (!ok) break;
+          tc::fence_proxy_async_shared();   // generic shared-memory writes -> the TMA (async proxy)
+          tc::mbar_arrive(&bars->dq_staged);
         }
-        tc::fence_before_sync();
-        tc::mbar_arrive(&bars->s_free);
       }
       // unit epilogue: dK (scaled by tau) and dV of key row r, written or added once
       if (ok && (ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->acc_full, par, abort)))) {
@@ -507,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();   // every role finished the unit (a failed wait set abort)
   }
 
-  if (warp >= 4 && (warp & 3) == 0 && lane == 0) tc::bulk_wait_group0();   // the dQ reductions have landed
+  if (warp == 2 && lane == 0) tc::bulk_wait_group0();   // the dQ reductions have landed
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {
