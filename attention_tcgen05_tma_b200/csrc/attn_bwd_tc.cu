@@ -413,20 +413,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_wait_ld();
           uint32_t pk[16], dk2[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float pv[2], dv[2];
+          for (int e4 = 0; e4 < 8; ++e4) {   // four query columns: the row statistics as float4
+            const int q4 = 32 * c + 4 * e4;
+            const float4 l4 = *reinterpret_cast<const float4*>(s_lse + q4);
+            const float4 g4 = *reinterpret_cast<const float4*>(s_sig + q4);
+            const float4 d4 = *reinterpret_cast<const float4*>(s_dsum + q4);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w},
+                        dsv[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], dv[4];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int q = 32 * c + 2 * e + h2;
-              const int qpos = 64 * i + (q & 63);
+            for (int h = 0; h < 4; ++h) {
+              const int qpos = 64 * i + ((q4 + h) & 63);
               bool vis = row_on && kp <= qpos;
               if (MODE == kModeWindow) vis = vis && kp > qpos - p.window;
-              const float pe = vis ? exp2f(fmaf(__uint_as_float(sr[2 * e + h2]), p.sc, -s_lse[q])) : 0.0f;
-              pv[h2] = pe * s_sig[q];
-              dv[h2] = pe * fmaf(s_sig[q], __uint_as_float(dr[2 * e + h2]), -s_dsum[q]);
+              const float pe = vis ? exp2f(fmaf(__uint_as_float(sr[4 * e4 + h]), p.sc, -lv[h])) : 0.0f;
+              pv[h] = pe * gv[h];
+              dv[h] = pe * fmaf(gv[h], __uint_as_float(dr[4 * e4 + h]), -dsv[h]);
             }
-            pk[e] = tc::pack_bf16x2(pv[0], pv[1]);
-            dk2[e] = tc::pack_bf16x2(dv[0], dv[1]);
+            pk[2 * e4] = tc::pack_bf16x2(pv[0], pv[1]);
+            pk[2 * e4 + 1] = tc::pack_bf16x2(pv[2], pv[3]);
+            dk2[2 * e4] = tc::pack_bf16x2(dv[0], dv[1]);
+            dk2[2 * e4 + 1] = tc::pack_bf16x2(dv[2], dv[3]);
           }
           // packed bf16 pairs over this group's own fp32 columns, behind its reads (the other group
           // is still reading its half): group wg's 32 packed columns start at column 64 wg
