@@ -36,6 +36,8 @@
 // copies and MMAs already issued and frees TMEM.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -405,6 +407,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // visibility of this key row: valid key, selected half (sparse), then per query column
         // the causal line (and the window's lower edge)
         const bool row_on = kp < p.N && (MODE != kModeSparse || ((mask >> (r >> 6)) & 1));
+        // warp-uniform cases: every pair of the warp's rows visible (a key tile wholly before the
+        // query tile, full and selected-block modes), or no visible pair (a key row past N or a
+        // half the query tile did not select): the per-column tests and the exponentials go
+        const int vis_mode = __all_sync(0xffffffffu, row_on && MODE != kModeWindow && 128 * j + 127 <= 64 * i) ? 1
+                             : (__all_sync(0xffffffffu, !row_on) ? 2 : 0);
 #pragma unroll 1
         for (int c = 2 * wg; c < 2 * wg + 2; ++c) {        // 32 query columns per chunk
           uint32_t sr[32], dr[32];
@@ -412,28 +419,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_ld32(tP + 32 * c + lane_off, dr);
           tc::tmem_wait_ld();
           uint32_t pk[16], dk2[16];
+          // P and dS for four query columns at a time (the row statistics as float4); ALL: every
+          // pair visible
+          auto pairs = [&](auto all_tag) {
+            constexpr bool ALL = decltype(all_tag)::value;
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {   // four query columns: the row statistics as float4
-            const int q4 = 32 * c + 4 * e4;
-            const float4 l4 = *reinterpret_cast<const float4*>(s_lse + q4);
-            const float4 g4 = *reinterpret_cast<const float4*>(s_sig + q4);
-            const float4 d4 = *reinterpret_cast<const float4*>(s_dsum + q4);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w},
-                        dsv[4] = {d4.x, d4.y, d4.z, d4.w};
-            float pv[4], dv[4];
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const int q4 = 32 * c + 4 * e4;
+              const float4 l4 = *reinterpret_cast<const float4*>(s_lse + q4);
+              const float4 g4 = *reinterpret_cast<const float4*>(s_sig + q4);
+              const float4 d4 = *reinterpret_cast<const float4*>(s_dsum + q4);
+              const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w},
+                          dsv[4] = {d4.x, d4.y, d4.z, d4.w};
+              float pv[4], dv[4];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int qpos = 64 * i + ((q4 + h) & 63);
-              bool vis = row_on && kp <= qpos;
-              if (MODE == kModeWindow) vis = vis && kp > qpos - p.window;
-              const float pe = vis ? exp2f(fmaf(__uint_as_float(sr[4 * e4 + h]), p.sc, -lv[h])) : 0.0f;
-              pv[h] = pe * gv[h];
-              dv[h] = pe * fmaf(gv[h], __uint_as_float(dr[4 * e4 + h]), -dsv[h]);
+              for (int h = 0; h < 4; ++h) {
+                float pe;
+                if (ALL) {
+                  pe = exp2f(fmaf(__uint_as_float(sr[4 * e4 + h]), p.sc, -lv[h]));
+                } else {
+                  const int qpos = 64 * i + ((q4 + h) & 63);
+                  bool vis = row_on && kp <= qpos;
+                  if (MODE == kModeWindow) vis = vis && kp > qpos - p.window;
+                  pe = vis ? exp2f(fmaf(__uint_as_float(sr[4 * e4 + h]), p.sc, -lv[h])) : 0.0f;
+                }
+                pv[h] = pe * gv[h];
+                dv[h] = pe * fmaf(gv[h], __uint_as_float(dr[4 * e4 + h]), -dsv[h]);
+              }
+              pk[2 * e4] = tc::pack_bf16x2(pv[0], pv[1]);
+              pk[2 * e4 + 1] = tc::pack_bf16x2(pv[2], pv[3]);
+              dk2[2 * e4] = tc::pack_bf16x2(dv[0], dv[1]);
+              dk2[2 * e4 + 1] = tc::pack_bf16x2(dv[2], dv[3]);
             }
-            pk[2 * e4] = tc::pack_bf16x2(pv[0], pv[1]);
-            pk[2 * e4 + 1] = tc::pack_bf16x2(pv[2], pv[3]);
-            dk2[2 * e4] = tc::pack_bf16x2(dv[0], dv[1]);
-            dk2[2 * e4 + 1] = tc::pack_bf16x2(dv[2], dv[3]);
+          };
+          if (vis_mode == 1) {
+            pairs(std::true_type{});
+          } else if (vis_mode == 2) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = dk2[e] = 0u;
+          } else {
+            pairs(std::false_type{});
           }
           // packed bf16 pairs over this group's own fp32 columns, behind its reads (the other group
           // is still reading its half): group wg's 32 packed columns start at column 64 wg
