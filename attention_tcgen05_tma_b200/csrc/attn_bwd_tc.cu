@@ -426,8 +426,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
               const int q4 = 32 * c + 4 * e4;
+              // (the full layer has no per-row factor: sigma = 1)
               const float4 l4 = *reinterpret_cast<const float4*>(s_lse + q4);
-              const float4 g4 = *reinterpret_cast<const float4*>(s_sig + q4);
+              const float4 g4 = MODE == kModeFull ? make_float4(1.0f, 1.0f, 1.0f, 1.0f)
+                                                  : *reinterpret_cast<const float4*>(s_sig + q4);
               const float4 d4 = *reinterpret_cast<const float4*>(s_dsum + q4);
               const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w},
                           dsv[4] = {d4.x, d4.y, d4.z, d4.w};
