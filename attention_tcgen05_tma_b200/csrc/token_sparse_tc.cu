@@ -26,6 +26,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdlib>
 
 #include "cluster_ptx.cuh"
 #include "common.cuh"
@@ -765,8 +766,14 @@ cudaError_t launch_typed(const PrefillDims& d, const void* q, const void* k, con
   p.status = device_status_ptr();
   p.scale_log2 = kLog2e / sqrtf((float)D);
   const int smem = Cfg<D>::kSmemBytes;
-  // four or more M-tiles per unit: a single CTA would gather every key tile once per round
-  const bool pair = HYS_TOKEN_PAIR && p.G / 2 >= 3;
+  // four or more M-tiles per unit: a single CTA would gather every key tile once per round.
+  // HYS_TOKEN_SINGLE_CTA=1 (tests only) keeps the single-CTA kernel, the path taken where no
+  // cluster of two fits, so that its rounds are checked too
+  static const bool single_forced = [] {
+    const char* e = getenv("HYS_TOKEN_SINGLE_CTA");
+    return e != nullptr && e[0] == '1';
+  }();
+  const bool pair = HYS_TOKEN_PAIR && p.G / 2 >= 3 && !single_forced;
   cudaError_t e = pair ? check_regs<D, true>() : check_regs<D, false>();
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(pair ? token_sparse_tc_kernel<D, true> : token_sparse_tc_kernel<D, false>,
