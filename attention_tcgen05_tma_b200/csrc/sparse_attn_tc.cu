@@ -46,6 +46,7 @@ constexpr int kStages = 4;
 constexpr int kMaxGrid = 148;
 constexpr int kMaxKb = 1024;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr float kRescaleSum = 256.0f;   // 2^kRescaleLog2
 #ifndef HYS_SPARSE_POLY_PAIRS
 #define HYS_SPARSE_POLY_PAIRS 4
 #endif
@@ -445,6 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               ++kv_it;
             }
             bool have_k = false;
+            // the next K tile before the first slot's P.V, so that S follows P.V without a wait
+            if (tau < ntiles) {
+              kst = kv_it % kStages;
+              if (!(ok = tc::mbar_wait(&bars->kv_full[kst], (kv_it / kStages) & 1u, abort))) break;
+              ++kv_it;
+              have_k = true;
+              tc::fence_after_sync();
+            }
             for (int s = 0; s < 2 && ok; ++s) {
               if (!act[s]) continue;
               // p_full: the softmax is done with S_s(tau-1) (and wrote P unless it was a statistics tile)
@@ -614,32 +623,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float2 sc2 = make_float2(sc, sc);
           // P = exp2(s sc - ms) for the whole row, written to TMEM as bf16 over S; returns the
-          // row sum and (three-input max chains on the ALU, beside the MUFU work) the row max
-          auto emit_p = [&](float ms, float& rmax) -> float {
+          // row sum
+          auto emit_p = [&](float ms) -> float {
             const float2 nm2 = make_float2(-ms, -ms);
             float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-            float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t pk[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float s0 = sv[32 * c + 2 * i], s1 = sv[32 * c + 2 * i + 1];
-                mk[i & 3] = tc::fmax3(mk[i & 3], s0, s1);
                 const float2 pv = exp2_pair(tc::ffma2(make_float2(s0, s1), sc2, nm2), 16 * c + i);
                 acc[i & 1] = tc::fadd2(acc[i & 1], pv);
                 pk[i] = tc::pack_bf16x2(pv.x, pv.y);
               }
               tc::tmem_st16(tSrow + 16 * c, pk);
             }
-            rmax = tc::fmax3(fmaxf(mk[0], mk[1]), mk[2], mk[3]);
             const float2 a = tc::fadd2(acc[0], acc[1]);
             return a.x + a.y;
           };
           if (kind == kWinPV) {
             // window P.V pass with the final statistics; pw holds the combined exponent offset
-            float unused;
-            emit_p(pw, unused);
+            emit_p(pw);
           } else if (kind == kWinStats) {
             // window statistics only: running max and sum, no P, no P.V
             const float mx = fmaxf(tc::max64(sv), tc::max64(sv + 64));
@@ -665,22 +670,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
             // Sparse tile.  The row max is needed first only while the row has none: later
-            // tiles compute P with the running max m_used straight away and find the tile max
-            // beside it; a row whose max rose by more than 2^kRescaleLog2 redoes the tile with
-            // the new max (rare), and O is rescaled.  Warp-uniform branches only: the TMEM
-            // loads and stores are warp-collective.
+            // tiles compute P with the running max m_used straight away.  While no score
+            // exceeds m_used every P is at most 1, so only a tile sum above 2^kRescaleLog2 can
+            // hide a P above 2^kRescaleLog2: such a row takes its tile max, redoes the tile
+            // with it (rare), and O is rescaled.  Warp-uniform branches only: the TMEM loads
+            // and stores are warp-collective.
             if (m_used == -INFINITY) m_used = fmaxf(tc::max64(sv), tc::max64(sv + 64));
-            float mx;
-            float lt = emit_p(m_used == -INFINITY ? 0.0f : m_used * sc, mx);
+            float lt = emit_p(m_used == -INFINITY ? 0.0f : m_used * sc);
             float alpha = 1.0f;
-            const bool rescale = mx > -INFINITY && (mx - m_used) * sc > kRescaleLog2;
-            if (__any_sync(0xffffffffu, rescale)) {
+            bool rescale = false;
+            if (__any_sync(0xffffffffu, lt > kRescaleSum)) {
+              const float mx = fmaxf(tc::max64(sv), tc::max64(sv + 64));
+              rescale = lt > kRescaleSum && mx > m_used;
               if (rescale) {
                 alpha = exp2f((m_used - mx) * sc);
                 m_used = mx;
               }
-              float unused;
-              lt = emit_p(m_used * sc, unused);   // unchanged rows write the same P again
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+              lt = emit_p(m_used * sc);   // unchanged rows write the same P again
               if (tau > 0) {
                 uint32_t ov[D];
 #pragma unroll
