@@ -328,7 +328,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const Unit x = make_unit(p, u, nsel, diag);
         const int ntiles = num_tiles(x);
+        // part kv (0: K, 1: V) of tile tau into the next stage
+        auto load_kv = [&](int tau, int kv) -> bool {
+          const int kind = tile_kind(x, tau);
+          const bool swa = kind != kSparse;
+          const int wi = kind == kWinStats ? tau - x.n_sp : tau - x.n_sp - x.n_sw;  // window pair
+          int jj[2];
+          for (int hh = 0; hh < 2; ++hh) {
+            if (!swa) {
+              const int e = 2 * tau + hh;
+              jj[hh] = e < x.nsel ? plist[e] : -1;
+            } else {
+              const int j = x.jw0 + 2 * wi + hh;
+              jj[hh] = j <= x.I ? j : -1;
+            }
+          }
+          const uint32_t st = kv_it % kStages;
+          if (!tc::mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1u) ^ 1u, abort)) return false;
+          tc::mbar_arrive_expect_tx(&bars->kv_full[st], C::kKVBytes);
+          uint8_t* dst = smem + C::kOffKV + st * C::kKVBytes;
+          const CUtensorMap* map = swa ? (kv ? &tmVs : &tmKs) : (kv ? &tmV : &tmK);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int row = jj[hh] >= 0 ? 64 * jj[hh] : p.N;  // empty half: rows past the end read as zeros
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tc::tma_load_3d(map, &bars->kv_full[st], dst + ch * 16384 + hh * 8192, ch * 64, row,
+                              x.b * p.Hkv + x.g);
+          }
+          ++kv_it;
+          return true;
+        };
         for (int r = 0; r < rounds && ok; ++r) {
+          // The round's first K tile goes ahead of its Q tiles: its stage is free well before the
+          // previous round's last MMA releases Q, and the Q tiles (HBM reads that the TMA unit
+          // serves one after another) would otherwise hold it back.
+          if (!(ok = load_kv(0, 0))) break;
           for (int s = 0; s < 2 && ok; ++s) {
             const int mt = 2 * r + s;
             if (mt >= MT) continue;
@@ -342,35 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::tma_load_3d(&tmQ, &bars->q_full[s], qdst + ch * 16384 + hh * 8192, ch * 64, 64 * x.I,
                                 x.b * p.Hq + h0 + hh);
           }
-          for (int tau = 0; tau < ntiles && ok; ++tau) {
-            const int kind = tile_kind(x, tau);
-            const bool swa = kind != kSparse;
-            const int wi = kind == kWinStats ? tau - x.n_sp : tau - x.n_sp - x.n_sw;  // window pair
-            int jj[2];
-            for (int hh = 0; hh < 2; ++hh) {
-              if (!swa) {
-                const int e = 2 * tau + hh;
-                jj[hh] = e < x.nsel ? plist[e] : -1;
-              } else {
-                const int j = x.jw0 + 2 * wi + hh;
-                jj[hh] = j <= x.I ? j : -1;
-              }
-            }
-            for (int kv = 0; kv < (kind == kWinStats ? 1 : 2); ++kv) {
-              const uint32_t st = kv_it % kStages;
-              if (!(ok = tc::mbar_wait(&bars->kv_empty[st], ((kv_it / kStages) & 1u) ^ 1u, abort))) break;
-              tc::mbar_arrive_expect_tx(&bars->kv_full[st], C::kKVBytes);
-              uint8_t* dst = smem + C::kOffKV + st * C::kKVBytes;
-              const CUtensorMap* map = swa ? (kv ? &tmVs : &tmKs) : (kv ? &tmV : &tmK);
-              for (int hh = 0; hh < 2; ++hh) {
-                const int row = jj[hh] >= 0 ? 64 * jj[hh] : p.N;  // empty half: rows past the end read as zeros
-                for (int ch = 0; ch < C::kChunks; ++ch)
-                  tc::tma_load_3d(map, &bars->kv_full[st], dst + ch * 16384 + hh * 8192, ch * 64, row,
-                                  x.b * p.Hkv + x.g);
-              }
-              ++kv_it;
-            }
-          }
+          for (int tau = 0; tau < ntiles && ok; ++tau)
+            for (int kv = (tau == 0 ? 1 : 0); kv < (tile_kind(x, tau) == kWinStats ? 1 : 2) && ok; ++kv)
+              ok = load_kv(tau, kv);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -418,23 +425,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ntiles = num_tiles(x);
         for (int r = 0; r < rounds && ok; ++r) {
           bool act[2];
-          for (int s = 0; s < 2; ++s) {
-            act[s] = (2 * r + s) < MT;
-            if (act[s] && ok) {
-              ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort);
-              ++q_cnt[s];
-            }
-          }
-          if (!ok) break;
+          for (int s = 0; s < 2; ++s) act[s] = (2 * r + s) < MT;
+          // the round's first K tile (loaded ahead of the Q tiles), then each slot's S as soon as
+          // its Q has landed
           uint32_t kst = kv_it % kStages;
           if (!(ok = tc::mbar_wait(&bars->kv_full[kst], (kv_it / kStages) & 1u, abort))) break;
           ++kv_it;
-          tc::fence_after_sync();
-          for (int s = 0; s < 2; ++s)
+          for (int s = 0; s < 2 && ok; ++s)
             if (act[s]) {
+              if (!(ok = tc::mbar_wait(&bars->q_full[s], q_cnt[s] & 1u, abort))) break;
+              ++q_cnt[s];
+              tc::fence_after_sync();
               issue_S(s, kst);
               tc::mma_commit(&bars->s_full[s]);
             }
+          if (!ok) break;
           tc::mma_commit(&bars->kv_empty[kst]);
           bool pv_started = false;  // O of this round already holds a P.V product
           for (int tau = 1; tau <= ntiles && ok; ++tau) {
