@@ -692,17 +692,22 @@ def run_decode(args, torch, dist, rank, world, dev, peaks, peak_src):
 
 
 def token_sparse_flops(idx_np, N, G, D, W, block=64):
-    """Algorithmic flops of one token-sparse layer: 4*D per (row, head, attended key), the
-    attended set being the tile's selected tokens (all before the row's window) plus the
-    row's newest W tokens."""
+    """Algorithmic flops of one token-sparse layer: 4*D per (row, head, attended key).  Row t of
+    tile I attends Sel_I and its newest W tokens [max(0, t-W+1), t], each key once.  Every
+    selected token is at most e_I - W < 64 I <= t, so the selected tokens at or after t - W + 1
+    are the ones the two sets share."""
     B, Hkv, T, k = idx_np.shape
-    nsel = (idx_np >= 0).sum(-1)                                  # [B, Hkv, T]
-    rows = np.arange(N)
-    win = np.minimum(rows + 1, W)
-    per_tile_rows = np.array([min(N, (I + 1) * block) - I * block for I in range(T)])
-    win_tile = np.add.reduceat(win, np.arange(0, N, block))
-    total = int((nsel * per_tile_rows[None, None, :]).sum()) * G + int(win_tile.sum()) * B * Hkv * G
-    return 4.0 * D * total
+    win = np.minimum(np.arange(N) + 1, W)
+    total = 0
+    for b in range(B):
+        for g in range(Hkv):
+            for I in range(T):
+                sel = idx_np[b, g, I]
+                sel = np.sort(sel[sel >= 0])
+                t = np.arange(I * block, min(N, (I + 1) * block))
+                shared = sel.size - np.searchsorted(sel, t - W + 1, side="left")
+                total += int((sel.size + win[t] - shared).sum())
+    return 4.0 * D * total * G
 
 
 def run_token(args, torch, dist, rank, world, dev, peaks, peak_src):

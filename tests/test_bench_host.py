@@ -54,3 +54,38 @@ def test_cpu_baseline_is_unbiased_over_tile_position():
     b = bench.cpu_baseline(w, budget_s=60.0, n_tiles=16, seed=2)
     assert a["tiles"] == 1 and b["tiles"] == 16
     assert 0.2 < a["value"] / b["value"] < 5.0
+
+
+def _brute_attended(idx, N, W, block):
+    """Per (b, g, row): |Sel_I ∪ [max(0, t-W+1), t]| by explicit sets."""
+    B, Hkv, T, _ = idx.shape
+    n = 0
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(N):
+                sel = {int(i) for i in idx[b, g, t // block] if i >= 0}
+                n += len(sel | set(range(max(0, t - W + 1), t + 1)))
+    return n
+
+
+def test_token_sparse_flops_count_each_attended_key_once():
+    """The token-sparse layer's algorithmic flops: 4*D per (row, head, key of the union of the
+    tile's selected tokens and the row's newest W), checked against explicit sets on a small
+    ragged case whose selections reach up to the window."""
+    import numpy as np
+    rng = np.random.default_rng(5)
+    B, Hkv, G, D, N, W, block, kt = 1, 2, 3, 16, 333, 128, 64, 24
+    T = (N + block - 1) // block
+    idx = np.full((B, Hkv, T, kt), -1, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            for I in range(T):
+                e_I = min(64 * I + 63, N - 1)
+                cand = np.arange(0, e_I - W + 1)
+                if cand.size == 0:
+                    continue
+                pick = np.sort(rng.choice(cand, size=min(kt, cand.size), replace=False))
+                pick[-1] = cand[-1]   # the last candidate sits inside every row's window but the tile's last
+                idx[b, g, I, :pick.size] = pick
+    want = 4.0 * D * G * _brute_attended(idx, N, W, block)
+    assert bench.token_sparse_flops(idx, N, G, D, W, block) == want
