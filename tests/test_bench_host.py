@@ -89,3 +89,26 @@ def test_token_sparse_flops_count_each_attended_key_once():
                 idx[b, g, I, :pick.size] = pick
     want = 4.0 * D * G * _brute_attended(idx, N, W, block)
     assert bench.token_sparse_flops(idx, N, G, D, W, block) == want
+
+
+def test_block_sparse_flops_count_visible_keys_of_both_branches():
+    """The block-sparse layer's algorithmic flops: 4*D per (row, head) for each causally visible
+    key of the selected blocks plus each key of the row's window branch, against explicit counts
+    on a small ragged case."""
+    import numpy as np
+    rng = np.random.default_rng(7)
+    B, Hkv, G, D, N, W, block, kb = 2, 1, 2, 8, 300, 100, 64, 3
+    T = (N + block - 1) // block
+    idx = np.full((B, Hkv, T, kb), -1, dtype=np.int32)
+    for b in range(B):
+        for I in range(T):
+            pick = np.sort(rng.choice(I + 1, size=min(kb, I + 1), replace=False))
+            idx[b, 0, I, :pick.size] = pick
+    n = 0
+    for b in range(B):
+        for t in range(N):
+            for j in idx[b, 0, t // block]:
+                if j >= 0:
+                    n += len([i for i in range(64 * j, 64 * j + 64) if i <= t])
+            n += len(range(max(0, t - W + 1), t + 1))
+    assert bench.sparse_flops(idx, N, G, D, W, block) == 4.0 * D * G * n
